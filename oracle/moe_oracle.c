@@ -1,0 +1,351 @@
+/*
+ * Plain CPU oracle of the forward pass of the biased-sigmoid-routed MoE FFN layer
+ * (Step-3.5-Flash / Step-5-Preview), written from the method's description.
+ *
+ * TEST INFRASTRUCTURE ONLY. Tests, the package's smoke check and the benchmark's
+ * CPU-baseline leg may load this library; the product path never does. It shares
+ * no code, header or constant with the CUDA library.
+ *
+ * Sources (page titles and sections):
+ *  [MAX-MoE]    "MAX 中 Step-3.5-Flash 架构解析", section "MoE共享专家、sigmoid 路由与激活裁剪":
+ *               scores = sigmoid(gate(x)) with the gate matmul forced to FP32; the fp32
+ *               per-expert router_bias is added for top-k selection only; the weights
+ *               come from the uncorrected scores, are optionally normalised to sum 1
+ *               and then multiplied by the routing scale; indices are clamped to
+ *               [0, E-1]; output = routed_moe(x) + shared_expert(x); routed and shared
+ *               experts take their own SwiGLU clip limit.
+ *  [MAX-Config] same page, section "Step3p5Config配置项全解": moe_top_k,
+ *               moe_router_scaling_factor = 3.0, norm_expert_weight, swiglu_limits /
+ *               swiglu_limits_shared with 0.0 meaning no clip.
+ *  [MAX-Weights] same page, section "权重适配从 HF checkpoint 到 MAX 布局": experts
+ *               stacked [num_experts, ...], router_bias kept in float32.
+ *  [miles-5.3]  miles Step-5-Preview recipe page, section 5.3: 24 MiB and 12 MiB BF16
+ *               expert tensors, i.e. a fused [2I, H] gate_up and a [H, I] down matrix.
+ *
+ * Readings where the pages leave a step open (all restated in the design notes):
+ *  - clip form: a = min(silu(g), L), u = clamp(u, -L, L), h = a*u; L = 0 means no clip;
+ *  - gate_up rows: gate rows first, then up rows;
+ *  - selection order: biased score descending, ties to the lower expert index, a NaN
+ *    biased score below every number (ties among NaNs by index), -0.0 equal to +0.0;
+ *  - normalisation has no epsilon; if the selected scores sum to 0 every selected
+ *    weight is scale/k; without normalisation the weight is scale*s;
+ *  - margin = (k-th biased score) - ((k+1)-th biased score) in fp32, +inf when k = E.
+ *
+ * Precision: inputs are bf16 bit patterns (decoded exactly). The router logit is the
+ * dot product accumulated in double and rounded once to fp32 (the FP32 gate); the
+ * score is sigmoid evaluated in double from that fp32 logit and rounded to fp32; the
+ * biased score is an fp32 addition. Everything after selection (weights, expert
+ * MLPs, combine) is evaluated in double; nothing is rounded to bf16.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double bf(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* [MAX-MoE] gate(x) in FP32: logits[t,e] = fp32( sum_h x[t,h] * Wr[e,h] ), summed in
+ * ascending h in double. */
+void oracle_router_logits(int64_t T, int H, int E, const uint16_t *x, const uint16_t *Wr,
+                          float *logits)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *xr = x + t * (int64_t)H;
+        for (int e = 0; e < E; ++e) {
+            const uint16_t *wr = Wr + (int64_t)e * H;
+            double acc = 0.0;
+            for (int h = 0; h < H; ++h)
+                acc += bf(xr[h]) * bf(wr[h]);
+            logits[t * (int64_t)E + e] = (float)acc;
+        }
+    }
+}
+
+/* Selection order (reading stated above): is expert a ranked before expert b? */
+static int ranks_before(float ba, int ea, float bb, int eb)
+{
+    int na = isnan(ba), nb = isnan(bb);
+    if (na != nb)
+        return nb; /* the number ranks before the NaN */
+    if (!na && ba != bb)
+        return ba > bb;
+    return ea < eb;
+}
+
+/* [MAX-MoE], [MAX-Config]: for each token, s = sigmoid(logit) in fp32,
+ * corrected = s + router_bias (fp32), top-k on corrected, weights from s,
+ * normalised to sum 1 when norm != 0, times scale. Ids are reported in rank order.
+ * w64 (double) and w32 (fp32 rounding of w64) may each be NULL, as may margin and
+ * scores. */
+void oracle_router_select(int64_t T, int E, int k, const float *logits, const float *bias,
+                          float scale, int norm, int32_t *idx, float *w32, double *w64,
+                          float *margin, float *scores)
+{
+#pragma omp parallel
+    {
+        float *s = (float *)malloc(sizeof(float) * (size_t)E);
+        float *b = (float *)malloc(sizeof(float) * (size_t)E);
+        char *taken = (char *)malloc((size_t)E);
+        int *order = (int *)malloc(sizeof(int) * (size_t)(k + 1));
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            const float *l = logits + t * (int64_t)E;
+            for (int e = 0; e < E; ++e) {
+                s[e] = (float)(1.0 / (1.0 + exp(-(double)l[e])));
+                b[e] = s[e] + bias[e];
+                taken[e] = 0;
+                if (scores)
+                    scores[t * (int64_t)E + e] = s[e];
+            }
+            int nrank = k < E ? k + 1 : E;
+            /* selection by repeated scan: rank r takes the best expert not yet taken */
+            for (int r = 0; r < nrank; ++r) {
+                int best = -1;
+                for (int e = 0; e < E; ++e) {
+                    if (taken[e])
+                        continue;
+                    if (best < 0 || ranks_before(b[e], e, b[best], best))
+                        best = e;
+                }
+                taken[best] = 1;
+                order[r] = best;
+            }
+            double sum = 0.0;
+            for (int j = 0; j < k; ++j)
+                sum += (double)s[order[j]];
+            for (int j = 0; j < k; ++j) {
+                int e = order[j];
+                /* [MAX-MoE] clamp to [0, E-1] as a guard (always in range here) */
+                if (e < 0)
+                    e = 0;
+                if (e > E - 1)
+                    e = E - 1;
+                double w;
+                if (norm)
+                    w = sum > 0.0 ? (double)scale * (double)s[e] / sum : (double)scale / k;
+                else
+                    w = (double)scale * (double)s[e];
+                idx[t * k + j] = e;
+                if (w64)
+                    w64[t * k + j] = w;
+                if (w32)
+                    w32[t * k + j] = (float)w;
+            }
+            if (margin)
+                margin[t] = k < E ? b[order[k - 1]] - b[order[k]] : INFINITY;
+        }
+        free(s);
+        free(b);
+        free(taken);
+        free(order);
+    }
+}
+
+/* Token -> slot permutation (histogram, exclusive scan, stable scatter) as a plain
+ * counting sort by expert, stable in token order. Group E is the shared expert: it
+ * holds every token in order. counts[E+1], offsets[E+2], perm_token[T*k+T],
+ * slot_of[T*k]. Returns -1 (and writes nothing further) on an id outside [0, E-1]. */
+int oracle_permute(int64_t T, int k, int E, const int32_t *idx, int32_t *counts,
+                   int32_t *offsets, int32_t *perm_token, int32_t *slot_of)
+{
+    for (int e = 0; e <= E; ++e)
+        counts[e] = 0;
+    for (int64_t n = 0; n < T * k; ++n) {
+        if (idx[n] < 0 || idx[n] >= E)
+            return -1;
+        counts[idx[n]] += 1;
+    }
+    counts[E] = (int32_t)T;
+    offsets[0] = 0;
+    for (int e = 0; e <= E; ++e)
+        offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *cursor = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E + 1));
+    for (int e = 0; e <= E; ++e)
+        cursor[e] = offsets[e];
+    for (int64_t t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int e = idx[t * k + j];
+            int32_t slot = cursor[e]++;
+            perm_token[slot] = (int32_t)t;
+            slot_of[t * k + j] = slot;
+        }
+        perm_token[cursor[E]++] = (int32_t)t;
+    }
+    free(cursor);
+    return 0;
+}
+
+/* SwiGLU hidden activation of one token through one expert ([MAX-MoE] clipped
+ * activation; [miles-5.3] fused [2I, H] gate_up, gate rows first):
+ *   g_i = sum_h Wgu[i,h] x_h, u_i = sum_h Wgu[I+i,h] x_h,
+ *   a_i = silu(g_i), clipped a_i = min(a_i, L), u_i = clamp(u_i, -L, L) when L > 0,
+ *   hid_i = a_i * u_i. */
+void oracle_swiglu_hidden(int H, int Iw, const uint16_t *x_row, const uint16_t *Wgu,
+                          double limit, double *hid)
+{
+    for (int i = 0; i < Iw; ++i) {
+        const uint16_t *wg = Wgu + (int64_t)i * H;
+        const uint16_t *wu = Wgu + (int64_t)(Iw + i) * H;
+        double g = 0.0, u = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double xv = bf(x_row[h]);
+            g += bf(wg[h]) * xv;
+            u += bf(wu[h]) * xv;
+        }
+        double a = g / (1.0 + exp(-g));
+        if (limit > 0.0) {
+            if (a > limit)
+                a = limit;
+            if (u > limit)
+                u = limit;
+            if (u < -limit)
+                u = -limit;
+        }
+        hid[i] = a * u;
+    }
+}
+
+/* One expert MLP on one token: out_f = sum_i Wd[f,i] * hid_i, Wd [H, Iw]. */
+void oracle_swiglu_mlp(int H, int Iw, const uint16_t *x_row, const uint16_t *Wgu,
+                       const uint16_t *Wd, double limit, double *out, double *hid)
+{
+    oracle_swiglu_hidden(H, Iw, x_row, Wgu, limit, hid);
+    for (int f = 0; f < H; ++f) {
+        const uint16_t *wd = Wd + (int64_t)f * Iw;
+        double acc = 0.0;
+        for (int i = 0; i < Iw; ++i)
+            acc += bf(wd[i]) * hid[i];
+        out[f] = acc;
+    }
+}
+
+/* [MAX-MoE] layer output for a list of tokens:
+ *   y = sum_j w_j * MLP_{e_j}(x; L_routed) + MLP_shared(x; L_shared),
+ * routed terms summed in rank order, then the shared expert, in double.
+ * Routed weights are given per expert id (Wgu_by_e[e] -> [2I, H], Wd_by_e[e] ->
+ * [H, I]); an entry may be NULL when no listed token selects that expert.
+ * Returns -1 if a selected expert's pointer is NULL, else 0. idx, w and margin
+ * (each optional) receive the routing of every listed token. */
+int oracle_forward_tokens(int64_t ntok, int H, int E, int k, int I, int Is, float scale,
+                          int norm, float limit_routed, float limit_shared,
+                          const uint16_t *x_rows, const uint16_t *Wr, const float *bias,
+                          const uint16_t *const *Wgu_by_e, const uint16_t *const *Wd_by_e,
+                          const uint16_t *Wsh_gu, const uint16_t *Wsh_d, double *y,
+                          int32_t *idx_out, double *w_out, float *margin_out)
+{
+    float *logits = (float *)malloc(sizeof(float) * (size_t)(ntok * E));
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)(ntok * k));
+    double *w = (double *)malloc(sizeof(double) * (size_t)(ntok * k));
+    float *margin = (float *)malloc(sizeof(float) * (size_t)ntok);
+    oracle_router_logits(ntok, H, E, x_rows, Wr, logits);
+    oracle_router_select(ntok, E, k, logits, bias, scale, norm, idx, NULL, w, margin, NULL);
+    int missing = 0;
+    for (int64_t n = 0; n < ntok * k; ++n)
+        if (!Wgu_by_e[idx[n]] || !Wd_by_e[idx[n]])
+            missing = 1;
+    if (!missing) {
+#pragma omp parallel
+        {
+            int Imax = I > Is ? I : Is;
+            double *hid = (double *)malloc(sizeof(double) * (size_t)Imax);
+            double *o = (double *)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t t = 0; t < ntok; ++t) {
+                const uint16_t *xr = x_rows + t * (int64_t)H;
+                double *yr = y + t * (int64_t)H;
+                for (int f = 0; f < H; ++f)
+                    yr[f] = 0.0;
+                for (int j = 0; j < k; ++j) {
+                    int e = idx[t * k + j];
+                    oracle_swiglu_mlp(H, I, xr, Wgu_by_e[e], Wd_by_e[e], limit_routed, o, hid);
+                    for (int f = 0; f < H; ++f)
+                        yr[f] += w[t * k + j] * o[f];
+                }
+                oracle_swiglu_mlp(H, Is, xr, Wsh_gu, Wsh_d, limit_shared, o, hid);
+                for (int f = 0; f < H; ++f)
+                    yr[f] += o[f];
+            }
+            free(hid);
+            free(o);
+        }
+    }
+    if (idx_out)
+        memcpy(idx_out, idx, sizeof(int32_t) * (size_t)(ntok * k));
+    if (w_out)
+        memcpy(w_out, w, sizeof(double) * (size_t)(ntok * k));
+    if (margin_out)
+        memcpy(margin_out, margin, sizeof(float) * (size_t)ntok);
+    free(logits);
+    free(idx);
+    free(w);
+    free(margin);
+    return missing ? -1 : 0;
+}
+
+/* Dense brute force of the same layer: every expert runs on every token and a
+ * [T, E] mask-weight matrix (the selection weight, 0 for unselected experts) mixes
+ * them, experts summed in ascending index order, plus the shared expert. Stacked
+ * weights: W_gate_up [E, 2I, H], W_down [E, H, I]. */
+void oracle_forward_dense(int64_t T, int H, int E, int k, int I, int Is, float scale,
+                          int norm, float limit_routed, float limit_shared,
+                          const uint16_t *x, const uint16_t *Wr, const float *bias,
+                          const uint16_t *W_gate_up, const uint16_t *W_down,
+                          const uint16_t *Wsh_gu, const uint16_t *Wsh_d, double *y)
+{
+    float *logits = (float *)malloc(sizeof(float) * (size_t)(T * E));
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T * k));
+    double *w = (double *)malloc(sizeof(double) * (size_t)(T * k));
+    double *mask = (double *)calloc((size_t)(T * E), sizeof(double));
+    oracle_router_logits(T, H, E, x, Wr, logits);
+    oracle_router_select(T, E, k, logits, bias, scale, norm, idx, NULL, w, NULL, NULL);
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j)
+            mask[t * E + idx[t * k + j]] = w[t * k + j];
+#pragma omp parallel
+    {
+        int Imax = I > Is ? I : Is;
+        double *hid = (double *)malloc(sizeof(double) * (size_t)Imax);
+        double *o = (double *)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < T; ++t) {
+            const uint16_t *xr = x + t * (int64_t)H;
+            double *yr = y + t * (int64_t)H;
+            for (int f = 0; f < H; ++f)
+                yr[f] = 0.0;
+            for (int e = 0; e < E; ++e) {
+                oracle_swiglu_mlp(H, I, xr, W_gate_up + (int64_t)e * 2 * I * H,
+                                  W_down + (int64_t)e * H * I, limit_routed, o, hid);
+                for (int f = 0; f < H; ++f)
+                    yr[f] += mask[t * E + e] * o[f];
+            }
+            oracle_swiglu_mlp(H, Is, xr, Wsh_gu, Wsh_d, limit_shared, o, hid);
+            for (int f = 0; f < H; ++f)
+                yr[f] += o[f];
+        }
+        free(hid);
+        free(o);
+    }
+    free(logits);
+    free(idx);
+    free(w);
+    free(mask);
+}
