@@ -1,0 +1,358 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 MoE layer forward pass (biased-sigmoid routing, clipped SwiGLU
+experts, shared expert) through the C ABI.
+
+One step = one moe_forward over one batch: router -> permutation -> gather / tile table ->
+grouped gate_up GEMM + clipped SwiGLU -> grouped down GEMM + weighted scatter-add.
+Default workload: Step-3.5-Flash-shaped prefill layer (T=4096, H=4096, E=288, top-8,
+I=Is=1280). Inputs are seeded synthetic tensors drawn on the device; the expert weights
+(9.1 GB) are larger than L2, so every step streams them from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl b200|reference]
+
+Multi-GPU (torchrun, one process per GPU): independent replicas, no collective on the data
+path ("replicas only"); value = tokens processed by all ranks / max-over-ranks time.
+--impl reference times the CPU oracle on a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd tokens/s on 1 B200; % of BF16 tensor peak / HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="step35_prefill")
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--deterministic", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
+    ap.add_argument("--experts", type=int, default=None, help="override E (profiling runs)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.lines = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-i", self.gpu_id,
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def workload_config(shape, extra=None):
+    c = {"workload": shape.name, "T": shape.T, "H": shape.H, "E": shape.E, "k": shape.k, "I": shape.I,
+         "Is": shape.Is, "scale": shape.scale, "norm_expert_weight": shape.norm_expert_weight,
+         "limit_routed": shape.limit_routed, "limit_shared": shape.limit_shared, "seed": shape.seed,
+         "bias": shape.bias_kind}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def cpu_oracle_sample(shape, inp, target_s: float, max_tokens: int = 4096, start: int = 0):
+    """Times the CPU oracle on a token sample of the workload; returns (tokens/s, n, seconds)."""
+    import numpy as np
+    import oracle
+    from sparse_moe_layer_biased_b200.inputs import bf16_bits
+
+    host = {k: v.cpu() for k, v in inp.items() if k in ("Wr", "bias", "Wsh_gate_up", "Wsh_down")}
+    gu = inp["W_gate_up"]
+    wd = inp["W_down"]
+    Wr = bf16_bits(host["Wr"])
+    bias = host["bias"].numpy()
+    Wsh_gu = bf16_bits(host["Wsh_gate_up"])
+    Wsh_d = bf16_bits(host["Wsh_down"])
+    cache = {}
+
+    def run(rows):
+        x_rows = bf16_bits(inp["x"][rows])
+        r = oracle.router(x_rows, Wr, bias, shape.k, shape.scale, shape.norm_expert_weight)
+        for e in np.unique(r["idx"]):
+            if int(e) not in cache:
+                cache[int(e)] = (bf16_bits(gu[int(e)]), bf16_bits(wd[int(e)]))
+        experts = {int(e): cache[int(e)] for e in np.unique(r["idx"])}
+        t0 = time.perf_counter()
+        oracle.forward_tokens(x_rows, Wr, bias, experts, Wsh_gu, Wsh_d, k=shape.k, scale=shape.scale,
+                              norm=shape.norm_expert_weight, limit_routed=shape.limit_routed,
+                              limit_shared=shape.limit_shared)
+        return time.perf_counter() - t0
+
+    nthreads = oracle.num_threads()
+    n0 = max(1, min(nthreads, shape.T))
+    rows = [(start + i) % shape.T for i in range(n0)]
+    dt = run(rows)
+    per_tok = dt / n0
+    n = int(min(max_tokens, shape.T, max(n0, target_s / max(per_tok, 1e-9))))
+    rows = [(start + n0 + i) % shape.T for i in range(n)]
+    dt = run(rows)
+    return n / dt, n, dt, nthreads
+
+
+def run_reference(args, shape):
+    """CPU oracle arm: each step runs the oracle on a bounded token sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    from sparse_moe_layer_biased_b200.inputs import draw
+
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = draw(shape, device=dev)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    rates, times = [], []
+    n_used = None
+    threads = None
+    for i in range(args.warmup + args.steps):
+        rate, n, dt, threads = cpu_oracle_sample(shape, inp, target_s=budget, start=i * 97)
+        if i >= args.warmup:
+            rates.append(rate)
+            times.append(dt * 1e3)
+            n_used = n
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; same draw as the b200 arm)",
+        "config": workload_config(shape, {"parallelism": "rank 0 only (CPU oracle)"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{n_used} tokens per step of {shape.name}, oracle forward (router + k routed "
+                                   f"+ shared expert MLPs in fp64)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def gate_up_bytes(shape, counts):
+    """Algorithmic HBM bytes of one gate_up launch: weights of every expert that received
+    tokens (2I x H bf16 each) + shared gate_up + permuted token rows + shared token rows +
+    hidden activations written."""
+    touched = int((counts[: shape.E] > 0).sum())
+    T, H, k, I, Is = shape.T, shape.H, shape.k, shape.I, shape.Is
+    w = touched * 2 * I * H * 2 + 2 * Is * H * 2
+    acts = T * k * H * 2 + T * H * 2
+    out = T * k * I * 2 + T * Is * 2
+    return w + acts + out, touched
+
+
+def run_b200(args, shape):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from sparse_moe_layer_biased_b200 import _abi
+    from sparse_moe_layer_biased_b200.inputs import draw
+    from sparse_moe_layer_biased_b200.layer import MoeLayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    inp = draw(shape, device="cuda")
+    layer = MoeLayer(shape, inp, deterministic=args.deterministic)
+    x = inp["x"]
+    y = torch.empty((shape.T, shape.H), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    # warm-up (also yields the routing used for the algorithmic byte count)
+    _, idx, _ = layer.forward(x, y=y, routing=True)
+    for _ in range(max(0, args.warmup - 1)):
+        layer.forward(x, y=y)
+    torch.cuda.synchronize()
+    _abi.moe_check_device()
+    counts = np.bincount(idx.cpu().numpy().ravel(), minlength=shape.E)
+
+    nstage = 7 if args.deterministic else 6
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_name = str(torch.cuda.get_device_properties(local).uuid)
+    sampler = ClockSampler("GPU-" + gpu_name if not gpu_name.startswith("GPU-") else gpu_name)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        _abi.moe_set_stage_events(evs[i])
+        layer.forward(x, y=y)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    _abi.moe_set_stage_events([])
+    barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    names = ["router", "permute", "gather_tiles", "gate_up", "down", "combine"][: nstage - 1]
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                for j, n in enumerate(names)}
+    _abi.moe_check_device()
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        x_h = x.cpu().pin_memory()
+        y_h = torch.empty((shape.T, shape.H), dtype=torch.float32).pin_memory()
+        x_d = torch.empty_like(x)
+        for _ in range(2):
+            x_d.copy_(x_h, non_blocking=True)
+            layer.forward(x_d, y=y)
+            y_h.copy_(y, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            x_d.copy_(x_h, non_blocking=True)
+            layer.forward(x_d, y=y)
+            y_h.copy_(y, non_blocking=True)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        ms2 = s2.elapsed_time(e2)
+        if world > 1:
+            t = torch.tensor([ms2], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms2 = float(t.item())
+        e2e = {"value": world * shape.T * args.steps / (ms2 / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": shape.T * shape.H * 2, "d2h_bytes_per_step": shape.T * shape.H * 4}
+
+    peaks, peak_kind = load_peaks()
+    gbytes, touched = gate_up_bytes(shape, counts)
+    gate_ms = stage_ms["gate_up"]
+    achieved = gbytes / (gate_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "gate_up_kernel", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": gbytes, "launch_ms": gate_ms,
+                "touched_experts": touched}
+    flops = shape.flops_per_token * shape.T
+    step_ms = ms / args.steps
+    value = world * shape.T * args.steps / (ms / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded draw on device; random-init weights)",
+        "config": workload_config(shape, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                                          "l2": "inputs larger than L2 (expert weights streamed every step)",
+                                          "deterministic": bool(args.deterministic)}),
+        "roofline": roofline,
+        "tensor": {"achieved_tflops": flops / (step_ms / 1e3) / 1e12,
+                   "frac_of_bf16_peak": flops / (step_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+        "stages_ms": stage_ms,
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": (nstage) * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, dt, threads = cpu_oracle_sample(shape, inp, target_s=15.0)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"{n} tokens of {shape.name} through the CPU oracle forward "
+                                          f"({dt:.1f} s, fp64)"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from sparse_moe_layer_biased_b200.inputs import WORKLOADS
+
+    shape = WORKLOADS[args.workload]
+    if args.tokens or args.experts:
+        shape = shape.replace(name=f"{shape.name}_T{args.tokens or shape.T}_E{args.experts or shape.E}",
+                              T=args.tokens or shape.T, E=args.experts or shape.E)
+    if args.impl == "reference":
+        run_reference(args, shape)
+    else:
+        run_b200(args, shape)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,166 @@
+/*
+ * moe_b200.h — C ABI of the B200 (sm_100a) forward pass of the biased-sigmoid-routed
+ * Mixture-of-Experts FFN layer of Step-3.5-Flash / Step-5-Preview.
+ *
+ * The layer ("MAX 中 Step-3.5-Flash 架构解析", section "MoE共享专家、sigmoid 路由与激活裁剪",
+ * config keys from section "Step3p5Config配置项全解"):
+ *   logits  = x · Wr^T                      computed in FP32 (the FP32 gate)
+ *   s       = sigmoid(logits)
+ *   ids     = top-k of (s + router_bias)    bias used for selection only; ties to the
+ *                                           lower expert index; a NaN score ranks last
+ *   w_j     = scale · s_j / Σ_j s_j         (norm_expert_weight; no epsilon; if the sum
+ *                                           is 0 every weight is scale/k), or scale · s_j
+ *   y       = Σ_j w_j · SwiGLU_{ids_j}(x; L_routed) + SwiGLU_shared(x; L_shared)
+ *   SwiGLU(x; L) = Wd · (min(silu(g), L) ⊙ clamp(u, −L, L)), g = Wg·x, u = Wu·x; L = 0: no clip.
+ *
+ * Conventions for every entry point:
+ *  - All array arguments are DEVICE pointers on the current CUDA device, allocated and
+ *    owned by the caller. The library never allocates, frees or synchronises; it only
+ *    enqueues kernels (and, where stated, a memset) on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).
+ *  - bf16 arrays are passed as uint16_t bit patterns. Matrices are row-major with the
+ *    reduction dimension innermost (PyTorch [out, in]).
+ *  - Argument checks run on the host before anything is enqueued; on any error nothing
+ *    is enqueued and the outputs are untouched. MOE_ERR_INVALID_ARG: NULL pointer, bad
+ *    sizes or k outside [1, min(E, 32)]. MOE_ERR_UNSUPPORTED: H not a multiple of 128,
+ *    I or Is not a multiple of 64, E > 512, a bf16/fp32 array not 16-byte aligned, or
+ *    sizes whose index arithmetic would overflow 32-bit row counts. MOE_ERR_WORKSPACE:
+ *    ws_bytes below moe_workspace_size(). MOE_ERR_CUDA: a launch failed (the CUDA error
+ *    is left for cudaGetLastError()).
+ *  - Device-side waits are bounded; a wait that expires sets a device error word that
+ *    moe_check_device() reports as MOE_ERR_TIMEOUT. Kernels never trap.
+ *  - T = 0 is valid: after the descriptor check the call returns MOE_OK without
+ *    enqueueing anything, and the array pointers may then be NULL.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_WORKSPACE = 3,
+    MOE_ERR_CUDA = 4,
+    MOE_ERR_TIMEOUT = 5
+} moe_status_t;
+
+/* One MoE layer call. Field names follow Step3p5Config ("Step3p5Config配置项全解"):
+ * E = moe_num_experts, k = moe_top_k, I = moe_intermediate_size, Is = share_expert_dim,
+ * scale = moe_router_scaling_factor, norm_expert_weight, limit_routed =
+ * swiglu_limits[layer], limit_shared = swiglu_limits_shared[layer] (0 = no clip).
+ * deterministic = 1 selects the fixed-order combine (moe_combine) instead of fp32
+ * atomic accumulation into y; both give the same value up to fp32 summation order. */
+typedef struct {
+    int32_t T;  /* tokens */
+    int32_t H;  /* hidden size */
+    int32_t E;  /* routed experts */
+    int32_t k;  /* experts per token */
+    int32_t I;  /* routed expert intermediate size */
+    int32_t Is; /* shared expert intermediate size */
+    float scale;
+    int32_t norm_expert_weight;
+    float limit_routed;
+    float limit_shared;
+    int32_t deterministic;
+} moe_layer_desc;
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char *moe_status_string(int status);
+
+/* Bytes of device workspace that moe_expert_ffn and moe_forward need for `desc`
+ * (written to *bytes). The workspace holds the permuted activations, the hidden
+ * SwiGLU activations, per-slot weights, the tile table and (moe_forward) the routing
+ * tables. Its contents need not be initialised. */
+MOE_API moe_status_t moe_workspace_size(const moe_layer_desc *desc, size_t *bytes);
+
+/* Router ("MoE共享专家、sigmoid 路由与激活裁剪": FP32 gate, sigmoid, router_bias for selection
+ * only, top-k, normalisation, scaling; index clamp to [0, E-1]).
+ *   x [T, H] bf16, Wr [E, H] bf16, bias [E] fp32 (inputs, read-only)
+ *   topk_idx [T, k] int32: selected experts in rank order (biased score descending,
+ *                          ties to the lower index)
+ *   topk_w   [T, k] fp32:  routing weights (from the unbiased scores)
+ *   margin   [T] fp32 or NULL: (k-th biased score) - ((k+1)-th), +inf when k = E. */
+MOE_API moe_status_t moe_router(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr,
+                        const float *bias, int32_t *topk_idx, float *topk_w, float *margin,
+                        void *stream);
+
+/* Token -> slot permutation, bit-exact and deterministic: per-expert histogram,
+ * exclusive scan, and a scatter stable in token order. Group E is the shared expert and
+ * holds every token in order.
+ *   topk_idx [T, k] int32 (input; ids outside [0, E-1] are clamped)
+ *   counts [E+1]: tokens per group (counts[E] = T)
+ *   offsets [E+2]: exclusive scan of counts (offsets[E] = T*k, offsets[E+1] = T*k + T)
+ *   perm_token [T*k + T]: token of each slot; slots of group e are
+ *              [offsets[e], offsets[e+1]) in ascending token order
+ *   slot_of [T, k]: slot of (token, rank j); the inverse of perm_token on routed slots. */
+MOE_API moe_status_t moe_permute(const moe_layer_desc *desc, const int32_t *topk_idx, int32_t *counts,
+                         int32_t *offsets, int32_t *perm_token, int32_t *slot_of, void *stream);
+
+/* Routed and shared expert FFNs with the clipped SwiGLU ("MoE共享专家、sigmoid 路由与激活裁剪":
+ * routed_moe(x) + shared_expert(x), make_concatenated_gated_activation_fn(silu, limit)).
+ *   x [T, H] bf16; topk_w [T, k] fp32; offsets, perm_token, slot_of from moe_permute
+ *   W_gate_up [E, 2I, H] bf16 (rows [0, I) gate, [I, 2I) up); W_down [E, H, I] bf16
+ *   Wsh_gate_up [2Is, H] bf16; Wsh_down [H, Is] bf16
+ *   out: deterministic = 0 -> y [T, H] fp32, overwritten (zeroed, then accumulated);
+ *        deterministic = 1 -> o_perm [T*k + T, H] fp32: row slot_of[t, j] holds
+ *        topk_w[t, j] * expert output, row T*k + t holds the shared expert output;
+ *        moe_combine then sums them in a fixed order.
+ *   ws, ws_bytes: workspace of at least moe_workspace_size() bytes. */
+MOE_API moe_status_t moe_expert_ffn(const moe_layer_desc *desc, const uint16_t *x, const float *topk_w,
+                            const int32_t *offsets, const int32_t *perm_token,
+                            const int32_t *slot_of, const uint16_t *W_gate_up,
+                            const uint16_t *W_down, const uint16_t *Wsh_gate_up,
+                            const uint16_t *Wsh_down, float *out, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/* Fixed-order combine: y[t] = Σ_{j<k} o_perm[slot_of[t, j]] + o_perm[T*k + t], summed in
+ * rank order, then the shared row. o_perm [T*k + T, H] fp32, slot_of [T, k], y [T, H]
+ * fp32 (overwritten). */
+MOE_API moe_status_t moe_combine(const moe_layer_desc *desc, const float *o_perm, const int32_t *slot_of,
+                         float *y, void *stream);
+
+/* The whole layer: moe_router -> moe_permute -> moe_expert_ffn (-> moe_combine when
+ * deterministic). y [T, H] fp32 is overwritten. topk_idx_out / topk_w_out ([T, k]) may be
+ * NULL; when given they receive the routing. */
+MOE_API moe_status_t moe_forward(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr,
+                         const float *bias, const uint16_t *W_gate_up, const uint16_t *W_down,
+                         const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y,
+                         int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/* Waits for the current device, then reports and clears the device error word:
+ * MOE_ERR_TIMEOUT if a bounded device wait expired since the last call, MOE_ERR_CUDA if
+ * the device reports an error, else MOE_OK. This call synchronises the device. */
+MOE_API moe_status_t moe_check_device(void);
+
+/* Stage timing hook (profiling). When n > 0, every later moe_forward on this process
+ * records events[0] before the router, events[1] before the permutation, events[2] before
+ * the gather / tile table, events[3] before the gate_up GEMM, events[4] before the down
+ * GEMM, events[5] after the down GEMM and, when n >= 7, events[6] after the combine
+ * (deterministic mode), each with cudaEventRecord on the call's stream. `events` are
+ * cudaEvent_t handles owned by the caller; the array is copied. n = 0 turns it off.
+ * Returns MOE_ERR_INVALID_ARG if n < 0, n > 7 or events is NULL with n > 0. */
+MOE_API moe_status_t moe_set_stage_events(void *const *events, int n);
+
+/* Upper bound, in nanoseconds, of every device-side wait in later launches on this
+ * process (default 2e9). Values below 1000 are raised to 1000. Returns the old value. */
+MOE_API uint64_t moe_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,437 @@
+// expert_gemm.cu — grouped expert GEMMs of the MoE layer on sm_100a (tcgen05 + TMEM + TMA).
+//
+// Layer step ("MAX 中 Step-3.5-Flash 架构解析", section "MoE共享专家、sigmoid 路由与激活裁剪"):
+// output = routed_moe(x) + shared_expert(x); each expert is a SwiGLU MLP whose gated
+// activation is built from the concatenated gate/up projection with a per-layer clip
+// limit (swiglu_limits / swiglu_limits_shared, 0 = no clip, section
+// "Step3p5Config配置项全解"). The fused [2I, H] gate_up and [H, I] down layouts follow
+// the 24 MiB / 12 MiB BF16 expert tensors of the miles Step-5-Preview page, section 5.3.
+//
+// Both kernels are "swap-AB": the expert weight rows fill the 128-lane M side of the
+// UMMA and the tokens of one expert chunk (16..256, a multiple of 16) are the N side, so
+// a ragged group wastes at most 15 token columns, and a decode-sized group of one or
+// two tokens still streams full 128-row weight tiles.
+//
+// Roles per CTA (persistent, one CTA per SM, static round-robin over tiles):
+//   warp 0      TMA producer: weight tile + token rows (16-row boxes) per 64-wide K slice
+//   warp 1      MMA issuer (one thread) and TMEM owner; 2 x 256-column fp32 accumulators
+//   warps 2..5  epilogue: TMEM -> registers -> activation / weighting -> global
+// Every wait is bounded (mbar_wait); on expiry the CTA drains its own copies and MMAs,
+// frees TMEM and returns with the device error word set.
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 4;
+constexpr int kBK = 64;
+constexpr uint32_t kABytes = 128 * 128;     // 128 weight rows x 64 bf16
+constexpr uint32_t kBBytes = 256 * 128;     // up to 256 token rows x 64 bf16
+constexpr uint32_t kBoxBytes = 16 * 128;    // one 16-row token box
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kBarOff = kStages * kStageBytes;
+constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * kStages + 5);
+constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
+constexpr uint32_t kAccCols = 256;
+constexpr uint32_t kTmemCols = 512;
+
+struct Ring {
+    uint64_t *full, *empty, *accf, *acce, *drain;
+    uint32_t *holder;
+    volatile int *abort_flag;
+};
+
+__device__ __forceinline__ uint8_t *ring_setup(uint8_t *smem_raw, Ring &r)
+{
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    uint8_t *smem = smem_raw + pad;
+    r.full = reinterpret_cast<uint64_t *>(smem + kBarOff);
+    r.empty = r.full + kStages;
+    r.accf = r.empty + kStages;
+    r.acce = r.accf + 2;
+    r.drain = r.acce + 2;
+    r.holder = reinterpret_cast<uint32_t *>(smem + kMiscOff);
+    r.abort_flag = reinterpret_cast<volatile int *>(smem + kMiscOff + 4);
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&r.full[s], 1);
+            mbar_init(&r.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&r.accf[b], 1);
+            mbar_init(&r.acce[b], 4);  // one arrival per epilogue warp
+        }
+        mbar_init(r.drain, 1);
+        *r.abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(r.holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return smem;
+}
+
+__device__ __forceinline__ void ring_teardown(uint32_t tmem)
+{
+    tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Lane 0 waits, the whole warp learns the outcome (keeps warp-collective ops converged).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const WaitCfg &wc, volatile int *ab)
+{
+    bool ok = false;
+    if ((threadIdx.x & 31) == 0)
+        ok = mbar_wait(bar, parity, wc, ab);
+    return __shfl_sync(0xFFFFFFFFu, ok, 0);
+}
+
+__device__ __forceinline__ void producer_drain(const Ring &r, int issued, const WaitCfg &wc)
+{
+    for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it)
+        mbar_wait_drain(&r.full[it % kStages], (it / kStages) & 1, wc);
+}
+
+// MMA issue for one tile: nkb K-slices of 64 into accumulator d (N = n columns).
+// Returns false if a wait gave up.
+__device__ __forceinline__ bool mma_tile(const Ring &r, uint8_t *smem, uint32_t d, int n, int nkb, int &it,
+                                         const WaitCfg &wc)
+{
+    const uint32_t idesc = idesc_bf16_f32(128, n);
+    for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(&r.full[s], (it / kStages) & 1, wc, r.abort_flag))
+            return false;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+        const uint64_t ad = sdesc_kmajor_sw128(a_addr);
+        const uint64_t bd = sdesc_kmajor_sw128(a_addr + kABytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+        umma_commit(&r.empty[s]);
+    }
+    return true;
+}
+
+__device__ __forceinline__ float swiglu_clip(float g, float u, float L)
+{
+    float a = g / (1.0f + expf(-g));
+    if (L > 0.0f) {
+        a = a > L ? L : a;
+        u = u > L ? L : (u < -L ? -L : u);
+    }
+    return a * u;
+}
+
+// ------------------------------------------------------------------------------------
+// gate_up: h[slot, f] = act(Wg_e[f]·x[tok], Wu_e[f]·x[tok]) for one chunk of an expert.
+// A tile = 64 (gate, up) row pairs of one expert, interleaved by the 4-D tensor map
+// (H, half, row, expert) so TMEM lane 2i holds gate row i and lane 2i+1 its up row; the
+// epilogue pairs them with one shuffle. Routed chunks read x_perm; the shared expert's
+// chunks read x directly (identity permutation).
+__device__ __forceinline__ void decode_gate_up(const GateUpArgs &a, int nrc, int tiles_r, int tile, int &g,
+                                               int &row0, int &ntok, int &fb)
+{
+    int ci;
+    if (tile < tiles_r) {
+        const int nfb = a.I / 64;
+        ci = tile / nfb;
+        fb = tile - ci * nfb;
+    } else {
+        const int nfb = a.Is / 64;
+        const int tt = tile - tiles_r;
+        ci = nrc + tt / nfb;
+        fb = tt - (tt / nfb) * nfb;
+    }
+    const int4 c = a.chunks[ci];
+    g = c.x;
+    row0 = c.y;
+    ntok = c.z;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gate_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_wsh,
+                   const __grid_constant__ CUtensorMap tm_xp, const __grid_constant__ CUtensorMap tm_x,
+                   const GateUpArgs a, const WaitCfg wc)
+{
+    extern __shared__ uint8_t smem_raw[];
+    Ring r;
+    uint8_t *smem = ring_setup(smem_raw, r);
+    const uint32_t tmem = *r.holder;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nrc = a.hdr[0];
+    const int ntot = a.hdr[1];
+    const int tiles_r = nrc * (a.I / 64);
+    const int tiles = tiles_r + (ntot - nrc) * (a.Is / 64);
+    const int nkb = a.H / kBK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_map(&tm_w);
+            tma_prefetch_map(&tm_wsh);
+            tma_prefetch_map(&tm_xp);
+            tma_prefetch_map(&tm_x);
+            int it = 0;
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x) {
+                int g, row0, ntok, fb;
+                decode_gate_up(a, nrc, tiles_r, tile, g, row0, ntok, fb);
+                const bool sh = g == a.E;
+                const int nb = (ntok + 15) >> 4;
+                const uint32_t tx = kABytes + nb * kBoxBytes;
+                const CUtensorMap *mb = sh ? &tm_x : &tm_xp;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(&r.empty[s], ((it / kStages) & 1) ^ 1, wc, r.abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&r.full[s], tx);
+                    uint8_t *A = smem + s * kStageBytes;
+                    uint8_t *B = A + kABytes;
+                    if (sh)
+                        tma_load_4d(A, &tm_wsh, &r.full[s], kb * kBK, 0, fb * 64, 0);
+                    else
+                        tma_load_4d(A, &tm_w, &r.full[s], kb * kBK, 0, fb * 64, g);
+                    for (int i = 0; i < nb; ++i)
+                        tma_load_2d(B + i * kBoxBytes, mb, &r.full[s], kb * kBK, row0 + 16 * i);
+                }
+            }
+            producer_drain(r, it, wc);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int it = 0, tc = 0;
+            for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+                int g, row0, ntok, fb;
+                decode_gate_up(a, nrc, tiles_r, tile, g, row0, ntok, fb);
+                const int buf = tc & 1;
+                if (!mbar_wait(&r.acce[buf], ((tc >> 1) & 1) ^ 1, wc, r.abort_flag))
+                    break;
+                tc_fence_after();
+                if (!mma_tile(r, smem, tmem + buf * kAccCols, (ntok + 15) & ~15, nkb, it, wc))
+                    break;
+                umma_commit(&r.accf[buf]);
+            }
+            umma_commit(r.drain);
+            mbar_wait_drain(r.drain, 0, wc);
+        }
+    } else {
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int pair = row >> 1;
+        const bool is_up = row & 1;
+        int tc = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+            int g, row0, ntok, fb;
+            decode_gate_up(a, nrc, tiles_r, tile, g, row0, ntok, fb);
+            const int buf = tc & 1;
+            if (!warp_wait(&r.accf[buf], (tc >> 1) & 1, wc, r.abort_flag))
+                break;
+            tc_fence_after();
+            const bool sh = g == a.E;
+            const float L = sh ? a.lim_s : a.lim_r;
+            uint16_t *out = sh ? a.h_sh : a.h;
+            const int64_t ld = sh ? a.Is : a.I;
+            const int64_t feat = fb * 64 + pair;
+            const uint32_t tb = tmem + buf * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
+            for (int cb = 0; cb < ntok; cb += 32) {
+                float v[32];
+                tmem_load32(tb + cb, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    // even lane finishes column cb+i (needs the up value), odd lane column
+                    // cb+16+i (needs the gate value)
+                    const float send = is_up ? v[i] : v[16 + i];
+                    const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+                    const float gv = is_up ? recv : v[i];
+                    const float uv = is_up ? v[16 + i] : recv;
+                    const int col = cb + (is_up ? 16 + i : i);
+                    const float hv = swiglu_clip(gv, uv, L);
+                    if (col < ntok)
+                        out[(row0 + col) * ld + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&r.acce[buf]);
+        }
+    }
+    ring_teardown(tmem);
+}
+
+// ------------------------------------------------------------------------------------
+// down: o[f, slot] = Wd_e[f]·h[slot]; routed slots add w_slot * o into y[token] (fp32
+// atomics) or store it in o_perm[slot] (deterministic mode); shared rows add o (weight 1).
+__device__ __forceinline__ void decode_down(const DownArgs &a, int tile, int &g, int &row0, int &ntok, int &fb)
+{
+    const int nfb = a.H / 128;
+    const int ci = tile / nfb;
+    fb = tile - ci * nfb;
+    const int4 c = a.chunks[ci];
+    g = c.x;
+    row0 = c.y;
+    ntok = c.z;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    down_kernel(const __grid_constant__ CUtensorMap tm_wd, const __grid_constant__ CUtensorMap tm_wdsh,
+                const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_hsh,
+                const DownArgs a, const WaitCfg wc)
+{
+    extern __shared__ uint8_t smem_raw[];
+    Ring r;
+    uint8_t *smem = ring_setup(smem_raw, r);
+    const uint32_t tmem = *r.holder;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int ntot = a.hdr[1];
+    const int tiles = ntot * (a.H / 128);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_map(&tm_wd);
+            tma_prefetch_map(&tm_wdsh);
+            tma_prefetch_map(&tm_h);
+            tma_prefetch_map(&tm_hsh);
+            int it = 0;
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x) {
+                int g, row0, ntok, fb;
+                decode_down(a, tile, g, row0, ntok, fb);
+                const bool sh = g == a.E;
+                const int nkb = (sh ? a.Is : a.I) / kBK;
+                const int nb = (ntok + 15) >> 4;
+                const uint32_t tx = kABytes + nb * kBoxBytes;
+                const CUtensorMap *mb = sh ? &tm_hsh : &tm_h;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(&r.empty[s], ((it / kStages) & 1) ^ 1, wc, r.abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&r.full[s], tx);
+                    uint8_t *A = smem + s * kStageBytes;
+                    uint8_t *B = A + kABytes;
+                    if (sh)
+                        tma_load_2d(A, &tm_wdsh, &r.full[s], kb * kBK, fb * 128);
+                    else
+                        tma_load_2d(A, &tm_wd, &r.full[s], kb * kBK, g * a.H + fb * 128);
+                    for (int i = 0; i < nb; ++i)
+                        tma_load_2d(B + i * kBoxBytes, mb, &r.full[s], kb * kBK, row0 + 16 * i);
+                }
+            }
+            producer_drain(r, it, wc);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int it = 0, tc = 0;
+            for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+                int g, row0, ntok, fb;
+                decode_down(a, tile, g, row0, ntok, fb);
+                const int nkb = (g == a.E ? a.Is : a.I) / kBK;
+                const int buf = tc & 1;
+                if (!mbar_wait(&r.acce[buf], ((tc >> 1) & 1) ^ 1, wc, r.abort_flag))
+                    break;
+                tc_fence_after();
+                if (!mma_tile(r, smem, tmem + buf * kAccCols, (ntok + 15) & ~15, nkb, it, wc))
+                    break;
+                umma_commit(&r.accf[buf]);
+            }
+            umma_commit(r.drain);
+            mbar_wait_drain(r.drain, 0, wc);
+        }
+    } else {
+        const int q = warp & 3;
+        const int64_t f = q * 32 + lane;
+        const int64_t H = a.H;
+        const int64_t shared_base = static_cast<int64_t>(a.T) * a.k;
+        int tc = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+            int g, row0, ntok, fb;
+            decode_down(a, tile, g, row0, ntok, fb);
+            const int buf = tc & 1;
+            if (!warp_wait(&r.accf[buf], (tc >> 1) & 1, wc, r.abort_flag))
+                break;
+            tc_fence_after();
+            const bool sh = g == a.E;
+            const int64_t feat = fb * 128 + f;
+            const uint32_t tb = tmem + buf * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
+            for (int cb = 0; cb < ntok; cb += 32) {
+                // lane l fetches the token / slot and weight of column cb + l
+                const int mycol = cb + lane;
+                int64_t dst_row = 0;
+                float wgt = 0.0f;
+                if (mycol < ntok) {
+                    const int64_t rr = row0 + mycol;
+                    if (a.deterministic) {
+                        dst_row = sh ? shared_base + rr : rr;
+                    } else {
+                        dst_row = sh ? rr : a.perm_token[rr];
+                    }
+                    wgt = sh ? 1.0f : a.w_perm[rr];
+                }
+                float v[32];
+                tmem_load32(tb + cb, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int64_t drow = __shfl_sync(0xFFFFFFFFu, dst_row, i);
+                    const float w = __shfl_sync(0xFFFFFFFFu, wgt, i);
+                    if (cb + i < ntok) {
+                        float *p = a.out + drow * H + feat;
+                        if (a.deterministic)
+                            *p = w * v[i];
+                        else
+                            atomicAdd(p, w * v[i]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&r.acce[buf]);
+        }
+    }
+    ring_teardown(tmem);
+}
+
+}  // namespace
+
+cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
+                           const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
+                           cudaStream_t stream)
+{
+    cudaError_t err =
+        cudaFuncSetAttribute(gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+    if (err != cudaSuccess)
+        return err;
+    gate_up_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_w, tm_wsh, tm_xp, tm_x, a, wc);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
+                        const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
+                        cudaStream_t stream)
+{
+    cudaError_t err =
+        cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+    if (err != cudaSuccess)
+        return err;
+    down_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,71 @@
+// internal.h — launchers shared between the kernel translation units and the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sm100.cuh"
+
+namespace moe {
+
+// Largest dynamic shared memory a CTA may request on sm_100 (227 KB).
+constexpr int kMaxDynSmem = 232448;
+
+struct RouterArgs {
+    const float *bias;
+    int32_t *idx;
+    float *w;
+    float *margin;  // may be null
+    int T, H, E, k;
+    float scale;
+    int norm;
+};
+cudaError_t launch_router(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const RouterArgs &a,
+                          const WaitCfg &wc, cudaStream_t stream);
+
+cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int32_t *counts, int32_t *offsets,
+                           int32_t *perm_token, int32_t *slot_of, cudaStream_t stream);
+
+cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
+                          uint16_t *x_perm, float *w_perm, int num_sms, cudaStream_t stream);
+
+// Splits every group (E routed experts, then the shared expert) into chunks of at most
+// kChunkTokens rows. hdr[0] = routed chunk count, hdr[1] = total chunk count.
+constexpr int kChunkTokens = 256;
+cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int k, int4 *chunks, int32_t *hdr,
+                          cudaStream_t stream);
+inline int64_t max_chunks(int64_t T, int64_t k, int64_t E)
+{
+    return (T * k + T) / kChunkTokens + E + 2;
+}
+
+struct GateUpArgs {
+    const int4 *chunks;
+    const int32_t *hdr;
+    uint16_t *h;     // [T*k, I] bf16
+    uint16_t *h_sh;  // [T, Is] bf16
+    int E, H, I, Is;
+    float lim_r, lim_s;
+};
+cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
+                           const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
+                           cudaStream_t stream);
+
+struct DownArgs {
+    const int4 *chunks;
+    const int32_t *hdr;
+    const int32_t *perm_token;
+    const float *w_perm;
+    float *out;  // y [T, H] (atomic) or o_perm [T*k + T, H] (deterministic)
+    int E, H, I, Is, T, k;
+    int deterministic;
+};
+cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
+                        const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
+                        cudaStream_t stream);
+
+cudaError_t launch_combine(const float *o_perm, const int32_t *slot_of, int T, int k, int H, float *y,
+                           cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,440 @@
+// moe_api.cu — C ABI of the B200 MoE layer (declarations and contract in include/moe_b200.h).
+//
+// Host side only: argument validation (before anything is enqueued), workspace layout,
+// TMA tensor-map encoding, and the launch sequence router -> permute -> gather/tile
+// table -> gate_up GEMM -> down GEMM (-> combine). The library allocates nothing and never
+// synchronises except in moe_check_device().
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe_b200.h"
+#include "internal.h"
+
+namespace {
+
+// Device error word (bit flags of moe::kDevErr*), one per device context.
+__device__ uint32_t g_moe_err;
+
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+
+// Optional stage events recorded by moe_forward (profiling hook).
+constexpr int kMaxStageEvents = 7;
+std::mutex g_ev_mu;
+cudaEvent_t g_stage_ev[kMaxStageEvents];
+int g_stage_n = 0;
+
+void stage_mark(int i, cudaStream_t s)
+{
+    std::lock_guard<std::mutex> lk(g_ev_mu);
+    if (i < g_stage_n)
+        cudaEventRecord(g_stage_ev[i], s);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int num_sms = 0;
+    uint32_t *err = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+moe_status_t device_info(DeviceInfo &out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return MOE_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_moe_err) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        d.err = static_cast<uint32_t *>(p);
+        d.ready = true;
+    }
+    out = d;
+    return MOE_OK;
+}
+
+moe::WaitCfg wait_cfg(const DeviceInfo &d)
+{
+    return moe::WaitCfg{g_wait_limit_ns.load(), d.err};
+}
+
+// bf16 tensor map, 128-byte swizzle, 64-element inner box. dims/strides innermost first;
+// strides (bytes) are given for dims 1..rank-1.
+bool encode_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
+                 const cuuint32_t *box)
+{
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+                                const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool map_rows(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, uint32_t box_rows)
+{
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    return encode_bf16(m, base, 2, dims, strides, box);
+}
+
+// Stacked gate_up weights [G, 2*Iw, H] viewed as (H, half, row, group) so one box of
+// (64, 2, 64, 1) lands as 128 rows alternating gate row i / up row i.
+bool map_gate_up(CUtensorMap *m, const void *base, int64_t H, int64_t Iw, int64_t G)
+{
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(H), 2, static_cast<cuuint64_t>(Iw),
+                                static_cast<cuuint64_t>(G)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(Iw * H * 2), static_cast<cuuint64_t>(H * 2),
+                                   static_cast<cuuint64_t>(2 * Iw * H * 2)};
+    const cuuint32_t box[4] = {64, 2, 64, 1};
+    return encode_bf16(m, base, 4, dims, strides, box);
+}
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+moe_status_t check_desc(const moe_layer_desc *d)
+{
+    if (!d)
+        return MOE_ERR_INVALID_ARG;
+    if (d->T < 0 || d->H <= 0 || d->E <= 0 || d->k <= 0 || d->I <= 0 || d->Is <= 0)
+        return MOE_ERR_INVALID_ARG;
+    if (d->k > d->E || d->k > 32)
+        return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(d->scale) || !std::isfinite(d->limit_routed) || !std::isfinite(d->limit_shared) ||
+        d->limit_routed < 0.0f || d->limit_shared < 0.0f)
+        return MOE_ERR_INVALID_ARG;
+    if ((d->norm_expert_weight != 0 && d->norm_expert_weight != 1) ||
+        (d->deterministic != 0 && d->deterministic != 1))
+        return MOE_ERR_INVALID_ARG;
+    if (d->E > 512 || d->H % 128 != 0 || d->I % 64 != 0 || d->Is % 64 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    const int64_t rows = static_cast<int64_t>(d->T) * (d->k + 1);
+    if (rows >= (int64_t(1) << 31) - 512 || static_cast<int64_t>(d->E) * d->H >= (int64_t(1) << 31))
+        return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+struct WsLayout {
+    size_t x_perm, w_perm, h, h_sh, chunks, hdr, o_perm, idx, w, counts, offsets, perm_token, slot_of, total;
+};
+
+size_t up256(size_t v)
+{
+    return (v + 255) / 256 * 256;
+}
+
+WsLayout ws_layout(const moe_layer_desc &d)
+{
+    const size_t T = d.T, H = d.H, E = d.E, k = d.k, I = d.I, Is = d.Is;
+    WsLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += up256(bytes);
+        return o;
+    };
+    L.x_perm = take(T * k * H * 2);
+    L.w_perm = take(T * k * 4);
+    L.h = take(T * k * I * 2);
+    L.h_sh = take(T * Is * 2);
+    L.chunks = take(static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E)) * 16);
+    L.hdr = take(64);
+    L.o_perm = take(d.deterministic ? (T * k + T) * H * 4 : 0);
+    L.idx = take(T * k * 4);
+    L.w = take(T * k * 4);
+    L.counts = take((E + 1) * 4);
+    L.offsets = take((E + 2) * 4);
+    L.perm_token = take((T * k + T) * 4);
+    L.slot_of = take(T * k * 4);
+    L.total = off;
+    return L;
+}
+
+template <typename P>
+P *at(void *ws, size_t off)
+{
+    return reinterpret_cast<P *>(static_cast<uint8_t *>(ws) + off);
+}
+
+moe_status_t cuda_status(cudaError_t e)
+{
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t run_router(const moe_layer_desc &d, const DeviceInfo &di, const uint16_t *x, const uint16_t *Wr,
+                        const float *bias, int32_t *idx, float *w, float *margin, cudaStream_t s)
+{
+    CUtensorMap tm_x, tm_wr;
+    if (!map_rows(&tm_x, x, d.H, d.T, 128) || !map_rows(&tm_wr, Wr, d.H, d.E, 16))
+        return MOE_ERR_CUDA;
+    moe::RouterArgs a{bias, idx, w, margin, d.T, d.H, d.E, d.k, d.scale, d.norm_expert_weight};
+    return cuda_status(moe::launch_router(tm_x, tm_wr, a, wait_cfg(di), s));
+}
+
+moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const uint16_t *x, const float *topk_w,
+                            const int32_t *offsets, const int32_t *perm_token, const int32_t *slot_of,
+                            const uint16_t *Wgu, const uint16_t *Wd, const uint16_t *Wsh_gu, const uint16_t *Wsh_d,
+                            float *out, void *ws, cudaStream_t s)
+{
+    const WsLayout L = ws_layout(d);
+    uint16_t *x_perm = at<uint16_t>(ws, L.x_perm);
+    float *w_perm = at<float>(ws, L.w_perm);
+    uint16_t *h = at<uint16_t>(ws, L.h);
+    uint16_t *h_sh = at<uint16_t>(ws, L.h_sh);
+    int4 *chunks = at<int4>(ws, L.chunks);
+    int32_t *hdr = at<int32_t>(ws, L.hdr);
+    const int64_t Tk = static_cast<int64_t>(d.T) * d.k;
+
+    CUtensorMap tm_w, tm_wsh, tm_xp, tm_x, tm_wd, tm_wdsh, tm_h, tm_hsh;
+    bool ok = map_gate_up(&tm_w, Wgu, d.H, d.I, d.E) && map_gate_up(&tm_wsh, Wsh_gu, d.H, d.Is, 1) &&
+              map_rows(&tm_xp, x_perm, d.H, Tk, 16) && map_rows(&tm_x, x, d.H, d.T, 16) &&
+              map_rows(&tm_wd, Wd, d.I, static_cast<int64_t>(d.E) * d.H, 128) &&
+              map_rows(&tm_wdsh, Wsh_d, d.Is, d.H, 128) && map_rows(&tm_h, h, d.I, Tk, 16) &&
+              map_rows(&tm_hsh, h_sh, d.Is, d.T, 16);
+    if (!ok)
+        return MOE_ERR_CUDA;
+
+    stage_mark(2, s);
+    cudaError_t e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, s);
+    if (e == cudaSuccess)
+        e = moe::launch_chunks(offsets, d.E, d.T, d.k, chunks, hdr, s);
+    if (e == cudaSuccess && !d.deterministic)
+        e = cudaMemsetAsync(out, 0, static_cast<size_t>(d.T) * d.H * 4, s);
+    if (e != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const moe::WaitCfg wc = wait_cfg(di);
+    moe::GateUpArgs ga{chunks, hdr, h, h_sh, d.E, d.H, d.I, d.Is, d.limit_routed, d.limit_shared};
+    stage_mark(3, s);
+    e = moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, s);
+    if (e != cudaSuccess)
+        return MOE_ERR_CUDA;
+    moe::DownArgs da{chunks, hdr, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic};
+    stage_mark(4, s);
+    e = moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, s);
+    stage_mark(5, s);
+    return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(int status)
+{
+    switch (status) {
+    case MOE_OK:
+        return "ok";
+    case MOE_ERR_INVALID_ARG:
+        return "invalid argument";
+    case MOE_ERR_UNSUPPORTED:
+        return "unsupported shape or alignment";
+    case MOE_ERR_WORKSPACE:
+        return "workspace too small";
+    case MOE_ERR_CUDA:
+        return "CUDA error";
+    case MOE_ERR_TIMEOUT:
+        return "device wait timed out";
+    default:
+        return "unknown status";
+    }
+}
+
+moe_status_t moe_workspace_size(const moe_layer_desc *desc, size_t *bytes)
+{
+    if (!bytes)
+        return MOE_ERR_INVALID_ARG;
+    const moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    *bytes = ws_layout(*desc).total;
+    return MOE_OK;
+}
+
+moe_status_t moe_router(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr, const float *bias,
+                        int32_t *topk_idx, float *topk_w, float *margin, void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->T == 0)
+        return MOE_OK;  // nothing to do; array pointers may be NULL
+    if (!x || !Wr || !bias || !topk_idx || !topk_w)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wr))
+        return MOE_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    return run_router(*desc, di, x, Wr, bias, topk_idx, topk_w, margin, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_permute(const moe_layer_desc *desc, const int32_t *topk_idx, int32_t *counts, int32_t *offsets,
+                         int32_t *perm_token, int32_t *slot_of, void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->T == 0)
+        return MOE_OK;  // nothing to do; array pointers may be NULL
+    if (!topk_idx || !counts || !offsets || !perm_token || !slot_of)
+        return MOE_ERR_INVALID_ARG;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    return cuda_status(moe::launch_permute(topk_idx, desc->T, desc->k, desc->E, counts, offsets, perm_token, slot_of,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_ffn(const moe_layer_desc *desc, const uint16_t *x, const float *topk_w,
+                            const int32_t *offsets, const int32_t *perm_token, const int32_t *slot_of,
+                            const uint16_t *W_gate_up, const uint16_t *W_down, const uint16_t *Wsh_gate_up,
+                            const uint16_t *Wsh_down, float *out, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->T == 0)
+        return MOE_OK;  // nothing to do; array pointers may be NULL
+    if (!x || !topk_w || !offsets || !perm_token || !slot_of || !W_gate_up || !W_down || !Wsh_gate_up ||
+        !Wsh_down || !out || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W_gate_up) || !aligned16(W_down) || !aligned16(Wsh_gate_up) ||
+        !aligned16(Wsh_down) || !aligned16(out) || !aligned16(ws))
+        return MOE_ERR_UNSUPPORTED;
+    if (ws_bytes < ws_layout(*desc).total)
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    return run_expert_ffn(*desc, di, x, topk_w, offsets, perm_token, slot_of, W_gate_up, W_down, Wsh_gate_up,
+                          Wsh_down, out, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_combine(const moe_layer_desc *desc, const float *o_perm, const int32_t *slot_of, float *y,
+                         void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->T == 0)
+        return MOE_OK;  // nothing to do; array pointers may be NULL
+    if (!o_perm || !slot_of || !y)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(o_perm) || !aligned16(y))
+        return MOE_ERR_UNSUPPORTED;
+    return cuda_status(
+        moe::launch_combine(o_perm, slot_of, desc->T, desc->k, desc->H, y, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr, const float *bias,
+                         const uint16_t *W_gate_up, const uint16_t *W_down, const uint16_t *Wsh_gate_up,
+                         const uint16_t *Wsh_down, float *y, int32_t *topk_idx_out, float *topk_w_out, void *ws,
+                         size_t ws_bytes, void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->T == 0)
+        return MOE_OK;  // nothing to do; array pointers may be NULL
+    if (!x || !Wr || !bias || !W_gate_up || !W_down || !Wsh_gate_up || !Wsh_down || !y || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wr) || !aligned16(W_gate_up) || !aligned16(W_down) ||
+        !aligned16(Wsh_gate_up) || !aligned16(Wsh_down) || !aligned16(y) || !aligned16(ws))
+        return MOE_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(*desc);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const moe_layer_desc &d = *desc;
+    int32_t *idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+    float *w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
+    int32_t *counts = at<int32_t>(ws, L.counts);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *perm_token = at<int32_t>(ws, L.perm_token);
+    int32_t *slot_of = at<int32_t>(ws, L.slot_of);
+    stage_mark(0, s);
+    if ((st = run_router(d, di, x, Wr, bias, idx, w, nullptr, s)) != MOE_OK)
+        return st;
+    stage_mark(1, s);
+    if (moe::launch_permute(idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    float *out = d.deterministic ? at<float>(ws, L.o_perm) : y;
+    if ((st = run_expert_ffn(d, di, x, w, offsets, perm_token, slot_of, W_gate_up, W_down, Wsh_gate_up, Wsh_down,
+                             out, ws, s)) != MOE_OK)
+        return st;
+    if (d.deterministic) {
+        st = cuda_status(moe::launch_combine(out, slot_of, d.T, d.k, d.H, y, s));
+        stage_mark(6, s);
+        return st;
+    }
+    return MOE_OK;
+}
+
+moe_status_t moe_check_device(void)
+{
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK)
+        return st;
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return MOE_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_moe_err, sizeof v) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (v != 0) {
+        const uint32_t zero = 0;
+        if (cudaMemcpyToSymbol(g_moe_err, &zero, sizeof zero) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    return (v & moe::kDevErrTimeout) ? MOE_ERR_TIMEOUT : MOE_OK;
+}
+
+moe_status_t moe_set_stage_events(void *const *events, int n)
+{
+    if (n < 0 || n > kMaxStageEvents || (n > 0 && !events))
+        return MOE_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_ev_mu);
+    for (int i = 0; i < n; ++i)
+        g_stage_ev[i] = static_cast<cudaEvent_t>(events[i]);
+    g_stage_n = n;
+    return MOE_OK;
+}
+
+uint64_t moe_set_wait_limit_ns(uint64_t ns)
+{
+    if (ns < 1000)
+        ns = 1000;
+    return g_wait_limit_ns.exchange(ns);
+}
+
+}  // extern "C"

@@ -1,0 +1,263 @@
+// permute.cu — integer stages of the MoE layer on sm_100a: the token -> slot
+// permutation (histogram, exclusive scan, stable scatter), the gather of token rows into
+// expert-contiguous order, the tile table of the grouped GEMMs, and the fixed-order
+// combine of the deterministic mode.
+//
+// The permutation is the local form of an expert-parallel dispatch ("MAX 中 Step-3.5-Flash
+// 架构解析", section "并行模式TP_TP / TP_EP / DP_EP"): slots of expert e are
+// [offsets[e], offsets[e+1]), ordered by token. Group E is the always-on shared expert
+// (section "MoE共享专家、sigmoid 路由与激活裁剪") holding every token in order.
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kPermThreads = 1024;  // 32 warps; warp w owns a contiguous token range
+
+// Single CTA. Pass 1: per-warp per-expert counts, built 32 entries at a time with
+// __match_any_sync (one leader per distinct expert adds the group size). Pass 2: per
+// expert, exclusive prefix over warps; exclusive scan over experts. Pass 3: the same
+// walk again; an entry's slot = its warp's base for that expert + the number of earlier
+// lanes in its round with the same expert. Entries are visited in (token, rank) order,
+// so slots within an expert are in token order: the result is unique and deterministic.
+__global__ void __launch_bounds__(kPermThreads)
+    permute_kernel(const int32_t *__restrict__ idx, int T, int k, int E, int32_t *__restrict__ counts,
+                   int32_t *__restrict__ offsets, int32_t *__restrict__ perm_token, int32_t *__restrict__ slot_of)
+{
+    extern __shared__ int32_t sm[];
+    int32_t *cnt = sm;           // [32][E]
+    int32_t *tot = sm + 32 * E;  // [E]
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < 32 * E; i += kPermThreads)
+        cnt[i] = 0;
+    __syncthreads();
+
+    const int per_warp = (T + 31) / 32;
+    const int64_t t_begin = static_cast<int64_t>(warp) * per_warp < T ? static_cast<int64_t>(warp) * per_warp : T;
+    const int64_t t_end = t_begin + per_warp < T ? t_begin + per_warp : T;
+    const int64_t begin = t_begin * k, end = t_end * k;
+    int32_t *mine = cnt + warp * E;
+
+    for (int64_t b = begin; b < end; b += 32) {
+        const int64_t n = b + lane;
+        const bool valid = n < end;
+        int e = E + lane;  // distinct sentinel for idle lanes
+        if (valid) {
+            e = idx[n];
+            e = e < 0 ? 0 : (e > E - 1 ? E - 1 : e);
+        }
+        const unsigned m = __match_any_sync(0xFFFFFFFFu, e);
+        if (valid && lane == 31 - __clz(m))
+            mine[e] += __popc(m);
+        __syncwarp();
+    }
+    __syncthreads();
+
+    for (int e = threadIdx.x; e < E; e += kPermThreads) {
+        int run = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int c = cnt[w * E + e];
+            cnt[w * E + e] = run;
+            run += c;
+        }
+        tot[e] = run;
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        const int per = (E + 31) / 32;
+        const int lo = lane * per;
+        const int hi = lo + per < E ? lo + per : E;
+        int s = 0;
+        for (int e = lo; e < hi; ++e)
+            s += tot[e];
+        int incl = s;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o)
+                incl += v;
+        }
+        int run = incl - s;
+        for (int e = lo; e < hi; ++e) {
+            const int c = tot[e];
+            counts[e] = c;
+            offsets[e] = run;
+            tot[e] = run;
+            run += c;
+        }
+        if (lane == 31) {
+            counts[E] = T;
+            offsets[E] = incl;
+            offsets[E + 1] = incl + T;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 32 * E; i += kPermThreads)
+        cnt[i] += tot[i % E];
+    __syncthreads();
+
+    for (int64_t b = begin; b < end; b += 32) {
+        const int64_t n = b + lane;
+        const bool valid = n < end;
+        int e = E + lane;
+        if (valid) {
+            e = idx[n];
+            e = e < 0 ? 0 : (e > E - 1 ? E - 1 : e);
+        }
+        const unsigned m = __match_any_sync(0xFFFFFFFFu, e);
+        if (valid) {
+            const int slot = mine[e] + __popc(m & ((1u << lane) - 1u));
+            slot_of[n] = slot;
+            perm_token[slot] = static_cast<int32_t>(n / k);
+        }
+        __syncwarp();
+        if (valid && lane == 31 - __clz(m))
+            mine[e] += __popc(m);
+        __syncwarp();
+    }
+    const int64_t shared_base = static_cast<int64_t>(T) * k;
+    for (int t = threadIdx.x; t < T; t += kPermThreads)
+        perm_token[shared_base + t] = t;
+}
+
+// One warp per (token, rank) entry: copies the token's row of x into its slot and
+// records the slot's routing weight.
+__global__ void __launch_bounds__(256)
+    gather_kernel(const uint4 *__restrict__ x, const float *__restrict__ topk_w,
+                  const int32_t *__restrict__ slot_of, int64_t nent, int k, int vec_per_row,
+                  uint4 *__restrict__ x_perm, float *__restrict__ w_perm)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t n = gw; n < nent; n += nw) {
+        const int64_t slot = slot_of[n];
+        const int64_t t = n / k;
+        const uint4 *src = x + t * vec_per_row;
+        uint4 *dst = x_perm + slot * vec_per_row;
+#pragma unroll 4
+        for (int v = lane; v < vec_per_row; v += 32)
+            dst[v] = __ldg(src + v);
+        if (lane == 0)
+            w_perm[slot] = topk_w[n];
+    }
+}
+
+// One thread per group g in [0, E] (E = shared expert). A group of n rows becomes
+// ceil(n / 256) chunks of equal size rounded up to 16 rows (the last one shorter).
+__global__ void __launch_bounds__(1024)
+    chunks_kernel(const int32_t *__restrict__ offsets, int E, int T, int4 *__restrict__ chunks,
+                  int32_t *__restrict__ hdr)
+{
+    __shared__ int warp_sums[32];
+    const int g = threadIdx.x;
+    const int lane = g & 31, warp = g >> 5;
+    int n = 0, base = 0;
+    if (g < E) {
+        base = offsets[g];
+        n = offsets[g + 1] - base;
+    } else if (g == E) {
+        n = T;
+    }
+    const int nch = n > 0 ? (n + kChunkTokens - 1) / kChunkTokens : 0;
+    const int csz = nch > 0 ? ((n + nch - 1) / nch + 15) / 16 * 16 : 0;
+    int incl = nch;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o)
+            incl += v;
+    }
+    if (lane == 31)
+        warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int ws = warp_sums[lane];
+        int wi = ws;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+            if (lane >= o)
+                wi += v;
+        }
+        warp_sums[lane] = wi - ws;
+    }
+    __syncthreads();
+    const int start = warp_sums[warp] + incl - nch;
+    for (int c = 0; c < nch; ++c) {
+        const int r = c * csz;
+        const int len = n - r < csz ? n - r : csz;
+        chunks[start + c] = make_int4(g, base + r, len, 0);
+    }
+    if (g == E) {
+        hdr[0] = start;
+        hdr[1] = start + nch;
+    }
+}
+
+// y[t] = sum_{j<k} o_perm[slot_of[t, j]] + o_perm[T*k + t], in that order.
+__global__ void __launch_bounds__(256)
+    combine_kernel(const float4 *__restrict__ o_perm, const int32_t *__restrict__ slot_of, int T, int k,
+                   int vec_per_row, float4 *__restrict__ y)
+{
+    const int t = blockIdx.x;
+    const int64_t shared_row = static_cast<int64_t>(T) * k + t;
+    for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const float4 o = __ldg(o_perm + static_cast<int64_t>(slot_of[static_cast<int64_t>(t) * k + j]) * vec_per_row + v);
+            acc.x += o.x;
+            acc.y += o.y;
+            acc.z += o.z;
+            acc.w += o.w;
+        }
+        const float4 o = __ldg(o_perm + shared_row * vec_per_row + v);
+        acc.x += o.x;
+        acc.y += o.y;
+        acc.z += o.z;
+        acc.w += o.w;
+        y[static_cast<int64_t>(t) * vec_per_row + v] = acc;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int32_t *counts, int32_t *offsets,
+                           int32_t *perm_token, int32_t *slot_of, cudaStream_t stream)
+{
+    const int smem = (32 * E + E) * 4;
+    cudaError_t err = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess)
+        return err;
+    permute_kernel<<<1, kPermThreads, smem, stream>>>(idx, T, k, E, counts, offsets, perm_token, slot_of);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
+                          uint16_t *x_perm, float *w_perm, int num_sms, cudaStream_t stream)
+{
+    const int64_t nent = static_cast<int64_t>(T) * k;
+    const int64_t blocks_needed = (nent + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
+    gather_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(x), topk_w, slot_of, nent, k, H / 8,
+                                            reinterpret_cast<uint4 *>(x_perm), w_perm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int k, int4 *chunks, int32_t *hdr,
+                          cudaStream_t stream)
+{
+    (void)k;
+    chunks_kernel<<<1, 1024, 0, stream>>>(offsets, E, T, chunks, hdr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float *o_perm, const int32_t *slot_of, int T, int k, int H, float *y,
+                           cudaStream_t stream)
+{
+    combine_kernel<<<T, 256, 0, stream>>>(reinterpret_cast<const float4 *>(o_perm), slot_of, T, k, H / 4,
+                                          reinterpret_cast<float4 *>(y));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

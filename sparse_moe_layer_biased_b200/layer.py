@@ -1,0 +1,43 @@
+"""MoeLayer: device-resident weights + workspace around the moe_forward entry point.
+
+PyTorch only allocates device memory and supplies the stream; the layer's arithmetic
+runs in libmoe_b200.so.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _abi
+
+
+class MoeLayer:
+    """One MoE layer call shape (inputs.LayerShape) with its weights on a CUDA device.
+
+    weights: dict with Wr [E, H] bf16, bias [E] fp32, W_gate_up [E, 2I, H] bf16,
+    W_down [E, H, I] bf16, Wsh_gate_up [2Is, H] bf16, Wsh_down [H, Is] bf16.
+    """
+
+    def __init__(self, shape, weights: dict, deterministic: bool = False, max_tokens: int | None = None):
+        self.shape = shape
+        self.deterministic = deterministic
+        self.w = weights
+        dev = weights["Wr"].device
+        self.max_tokens = shape.T if max_tokens is None else max_tokens
+        nbytes = _abi.moe_workspace_size(_abi.desc_of(shape, T=self.max_tokens, deterministic=deterministic))
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, routing: bool = False, stream=None):
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError(f"{T} tokens exceed the workspace size of {self.max_tokens}")
+        desc = _abi.desc_of(self.shape, T=T, deterministic=self.deterministic)
+        if y is None:
+            y = torch.empty((T, self.shape.H), dtype=torch.float32, device=x.device)
+        idx = w = None
+        if routing:
+            idx = torch.empty((T, self.shape.k), dtype=torch.int32, device=x.device)
+            w = torch.empty((T, self.shape.k), dtype=torch.float32, device=x.device)
+        W = self.w
+        _abi.moe_forward(desc, x, W["Wr"], W["bias"], W["W_gate_up"], W["W_down"], W["Wsh_gate_up"],
+                         W["Wsh_down"], y, self.ws, idx, w, stream=stream)
+        return (y, idx, w) if routing else y
