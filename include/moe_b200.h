@@ -152,7 +152,8 @@ MOE_API moe_status_t moe_check_device(void);
  * GEMM, events[5] after the down GEMM and, when n >= 7, events[6] after the combine
  * (deterministic mode), each with cudaEventRecord on the call's stream. `events` are
  * cudaEvent_t handles owned by the caller; the array is copied. n = 0 turns it off.
- * Returns MOE_ERR_INVALID_ARG if n < 0, n > 7 or events is NULL with n > 0. */
+ * Returns MOE_ERR_INVALID_ARG if n < 0, n > 7, or n > 0 and events or one of its
+ * entries is NULL. A moe_forward whose event record fails returns MOE_ERR_CUDA. */
 MOE_API moe_status_t moe_set_stage_events(void *const *events, int n);
 
 /* Upper bound, in nanoseconds, of every device-side wait in later launches on this

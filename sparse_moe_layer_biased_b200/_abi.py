@@ -144,7 +144,14 @@ def moe_set_wait_limit_ns(ns: int) -> int:
 
 
 def moe_set_stage_events(events) -> None:
-    """events: list of torch.cuda.Event (enable_timing=True), or [] to turn the hook off."""
+    """events: list of torch.cuda.Event (enable_timing=True), or [] to turn the hook off.
+
+    torch creates an event's CUDA handle on its first record, so events without a handle
+    are recorded once here on the current stream to materialise it.
+    """
+    for ev in events:
+        if not ev.cuda_event:
+            ev.record()
     n = len(events)
     arr = (ctypes.c_void_p * max(n, 1))(*[ev.cuda_event for ev in events])
     _check("moe_set_stage_events", lib().moe_set_stage_events(arr if n else None, n))

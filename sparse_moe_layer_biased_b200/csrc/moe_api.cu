@@ -25,11 +25,10 @@ std::mutex g_ev_mu;
 cudaEvent_t g_stage_ev[kMaxStageEvents];
 int g_stage_n = 0;
 
-void stage_mark(int i, cudaStream_t s)
+bool stage_mark(int i, cudaStream_t s)
 {
     std::lock_guard<std::mutex> lk(g_ev_mu);
-    if (i < g_stage_n)
-        cudaEventRecord(g_stage_ev[i], s);
+    return i >= g_stage_n || cudaEventRecord(g_stage_ev[i], s) == cudaSuccess;
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -221,7 +220,8 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     if (!ok)
         return MOE_ERR_CUDA;
 
-    stage_mark(2, s);
+    if (!stage_mark(2, s))
+        return MOE_ERR_CUDA;
     cudaError_t e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, s);
     if (e == cudaSuccess)
         e = moe::launch_chunks(offsets, d.E, d.T, d.k, chunks, hdr, s);
@@ -231,15 +231,18 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
         return MOE_ERR_CUDA;
     const moe::WaitCfg wc = wait_cfg(di);
     moe::GateUpArgs ga{chunks, hdr, h, h_sh, d.E, d.H, d.I, d.Is, d.limit_routed, d.limit_shared};
-    stage_mark(3, s);
+    if (!stage_mark(3, s))
+        return MOE_ERR_CUDA;
     e = moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, s);
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
     moe::DownArgs da{chunks, hdr, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic};
-    stage_mark(4, s);
+    if (!stage_mark(4, s))
+        return MOE_ERR_CUDA;
     e = moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, s);
-    stage_mark(5, s);
-    return cuda_status(e);
+    if (e != cudaSuccess || !stage_mark(5, s))
+        return MOE_ERR_CUDA;
+    return MOE_OK;
 }
 
 }  // namespace
@@ -382,10 +385,12 @@ moe_status_t moe_forward(const moe_layer_desc *desc, const uint16_t *x, const ui
     int32_t *offsets = at<int32_t>(ws, L.offsets);
     int32_t *perm_token = at<int32_t>(ws, L.perm_token);
     int32_t *slot_of = at<int32_t>(ws, L.slot_of);
-    stage_mark(0, s);
+    if (!stage_mark(0, s))
+        return MOE_ERR_CUDA;
     if ((st = run_router(d, di, x, Wr, bias, idx, w, nullptr, s)) != MOE_OK)
         return st;
-    stage_mark(1, s);
+    if (!stage_mark(1, s))
+        return MOE_ERR_CUDA;
     if (moe::launch_permute(idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     float *out = d.deterministic ? at<float>(ws, L.o_perm) : y;
@@ -394,7 +399,8 @@ moe_status_t moe_forward(const moe_layer_desc *desc, const uint16_t *x, const ui
         return st;
     if (d.deterministic) {
         st = cuda_status(moe::launch_combine(out, slot_of, d.T, d.k, d.H, y, s));
-        stage_mark(6, s);
+        if (st == MOE_OK && !stage_mark(6, s))
+            st = MOE_ERR_CUDA;
         return st;
     }
     return MOE_OK;
@@ -423,6 +429,9 @@ moe_status_t moe_set_stage_events(void *const *events, int n)
 {
     if (n < 0 || n > kMaxStageEvents || (n > 0 && !events))
         return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i)
+        if (!events[i])
+            return MOE_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lk(g_ev_mu);
     for (int i = 0; i < n; ++i)
         g_stage_ev[i] = static_cast<cudaEvent_t>(events[i]);

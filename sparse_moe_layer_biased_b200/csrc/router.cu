@@ -240,13 +240,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         a.idx[static_cast<int64_t>(t) * k + j] = e;
                         a.w[static_cast<int64_t>(t) * k + j] = w;
                     }
-                    if (j == k - 1)
-                        bk = key_value(keys[j]);
+
                 }
+                // k-th and (k+1)-th keys picked by a compare-and-select chain (a dynamic
+                // index would move the list to local memory)
+                uint64_t key_k = 0, key_k1 = 0;
 #pragma unroll
-                for (int j = 1; j <= KMAX; ++j)
-                    if (j == k)
-                        bk1 = key_value(keys[j]);
+                for (int j = 0; j <= KMAX; ++j) {
+                    const bool at_k = (j + 1 == k), at_k1 = (j == k);
+                    key_k = at_k ? keys[j] : key_k;
+                    key_k1 = at_k1 ? keys[j] : key_k1;
+                    asm volatile("" : "+l"(key_k), "+l"(key_k1));
+                }
+                bk = key_value(key_k);
+                bk1 = key_value(key_k1);
                 if (a.margin)
                     a.margin[t] = k < a.E ? bk - bk1 : __int_as_float(0x7F800000);
             }

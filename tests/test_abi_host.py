@@ -105,3 +105,12 @@ def test_wait_limit_roundtrip():
     old = moe.moe_set_wait_limit_ns(5_000_000)
     assert moe.moe_set_wait_limit_ns(old) == 5_000_000
     assert moe.moe_set_wait_limit_ns(old) == old
+
+
+def test_stage_events_validation():
+    L = moe.lib()
+    arr = (ctypes.c_void_p * 2)(FAKE, None)
+    assert L.moe_set_stage_events(arr, 2) == 1
+    assert L.moe_set_stage_events(None, 1) == 1
+    assert L.moe_set_stage_events(arr, 8) == 1
+    assert L.moe_set_stage_events(None, 0) == 0
