@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 
 # Every exported entry point; the header include/moe_b200.h declares exactly these.
 EXPORTS = ["moe_status_string", "moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn",
-           "moe_combine", "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events"]
+           "moe_combine", "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events",
+           "moe_forward_noalloc"]
 
 
 class MoeError(RuntimeError):
@@ -68,6 +69,8 @@ def lib():
         L.moe_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.moe_set_wait_limit_ns.restype = ctypes.c_uint64
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(vp), i32]
+        L.moe_forward_noalloc.argtypes = [dp] + [vp] * 11
+        L.moe_forward_noalloc.restype = i32
         for name in ("moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn", "moe_combine",
                      "moe_forward", "moe_check_device", "moe_set_stage_events"):
             getattr(L, name).restype = i32
@@ -155,3 +158,11 @@ def moe_set_stage_events(events) -> None:
     n = len(events)
     arr = (ctypes.c_void_p * max(n, 1))(*[ev.cuda_event for ev in events])
     _check("moe_set_stage_events", lib().moe_set_stage_events(arr if n else None, n))
+
+
+def moe_forward_noalloc(desc, x, Wr, bias, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y, topk_idx_out=None,
+                        topk_w_out=None, stream=None):
+    """moe_forward on the library's built-in 16 MiB scratch instead of a caller workspace."""
+    _check("moe_forward_noalloc", lib().moe_forward_noalloc(
+        ctypes.byref(desc), _p(x), _p(Wr), _p(bias), _p(W_gate_up), _p(W_down), _p(Wsh_gate_up), _p(Wsh_down),
+        _p(y), _p(topk_idx_out), _p(topk_w_out), _stream(stream)))
