@@ -7,14 +7,17 @@
 // "Step3p5Config配置项全解"). The fused [2I, H] gate_up and [H, I] down layouts follow
 // the 24 MiB / 12 MiB BF16 expert tensors of the miles Step-5-Preview page, section 5.3.
 //
-// Both kernels are "swap-AB": the expert weight rows fill the 128-lane M side of the
-// UMMA and the tokens of one expert chunk (16..256, a multiple of 16) are the N side, so
-// a ragged group wastes at most 15 token columns, and a decode-sized group of one or
-// two tokens still streams full 128-row weight tiles.
+// Both kernels are "swap-AB": expert weight rows fill the 128-lane M side of the UMMA
+// and the tokens of one expert chunk (up to BN rows, rounded up to a multiple of 16) are
+// the N side, so a ragged group wastes at most 15 token columns and a decode-sized group
+// of one or two tokens still streams full weight tiles. A stage holds MT weight tiles of
+// 128 rows that share one token tile: MT = 2 halves how often a token chunk is re-read
+// from L2 per weight byte (the token tile is reused by two MMAs per K step).
 //
 // Roles per CTA (persistent, one CTA per SM, static round-robin over tiles):
-//   warp 0      TMA producer: weight tile + token rows (16-row boxes) per 64-wide K slice
-//   warp 1      MMA issuer (one thread) and TMEM owner; 2 x 256-column fp32 accumulators
+//   warp 0      TMA producer: MT weight tiles + token rows (16-row boxes) per 64-wide K slice
+//   warp 1      MMA issuer (one thread) and TMEM owner; 2 buffers x MT accumulators x BN
+//               fp32 columns, so the epilogue of one tile overlaps the mainloop of the next
 //   warps 2..5  epilogue: TMEM -> registers -> activation / weighting -> global
 // Every wait is bounded (mbar_wait); on expiry the CTA drains its own copies and MMAs,
 // frees TMEM and returns with the device error word set.
@@ -24,17 +27,25 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 4;
 constexpr int kBK = 64;
-constexpr uint32_t kABytes = 128 * 128;     // 128 weight rows x 64 bf16
-constexpr uint32_t kBBytes = 256 * 128;     // up to 256 token rows x 64 bf16
-constexpr uint32_t kBoxBytes = 16 * 128;    // one 16-row token box
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kBarOff = kStages * kStageBytes;
-constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * kStages + 5);
-constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
-constexpr uint32_t kAccCols = 256;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kATileBytes = 128 * 128;  // 128 weight rows x 64 bf16
+constexpr uint32_t kBoxBytes = 16 * 128;     // one 16-row token box
+
+// Ring geometry: token chunks of at most BN rows, S stages, MT weight tiles per stage.
+template <int BN, int S, int MT>
+struct Geo {
+    static constexpr uint32_t kABytes = MT * kATileBytes;
+    static constexpr uint32_t kBBytes = BN * 128;
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+    static constexpr uint32_t kBarOff = S * kStageBytes;
+    static constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * S + 5);
+    static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
+    static constexpr uint32_t kBufCols = MT * BN;  // one TMEM buffer: MT accumulators of BN columns
+    static constexpr uint32_t kTmemCols = 2 * kBufCols < 32 ? 32 : 2 * kBufCols;
+    static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
+    static_assert(kSmemBytes <= kMaxDynSmem, "ring exceeds shared memory");
+    static_assert((kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512, "TMEM allocation");
+};
 
 struct Ring {
     uint64_t *full, *empty, *accf, *acce, *drain;
@@ -42,20 +53,21 @@ struct Ring {
     volatile int *abort_flag;
 };
 
+template <class G, int S>
 __device__ __forceinline__ uint8_t *ring_setup(uint8_t *smem_raw, Ring &r)
 {
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *smem = smem_raw + pad;
-    r.full = reinterpret_cast<uint64_t *>(smem + kBarOff);
-    r.empty = r.full + kStages;
-    r.accf = r.empty + kStages;
+    r.full = reinterpret_cast<uint64_t *>(smem + G::kBarOff);
+    r.empty = r.full + S;
+    r.accf = r.empty + S;
     r.acce = r.accf + 2;
     r.drain = r.acce + 2;
-    r.holder = reinterpret_cast<uint32_t *>(smem + kMiscOff);
-    r.abort_flag = reinterpret_cast<volatile int *>(smem + kMiscOff + 4);
+    r.holder = reinterpret_cast<uint32_t *>(smem + G::kMiscOff);
+    r.abort_flag = reinterpret_cast<volatile int *>(smem + G::kMiscOff + 4);
     const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&r.full[s], 1);
             mbar_init(&r.empty[s], 1);
         }
@@ -68,7 +80,7 @@ __device__ __forceinline__ uint8_t *ring_setup(uint8_t *smem_raw, Ring &r)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(r.holder, kTmemCols);
+        tmem_alloc(r.holder, G::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -77,13 +89,14 @@ __device__ __forceinline__ uint8_t *ring_setup(uint8_t *smem_raw, Ring &r)
     return smem;
 }
 
+template <class G>
 __device__ __forceinline__ void ring_teardown(uint32_t tmem)
 {
     tc_fence_before();
     __syncthreads();
     if ((threadIdx.x >> 5) == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, G::kTmemCols);
     }
 }
 
@@ -96,29 +109,35 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const 
     return __shfl_sync(0xFFFFFFFFu, ok, 0);
 }
 
+template <int S>
 __device__ __forceinline__ void producer_drain(const Ring &r, int issued, const WaitCfg &wc)
 {
-    for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it)
-        mbar_wait_drain(&r.full[it % kStages], (it / kStages) & 1, wc);
+    for (int it = issued > S ? issued - S : 0; it < issued; ++it)
+        mbar_wait_drain(&r.full[it % S], (it / S) & 1, wc);
 }
 
-// MMA issue for one tile: nkb K-slices of 64 into accumulator d (N = n columns).
-// Returns false if a wait gave up.
+// MMA issue for one tile: nkb K-slices of 64; weight tile m of the stage accumulates into
+// columns [d + m*BN, d + m*BN + n). Returns false if a wait gave up.
+template <class G, int S, int BN, int MT>
 __device__ __forceinline__ bool mma_tile(const Ring &r, uint8_t *smem, uint32_t d, int n, int nkb, int &it,
                                          const WaitCfg &wc)
 {
     const uint32_t idesc = idesc_bf16_f32(128, n);
     for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % kStages;
-        if (!mbar_wait(&r.full[s], (it / kStages) & 1, wc, r.abort_flag))
+        const int s = it % S;
+        if (!mbar_wait(&r.full[s], (it / S) & 1, wc, r.abort_flag))
             return false;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
-        const uint64_t ad = sdesc_kmajor_sw128(a_addr);
-        const uint64_t bd = sdesc_kmajor_sw128(a_addr + kABytes);
+        const uint32_t a_addr = smem_u32(smem + s * G::kStageBytes);
+        const uint64_t bd = sdesc_kmajor_sw128(a_addr + G::kABytes);
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const uint64_t ad = sdesc_kmajor_sw128(a_addr + m * kATileBytes);
+                umma_bf16(d + m * BN, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+            }
+        }
         umma_commit(&r.empty[s]);
     }
     return true;
@@ -136,20 +155,21 @@ __device__ __forceinline__ float swiglu_clip(float g, float u, float L)
 
 // ------------------------------------------------------------------------------------
 // gate_up: h[slot, f] = act(Wg_e[f]·x[tok], Wu_e[f]·x[tok]) for one chunk of an expert.
-// A tile = 64 (gate, up) row pairs of one expert, interleaved by the 4-D tensor map
-// (H, half, row, expert) so TMEM lane 2i holds gate row i and lane 2i+1 its up row; the
-// epilogue pairs them with one shuffle. Routed chunks read x_perm; the shared expert's
-// chunks read x directly (identity permutation).
+// A weight tile = 64 (gate, up) row pairs of one expert, interleaved by the 4-D tensor
+// map (H, half, row, expert) so TMEM lane 2i holds gate row i and lane 2i+1 its up row;
+// the epilogue pairs them with one shuffle. A tile covers MT * 64 features. Routed
+// chunks read x_perm; the shared expert's chunks read x directly (identity permutation).
+template <int MT>
 __device__ __forceinline__ void decode_gate_up(const GateUpArgs &a, int nrc, int tiles_r, int tile, int &g,
                                                int &row0, int &ntok, int &fb)
 {
     int ci;
     if (tile < tiles_r) {
-        const int nfb = a.I / 64;
+        const int nfb = a.I / (64 * MT);
         ci = tile / nfb;
         fb = tile - ci * nfb;
     } else {
-        const int nfb = a.Is / 64;
+        const int nfb = a.Is / (64 * MT);
         const int tt = tile - tiles_r;
         ci = nrc + tt / nfb;
         fb = tt - (tt / nfb) * nfb;
@@ -160,21 +180,23 @@ __device__ __forceinline__ void decode_gate_up(const GateUpArgs &a, int nrc, int
     ntok = c.z;
 }
 
+template <int BN, int S, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
     gate_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_wsh,
                    const __grid_constant__ CUtensorMap tm_xp, const __grid_constant__ CUtensorMap tm_x,
                    const GateUpArgs a, const WaitCfg wc)
 {
+    using G = Geo<BN, S, MT>;
     extern __shared__ uint8_t smem_raw[];
     Ring r;
-    uint8_t *smem = ring_setup(smem_raw, r);
+    uint8_t *smem = ring_setup<G, S>(smem_raw, r);
     const uint32_t tmem = *r.holder;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nrc = a.hdr[0];
     const int ntot = a.hdr[1];
-    const int tiles_r = nrc * (a.I / 64);
-    const int tiles = tiles_r + (ntot - nrc) * (a.Is / 64);
+    const int tiles_r = nrc * (a.I / (64 * MT));
+    const int tiles = tiles_r + (ntot - nrc) * (a.Is / (64 * MT));
     const int nkb = a.H / kBK;
 
     if (warp == 0) {
@@ -187,41 +209,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool stop = false;
             for (int tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x) {
                 int g, row0, ntok, fb;
-                decode_gate_up(a, nrc, tiles_r, tile, g, row0, ntok, fb);
+                decode_gate_up<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
                 const bool sh = g == a.E;
                 const int nb = (ntok + 15) >> 4;
-                const uint32_t tx = kABytes + nb * kBoxBytes;
+                const uint32_t tx = G::kABytes + nb * kBoxBytes;
+                const CUtensorMap *mw = sh ? &tm_wsh : &tm_w;
                 const CUtensorMap *mb = sh ? &tm_x : &tm_xp;
+                const int ge = sh ? 0 : g;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int s = it % kStages;
-                    if (!mbar_wait(&r.empty[s], ((it / kStages) & 1) ^ 1, wc, r.abort_flag)) {
+                    const int s = it % S;
+                    if (!mbar_wait(&r.empty[s], ((it / S) & 1) ^ 1, wc, r.abort_flag)) {
                         stop = true;
                         break;
                     }
                     mbar_arrive_expect_tx(&r.full[s], tx);
-                    uint8_t *A = smem + s * kStageBytes;
-                    uint8_t *B = A + kABytes;
-                    if (sh)
-                        tma_load_4d(A, &tm_wsh, &r.full[s], kb * kBK, 0, fb * 64, 0);
-                    else
-                        tma_load_4d(A, &tm_w, &r.full[s], kb * kBK, 0, fb * 64, g);
+                    uint8_t *A = smem + s * G::kStageBytes;
+                    uint8_t *B = A + G::kABytes;
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        tma_load_4d(A + m * kATileBytes, mw, &r.full[s], kb * kBK, 0, (fb * MT + m) * 64, ge);
                     for (int i = 0; i < nb; ++i)
                         tma_load_2d(B + i * kBoxBytes, mb, &r.full[s], kb * kBK, row0 + 16 * i);
                 }
             }
-            producer_drain(r, it, wc);
+            producer_drain<S>(r, it, wc);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             int it = 0, tc = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
                 int g, row0, ntok, fb;
-                decode_gate_up(a, nrc, tiles_r, tile, g, row0, ntok, fb);
+                decode_gate_up<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
                 const int buf = tc & 1;
                 if (!mbar_wait(&r.acce[buf], ((tc >> 1) & 1) ^ 1, wc, r.abort_flag))
                     break;
                 tc_fence_after();
-                if (!mma_tile(r, smem, tmem + buf * kAccCols, (ntok + 15) & ~15, nkb, it, wc))
+                if (!mma_tile<G, S, BN, MT>(r, smem, tmem + buf * G::kBufCols, (ntok + 15) & ~15, nkb, it, wc))
                     break;
                 umma_commit(&r.accf[buf]);
             }
@@ -236,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tc = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
             int g, row0, ntok, fb;
-            decode_gate_up(a, nrc, tiles_r, tile, g, row0, ntok, fb);
+            decode_gate_up<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
             const int buf = tc & 1;
             if (!warp_wait(&r.accf[buf], (tc >> 1) & 1, wc, r.abort_flag))
                 break;
@@ -245,23 +268,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float L = sh ? a.lim_s : a.lim_r;
             uint16_t *out = sh ? a.h_sh : a.h;
             const int64_t ld = sh ? a.Is : a.I;
-            const int64_t feat = fb * 64 + pair;
-            const uint32_t tb = tmem + buf * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
-            for (int cb = 0; cb < ntok; cb += 32) {
-                float v[32];
-                tmem_load32(tb + cb, v);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    // even lane finishes column cb+i (needs the up value), odd lane column
-                    // cb+16+i (needs the gate value)
-                    const float send = is_up ? v[i] : v[16 + i];
-                    const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-                    const float gv = is_up ? recv : v[i];
-                    const float uv = is_up ? v[16 + i] : recv;
-                    const int col = cb + (is_up ? 16 + i : i);
-                    const float hv = swiglu_clip(gv, uv, L);
-                    if (col < ntok)
-                        out[(row0 + col) * ld + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+            for (int m = 0; m < MT; ++m) {
+                const int64_t feat = (fb * MT + m) * 64 + pair;
+                const uint32_t tb =
+                    tmem + buf * G::kBufCols + m * BN + (static_cast<uint32_t>(q * 32) << 16);
+                for (int cb = 0; cb < ntok; cb += 32) {
+                    float v[32];
+                    tmem_load32(tb + cb, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        // even lane finishes column cb+i (needs the up value), odd lane
+                        // column cb+16+i (needs the gate value)
+                        const float send = is_up ? v[i] : v[16 + i];
+                        const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+                        const float gv = is_up ? recv : v[i];
+                        const float uv = is_up ? v[16 + i] : recv;
+                        const int col = cb + (is_up ? 16 + i : i);
+                        const float hv = swiglu_clip(gv, uv, L);
+                        if (col < ntok)
+                            out[(row0 + col) * ld + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+                    }
                 }
             }
             tc_fence_before();
@@ -270,15 +297,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&r.acce[buf]);
         }
     }
-    ring_teardown(tmem);
+    ring_teardown<G>(tmem);
 }
 
 // ------------------------------------------------------------------------------------
 // down: o[f, slot] = Wd_e[f]·h[slot]; routed slots add w_slot * o into y[token] (fp32
 // atomics) or store it in o_perm[slot] (deterministic mode); shared rows add o (weight 1).
+// A tile covers MT * 128 output features.
+template <int MT>
 __device__ __forceinline__ void decode_down(const DownArgs &a, int tile, int &g, int &row0, int &ntok, int &fb)
 {
-    const int nfb = a.H / 128;
+    const int nfb = a.H / (128 * MT);
     const int ci = tile / nfb;
     fb = tile - ci * nfb;
     const int4 c = a.chunks[ci];
@@ -287,19 +316,21 @@ __device__ __forceinline__ void decode_down(const DownArgs &a, int tile, int &g,
     ntok = c.z;
 }
 
+template <int BN, int S, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
     down_kernel(const __grid_constant__ CUtensorMap tm_wd, const __grid_constant__ CUtensorMap tm_wdsh,
                 const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_hsh,
                 const DownArgs a, const WaitCfg wc)
 {
+    using G = Geo<BN, S, MT>;
     extern __shared__ uint8_t smem_raw[];
     Ring r;
-    uint8_t *smem = ring_setup(smem_raw, r);
+    uint8_t *smem = ring_setup<G, S>(smem_raw, r);
     const uint32_t tmem = *r.holder;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int ntot = a.hdr[1];
-    const int tiles = ntot * (a.H / 128);
+    const int tiles = ntot * (a.H / (128 * MT));
 
     if (warp == 0) {
         if (lane == 0) {
@@ -311,43 +342,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool stop = false;
             for (int tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x) {
                 int g, row0, ntok, fb;
-                decode_down(a, tile, g, row0, ntok, fb);
+                decode_down<MT>(a, tile, g, row0, ntok, fb);
                 const bool sh = g == a.E;
                 const int nkb = (sh ? a.Is : a.I) / kBK;
                 const int nb = (ntok + 15) >> 4;
-                const uint32_t tx = kABytes + nb * kBoxBytes;
+                const uint32_t tx = G::kABytes + nb * kBoxBytes;
+                const CUtensorMap *mw = sh ? &tm_wdsh : &tm_wd;
                 const CUtensorMap *mb = sh ? &tm_hsh : &tm_h;
+                const int wrow = (sh ? 0 : g * a.H) + fb * MT * 128;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int s = it % kStages;
-                    if (!mbar_wait(&r.empty[s], ((it / kStages) & 1) ^ 1, wc, r.abort_flag)) {
+                    const int s = it % S;
+                    if (!mbar_wait(&r.empty[s], ((it / S) & 1) ^ 1, wc, r.abort_flag)) {
                         stop = true;
                         break;
                     }
                     mbar_arrive_expect_tx(&r.full[s], tx);
-                    uint8_t *A = smem + s * kStageBytes;
-                    uint8_t *B = A + kABytes;
-                    if (sh)
-                        tma_load_2d(A, &tm_wdsh, &r.full[s], kb * kBK, fb * 128);
-                    else
-                        tma_load_2d(A, &tm_wd, &r.full[s], kb * kBK, g * a.H + fb * 128);
+                    uint8_t *A = smem + s * G::kStageBytes;
+                    uint8_t *B = A + G::kABytes;
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        tma_load_2d(A + m * kATileBytes, mw, &r.full[s], kb * kBK, wrow + m * 128);
                     for (int i = 0; i < nb; ++i)
                         tma_load_2d(B + i * kBoxBytes, mb, &r.full[s], kb * kBK, row0 + 16 * i);
                 }
             }
-            producer_drain(r, it, wc);
+            producer_drain<S>(r, it, wc);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             int it = 0, tc = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
                 int g, row0, ntok, fb;
-                decode_down(a, tile, g, row0, ntok, fb);
+                decode_down<MT>(a, tile, g, row0, ntok, fb);
                 const int nkb = (g == a.E ? a.Is : a.I) / kBK;
                 const int buf = tc & 1;
                 if (!mbar_wait(&r.acce[buf], ((tc >> 1) & 1) ^ 1, wc, r.abort_flag))
                     break;
                 tc_fence_after();
-                if (!mma_tile(r, smem, tmem + buf * kAccCols, (ntok + 15) & ~15, nkb, it, wc))
+                if (!mma_tile<G, S, BN, MT>(r, smem, tmem + buf * G::kBufCols, (ntok + 15) & ~15, nkb, it, wc))
                     break;
                 umma_commit(&r.accf[buf]);
             }
@@ -362,40 +394,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tc = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
             int g, row0, ntok, fb;
-            decode_down(a, tile, g, row0, ntok, fb);
+            decode_down<MT>(a, tile, g, row0, ntok, fb);
             const int buf = tc & 1;
             if (!warp_wait(&r.accf[buf], (tc >> 1) & 1, wc, r.abort_flag))
                 break;
             tc_fence_after();
             const bool sh = g == a.E;
-            const int64_t feat = fb * 128 + f;
-            const uint32_t tb = tmem + buf * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
             for (int cb = 0; cb < ntok; cb += 32) {
-                // lane l fetches the token / slot and weight of column cb + l
+                // lane l fetches the destination row and weight of column cb + l
                 const int mycol = cb + lane;
                 int64_t dst_row = 0;
                 float wgt = 0.0f;
                 if (mycol < ntok) {
                     const int64_t rr = row0 + mycol;
-                    if (a.deterministic) {
+                    if (a.deterministic)
                         dst_row = sh ? shared_base + rr : rr;
-                    } else {
+                    else
                         dst_row = sh ? rr : a.perm_token[rr];
-                    }
                     wgt = sh ? 1.0f : a.w_perm[rr];
                 }
-                float v[32];
-                tmem_load32(tb + cb, v);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int64_t drow = __shfl_sync(0xFFFFFFFFu, dst_row, i);
-                    const float w = __shfl_sync(0xFFFFFFFFu, wgt, i);
-                    if (cb + i < ntok) {
-                        float *p = a.out + drow * H + feat;
-                        if (a.deterministic)
-                            *p = w * v[i];
-                        else
-                            atomicAdd(p, w * v[i]);
+                for (int m = 0; m < MT; ++m) {
+                    const int64_t feat = (fb * MT + m) * 128 + f;
+                    float v[32];
+                    tmem_load32(tmem + buf * G::kBufCols + m * BN + (static_cast<uint32_t>(q * 32) << 16) + cb, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int64_t drow = __shfl_sync(0xFFFFFFFFu, dst_row, i);
+                        const float w = __shfl_sync(0xFFFFFFFFu, wgt, i);
+                        if (cb + i < ntok) {
+                            float *p = a.out + drow * H + feat;
+                            if (a.deterministic)
+                                *p = w * v[i];
+                            else
+                                atomicAdd(p, w * v[i]);
+                        }
                     }
                 }
             }
@@ -405,33 +438,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&r.acce[buf]);
         }
     }
-    ring_teardown(tmem);
+    ring_teardown<G>(tmem);
+}
+
+template <int BN, int S, int MT>
+cudaError_t gate_up_impl(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
+                         const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
+                         cudaStream_t stream)
+{
+    constexpr int smem = static_cast<int>(Geo<BN, S, MT>::kSmemBytes);
+    cudaError_t err =
+        cudaFuncSetAttribute(gate_up_kernel<BN, S, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess)
+        return err;
+    gate_up_kernel<BN, S, MT><<<grid, kThreads, smem, stream>>>(tm_w, tm_wsh, tm_xp, tm_x, a, wc);
+    return cudaGetLastError();
+}
+
+template <int BN, int S, int MT>
+cudaError_t down_impl(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
+                      const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid, cudaStream_t stream)
+{
+    constexpr int smem = static_cast<int>(Geo<BN, S, MT>::kSmemBytes);
+    cudaError_t err = cudaFuncSetAttribute(down_kernel<BN, S, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess)
+        return err;
+    down_kernel<BN, S, MT><<<grid, kThreads, smem, stream>>>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
+// Configurations (chosen by gemm_config): decode chunks of <= 32 tokens with one weight
+// tile per stage and a 10-deep ring of 20 KB stages; prefill chunks of <= 128 tokens with
+// two weight tiles per stage (48 KB stages, 4 deep); prefill shapes whose I, Is or H do
+// not split into two tiles use one weight tile and chunks of <= 256 tokens.
 cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
                            const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
-                           cudaStream_t stream)
+                           const GemmConfig &c, cudaStream_t stream)
 {
-    cudaError_t err =
-        cudaFuncSetAttribute(gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
-    if (err != cudaSuccess)
-        return err;
-    gate_up_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_w, tm_wsh, tm_xp, tm_x, a, wc);
-    return cudaGetLastError();
+    if (c.cap == 32)
+        return gate_up_impl<32, 10, 1>(tm_w, tm_wsh, tm_xp, tm_x, a, wc, grid, stream);
+    if (c.mt == 2)
+        return gate_up_impl<128, 4, 2>(tm_w, tm_wsh, tm_xp, tm_x, a, wc, grid, stream);
+    return gate_up_impl<256, 4, 1>(tm_w, tm_wsh, tm_xp, tm_x, a, wc, grid, stream);
 }
 
 cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
                         const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
-                        cudaStream_t stream)
+                        const GemmConfig &c, cudaStream_t stream)
 {
-    cudaError_t err =
-        cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
-    if (err != cudaSuccess)
-        return err;
-    down_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
-    return cudaGetLastError();
+    if (c.cap == 32)
+        return down_impl<32, 10, 1>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
+    if (c.mt == 2)
+        return down_impl<128, 4, 2>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
+    return down_impl<256, 4, 1>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
 }
 
 }  // namespace moe

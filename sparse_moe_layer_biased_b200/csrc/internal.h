@@ -30,14 +30,31 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int32_t *cou
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
                           uint16_t *x_perm, float *w_perm, int num_sms, cudaStream_t stream);
 
-// Splits every group (E routed experts, then the shared expert) into chunks of at most
-// kChunkTokens rows. hdr[0] = routed chunk count, hdr[1] = total chunk count.
-constexpr int kChunkTokens = 256;
-cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int k, int4 *chunks, int32_t *hdr,
-                          cudaStream_t stream);
-inline int64_t max_chunks(int64_t T, int64_t k, int64_t E)
+// Grouped-GEMM configuration: `cap` = token rows per chunk (the N side of one tile),
+// `mt` = 128-row weight tiles per pipeline stage. Decode-sized calls (at most 16 tokens
+// per expert on average) use 32-row chunks with one weight tile and a deep ring; larger
+// calls use 128-row chunks with two weight tiles per stage when I, Is and H split into
+// such tiles, else 256-row chunks with one.
+struct GemmConfig {
+    int cap;
+    int mt;
+};
+inline GemmConfig gemm_config(int64_t T, int64_t k, int64_t E, int64_t H, int64_t I, int64_t Is)
 {
-    return (T * k + T) / kChunkTokens + E + 2;
+    if (T * k <= 16 * E)
+        return {32, 1};
+    if (I % 128 == 0 && Is % 128 == 0 && H % 256 == 0)
+        return {128, 2};
+    return {256, 1};
+}
+
+// Splits every group (E routed experts, then the shared expert) into chunks of at most
+// `cap` rows. hdr[0] = routed chunk count, hdr[1] = total chunk count.
+cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr,
+                          cudaStream_t stream);
+inline int64_t max_chunks(int64_t T, int64_t k, int64_t E, int64_t H, int64_t I, int64_t Is)
+{
+    return (T * k + T) / gemm_config(T, k, E, H, I, Is).cap + E + 2;
 }
 
 struct GateUpArgs {
@@ -50,7 +67,7 @@ struct GateUpArgs {
 };
 cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
                            const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
-                           cudaStream_t stream);
+                           const GemmConfig &c, cudaStream_t stream);
 
 struct DownArgs {
     const int4 *chunks;
@@ -63,7 +80,7 @@ struct DownArgs {
 };
 cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
                         const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
-                        cudaStream_t stream);
+                        const GemmConfig &c, cudaStream_t stream);
 
 cudaError_t launch_combine(const float *o_perm, const int32_t *slot_of, int T, int k, int H, float *y,
                            cudaStream_t stream);

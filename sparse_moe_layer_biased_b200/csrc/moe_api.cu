@@ -163,7 +163,7 @@ WsLayout ws_layout(const moe_layer_desc &d)
     L.w_perm = take(T * k * 4);
     L.h = take(T * k * I * 2);
     L.h_sh = take(T * Is * 2);
-    L.chunks = take(static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E)) * 16);
+    L.chunks = take(static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, d.H, d.I, d.Is)) * 16);
     L.hdr = take(64);
     L.o_perm = take(d.deterministic ? (T * k + T) * H * 4 : 0);
     L.idx = take(T * k * 4);
@@ -222,9 +222,10 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
 
     if (!stage_mark(2, s))
         return MOE_ERR_CUDA;
+    const moe::GemmConfig cfg = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
     cudaError_t e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, s);
     if (e == cudaSuccess)
-        e = moe::launch_chunks(offsets, d.E, d.T, d.k, chunks, hdr, s);
+        e = moe::launch_chunks(offsets, d.E, d.T, cfg.cap, chunks, hdr, s);
     if (e == cudaSuccess && !d.deterministic)
         e = cudaMemsetAsync(out, 0, static_cast<size_t>(d.T) * d.H * 4, s);
     if (e != cudaSuccess)
@@ -233,13 +234,13 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     moe::GateUpArgs ga{chunks, hdr, h, h_sh, d.E, d.H, d.I, d.Is, d.limit_routed, d.limit_shared};
     if (!stage_mark(3, s))
         return MOE_ERR_CUDA;
-    e = moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, s);
+    e = moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s);
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
     moe::DownArgs da{chunks, hdr, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic};
     if (!stage_mark(4, s))
         return MOE_ERR_CUDA;
-    e = moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, s);
+    e = moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s);
     if (e != cudaSuccess || !stage_mark(5, s))
         return MOE_ERR_CUDA;
     return MOE_OK;

@@ -145,9 +145,9 @@ __global__ void __launch_bounds__(256)
 }
 
 // One thread per group g in [0, E] (E = shared expert). A group of n rows becomes
-// ceil(n / 256) chunks of equal size rounded up to 16 rows (the last one shorter).
+// ceil(n / cap) chunks of equal size rounded up to 16 rows (the last one shorter).
 __global__ void __launch_bounds__(1024)
-    chunks_kernel(const int32_t *__restrict__ offsets, int E, int T, int4 *__restrict__ chunks,
+    chunks_kernel(const int32_t *__restrict__ offsets, int E, int T, int cap, int4 *__restrict__ chunks,
                   int32_t *__restrict__ hdr)
 {
     __shared__ int warp_sums[32];
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(1024)
     } else if (g == E) {
         n = T;
     }
-    const int nch = n > 0 ? (n + kChunkTokens - 1) / kChunkTokens : 0;
+    const int nch = n > 0 ? (n + cap - 1) / cap : 0;
     const int csz = nch > 0 ? ((n + nch - 1) / nch + 15) / 16 * 16 : 0;
     int incl = nch;
     for (int o = 1; o < 32; o <<= 1) {
@@ -244,11 +244,10 @@ cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t 
     return cudaGetLastError();
 }
 
-cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int k, int4 *chunks, int32_t *hdr,
+cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr,
                           cudaStream_t stream)
 {
-    (void)k;
-    chunks_kernel<<<1, 1024, 0, stream>>>(offsets, E, T, chunks, hdr);
+    chunks_kernel<<<1, 1024, 0, stream>>>(offsets, E, T, cap, chunks, hdr);
     return cudaGetLastError();
 }
 

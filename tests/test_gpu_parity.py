@@ -29,6 +29,12 @@ SMALL = {
     "wideE": LayerShape("wideE", T=700, H=256, E=300, k=8, I=64, Is=64, seed=24),
     "k32": LayerShape("k32", T=129, H=256, E=64, k=32, I=128, Is=64, seed=25),
     "nonorm": WORKLOADS["tiny"].replace(name="nonorm", norm_expert_weight=False, scale=2.5),
+    # two weight tiles per stage (I, Is multiples of 128, H of 256; > 16 tokens per expert)
+    "mt2": LayerShape("mt2", T=300, H=512, E=12, k=4, I=256, Is=128, limit_routed=0.25, limit_shared=0.125,
+                      seed=27, weight_std=0.03),
+    # decode-sized: <= 16 tokens per expert on average
+    "decode": LayerShape("decode", T=24, H=512, E=40, k=8, I=192, Is=128, limit_routed=0.25, seed=28,
+                         weight_std=0.03),
 }
 
 
