@@ -20,6 +20,7 @@ struct RouterArgs {
     int T, H, E, k;
     float scale;
     int norm;
+    int num_sms;
 };
 cudaError_t launch_router(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const RouterArgs &a,
                           const WaitCfg &wc, cudaStream_t stream);

@@ -193,7 +193,7 @@ moe_status_t run_router(const moe_layer_desc &d, const DeviceInfo &di, const uin
     CUtensorMap tm_x, tm_wr;
     if (!map_rows(&tm_x, x, d.H, d.T, 128) || !map_rows(&tm_wr, Wr, d.H, d.E, 16))
         return MOE_ERR_CUDA;
-    moe::RouterArgs a{bias, idx, w, margin, d.T, d.H, d.E, d.k, d.scale, d.norm_expert_weight};
+    moe::RouterArgs a{bias, idx, w, margin, d.T, d.H, d.E, d.k, d.scale, d.norm_expert_weight, di.num_sms};
     return cuda_status(moe::launch_router(tm_x, tm_wr, a, wait_cfg(di), s));
 }
 

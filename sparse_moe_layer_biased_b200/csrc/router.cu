@@ -6,11 +6,15 @@
 // sum 1 (norm_expert_weight) and multiplied by moe_router_scaling_factor; indices clamped
 // to [0, E-1].
 //
-// One CTA owns 128 tokens. The logits tile [128 tokens x E] is one tcgen05 GEMM
-// (bf16 x bf16 products, fp32 accumulation in TMEM; E up to 512 columns as two MMAs of
-// N <= 256). TMA streams x and Wr K-slices through a 2-4 stage mbarrier ring. The
-// epilogue gives each TMEM lane (= token) to one thread, which reads its E logits in
-// 32-column chunks and keeps a sorted top-(k+1) list in registers: no logits reach HBM.
+// A thread-block cluster of NS CTAs owns 128 tokens; CTA r owns the experts of slice r
+// (SL experts, a multiple of 16, up to 512). Each CTA computes its logits tile
+// [128 tokens x SL] with tcgen05 MMAs (bf16 x bf16 products, fp32 accumulation in TMEM;
+// two MMAs when SL > 256) fed by a TMA ring,
+// then gives each TMEM lane (= token) to one thread, which keeps a sorted top-(k+1) list
+// of its slice in registers. The lists meet in CTA 0 through distributed shared memory,
+// where each thread merges the NS lists of its token and writes ids, weights and margin.
+// No logits reach global memory. NS is chosen so the grid covers the SMs about once:
+// decode-sized calls split the experts over up to 8 CTAs, large calls use NS = 1.
 #include "internal.h"
 
 namespace moe {
@@ -18,40 +22,56 @@ namespace {
 
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
 constexpr int kTileM = 128;
-constexpr int kBK = 64;                          // bf16 elements per 128-byte swizzled row
-constexpr uint32_t kABytes = kTileM * kBK * 2;   // 16 KB
-constexpr int kBRows = 16;                       // rows per Wr TMA box
+constexpr int kBK = 64;                         // bf16 elements per 128-byte swizzled row
+constexpr uint32_t kABytes = kTileM * kBK * 2;  // 16 KB
+constexpr int kBRows = 16;                      // rows per Wr TMA box
+constexpr int kMaxStages = 8;
 
-struct Layout {
-    int e_pad, n0, n1, stages;
-    uint32_t b_bytes, stage_bytes, bias_off, bar_off, misc_off, total;
-    uint32_t tmem_cols;
+struct Split {
+    int sl;  // experts per CTA (multiple of 16, at most 512)
+    int ns;  // CTAs per cluster
 };
 
-__host__ __device__ inline Layout make_layout(int E)
+// Enough CTAs to cover the SMs once: with few token tiles (decode) the experts are split
+// over up to 8 CTAs; with many token tiles each CTA keeps all experts, so x is read once.
+inline Split make_split(int E, int T, int num_sms)
 {
-    Layout L{};
-    L.e_pad = (E + 15) / 16 * 16;
-    L.n0 = L.e_pad < 256 ? L.e_pad : 256;
-    L.n1 = L.e_pad - L.n0;
-    L.b_bytes = (static_cast<uint32_t>(L.e_pad) * 128 + 1023) / 1024 * 1024;
-    L.stage_bytes = kABytes + L.b_bytes;
-    const uint32_t budget = kMaxDynSmem - 1024 - 4096;
-    int s = static_cast<int>(budget / L.stage_bytes);
-    L.stages = s > 4 ? 4 : s;
-    L.bias_off = L.stages * L.stage_bytes;
-    L.bar_off = L.bias_off + (static_cast<uint32_t>(L.e_pad) * 4 + 15) / 16 * 16;
-    L.misc_off = L.bar_off + 8 * (2 * 4 + 2);
-    L.total = L.misc_off + 16;
-    uint32_t c = 32;
-    while (c < static_cast<uint32_t>(L.e_pad))
-        c <<= 1;
-    L.tmem_cols = c;
-    return L;
+    const int tiles = (T + kTileM - 1) / kTileM;
+    const int e_pad = (E + 15) / 16 * 16;
+    int ns = num_sms / tiles;
+    ns = ns < 1 ? 1 : (ns > 8 ? 8 : ns);
+    ns = ns > e_pad / 16 ? e_pad / 16 : ns;
+    const int sl = ((e_pad + ns - 1) / ns + 15) / 16 * 16;
+    return Split{sl, (E + sl - 1) / sl};
 }
 
+template <int KMAX>
+struct Layout {
+    uint32_t b_bytes, stage_bytes, list_off, bias_off, bar_off, misc_off, total, tmem_cols;
+    int stages;
+    __host__ __device__ explicit Layout(int sl)
+    {
+        b_bytes = (static_cast<uint32_t>(sl) * 128 + 1023) / 1024 * 1024;
+        stage_bytes = kABytes + b_bytes;
+        const uint32_t list_bytes = kTileM * (KMAX + 1) * 12;
+        const uint32_t fixed = list_bytes + static_cast<uint32_t>(sl) * 4 + 8 * (2 * kMaxStages + 2) + 64;
+        int s = static_cast<int>((kMaxDynSmem - 1024 - fixed) / stage_bytes);
+        stages = s > kMaxStages ? kMaxStages : s;
+        list_off = stages * stage_bytes;  // keys [128][KMAX+1] u64, then scores [128][KMAX+1] f32
+        bias_off = list_off + list_bytes;
+        bar_off = (bias_off + static_cast<uint32_t>(sl) * 4 + 7) / 8 * 8;
+        misc_off = bar_off + 8 * (2 * kMaxStages + 2);
+        total = misc_off + 16;
+        uint32_t c = 32;
+        while (c < static_cast<uint32_t>(sl))
+            c <<= 1;
+        tmem_cols = c;
+    }
+};
+
 // Rank key of a biased score: larger key = ranked earlier. Order: value descending
-// (-0 equal to +0), a NaN below every number, ties to the lower expert index.
+// (-0 equal to +0), a NaN below every number, ties to the lower expert index. Key 0
+// (an empty list entry) ranks below every real entry.
 __device__ __forceinline__ uint64_t rank_key(float b, int e)
 {
     uint32_t u;
@@ -75,30 +95,57 @@ __device__ __forceinline__ int key_expert(uint64_t key)
     return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
 }
 
+// Insert (key, s) into the descending register list keys[0..KMAX] (fully unrolled).
+template <int KMAX>
+__device__ __forceinline__ void list_insert(uint64_t (&keys)[KMAX + 1], float (&sv)[KMAX + 1], uint64_t key, float s)
+{
+    if (key > keys[KMAX]) {
+        keys[KMAX] = key;
+        sv[KMAX] = s;
+#pragma unroll
+        for (int j = KMAX; j > 0; --j) {
+            if (keys[j] > keys[j - 1]) {
+                const uint64_t tk = keys[j];
+                keys[j] = keys[j - 1];
+                keys[j - 1] = tk;
+                const float ts = sv[j];
+                sv[j] = sv[j - 1];
+                sv[j - 1] = ts;
+            }
+        }
+    }
+}
+
 template <int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     router_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wr,
-                  const RouterArgs a, const WaitCfg wc)
+                  const RouterArgs a, const int sl, const WaitCfg wc)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *smem = smem_raw + pad;
-    const Layout L = make_layout(a.E);
+    const Layout<KMAX> L(sl);
+    uint64_t *list_keys = reinterpret_cast<uint64_t *>(smem + L.list_off);
+    float *list_s = reinterpret_cast<float *>(smem + L.list_off + kTileM * (KMAX + 1) * 8);
     float *bias_s = reinterpret_cast<float *>(smem + L.bias_off);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);
-    uint64_t *empty = full + 4;
-    uint64_t *accf = empty + 4;
+    uint64_t *empty = full + kMaxStages;
+    uint64_t *accf = empty + kMaxStages;
     uint64_t *drain = accf + 1;
     uint32_t *holder = reinterpret_cast<uint32_t *>(smem + L.misc_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc_off + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kTileM;
+    const uint32_t rank = cluster_ctarank();
+    const int ns = static_cast<int>(gridDim.x);
+    const int e0 = static_cast<int>(blockIdx.x) * sl;
+    const int ne = (a.E - e0) < sl ? (a.E - e0) : sl;  // experts of this slice (>= 1)
+    const int m0 = blockIdx.y * kTileM;
     const int nkb = a.H / kBK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 4; ++s) {
+        for (int s = 0; s < kMaxStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -107,8 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    for (int e = threadIdx.x; e < L.e_pad; e += kThreads)
-        bias_s[e] = e < a.E ? a.bias[e] : 0.0f;
+    for (int e = threadIdx.x; e < sl; e += kThreads)
+        bias_s[e] = e < ne ? a.bias[e0 + e] : 0.0f;
     if (warp == 1) {
         tmem_alloc(holder, L.tmem_cols);
         tmem_relinquish();
@@ -118,11 +165,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *holder;
 
+    // registers of the epilogue thread's list (kept across the cluster barrier in CTA 0)
+    uint64_t keys[KMAX + 1];
+    float sv[KMAX + 1];
+#pragma unroll
+    for (int j = 0; j <= KMAX; ++j) {
+        keys[j] = 0;
+        sv[j] = 0.0f;
+    }
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+
     if (warp == 0) {
         if (lane == 0) {
             tma_prefetch_map(&tm_x);
             tma_prefetch_map(&tm_wr);
-            const uint32_t tx = kABytes + static_cast<uint32_t>(L.e_pad) * 128;
+            const uint32_t tx = kABytes + static_cast<uint32_t>(sl) * 128;
             int issued = 0;
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % L.stages;
@@ -133,8 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t *A = smem + s * L.stage_bytes;
                 uint8_t *B = A + kABytes;
                 tma_load_2d(A, &tm_x, &full[s], kb * kBK, m0);
-                for (int r = 0; r < L.e_pad; r += kBRows)
-                    tma_load_2d(B + r * 128, &tm_wr, &full[s], kb * kBK, r);
+                for (int r = 0; r < sl; r += kBRows)
+                    tma_load_2d(B + r * 128, &tm_wr, &full[s], kb * kBK, e0 + r);
                 ++issued;
             }
             for (int kb = issued > L.stages ? issued - L.stages : 0; kb < issued; ++kb)
@@ -142,8 +200,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id0 = idesc_bf16_f32(kTileM, L.n0);
-            const uint32_t id1 = idesc_bf16_f32(kTileM, L.n1 > 0 ? L.n1 : 16);
+            // N up to 256 per MMA: a slice of more than 256 experts takes two MMAs
+            const int n0 = sl < 256 ? sl : 256;
+            const int n1 = sl - n0;
+            const uint32_t id0 = idesc_bf16_f32(kTileM, n0);
+            const uint32_t id1 = idesc_bf16_f32(kTileM, n1 > 0 ? n1 : 16);
             bool ok = true;
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % L.stages;
@@ -154,16 +215,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(smem + s * L.stage_bytes);
-                const uint32_t b_addr = a_addr + kABytes;
                 const uint64_t ad = sdesc_kmajor_sw128(a_addr);
-                const uint64_t bd0 = sdesc_kmajor_sw128(b_addr);
-                const uint64_t bd1 = sdesc_kmajor_sw128(b_addr + static_cast<uint32_t>(L.n0) * 128);
+                const uint64_t bd0 = sdesc_kmajor_sw128(a_addr + kABytes);
+                const uint64_t bd1 = sdesc_kmajor_sw128(a_addr + kABytes + static_cast<uint32_t>(n0) * 128);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk) {
-                    const uint32_t acc = (kb | kk) != 0;
-                    umma_bf16(tmem, ad + 2 * kk, bd0 + 2 * kk, id0, acc);
-                    if (L.n1 > 0)
-                        umma_bf16(tmem + L.n0, ad + 2 * kk, bd1 + 2 * kk, id1, acc);
+                    umma_bf16(tmem, ad + 2 * kk, bd0 + 2 * kk, id0, (kb | kk) != 0);
+                    if (n1 > 0)
+                        umma_bf16(tmem + n0, ad + 2 * kk, bd1 + 2 * kk, id1, (kb | kk) != 0);
                 }
                 umma_commit(&empty[s]);
             }
@@ -173,92 +232,92 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_drain(drain, 0, wc);
         }
     } else {
-        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
-        const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const int t = m0 + row;
+        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31; one thread per token row
         bool ok = false;
         if (lane == 0)
             ok = mbar_wait(accf, 0, wc, abort_flag);
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         tc_fence_after();
         if (ok) {
-            uint64_t keys[KMAX + 1];
-            float sv[KMAX + 1];
-#pragma unroll
-            for (int j = 0; j <= KMAX; ++j) {
-                keys[j] = 0;
-                sv[j] = 0.0f;
-            }
             const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
-            for (int c0 = 0; c0 < a.E; c0 += 32) {
+            for (int c0 = 0; c0 < ne; c0 += 32) {
                 float v[32];
                 tmem_load32(tbase + c0, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int e = c0 + i;
-                    if (e < a.E) {
+                    if (e < ne) {
                         const float s = 1.0f / (1.0f + expf(-v[i]));
                         const float b = s + bias_s[e];
-                        const uint64_t key = rank_key(b, e);
-                        if (key > keys[KMAX]) {
-                            keys[KMAX] = key;
-                            sv[KMAX] = s;
-#pragma unroll
-                            for (int j = KMAX; j > 0; --j) {
-                                if (keys[j] > keys[j - 1]) {
-                                    const uint64_t tk = keys[j];
-                                    keys[j] = keys[j - 1];
-                                    keys[j - 1] = tk;
-                                    const float ts = sv[j];
-                                    sv[j] = sv[j - 1];
-                                    sv[j - 1] = ts;
-                                }
-                            }
-                        }
+                        list_insert<KMAX>(keys, sv, rank_key(b, e0 + e), s);
                     }
                 }
             }
-            if (t < a.T) {
-                const int k = a.k;
-                float sum = 0.0f;
+        }
+        if (rank != 0) {
 #pragma unroll
-                for (int j = 0; j < KMAX; ++j)
-                    if (j < k)
-                        sum += sv[j];
-                float bk = 0.0f, bk1 = 0.0f;
-#pragma unroll
-                for (int j = 0; j < KMAX; ++j) {
-                    if (j < k) {
-                        int e = key_expert(keys[j]);
-                        e = e < 0 ? 0 : (e > a.E - 1 ? a.E - 1 : e);
-                        float w;
-                        if (a.norm)
-                            w = sum > 0.0f ? a.scale * (sv[j] / sum) : a.scale / static_cast<float>(k);
-                        else
-                            w = a.scale * sv[j];
-                        a.idx[static_cast<int64_t>(t) * k + j] = e;
-                        a.w[static_cast<int64_t>(t) * k + j] = w;
-                    }
-
-                }
-                // k-th and (k+1)-th keys picked by a compare-and-select chain (a dynamic
-                // index would move the list to local memory)
-                uint64_t key_k = 0, key_k1 = 0;
-#pragma unroll
-                for (int j = 0; j <= KMAX; ++j) {
-                    const bool at_k = (j + 1 == k), at_k1 = (j == k);
-                    key_k = at_k ? keys[j] : key_k;
-                    key_k1 = at_k1 ? keys[j] : key_k1;
-                    asm volatile("" : "+l"(key_k), "+l"(key_k1));
-                }
-                bk = key_value(key_k);
-                bk1 = key_value(key_k1);
-                if (a.margin)
-                    a.margin[t] = k < a.E ? bk - bk1 : __int_as_float(0x7F800000);
+            for (int j = 0; j <= KMAX; ++j) {
+                list_keys[row * (KMAX + 1) + j] = keys[j];
+                list_s[row * (KMAX + 1) + j] = sv[j];
             }
         }
     }
+
+    // Lists of CTAs 1..ns-1 become visible to CTA 0; every thread of every CTA gets here.
+    cluster_sync_all();
+
+    if (rank == 0 && warp >= 2) {
+        const uint32_t keys_local = smem_u32(list_keys + row * (KMAX + 1));
+        const uint32_t s_local = smem_u32(list_s + row * (KMAX + 1));
+        for (int p = 1; p < ns; ++p) {
+            const uint32_t kp = dsmem_addr(keys_local, p);
+            const uint32_t sp = dsmem_addr(s_local, p);
+            for (int j = 0; j <= KMAX; ++j) {
+                const uint64_t key = dsmem_ld_u64(kp + 8 * j);
+                if (key <= keys[KMAX])
+                    break;  // peer lists are sorted: nothing further can enter
+                list_insert<KMAX>(keys, sv, key, dsmem_ld_f32(sp + 4 * j));
+            }
+        }
+        const int t = m0 + row;
+        if (t < a.T) {
+            const int k = a.k;
+            float sum = 0.0f;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+                if (j < k)
+                    sum += sv[j];
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j < k) {
+                    int e = key_expert(keys[j]);
+                    e = e < 0 ? 0 : (e > a.E - 1 ? a.E - 1 : e);
+                    float w;
+                    if (a.norm)
+                        w = sum > 0.0f ? a.scale * (sv[j] / sum) : a.scale / static_cast<float>(k);
+                    else
+                        w = a.scale * sv[j];
+                    a.idx[static_cast<int64_t>(t) * k + j] = e;
+                    a.w[static_cast<int64_t>(t) * k + j] = w;
+                }
+            }
+            // k-th and (k+1)-th keys picked by a compare-and-select chain (a dynamic
+            // index would move the list to local memory)
+            uint64_t key_k = 0, key_k1 = 0;
+#pragma unroll
+            for (int j = 0; j <= KMAX; ++j) {
+                const bool at_k = (j + 1 == k), at_k1 = (j == k);
+                key_k = at_k ? keys[j] : key_k;
+                key_k1 = at_k1 ? keys[j] : key_k1;
+                asm volatile("" : "+l"(key_k), "+l"(key_k1));
+            }
+            if (a.margin)
+                a.margin[t] = k < a.E ? key_value(key_k) - key_value(key_k1) : __int_as_float(0x7F800000);
+        }
+    }
+
+    // CTA 0 has finished reading its peers' shared memory before any CTA exits.
+    cluster_sync_all();
 
     tc_fence_before();
     __syncthreads();
@@ -272,13 +331,27 @@ template <int KMAX>
 cudaError_t launch_impl(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const RouterArgs &a,
                         const WaitCfg &wc, cudaStream_t stream)
 {
-    const Layout L = make_layout(a.E);
+    const Split sp = make_split(a.E, a.T, a.num_sms);
+    const Layout<KMAX> L(sp.sl);
     const int smem = static_cast<int>(L.total) + 1024;
     cudaError_t err = cudaFuncSetAttribute(router_kernel<KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
-    const int grid = (a.T + kTileM - 1) / kTileM;
-    router_kernel<KMAX><<<grid, kThreads, smem, stream>>>(tm_x, tm_wr, a, wc);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sp.ns, (a.T + kTileM - 1) / kTileM, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = sp.ns;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, router_kernel<KMAX>, tm_x, tm_wr, a, sp.sl, wc);
+    if (err != cudaSuccess)
+        return err;
     return cudaGetLastError();
 }
 
