@@ -113,6 +113,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value: float, device) -> float:
+    """Largest value over all ranks (the job's time is its slowest rank's time)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: tokens processed by all ranks over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
+
+
 def workload_config(shape, extra=None):
     c = {"workload": shape.name, "T": shape.T, "H": shape.H, "E": shape.E, "k": shape.k, "I": shape.I,
          "Is": shape.Is, "scale": shape.scale, "norm_expert_weight": shape.norm_expert_weight,
@@ -264,11 +281,7 @@ def run_b200(args, shape):
     clocks = sampler.stop()
     _abi.moe_set_stage_events([])
     barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), "cuda")
     names = ["router", "permute", "gather_tiles", "gate_up", "down", "combine"][: nstage - 1]
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
                 for j, n in enumerate(names)}
@@ -294,12 +307,8 @@ def run_b200(args, shape):
             y_h.copy_(y, non_blocking=True)
         e2.record(stream)
         torch.cuda.synchronize()
-        ms2 = s2.elapsed_time(e2)
-        if world > 1:
-            t = torch.tensor([ms2], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms2 = float(t.item())
-        e2e = {"value": world * shape.T * args.steps / (ms2 / 1e3), "unit": UNIT,
+        ms2 = max_over_ranks(s2.elapsed_time(e2), "cuda")
+        e2e = {"value": job_tokens_per_s(world, shape.T, args.steps, ms2), "unit": UNIT,
                "h2d_bytes_per_step": shape.T * shape.H * 2, "d2h_bytes_per_step": shape.T * shape.H * 4}
 
     peaks, peak_kind = load_peaks()
@@ -312,7 +321,7 @@ def run_b200(args, shape):
                 "touched_experts": touched}
     flops = shape.flops_per_token * shape.T
     step_ms = ms / args.steps
-    value = world * shape.T * args.steps / (ms / 1e3)
+    value = job_tokens_per_s(world, shape.T, args.steps, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
