@@ -21,6 +21,7 @@
 //   warps 2..5  epilogue: TMEM -> registers -> activation / weighting -> global
 // Every wait is bounded (mbar_wait); on expiry the CTA drains its own copies and MMAs,
 // frees TMEM and returns with the device error word set.
+#include "gemm_common.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -100,15 +101,6 @@ __device__ __forceinline__ void ring_teardown(uint32_t tmem)
     }
 }
 
-// Lane 0 waits, the whole warp learns the outcome (keeps warp-collective ops converged).
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const WaitCfg &wc, volatile int *ab)
-{
-    bool ok = false;
-    if ((threadIdx.x & 31) == 0)
-        ok = mbar_wait(bar, parity, wc, ab);
-    return __shfl_sync(0xFFFFFFFFu, ok, 0);
-}
-
 template <int S>
 __device__ __forceinline__ void producer_drain(const Ring &r, int issued, const WaitCfg &wc)
 {
@@ -141,16 +133,6 @@ __device__ __forceinline__ bool mma_tile(const Ring &r, uint8_t *smem, uint32_t 
         umma_commit(&r.empty[s]);
     }
     return true;
-}
-
-__device__ __forceinline__ float swiglu_clip(float g, float u, float L)
-{
-    float a = g / (1.0f + expf(-g));
-    if (L > 0.0f) {
-        a = a > L ? L : a;
-        u = u > L ? L : (u < -L ? -L : u);
-    }
-    return a * u;
 }
 
 // ------------------------------------------------------------------------------------
@@ -469,14 +451,16 @@ cudaError_t down_impl(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, cons
 
 }  // namespace
 
-// Configurations (chosen by gemm_config): decode chunks of <= 32 tokens with one weight
-// tile per stage and a 10-deep ring of 20 KB stages; prefill chunks of <= 128 tokens with
-// two weight tiles per stage (48 KB stages, 4 deep); prefill shapes whose I, Is or H do
-// not split into two tiles use one weight tile and chunks of <= 256 tokens.
+// Configurations (chosen by gemm_config): CTA pairs (expert_gemm_pair.cu); decode chunks
+// of <= 32 tokens with one weight tile per stage and a 10-deep ring of 20 KB stages;
+// chunks of <= 128 tokens with two weight tiles per stage (48 KB stages, 4 deep); shapes
+// whose I, Is or H do not split into two tiles use one weight tile and <= 256 tokens.
 cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
                            const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
                            const GemmConfig &c, cudaStream_t stream)
 {
+    if (c.pair)
+        return launch_gate_up_pair(tm_w, tm_wsh, tm_xp, tm_x, a, wc, grid, stream);
     if (c.cap == 32)
         return gate_up_impl<32, 10, 1>(tm_w, tm_wsh, tm_xp, tm_x, a, wc, grid, stream);
     if (c.mt == 2)
@@ -488,6 +472,8 @@ cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, co
                         const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
                         const GemmConfig &c, cudaStream_t stream)
 {
+    if (c.pair)
+        return launch_down_pair(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
     if (c.cap == 32)
         return down_impl<32, 10, 1>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
     if (c.mt == 2)

@@ -1,0 +1,499 @@
+// expert_gemm_pair.cu — grouped expert GEMMs on CTA pairs (tcgen05 cta_group::2).
+//
+// Same layer steps and layouts as expert_gemm.cu ("MAX 中 Step-3.5-Flash 架构解析",
+// section "MoE共享专家、sigmoid 路由与激活裁剪": routed_moe(x) + shared_expert(x) with the
+// clipped, concatenated gate/up activation), for prefill-sized calls. Two CTAs of a
+// cluster (an SM pair) work on one tile: each holds MT weight tiles of 128 rows and HALF
+// of the token rows of the chunk; the leader CTA issues M = 256 MMAs that read the weight
+// rows of both CTAs and the token rows of both, and each CTA's TMEM receives its own 128
+// weight rows x all N tokens. Per SM, the token bytes per stage halve and the ring gets a
+// fifth stage, so more weight bytes are in flight (the HBM-bound case) and each MMA reads
+// half as many token bytes from this SM's shared memory (the compute-bound case).
+//
+// Pair protocol (leader = cluster rank 0):
+//   - both producers load into their own shared memory; the transaction bytes of both
+//     complete on the LEADER's full barrier, which only the leader arms (expect_tx);
+//   - the leader's MMA commit arrives on the empty / accumulator-full / drain barriers of
+//     both CTAs (multicast commit), so each producer and epilogue waits locally;
+//   - both CTAs' epilogue warps arrive on the leader's accumulator-empty barrier (8 arrivals);
+//   - TMEM is allocated and freed by warp 1 of both CTAs together (cta_group::2).
+// Every mbarrier wait is bounded; the cluster barriers at the start and end are reached
+// by every thread of both CTAs on every path.
+#include "gemm_common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kBK = 64;
+constexpr uint32_t kATileBytes = 128 * 128;  // 128 weight rows x 64 bf16
+constexpr uint32_t kBoxBytes = 16 * 128;     // one 16-row token box
+
+// BN = token rows per pair tile (N of the pair MMA); each CTA holds BN/2 of them.
+// NB = accumulator buffers in TMEM (2: the epilogue of one tile overlaps the next tile's
+// mainloop; 1: larger tiles, the MMA waits for the epilogue between tiles).
+template <int BN, int S, int MT, int NB>
+struct PairGeo {
+    static constexpr uint32_t kABytes = MT * kATileBytes;
+    static constexpr uint32_t kBBytes = (BN / 2) * 128;
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+    static constexpr uint32_t kBarOff = S * kStageBytes;
+    static constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * S + 5);
+    static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
+    static constexpr uint32_t kBufCols = MT * BN;
+    static constexpr uint32_t kTmemCols = NB * kBufCols <= 32 ? 32 : (NB * kBufCols <= 64 ? 64 : (NB * kBufCols <= 128 ? 128 : (NB * kBufCols <= 256 ? 256 : 512)));
+    static_assert(NB * kBufCols <= 512, "accumulators exceed TMEM");
+    static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
+    static_assert(kSmemBytes <= kMaxDynSmem, "ring exceeds shared memory");
+
+    static_assert(BN % 32 == 0 && BN <= 256, "pair token tile");
+};
+
+struct PairRing {
+    uint64_t *full, *empty, *accf, *acce, *drain;
+    uint32_t *holder;
+    volatile int *abort_flag;
+    uint32_t rank;
+    uint32_t full_leader;  // shared::cluster address of the leader's full[0]
+    uint32_t acce_leader;  // shared::cluster address of the leader's acce[0]
+};
+
+template <class G, int S>
+__device__ __forceinline__ uint8_t *pair_setup(uint8_t *smem_raw, PairRing &r)
+{
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    uint8_t *smem = smem_raw + pad;
+    r.full = reinterpret_cast<uint64_t *>(smem + G::kBarOff);
+    r.empty = r.full + S;
+    r.accf = r.empty + S;
+    r.acce = r.accf + 2;
+    r.drain = r.acce + 2;
+    r.holder = reinterpret_cast<uint32_t *>(smem + G::kMiscOff);
+    r.abort_flag = reinterpret_cast<volatile int *>(smem + G::kMiscOff + 4);
+    r.rank = cluster_ctarank();
+    r.full_leader = dsmem_addr(smem_u32(r.full), 0);
+    r.acce_leader = dsmem_addr(smem_u32(r.acce), 0);
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&r.full[s], 1);
+            mbar_init(&r.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&r.accf[b], 1);
+            mbar_init(&r.acce[b], 8);  // 4 epilogue warps in each CTA of the pair
+        }
+        mbar_init(r.drain, 1);
+        *r.abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(r.holder, G::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // barriers of both CTAs are initialised before any remote arrival
+    tc_fence_after();
+    return smem;
+}
+
+template <class G>
+__device__ __forceinline__ void pair_teardown(uint32_t tmem)
+{
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs are done with TMEM, shared memory and each other's barriers
+    if ((threadIdx.x >> 5) == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, G::kTmemCols);
+    }
+}
+
+// Leader only: the loads of the last S stages (both CTAs' bytes count on the leader's
+// full barriers) have landed.
+template <int S>
+__device__ __forceinline__ void pair_producer_drain(const PairRing &r, int issued, const WaitCfg &wc)
+{
+    if (r.rank != 0)
+        return;
+    for (int it = issued > S ? issued - S : 0; it < issued; ++it)
+        mbar_wait_drain(&r.full[it % S], (it / S) & 1, wc);
+}
+
+// Leader's MMA issue for one pair tile: nkb K-slices; weight tile m accumulates into
+// columns [d + m*BN, d + m*BN + n) of both CTAs' TMEM.
+template <class G, int S, int BN, int MT>
+__device__ __forceinline__ bool pair_mma_tile(const PairRing &r, uint8_t *smem, uint32_t d, int n, int nkb,
+                                              int &it, const WaitCfg &wc)
+{
+    const uint32_t idesc = idesc_bf16_f32(256, n);
+    for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % S;
+        if (!mbar_wait(&r.full[s], (it / S) & 1, wc, r.abort_flag))
+            return false;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + s * G::kStageBytes);
+        const uint64_t bd = sdesc_kmajor_sw128(a_addr + G::kABytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const uint64_t ad = sdesc_kmajor_sw128(a_addr + m * kATileBytes);
+                umma_bf16_pair(d + m * BN, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+            }
+        }
+        umma_commit_pair_mc(&r.empty[s], 0x3);
+    }
+    return true;
+}
+
+// The leader runs the MMA loop; the peer's MMA warp only waits for the final drain.
+template <class G, int S, int BN, int MT, int NB, class NextTile>
+__device__ __forceinline__ void pair_mma_role(const PairRing &r, uint8_t *smem, uint32_t tmem, int first,
+                                              int tiles, int stride, NextTile tile_info, const WaitCfg &wc)
+{
+    if (r.rank == 0) {
+        int it = 0, tc = 0;
+        for (int tile = first; tile < tiles; tile += stride, ++tc) {
+            int ntok, nkb;
+            tile_info(tile, ntok, nkb);
+            const int buf = tc % NB;
+            if (!mbar_wait(&r.acce[buf], ((tc / NB) & 1) ^ 1, wc, r.abort_flag))
+                break;
+            tc_fence_after();
+            if (!pair_mma_tile<G, S, BN, MT>(r, smem, tmem + buf * G::kBufCols, (ntok + 15) & ~15, nkb, it, wc))
+                break;
+            umma_commit_pair_mc(&r.accf[buf], 0x3);
+        }
+        umma_commit_pair_mc(r.drain, 0x3);
+    }
+    mbar_wait_drain(r.drain, 0, wc);
+}
+
+// ------------------------------------------------------------------------------------
+// gate_up on pairs: a pair tile covers 2 * MT * 64 features (CTA r holds weight tiles
+// (fb * 2 + r) * MT + m of 64 (gate, up) row pairs each).
+template <int MT>
+__device__ __forceinline__ void decode_gate_up_pair(const GateUpArgs &a, int nrc, int tiles_r, int tile, int &g,
+                                                    int &row0, int &ntok, int &fb)
+{
+    int ci;
+    if (tile < tiles_r) {
+        const int nfb = a.I / (128 * MT);
+        ci = tile / nfb;
+        fb = tile - ci * nfb;
+    } else {
+        const int nfb = a.Is / (128 * MT);
+        const int tt = tile - tiles_r;
+        ci = nrc + tt / nfb;
+        fb = tt - (tt / nfb) * nfb;
+    }
+    const int4 c = a.chunks[ci];
+    g = c.x;
+    row0 = c.y;
+    ntok = c.z;
+}
+
+template <int BN, int S, int MT, int NB>
+__global__ void __launch_bounds__(kThreads, 1)
+    gate_up_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_wsh,
+                        const __grid_constant__ CUtensorMap tm_xp, const __grid_constant__ CUtensorMap tm_x,
+                        const GateUpArgs a, const WaitCfg wc)
+{
+    using G = PairGeo<BN, S, MT, NB>;
+    extern __shared__ uint8_t smem_raw[];
+    PairRing r;
+    uint8_t *smem = pair_setup<G, S>(smem_raw, r);
+    const uint32_t tmem = *r.holder;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nrc = a.hdr[0];
+    const int ntot = a.hdr[1];
+    const int tiles_r = nrc * (a.I / (128 * MT));
+    const int tiles = tiles_r + (ntot - nrc) * (a.Is / (128 * MT));
+    const int nkb = a.H / kBK;
+    const int first = blockIdx.x >> 1;
+    const int stride = gridDim.x >> 1;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_map(&tm_w);
+            tma_prefetch_map(&tm_wsh);
+            tma_prefetch_map(&tm_xp);
+            tma_prefetch_map(&tm_x);
+            int it = 0;
+            bool stop = false;
+            for (int tile = first; tile < tiles && !stop; tile += stride) {
+                int g, row0, ntok, fb;
+                decode_gate_up_pair<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
+                const bool sh = g == a.E;
+                const int half = ((ntok + 15) & ~15) >> 1;  // token rows held by each CTA
+                const int nb = (half + 15) >> 4;
+                const uint32_t tx = 2 * (G::kABytes + nb * kBoxBytes);
+                const CUtensorMap *mw = sh ? &tm_wsh : &tm_w;
+                const CUtensorMap *mb = sh ? &tm_x : &tm_xp;
+                const int ge = sh ? 0 : g;
+                const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
+                const int brow = row0 + static_cast<int>(r.rank) * half;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % S;
+                    if (!mbar_wait(&r.empty[s], ((it / S) & 1) ^ 1, wc, r.abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    if (r.rank == 0)
+                        mbar_arrive_expect_tx(&r.full[s], tx);
+                    const uint32_t bar = r.full_leader + 8 * s;
+                    uint8_t *A = smem + s * G::kStageBytes;
+                    uint8_t *B = A + G::kABytes;
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        tma_load_4d_pair(A + m * kATileBytes, mw, bar, kb * kBK, 0, (wt0 + m) * 64, ge);
+                    for (int i = 0; i < nb; ++i)
+                        tma_load_2d_pair(B + i * kBoxBytes, mb, bar, kb * kBK, brow + 16 * i);
+                }
+            }
+            pair_producer_drain<S>(r, it, wc);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            auto info = [&](int tile, int &ntok, int &nk) {
+                int g, row0, fb;
+                decode_gate_up_pair<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
+                nk = nkb;
+            };
+            pair_mma_role<G, S, BN, MT, NB>(r, smem, tmem, first, tiles, stride, info, wc);
+        }
+    } else {
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int pair = row >> 1;
+        const bool is_up = row & 1;
+        int tc = 0;
+        for (int tile = first; tile < tiles; tile += stride, ++tc) {
+            int g, row0, ntok, fb;
+            decode_gate_up_pair<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
+            const int buf = tc % NB;
+            if (!warp_wait(&r.accf[buf], (tc / NB) & 1, wc, r.abort_flag))
+                break;
+            tc_fence_after();
+            const bool sh = g == a.E;
+            const float L = sh ? a.lim_s : a.lim_r;
+            uint16_t *out = sh ? a.h_sh : a.h;
+            const int64_t ld = sh ? a.Is : a.I;
+            const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const int64_t feat = (wt0 + m) * 64 + pair;
+                const uint32_t tb =
+                    tmem + buf * G::kBufCols + m * BN + (static_cast<uint32_t>(q * 32) << 16);
+                for (int cb = 0; cb < ntok; cb += 32) {
+                    float v[32];
+                    tmem_load32(tb + cb, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float send = is_up ? v[i] : v[16 + i];
+                        const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+                        const float gv = is_up ? recv : v[i];
+                        const float uv = is_up ? v[16 + i] : recv;
+                        const int col = cb + (is_up ? 16 + i : i);
+                        const float hv = swiglu_clip(gv, uv, L);
+                        if (col < ntok)
+                            out[(row0 + col) * ld + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(r.acce_leader + 8 * buf);
+        }
+    }
+    pair_teardown<G>(tmem);
+}
+
+// ------------------------------------------------------------------------------------
+// down on pairs: a pair tile covers 2 * MT * 128 output features.
+template <int MT>
+__device__ __forceinline__ void decode_down_pair(const DownArgs &a, int tile, int &g, int &row0, int &ntok, int &fb)
+{
+    const int nfb = a.H / (256 * MT);
+    const int ci = tile / nfb;
+    fb = tile - ci * nfb;
+    const int4 c = a.chunks[ci];
+    g = c.x;
+    row0 = c.y;
+    ntok = c.z;
+}
+
+template <int BN, int S, int MT, int NB>
+__global__ void __launch_bounds__(kThreads, 1)
+    down_pair_kernel(const __grid_constant__ CUtensorMap tm_wd, const __grid_constant__ CUtensorMap tm_wdsh,
+                     const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_hsh,
+                     const DownArgs a, const WaitCfg wc)
+{
+    using G = PairGeo<BN, S, MT, NB>;
+    extern __shared__ uint8_t smem_raw[];
+    PairRing r;
+    uint8_t *smem = pair_setup<G, S>(smem_raw, r);
+    const uint32_t tmem = *r.holder;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int ntot = a.hdr[1];
+    const int tiles = ntot * (a.H / (256 * MT));
+    const int first = blockIdx.x >> 1;
+    const int stride = gridDim.x >> 1;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_map(&tm_wd);
+            tma_prefetch_map(&tm_wdsh);
+            tma_prefetch_map(&tm_h);
+            tma_prefetch_map(&tm_hsh);
+            int it = 0;
+            bool stop = false;
+            for (int tile = first; tile < tiles && !stop; tile += stride) {
+                int g, row0, ntok, fb;
+                decode_down_pair<MT>(a, tile, g, row0, ntok, fb);
+                const bool sh = g == a.E;
+                const int nkb = (sh ? a.Is : a.I) / kBK;
+                const int half = ((ntok + 15) & ~15) >> 1;
+                const int nb = (half + 15) >> 4;
+                const uint32_t tx = 2 * (G::kABytes + nb * kBoxBytes);
+                const CUtensorMap *mw = sh ? &tm_wdsh : &tm_wd;
+                const CUtensorMap *mb = sh ? &tm_hsh : &tm_h;
+                const int wrow = (sh ? 0 : g * a.H) + (fb * 2 + static_cast<int>(r.rank)) * MT * 128;
+                const int brow = row0 + static_cast<int>(r.rank) * half;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % S;
+                    if (!mbar_wait(&r.empty[s], ((it / S) & 1) ^ 1, wc, r.abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    if (r.rank == 0)
+                        mbar_arrive_expect_tx(&r.full[s], tx);
+                    const uint32_t bar = r.full_leader + 8 * s;
+                    uint8_t *A = smem + s * G::kStageBytes;
+                    uint8_t *B = A + G::kABytes;
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        tma_load_2d_pair(A + m * kATileBytes, mw, bar, kb * kBK, wrow + m * 128);
+                    for (int i = 0; i < nb; ++i)
+                        tma_load_2d_pair(B + i * kBoxBytes, mb, bar, kb * kBK, brow + 16 * i);
+                }
+            }
+            pair_producer_drain<S>(r, it, wc);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            auto info = [&](int tile, int &ntok, int &nk) {
+                int g, row0, fb;
+                decode_down_pair<MT>(a, tile, g, row0, ntok, fb);
+                nk = (g == a.E ? a.Is : a.I) / kBK;
+            };
+            pair_mma_role<G, S, BN, MT, NB>(r, smem, tmem, first, tiles, stride, info, wc);
+        }
+    } else {
+        const int q = warp & 3;
+        const int64_t f = q * 32 + lane;
+        const int64_t H = a.H;
+        const int64_t shared_base = static_cast<int64_t>(a.T) * a.k;
+        int tc = 0;
+        for (int tile = first; tile < tiles; tile += stride, ++tc) {
+            int g, row0, ntok, fb;
+            decode_down_pair<MT>(a, tile, g, row0, ntok, fb);
+            const int buf = tc % NB;
+            if (!warp_wait(&r.accf[buf], (tc / NB) & 1, wc, r.abort_flag))
+                break;
+            tc_fence_after();
+            const bool sh = g == a.E;
+            const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
+            for (int cb = 0; cb < ntok; cb += 32) {
+                const int mycol = cb + lane;
+                int64_t dst_row = 0;
+                float wgt = 0.0f;
+                if (mycol < ntok) {
+                    const int64_t rr = row0 + mycol;
+                    if (a.deterministic)
+                        dst_row = sh ? shared_base + rr : rr;
+                    else
+                        dst_row = sh ? rr : a.perm_token[rr];
+                    wgt = sh ? 1.0f : a.w_perm[rr];
+                }
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    const int64_t feat = (wt0 + m) * 128 + f;
+                    float v[32];
+                    tmem_load32(tmem + buf * G::kBufCols + m * BN + (static_cast<uint32_t>(q * 32) << 16) + cb, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int64_t drow = __shfl_sync(0xFFFFFFFFu, dst_row, i);
+                        const float w = __shfl_sync(0xFFFFFFFFu, wgt, i);
+                        if (cb + i < ntok) {
+                            float *p = a.out + drow * H + feat;
+                            if (a.deterministic)
+                                *p = w * v[i];
+                            else
+                                atomicAdd(p, w * v[i]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(r.acce_leader + 8 * buf);
+        }
+    }
+    pair_teardown<G>(tmem);
+}
+
+template <class Kernel, class... Args>
+cudaError_t launch_pairs(Kernel kernel, int smem, int grid, cudaStream_t stream, Args... args)
+{
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess)
+        return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid & ~1, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (err != cudaSuccess)
+        return err;
+    return cudaGetLastError();
+}
+
+// Pair configuration: 128 token rows per pair tile (64 per CTA), two weight tiles per
+// CTA and stage (40 KB stages, 5 deep), two TMEM accumulator buffers.
+constexpr int kPairBN = 128, kPairStages = 5, kPairMT = 2, kPairNB = 2;
+
+}  // namespace
+
+cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
+                                const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
+                                cudaStream_t stream)
+{
+    using G = PairGeo<kPairBN, kPairStages, kPairMT, kPairNB>;
+    return launch_pairs(gate_up_pair_kernel<kPairBN, kPairStages, kPairMT, kPairNB>, static_cast<int>(G::kSmemBytes), grid,
+                        stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
+}
+
+cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
+                             const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
+                             cudaStream_t stream)
+{
+    using G = PairGeo<kPairBN, kPairStages, kPairMT, kPairNB>;
+    return launch_pairs(down_pair_kernel<kPairBN, kPairStages, kPairMT, kPairNB>, static_cast<int>(G::kSmemBytes), grid,
+                        stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
+}
+
+}  // namespace moe

@@ -32,21 +32,26 @@ cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t 
                           uint16_t *x_perm, float *w_perm, int num_sms, cudaStream_t stream);
 
 // Grouped-GEMM configuration: `cap` = token rows per chunk (the N side of one tile),
-// `mt` = 128-row weight tiles per pipeline stage. Decode-sized calls (at most 16 tokens
-// per expert on average) use 32-row chunks with one weight tile and a deep ring; larger
-// calls use 128-row chunks with two weight tiles per stage when I, Is and H split into
-// such tiles, else 256-row chunks with one.
+// `mt` = 128-row weight tiles per pipeline stage and CTA, `pair` = tiles run on CTA pairs
+// (cta_group::2). Decode-sized calls (at most 16 tokens per expert on average) use 32-row
+// chunks with one weight tile and a deep ring. Larger calls run on CTA pairs with
+// 128-row chunks when I and Is split into 256-feature and H into 512-feature pair tiles,
+// else on single CTAs with two weight tiles per stage (I, Is multiples of 128, H of 256),
+// else with one weight tile and 256-row chunks.
 struct GemmConfig {
     int cap;
     int mt;
+    int pair;
 };
 inline GemmConfig gemm_config(int64_t T, int64_t k, int64_t E, int64_t H, int64_t I, int64_t Is)
 {
     if (T * k <= 16 * E)
-        return {32, 1};
+        return {32, 1, 0};
+    if (I % 256 == 0 && Is % 256 == 0 && H % 512 == 0)
+        return {128, 2, 1};
     if (I % 128 == 0 && Is % 128 == 0 && H % 256 == 0)
-        return {128, 2};
-    return {256, 1};
+        return {128, 2, 0};
+    return {256, 1, 0};
 }
 
 // Splits every group (E routed experts, then the shared expert) into chunks of at most
@@ -82,6 +87,13 @@ struct DownArgs {
 cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
                         const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
                         const GemmConfig &c, cudaStream_t stream);
+
+cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
+                                const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
+                                cudaStream_t stream);
+cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
+                             const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
+                             cudaStream_t stream);
 
 cudaError_t launch_combine(const float *o_perm, const int32_t *slot_of, int T, int k, int H, float *y,
                            cudaStream_t stream);

@@ -89,13 +89,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
     }
 }
 
-// Drain wait used on the way out of a kernel: bounded, and it ignores the abort flag
-// (it waits for this role's own copies or MMAs that are already in flight).
+// Drain wait used on the way out of a kernel: it ignores the abort flag (it waits for
+// this role's own copies or MMAs that are already in flight) and is bounded by at least
+// 2 s whatever the wait limit, so a short limit never frees TMEM or shared memory under
+// operations that are still running.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, const WaitCfg &w)
 {
+    const unsigned long long limit = w.limit_ns > 2000000000ull ? w.limit_ns : 2000000000ull;
     const unsigned long long t0 = global_ns();
     while (!mbar_test(bar, parity)) {
-        if (global_ns() - t0 > w.limit_ns) {
+        if (global_ns() - t0 > limit) {
             atomicOr(w.err, kDevErrTimeout);
             return false;
         }
@@ -164,6 +167,79 @@ __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr)
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
     return v;
+}
+
+// Arrive on a barrier that may live in another CTA of the cluster (address from dsmem_addr).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+// TMA loads issued by either CTA of a pair into its own shared memory; the transaction
+// bytes complete on `bar_cluster`, the leader CTA's barrier (a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m, uint32_t bar_cluster, int32_t c0,
+                                                 int32_t c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d_pair(void *dst, const CUtensorMap *m, uint32_t bar_cluster, int32_t c0,
+                                                 int32_t c1, int32_t c2, int32_t c3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+// TMEM allocation shared by the pair: one warp of each CTA issues it (same warp, same
+// holder offset); both CTAs receive the same address.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *holder, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(holder)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Pair MMA (issued by the leader CTA only): D (+)= A · B^T with M = 256 rows, the first
+// 128 in the leader's shared memory / TMEM and the next 128 in the peer's; B's N rows are
+// split N/2 + N/2 between the two CTAs' shared memory at the same offset.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// When the pair MMAs issued so far are done, arrive once on the barrier at this shared
+// memory offset in every CTA of `cta_mask` (bit r = cluster rank r).
+__device__ __forceinline__ void umma_commit_pair_mc(uint64_t *bar, uint16_t cta_mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05

@@ -32,6 +32,11 @@ SMALL = {
     # two weight tiles per stage (I, Is multiples of 128, H of 256; > 16 tokens per expert)
     "mt2": LayerShape("mt2", T=300, H=512, E=12, k=4, I=256, Is=128, limit_routed=0.25, limit_shared=0.125,
                       seed=27, weight_std=0.03),
+    # CTA pairs (I, Is multiples of 256, H of 512)
+    "pair": LayerShape("pair", T=300, H=512, E=12, k=4, I=256, Is=256, limit_routed=0.25, limit_shared=0.125,
+                       seed=29, weight_std=0.03),
+    "pair_ragged": LayerShape("pair_ragged", T=173, H=1024, E=7, k=3, I=512, Is=256, limit_routed=0.0,
+                              limit_shared=0.0, seed=30, weight_std=0.03),
     # decode-sized: <= 16 tokens per expert on average
     "decode": LayerShape("decode", T=24, H=512, E=40, k=8, I=192, Is=128, limit_routed=0.25, seed=28,
                          weight_std=0.03),
