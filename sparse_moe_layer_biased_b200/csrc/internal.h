@@ -25,8 +25,20 @@ struct RouterArgs {
 cudaError_t launch_router(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const RouterArgs &a,
                           const WaitCfg &wc, cudaStream_t stream);
 
-cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int32_t *counts, int32_t *offsets,
-                           int32_t *perm_token, int32_t *slot_of, cudaStream_t stream);
+struct PermuteArgs {
+    const int32_t *idx;
+    int T, k, E;
+    int32_t *counts;      // [E + 1]
+    int32_t *offsets;     // [E + 2]
+    int32_t *perm_token;  // [T*k + T]
+    int32_t *slot_of;     // [T*k]
+    const float *topk_w;  // optional, with w_perm: the routing weight of each slot
+    float *w_perm;        // [T*k] or null
+    int4 *chunks;         // optional tile table of the grouped GEMMs (with hdr, cap)
+    int32_t *hdr;
+    int cap;
+};
+cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream);
 
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
                           uint16_t *x_perm, float *w_perm, int num_sms, cudaStream_t stream);

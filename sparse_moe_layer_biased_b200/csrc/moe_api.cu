@@ -312,8 +312,9 @@ moe_status_t moe_permute(const moe_layer_desc *desc, const int32_t *topk_idx, in
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK)
         return st;
-    return cuda_status(moe::launch_permute(topk_idx, desc->T, desc->k, desc->E, counts, offsets, perm_token, slot_of,
-                                           static_cast<cudaStream_t>(stream)));
+    const moe::PermuteArgs pa{topk_idx, desc->T, desc->k, desc->E, counts, offsets, perm_token, slot_of,
+                              nullptr, nullptr, nullptr, nullptr, 0};
+    return cuda_status(moe::launch_permute(pa, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_expert_ffn(const moe_layer_desc *desc, const uint16_t *x, const float *topk_w,
@@ -392,7 +393,9 @@ moe_status_t moe_forward(const moe_layer_desc *desc, const uint16_t *x, const ui
         return st;
     if (!stage_mark(1, s))
         return MOE_ERR_CUDA;
-    if (moe::launch_permute(idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, s) != cudaSuccess)
+    const moe::PermuteArgs pa{idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, nullptr, nullptr, nullptr,
+                              nullptr, 0};
+    if (moe::launch_permute(pa, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     float *out = d.deterministic ? at<float>(ws, L.o_perm) : y;
     if ((st = run_expert_ffn(d, di, x, w, offsets, perm_token, slot_of, W_gate_up, W_down, Wsh_gate_up, Wsh_down,

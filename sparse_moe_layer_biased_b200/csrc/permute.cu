@@ -12,30 +12,98 @@
 namespace moe {
 namespace {
 
-constexpr int kPermThreads = 1024;  // 32 warps; warp w owns a contiguous token range
+constexpr int kPermThreads = 1024;  // 32 warps per CTA; warp w owns a contiguous token range
 
-// Single CTA. Pass 1: per-warp per-expert counts, built 32 entries at a time with
-// __match_any_sync (one leader per distinct expert adds the group size). Pass 2: per
-// expert, exclusive prefix over warps; exclusive scan over experts. Pass 3: the same
-// walk again; an entry's slot = its warp's base for that expert + the number of earlier
-// lanes in its round with the same expert. Entries are visited in (token, rank) order,
-// so slots within an expert are in token order: the result is unique and deterministic.
+// Tile table of the grouped GEMMs, built by all threads of one CTA from the exclusive
+// scan `offs` (E + 1 entries in shared or global memory): group g in [0, E] (E = shared
+// expert, T rows) of n rows becomes ceil(n / cap) chunks of equal size rounded up to 16
+// rows (the last one shorter). hdr[0] = routed chunk count, hdr[1] = total.
+__device__ void build_chunk_table(const int32_t *offs, int E, int T, int cap, int4 *chunks, int32_t *hdr)
+{
+    __shared__ int warp_sums[32];
+    for (int g0 = 0; g0 <= E; g0 += kPermThreads) {
+        // E <= 512 < kPermThreads: a single pass
+        const int g = g0 + static_cast<int>(threadIdx.x);
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        int n = 0, base = 0;
+        if (g < E) {
+            base = offs[g];
+            n = offs[g + 1] - base;
+        } else if (g == E) {
+            n = T;
+        }
+        const int nch = n > 0 ? (n + cap - 1) / cap : 0;
+        const int csz = nch > 0 ? ((n + nch - 1) / nch + 15) / 16 * 16 : 0;
+        int incl = nch;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o)
+                incl += v;
+        }
+        if (lane == 31)
+            warp_sums[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int ws = warp_sums[lane];
+            int wi = ws;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+                if (lane >= o)
+                    wi += v;
+            }
+            warp_sums[lane] = wi - ws;
+        }
+        __syncthreads();
+        const int start = warp_sums[warp] + incl - nch;
+        for (int c = 0; c < nch; ++c) {
+            const int r = c * csz;
+            const int len = n - r < csz ? n - r : csz;
+            chunks[start + c] = make_int4(g, base + r, len, 0);
+        }
+        if (g == E) {
+            hdr[0] = start;
+            hdr[1] = start + nch;
+        }
+        __syncthreads();
+    }
+}
+
+// One thread-block cluster of NC CTAs (one CTA for small calls). CTA c owns a contiguous
+// range of tokens; its warp w owns a contiguous sub-range.
+// Pass 1: per-warp per-expert counts, built 32 entries at a time with __match_any_sync
+// (one leader per distinct expert adds the group size).
+// Scan: per expert, exclusive prefix over the warps of the CTA; the CTA totals meet
+// through distributed shared memory, giving each CTA its base per expert and every CTA
+// the global counts and their exclusive scan over experts.
+// Pass 3: the same walk again; an entry's slot = offsets[e] + its CTA's base + its
+// warp's base + the number of earlier lanes in its round with the same expert. Entries
+// are visited in (token, rank) order, so slots within an expert are in token order: the
+// result is unique and deterministic. Optionally also the per-slot routing weight and
+// the grouped-GEMM tile table.
 __global__ void __launch_bounds__(kPermThreads)
-    permute_kernel(const int32_t *__restrict__ idx, int T, int k, int E, int32_t *__restrict__ counts,
-                   int32_t *__restrict__ offsets, int32_t *__restrict__ perm_token, int32_t *__restrict__ slot_of)
+    permute_kernel(const PermuteArgs a)
 {
     extern __shared__ int32_t sm[];
-    int32_t *cnt = sm;           // [32][E]
-    int32_t *tot = sm + 32 * E;  // [E]
+    const int E = a.E, T = a.T, k = a.k;
+    int32_t *cnt = sm;            // [32][E]
+    int32_t *ctot = cnt + 32 * E; // [E] this CTA's totals (read by peers)
+    int32_t *cbase = ctot + E;    // [E] sum of lower CTAs' totals
+    int32_t *offs = cbase + E;    // [E + 1] exclusive scan of the global counts
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int nc = static_cast<int>(gridDim.x);
+
     for (int i = threadIdx.x; i < 32 * E; i += kPermThreads)
         cnt[i] = 0;
     __syncthreads();
 
-    const int per_warp = (T + 31) / 32;
-    const int64_t t_begin = static_cast<int64_t>(warp) * per_warp < T ? static_cast<int64_t>(warp) * per_warp : T;
-    const int64_t t_end = t_begin + per_warp < T ? t_begin + per_warp : T;
+    const int per_cta = (T + nc - 1) / nc;
+    const int c0 = static_cast<int>(rank) * per_cta < T ? static_cast<int>(rank) * per_cta : T;
+    const int c1 = c0 + per_cta < T ? c0 + per_cta : T;
+    const int per_warp = (c1 - c0 + 31) / 32;
+    const int64_t t_begin = c0 + warp * per_warp < c1 ? c0 + warp * per_warp : c1;
+    const int64_t t_end = t_begin + per_warp < c1 ? t_begin + per_warp : c1;
     const int64_t begin = t_begin * k, end = t_end * k;
     int32_t *mine = cnt + warp * E;
 
@@ -44,7 +112,7 @@ __global__ void __launch_bounds__(kPermThreads)
         const bool valid = n < end;
         int e = E + lane;  // distinct sentinel for idle lanes
         if (valid) {
-            e = idx[n];
+            e = a.idx[n];
             e = e < 0 ? 0 : (e > E - 1 ? E - 1 : e);
         }
         const unsigned m = __match_any_sync(0xFFFFFFFFu, e);
@@ -61,7 +129,21 @@ __global__ void __launch_bounds__(kPermThreads)
             cnt[w * E + e] = run;
             run += c;
         }
-        tot[e] = run;
+        ctot[e] = run;
+    }
+    cluster_sync_all();  // every CTA's totals are visible to its peers
+
+    for (int e = threadIdx.x; e < E; e += kPermThreads) {
+        int below = 0, all = 0;
+        const uint32_t local = smem_u32(ctot + e);
+        for (int c = 0; c < nc; ++c) {
+            const int v = c == static_cast<int>(rank) ? ctot[e] : dsmem_ld_s32(dsmem_addr(local, c));
+            if (c < static_cast<int>(rank))
+                below += v;
+            all += v;
+        }
+        cbase[e] = below;
+        offs[e] = all;  // global count, scanned below
     }
     __syncthreads();
 
@@ -71,7 +153,7 @@ __global__ void __launch_bounds__(kPermThreads)
         const int hi = lo + per < E ? lo + per : E;
         int s = 0;
         for (int e = lo; e < hi; ++e)
-            s += tot[e];
+            s += offs[e];
         int incl = s;
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
@@ -80,21 +162,28 @@ __global__ void __launch_bounds__(kPermThreads)
         }
         int run = incl - s;
         for (int e = lo; e < hi; ++e) {
-            const int c = tot[e];
-            counts[e] = c;
-            offsets[e] = run;
-            tot[e] = run;
+            const int c = offs[e];
+            if (rank == 0) {
+                a.counts[e] = c;
+                a.offsets[e] = run;
+            }
+            offs[e] = run;
             run += c;
         }
         if (lane == 31) {
-            counts[E] = T;
-            offsets[E] = incl;
-            offsets[E + 1] = incl + T;
+            offs[E] = incl;
+            if (rank == 0) {
+                a.counts[E] = T;
+                a.offsets[E] = incl;
+                a.offsets[E + 1] = incl + T;
+            }
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < 32 * E; i += kPermThreads)
-        cnt[i] += tot[i % E];
+    for (int i = threadIdx.x; i < 32 * E; i += kPermThreads) {
+        const int e = i % E;
+        cnt[i] += offs[e] + cbase[e];
+    }
     __syncthreads();
 
     for (int64_t b = begin; b < end; b += 32) {
@@ -102,14 +191,16 @@ __global__ void __launch_bounds__(kPermThreads)
         const bool valid = n < end;
         int e = E + lane;
         if (valid) {
-            e = idx[n];
+            e = a.idx[n];
             e = e < 0 ? 0 : (e > E - 1 ? E - 1 : e);
         }
         const unsigned m = __match_any_sync(0xFFFFFFFFu, e);
         if (valid) {
             const int slot = mine[e] + __popc(m & ((1u << lane) - 1u));
-            slot_of[n] = slot;
-            perm_token[slot] = static_cast<int32_t>(n / k);
+            a.slot_of[n] = slot;
+            a.perm_token[slot] = static_cast<int32_t>(n / k);
+            if (a.w_perm)
+                a.w_perm[slot] = a.topk_w[n];
         }
         __syncwarp();
         if (valid && lane == 31 - __clz(m))
@@ -117,8 +208,12 @@ __global__ void __launch_bounds__(kPermThreads)
         __syncwarp();
     }
     const int64_t shared_base = static_cast<int64_t>(T) * k;
-    for (int t = threadIdx.x; t < T; t += kPermThreads)
-        perm_token[shared_base + t] = t;
+    for (int t = c0 + threadIdx.x; t < c1; t += kPermThreads)
+        a.perm_token[shared_base + t] = t;
+    if (rank == 0 && a.chunks)
+        build_chunk_table(offs, E, T, a.cap, a.chunks, a.hdr);
+
+    cluster_sync_all();  // no CTA leaves while a peer may still read its totals
 }
 
 // One warp per (token, rank) entry: copies the token's row of x into its slot and
@@ -144,54 +239,12 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// One thread per group g in [0, E] (E = shared expert). A group of n rows becomes
-// ceil(n / cap) chunks of equal size rounded up to 16 rows (the last one shorter).
-__global__ void __launch_bounds__(1024)
+// Tile table from an offsets array in global memory (the moe_expert_ffn entry point).
+__global__ void __launch_bounds__(kPermThreads)
     chunks_kernel(const int32_t *__restrict__ offsets, int E, int T, int cap, int4 *__restrict__ chunks,
                   int32_t *__restrict__ hdr)
 {
-    __shared__ int warp_sums[32];
-    const int g = threadIdx.x;
-    const int lane = g & 31, warp = g >> 5;
-    int n = 0, base = 0;
-    if (g < E) {
-        base = offsets[g];
-        n = offsets[g + 1] - base;
-    } else if (g == E) {
-        n = T;
-    }
-    const int nch = n > 0 ? (n + cap - 1) / cap : 0;
-    const int csz = nch > 0 ? ((n + nch - 1) / nch + 15) / 16 * 16 : 0;
-    int incl = nch;
-    for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o)
-            incl += v;
-    }
-    if (lane == 31)
-        warp_sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int ws = warp_sums[lane];
-        int wi = ws;
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xFFFFFFFFu, wi, o);
-            if (lane >= o)
-                wi += v;
-        }
-        warp_sums[lane] = wi - ws;
-    }
-    __syncthreads();
-    const int start = warp_sums[warp] + incl - nch;
-    for (int c = 0; c < nch; ++c) {
-        const int r = c * csz;
-        const int len = n - r < csz ? n - r : csz;
-        chunks[start + c] = make_int4(g, base + r, len, 0);
-    }
-    if (g == E) {
-        hdr[0] = start;
-        hdr[1] = start + nch;
-    }
+    build_chunk_table(offsets, E, T, cap, chunks, hdr);
 }
 
 // y[t] = sum_{j<k} o_perm[slot_of[t, j]] + o_perm[T*k + t], in that order.
@@ -221,14 +274,31 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, int32_t *counts, int32_t *offsets,
-                           int32_t *perm_token, int32_t *slot_of, cudaStream_t stream)
+cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream)
 {
-    const int smem = (32 * E + E) * 4;
+    const int smem = (32 * a.E + 3 * a.E + 1) * 4;
     cudaError_t err = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
-    permute_kernel<<<1, kPermThreads, smem, stream>>>(idx, T, k, E, counts, offsets, perm_token, slot_of);
+    // one CTA per 8192 (token, expert) entries, at most one portable cluster of 8
+    const int64_t entries = static_cast<int64_t>(a.T) * a.k;
+    int nc = static_cast<int>((entries + 8191) / 8192);
+    nc = nc < 1 ? 1 : (nc > 8 ? 8 : nc);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nc, 1, 1);
+    cfg.blockDim = dim3(kPermThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nc;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, permute_kernel, a);
+    if (err != cudaSuccess)
+        return err;
     return cudaGetLastError();
 }
 
@@ -247,7 +317,7 @@ cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t 
 cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr,
                           cudaStream_t stream)
 {
-    chunks_kernel<<<1, 1024, 0, stream>>>(offsets, E, T, cap, chunks, hdr);
+    chunks_kernel<<<1, kPermThreads, 0, stream>>>(offsets, E, T, cap, chunks, hdr);
     return cudaGetLastError();
 }
 

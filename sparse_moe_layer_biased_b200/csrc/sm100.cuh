@@ -162,6 +162,13 @@ __device__ __forceinline__ uint64_t dsmem_ld_u64(uint32_t addr)
     return v;
 }
 
+__device__ __forceinline__ int32_t dsmem_ld_s32(uint32_t addr)
+{
+    int32_t v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr)
 {
     float v;
