@@ -15,7 +15,8 @@
 // from L2 per weight byte (the token tile is reused by two MMAs per K step).
 //
 // Roles per CTA (persistent, one CTA per SM, static round-robin over tiles):
-//   warp 0      TMA producer: MT weight tiles + token rows (16-row boxes) per 64-wide K slice
+//   warp 0      TMA producer: per 64-wide K slice, one box with the MT weight tiles and
+//               one box of BN token rows
 //   warp 1      MMA issuer (one thread) and TMEM owner; 2 buffers x MT accumulators x BN
 //               fp32 columns, so the epilogue of one tile overlaps the mainloop of the next
 //   warps 2..5  epilogue: TMEM -> registers -> activation / weighting -> global
@@ -30,7 +31,6 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kBK = 64;
 constexpr uint32_t kATileBytes = 128 * 128;  // 128 weight rows x 64 bf16
-constexpr uint32_t kBoxBytes = 16 * 128;     // one 16-row token box
 
 // Ring geometry: token chunks of at most BN rows, S stages, MT weight tiles per stage.
 template <int BN, int S, int MT>
@@ -193,8 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int g, row0, ntok, fb;
                 decode_gate_up<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
                 const bool sh = g == a.E;
-                const int nb = (ntok + 15) >> 4;
-                const uint32_t tx = G::kABytes + nb * kBoxBytes;
                 const CUtensorMap *mw = sh ? &tm_wsh : &tm_w;
                 const CUtensorMap *mb = sh ? &tm_x : &tm_xp;
                 const int ge = sh ? 0 : g;
@@ -204,14 +202,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         stop = true;
                         break;
                     }
-                    mbar_arrive_expect_tx(&r.full[s], tx);
+                    // one box with the MT weight tiles, one box of BN token rows (rows past
+                    // the chunk are loaded and ignored)
+                    mbar_arrive_expect_tx(&r.full[s], G::kStageBytes);
                     uint8_t *A = smem + s * G::kStageBytes;
-                    uint8_t *B = A + G::kABytes;
-#pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        tma_load_4d(A + m * kATileBytes, mw, &r.full[s], kb * kBK, 0, (fb * MT + m) * 64, ge);
-                    for (int i = 0; i < nb; ++i)
-                        tma_load_2d(B + i * kBoxBytes, mb, &r.full[s], kb * kBK, row0 + 16 * i);
+                    tma_load_4d(A, mw, &r.full[s], kb * kBK, 0, fb * MT * 64, ge);
+                    tma_load_2d(A + G::kABytes, mb, &r.full[s], kb * kBK, row0);
                 }
             }
             producer_drain<S>(r, it, wc);
@@ -327,8 +323,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_down<MT>(a, tile, g, row0, ntok, fb);
                 const bool sh = g == a.E;
                 const int nkb = (sh ? a.Is : a.I) / kBK;
-                const int nb = (ntok + 15) >> 4;
-                const uint32_t tx = G::kABytes + nb * kBoxBytes;
                 const CUtensorMap *mw = sh ? &tm_wdsh : &tm_wd;
                 const CUtensorMap *mb = sh ? &tm_hsh : &tm_h;
                 const int wrow = (sh ? 0 : g * a.H) + fb * MT * 128;
@@ -338,14 +332,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         stop = true;
                         break;
                     }
-                    mbar_arrive_expect_tx(&r.full[s], tx);
+                    mbar_arrive_expect_tx(&r.full[s], G::kStageBytes);
                     uint8_t *A = smem + s * G::kStageBytes;
-                    uint8_t *B = A + G::kABytes;
-#pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        tma_load_2d(A + m * kATileBytes, mw, &r.full[s], kb * kBK, wrow + m * 128);
-                    for (int i = 0; i < nb; ++i)
-                        tma_load_2d(B + i * kBoxBytes, mb, &r.full[s], kb * kBK, row0 + 16 * i);
+                    tma_load_2d(A, mw, &r.full[s], kb * kBK, wrow);
+                    tma_load_2d(A + G::kABytes, mb, &r.full[s], kb * kBK, row0);
                 }
             }
             producer_drain<S>(r, it, wc);

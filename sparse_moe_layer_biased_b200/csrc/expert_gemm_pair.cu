@@ -28,7 +28,6 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kBK = 64;
 constexpr uint32_t kATileBytes = 128 * 128;  // 128 weight rows x 64 bf16
-constexpr uint32_t kBoxBytes = 16 * 128;     // one 16-row token box
 
 // BN = token rows per pair tile (N of the pair MMA); each CTA holds BN/2 of them.
 // NB = accumulator buffers in TMEM (2: the epilogue of one tile overlaps the next tile's
@@ -227,9 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int g, row0, ntok, fb;
                 decode_gate_up_pair<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
                 const bool sh = g == a.E;
-                const int half = ((ntok + 15) & ~15) >> 1;  // token rows held by each CTA
-                const int nb = (half + 15) >> 4;
-                const uint32_t tx = 2 * (G::kABytes + nb * kBoxBytes);
+                const int half = ((ntok + 15) & ~15) >> 1;  // token rows used from each CTA
                 const CUtensorMap *mw = sh ? &tm_wsh : &tm_w;
                 const CUtensorMap *mb = sh ? &tm_x : &tm_xp;
                 const int ge = sh ? 0 : g;
@@ -242,15 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (r.rank == 0)
-                        mbar_arrive_expect_tx(&r.full[s], tx);
+                        mbar_arrive_expect_tx(&r.full[s], 2 * G::kStageBytes);
                     const uint32_t bar = r.full_leader + 8 * s;
                     uint8_t *A = smem + s * G::kStageBytes;
-                    uint8_t *B = A + G::kABytes;
-#pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        tma_load_4d_pair(A + m * kATileBytes, mw, bar, kb * kBK, 0, (wt0 + m) * 64, ge);
-                    for (int i = 0; i < nb; ++i)
-                        tma_load_2d_pair(B + i * kBoxBytes, mb, bar, kb * kBK, brow + 16 * i);
+                    // one box with this CTA's MT weight tiles, one box of BN/2 token rows
+                    // starting at its half (rows past it are loaded and ignored)
+                    tma_load_4d_pair(A, mw, bar, kb * kBK, 0, wt0 * 64, ge);
+                    tma_load_2d_pair(A + G::kABytes, mb, bar, kb * kBK, brow);
                 }
             }
             pair_producer_drain<S>(r, it, wc);
@@ -358,8 +353,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool sh = g == a.E;
                 const int nkb = (sh ? a.Is : a.I) / kBK;
                 const int half = ((ntok + 15) & ~15) >> 1;
-                const int nb = (half + 15) >> 4;
-                const uint32_t tx = 2 * (G::kABytes + nb * kBoxBytes);
                 const CUtensorMap *mw = sh ? &tm_wdsh : &tm_wd;
                 const CUtensorMap *mb = sh ? &tm_hsh : &tm_h;
                 const int wrow = (sh ? 0 : g * a.H) + (fb * 2 + static_cast<int>(r.rank)) * MT * 128;
@@ -371,15 +364,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (r.rank == 0)
-                        mbar_arrive_expect_tx(&r.full[s], tx);
+                        mbar_arrive_expect_tx(&r.full[s], 2 * G::kStageBytes);
                     const uint32_t bar = r.full_leader + 8 * s;
                     uint8_t *A = smem + s * G::kStageBytes;
-                    uint8_t *B = A + G::kABytes;
-#pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        tma_load_2d_pair(A + m * kATileBytes, mw, bar, kb * kBK, wrow + m * 128);
-                    for (int i = 0; i < nb; ++i)
-                        tma_load_2d_pair(B + i * kBoxBytes, mb, bar, kb * kBK, brow + 16 * i);
+                    tma_load_2d_pair(A, mw, bar, kb * kBK, wrow);
+                    tma_load_2d_pair(A + G::kABytes, mb, bar, kb * kBK, brow);
                 }
             }
             pair_producer_drain<S>(r, it, wc);

@@ -102,14 +102,14 @@ bool map_rows(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, uint
 }
 
 // Stacked gate_up weights [G, 2*Iw, H] viewed as (H, half, row, group) so one box of
-// (64, 2, 64, 1) lands as 128 rows alternating gate row i / up row i.
-bool map_gate_up(CUtensorMap *m, const void *base, int64_t H, int64_t Iw, int64_t G)
+// (64, 2, feats, 1) lands as 2 * feats rows alternating gate row i / up row i.
+bool map_gate_up(CUtensorMap *m, const void *base, int64_t H, int64_t Iw, int64_t G, uint32_t feats)
 {
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(H), 2, static_cast<cuuint64_t>(Iw),
                                 static_cast<cuuint64_t>(G)};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(Iw * H * 2), static_cast<cuuint64_t>(H * 2),
                                    static_cast<cuuint64_t>(2 * Iw * H * 2)};
-    const cuuint32_t box[4] = {64, 2, 64, 1};
+    const cuuint32_t box[4] = {64, 2, feats, 1};
     return encode_bf16(m, base, 4, dims, strides, box);
 }
 
@@ -191,7 +191,8 @@ moe_status_t run_router(const moe_layer_desc &d, const DeviceInfo &di, const uin
                         const float *bias, int32_t *idx, float *w, float *margin, cudaStream_t s)
 {
     CUtensorMap tm_x, tm_wr;
-    if (!map_rows(&tm_x, x, d.H, d.T, 128) || !map_rows(&tm_wr, Wr, d.H, d.E, 16))
+    const moe::RouterSplit sp = moe::router_split(d.E, d.T, di.num_sms);
+    if (!map_rows(&tm_x, x, d.H, d.T, 128) || !map_rows(&tm_wr, Wr, d.H, d.E, sp.box_rows))
         return MOE_ERR_CUDA;
     moe::RouterArgs a{bias, idx, w, margin, d.T, d.H, d.E, d.k, d.scale, d.norm_expert_weight, di.num_sms};
     return cuda_status(moe::launch_router(tm_x, tm_wr, a, wait_cfg(di), s));
@@ -211,18 +212,24 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     int32_t *hdr = at<int32_t>(ws, L.hdr);
     const int64_t Tk = static_cast<int64_t>(d.T) * d.k;
 
+    // One TMA box per operand and pipeline stage: all weight tiles of a stage (64 * mt
+    // gate/up feature pairs, or 128 * mt down rows) and the stage's token rows (the chunk
+    // cap, halved on CTA pairs).
+    const moe::GemmConfig cfg = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
+    const uint32_t brows = static_cast<uint32_t>(cfg.pair ? cfg.cap / 2 : cfg.cap);
+    const uint32_t feats = static_cast<uint32_t>(64 * cfg.mt);
+    const uint32_t drows = static_cast<uint32_t>(128 * cfg.mt);
     CUtensorMap tm_w, tm_wsh, tm_xp, tm_x, tm_wd, tm_wdsh, tm_h, tm_hsh;
-    bool ok = map_gate_up(&tm_w, Wgu, d.H, d.I, d.E) && map_gate_up(&tm_wsh, Wsh_gu, d.H, d.Is, 1) &&
-              map_rows(&tm_xp, x_perm, d.H, Tk, 16) && map_rows(&tm_x, x, d.H, d.T, 16) &&
-              map_rows(&tm_wd, Wd, d.I, static_cast<int64_t>(d.E) * d.H, 128) &&
-              map_rows(&tm_wdsh, Wsh_d, d.Is, d.H, 128) && map_rows(&tm_h, h, d.I, Tk, 16) &&
-              map_rows(&tm_hsh, h_sh, d.Is, d.T, 16);
+    bool ok = map_gate_up(&tm_w, Wgu, d.H, d.I, d.E, feats) && map_gate_up(&tm_wsh, Wsh_gu, d.H, d.Is, 1, feats) &&
+              map_rows(&tm_xp, x_perm, d.H, Tk, brows) && map_rows(&tm_x, x, d.H, d.T, brows) &&
+              map_rows(&tm_wd, Wd, d.I, static_cast<int64_t>(d.E) * d.H, drows) &&
+              map_rows(&tm_wdsh, Wsh_d, d.Is, d.H, drows) && map_rows(&tm_h, h, d.I, Tk, brows) &&
+              map_rows(&tm_hsh, h_sh, d.Is, d.T, brows);
     if (!ok)
         return MOE_ERR_CUDA;
 
     if (!stage_mark(2, s))
         return MOE_ERR_CUDA;
-    const moe::GemmConfig cfg = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
     cudaError_t e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, s);
     if (e == cudaSuccess)
         e = moe::launch_chunks(offsets, d.E, d.T, cfg.cap, chunks, hdr, s);

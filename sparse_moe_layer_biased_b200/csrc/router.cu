@@ -24,26 +24,7 @@ constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5
 constexpr int kTileM = 128;
 constexpr int kBK = 64;                         // bf16 elements per 128-byte swizzled row
 constexpr uint32_t kABytes = kTileM * kBK * 2;  // 16 KB
-constexpr int kBRows = 16;                      // rows per Wr TMA box
 constexpr int kMaxStages = 8;
-
-struct Split {
-    int sl;  // experts per CTA (multiple of 16, at most 512)
-    int ns;  // CTAs per cluster
-};
-
-// Enough CTAs to cover the SMs once: with few token tiles (decode) the experts are split
-// over up to 8 CTAs; with many token tiles each CTA keeps all experts, so x is read once.
-inline Split make_split(int E, int T, int num_sms)
-{
-    const int tiles = (T + kTileM - 1) / kTileM;
-    const int e_pad = (E + 15) / 16 * 16;
-    int ns = num_sms / tiles;
-    ns = ns < 1 ? 1 : (ns > 8 ? 8 : ns);
-    ns = ns > e_pad / 16 ? e_pad / 16 : ns;
-    const int sl = ((e_pad + ns - 1) / ns + 15) / 16 * 16;
-    return Split{sl, (E + sl - 1) / sl};
-}
 
 template <int KMAX>
 struct Layout {
@@ -164,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *holder;
+    const int box = sl <= 256 ? sl : sl / 2;  // Wr rows per TMA box (one or two per stage)
 
     // registers of the epilogue thread's list (kept across the cluster barrier in CTA 0)
     uint64_t keys[KMAX + 1];
@@ -191,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t *A = smem + s * L.stage_bytes;
                 uint8_t *B = A + kABytes;
                 tma_load_2d(A, &tm_x, &full[s], kb * kBK, m0);
-                for (int r = 0; r < sl; r += kBRows)
+                for (int r = 0; r < sl; r += box)
                     tma_load_2d(B + r * 128, &tm_wr, &full[s], kb * kBK, e0 + r);
                 ++issued;
             }
@@ -331,7 +313,7 @@ template <int KMAX>
 cudaError_t launch_impl(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const RouterArgs &a,
                         const WaitCfg &wc, cudaStream_t stream)
 {
-    const Split sp = make_split(a.E, a.T, a.num_sms);
+    const RouterSplit sp = router_split(a.E, a.T, a.num_sms);
     const Layout<KMAX> L(sp.sl);
     const int smem = static_cast<int>(L.total) + 1024;
     cudaError_t err = cudaFuncSetAttribute(router_kernel<KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -356,6 +338,26 @@ cudaError_t launch_impl(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const
 }
 
 }  // namespace
+
+// Enough CTAs to cover the SMs once: with few token tiles (decode) the experts are split
+// over up to 8 CTAs; with many token tiles each CTA keeps all experts, so x is read once.
+// Slices above 256 experts are a multiple of 32, loaded as two Wr boxes of sl / 2 rows.
+RouterSplit router_split(int E, int T, int num_sms)
+{
+    const int tiles = (T + kTileM - 1) / kTileM;
+    const int e_pad = (E + 15) / 16 * 16;
+    int ns = num_sms / tiles;
+    ns = ns < 1 ? 1 : (ns > 8 ? 8 : ns);
+    ns = ns > e_pad / 16 ? e_pad / 16 : ns;
+    int sl = ((e_pad + ns - 1) / ns + 15) / 16 * 16;
+    if (sl > 256)
+        sl = (sl + 31) / 32 * 32;
+    RouterSplit r;
+    r.sl = sl;
+    r.ns = (E + sl - 1) / sl;
+    r.box_rows = sl <= 256 ? sl : sl / 2;
+    return r;
+}
 
 cudaError_t launch_router(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const RouterArgs &a,
                           const WaitCfg &wc, cudaStream_t stream)
