@@ -43,6 +43,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--deterministic", action="store_true")
+    ap.add_argument("--routing", default="router", choices=["router", "balanced"],
+                    help="router: full layer; balanced: fixed round-robin routing through moe_forward_with_ids "
+                         "(fake balanced static expert routing)")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling runs)")
     return ap.parse_args()
@@ -254,11 +257,28 @@ def run_b200(args, shape):
     x = inp["x"]
     y = torch.empty((shape.T, shape.H), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
+    if args.routing == "balanced":
+        t = torch.arange(shape.T, device="cuda")[:, None]
+        j = torch.arange(shape.k, device="cuda")[None, :]
+        fixed_idx = ((t * shape.k + j) % shape.E).to(torch.int32).contiguous()
+        fixed_w = torch.full((shape.T, shape.k), shape.scale / shape.k, dtype=torch.float32, device="cuda")
+        bdesc = _abi.desc_of(shape, deterministic=args.deterministic)
+
+        def step(xx, yy):
+            _abi.moe_forward_with_ids(bdesc, xx, fixed_idx, fixed_w, inp["W_gate_up"], inp["W_down"],
+                                      inp["Wsh_gate_up"], inp["Wsh_down"], yy, layer.ws)
+    else:
+        def step(xx, yy):
+            layer.forward(xx, y=yy)
 
     # warm-up (also yields the routing used for the algorithmic byte count)
-    _, idx, _ = layer.forward(x, y=y, routing=True)
+    if args.routing == "balanced":
+        idx = fixed_idx
+        step(x, y)
+    else:
+        _, idx, _ = layer.forward(x, y=y, routing=True)
     for _ in range(max(0, args.warmup - 1)):
-        layer.forward(x, y=y)
+        step(x, y)
     torch.cuda.synchronize()
     _abi.moe_check_device()
     counts = np.bincount(idx.cpu().numpy().ravel(), minlength=shape.E)
@@ -275,7 +295,7 @@ def run_b200(args, shape):
     start.record(stream)
     for i in range(args.steps):
         _abi.moe_set_stage_events(evs[i])
-        layer.forward(x, y=y)
+        step(x, y)
     end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -295,7 +315,7 @@ def run_b200(args, shape):
         x_d = torch.empty_like(x)
         for _ in range(2):
             x_d.copy_(x_h, non_blocking=True)
-            layer.forward(x_d, y=y)
+            step(x_d, y)
             y_h.copy_(y, non_blocking=True)
         torch.cuda.synchronize()
         barrier()
@@ -303,7 +323,7 @@ def run_b200(args, shape):
         s2.record(stream)
         for _ in range(args.steps):
             x_d.copy_(x_h, non_blocking=True)
-            layer.forward(x_d, y=y)
+            step(x_d, y)
             y_h.copy_(y, non_blocking=True)
         e2.record(stream)
         torch.cuda.synchronize()
@@ -328,6 +348,7 @@ def run_b200(args, shape):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded draw on device; random-init weights)",
         "config": workload_config(shape, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                                           "l2": "inputs larger than L2 (expert weights streamed every step)",
+                                          "routing": args.routing,
                                           "deterministic": bool(args.deterministic)}),
         "roofline": roofline,
         "tensor": {"achieved_tflops": flops / (step_ms / 1e3) / 1e12,
@@ -335,7 +356,7 @@ def run_b200(args, shape):
         "stages_ms": stage_ms,
         "clocks": clocks,
         "e2e": e2e,
-        "gpu_launches": (nstage) * args.steps,
+        "gpu_launches": (nstage - (1 if args.routing == "balanced" else 0)) * args.steps,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, n, dt, threads = cpu_oracle_sample(shape, inp, target_s=15.0)

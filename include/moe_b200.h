@@ -141,6 +141,20 @@ MOE_API moe_status_t moe_forward(const moe_layer_desc *desc, const uint16_t *x, 
                          int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
                          void *stream);
 
+/* The layer with the routing supplied by the caller instead of computed: rollout routing
+ * replay, where a trainer replays the expert choices its rollout engine made (miles
+ * Step-5-Preview recipe page, sections 5.2 "--use-rollout-routing-replay" and 5.4, which
+ * needs the engine's materialised top-k ids), and the fake balanced static expert routing
+ * of the NeMo AutoModel Step-5-Preview benchmark setup. moe_permute -> moe_expert_ffn
+ * (-> moe_combine when deterministic).
+ *   topk_idx [T, k] int32 (ids outside [0, E-1] are clamped; an id may repeat within a token,
+ *   each slot then adds its own weighted copy), topk_w [T, k] fp32 routing weights, used as
+ *   given (no normalisation or scaling). Other arguments as in moe_forward. */
+MOE_API moe_status_t moe_forward_with_ids(const moe_layer_desc *desc, const uint16_t *x, const int32_t *topk_idx,
+                                  const float *topk_w, const uint16_t *W_gate_up, const uint16_t *W_down,
+                                  const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y, void *ws,
+                                  size_t ws_bytes, void *stream);
+
 /* moe_forward without a caller-provided workspace. The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory at call time, such
  * as a serving runtime whose device memory is already handed to a fixed pool, a

@@ -42,6 +42,11 @@ def lib():
                                             ctypes.POINTER(_vp), ctypes.POINTER(_vp), _u16p, _u16p, _f64p,
                                             _i32p, _f64p, _f32p]
         L.oracle_forward_tokens.restype = ctypes.c_int
+        L.oracle_forward_given_routing.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                                   _u16p, _i32p, _f32p, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                                   _u16p, _u16p, _f64p]
+        L.oracle_forward_given_routing.restype = ctypes.c_int
         L.oracle_forward_dense.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                            ctypes.c_float, ctypes.c_float, _u16p, _u16p, _f32p, _u16p,
@@ -163,6 +168,39 @@ def forward_tokens(x_rows, Wr, bias, experts, Wsh_gu, Wsh_d, *, k, scale=3.0, no
     return {"y": y, "idx": idx, "w": w, "margin": margin}
 
 
+def forward_given_routing(x_rows, idx, w, experts, Wsh_gu, Wsh_d, *, E, limit_routed=0.0, limit_shared=0.0):
+    """Layer output for caller-supplied routing (ids [n, k] int32, weights [n, k] fp32).
+
+    experts: mapping expert id -> (W_gate_up[e], W_down[e]) holding every id used.
+    """
+    x_rows = _u16(x_rows)
+    idx = np.ascontiguousarray(idx, np.int32)
+    w = np.ascontiguousarray(w, np.float32)
+    n, H = x_rows.shape
+    k = idx.shape[1]
+    keep = {}
+    gu_ptrs = (_vp * E)()
+    d_ptrs = (_vp * E)()
+    I = None
+    for e, (gu, d) in experts.items():
+        gu, d = _u16(gu), _u16(d)
+        keep[e] = (gu, d)
+        gu_ptrs[e] = gu.ctypes.data
+        d_ptrs[e] = d.ctypes.data
+        I = gu.shape[0] // 2
+    Wsh_gu, Wsh_d = _u16(Wsh_gu), _u16(Wsh_d)
+    Is = Wsh_gu.shape[0] // 2
+    if I is None:
+        I = Is
+    y = np.empty((n, H), np.float64)
+    rc = lib().oracle_forward_given_routing(n, H, E, k, I, Is, limit_routed, limit_shared, x_rows, idx, w,
+                                            gu_ptrs, d_ptrs, Wsh_gu, Wsh_d, y)
+    del keep
+    if rc != 0:
+        raise ValueError("a used expert's weights were not supplied")
+    return y
+
+
 def forward_dense(x, Wr, bias, W_gate_up, W_down, Wsh_gu, Wsh_d, *, k, scale=3.0, norm=True,
                   limit_routed=0.0, limit_shared=0.0):
     """Brute force: all experts on all tokens, mixed by a mask-weight matrix."""
@@ -195,4 +233,4 @@ def forward_full(inp: dict, shape, *, limit_routed=None, limit_shared=None, scal
 
 
 __all__ = ["lib", "num_threads", "router_logits", "router_select", "router", "permute", "swiglu_hidden",
-           "swiglu_mlp", "forward_tokens", "forward_dense", "forward_full"]
+           "swiglu_mlp", "forward_tokens", "forward_given_routing", "forward_dense", "forward_full"]

@@ -301,6 +301,49 @@ int oracle_forward_tokens(int64_t ntok, int H, int E, int k, int I, int Is, floa
     return missing ? -1 : 0;
 }
 
+/* Layer output with the routing supplied by the caller (routing replay; the pages' fake
+ * balanced static expert routing): y = sum_j w[t,j] * MLP_{idx[t,j]}(x; L_routed) +
+ * MLP_shared(x; L_shared), routed terms summed in the given order, in double. Ids are
+ * clamped to [0, E-1] like the router's. Returns -1 if a used expert's pointer is NULL. */
+int oracle_forward_given_routing(int64_t ntok, int H, int E, int k, int I, int Is, float limit_routed,
+                                 float limit_shared, const uint16_t *x_rows, const int32_t *idx,
+                                 const float *w, const uint16_t *const *Wgu_by_e,
+                                 const uint16_t *const *Wd_by_e, const uint16_t *Wsh_gu,
+                                 const uint16_t *Wsh_d, double *y)
+{
+    for (int64_t n = 0; n < ntok * k; ++n) {
+        int e = idx[n] < 0 ? 0 : (idx[n] > E - 1 ? E - 1 : idx[n]);
+        if (!Wgu_by_e[e] || !Wd_by_e[e])
+            return -1;
+    }
+#pragma omp parallel
+    {
+        int Imax = I > Is ? I : Is;
+        double *hid = (double *)malloc(sizeof(double) * (size_t)Imax);
+        double *o = (double *)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < ntok; ++t) {
+            const uint16_t *xr = x_rows + t * (int64_t)H;
+            double *yr = y + t * (int64_t)H;
+            for (int f = 0; f < H; ++f)
+                yr[f] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int e = idx[t * k + j];
+                e = e < 0 ? 0 : (e > E - 1 ? E - 1 : e);
+                oracle_swiglu_mlp(H, I, xr, Wgu_by_e[e], Wd_by_e[e], limit_routed, o, hid);
+                for (int f = 0; f < H; ++f)
+                    yr[f] += (double)w[t * k + j] * o[f];
+            }
+            oracle_swiglu_mlp(H, Is, xr, Wsh_gu, Wsh_d, limit_shared, o, hid);
+            for (int f = 0; f < H; ++f)
+                yr[f] += o[f];
+        }
+        free(hid);
+        free(o);
+    }
+    return 0;
+}
+
 /* Dense brute force of the same layer: every expert runs on every token and a
  * [T, E] mask-weight matrix (the selection weight, 0 for unselected experts) mixes
  * them, experts summed in ascending index order, plus the shared expert. Stacked

@@ -7,7 +7,7 @@ synthetic input generator is in inputs.py. Importing the package does not load t
 library; the first call does, and raises if it is not built.
 """
 _ABI = {"moe_status_string", "moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn", "moe_combine",
-        "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events", "moe_forward_noalloc", "MoeError", "LayerDesc", "desc_of", "lib",
+        "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events", "moe_forward_noalloc", "moe_forward_with_ids", "MoeError", "LayerDesc", "desc_of", "lib",
         "EXPORTS", "LIB_PATH"}
 
 

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 # Every exported entry point; the header include/moe_b200.h declares exactly these.
 EXPORTS = ["moe_status_string", "moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events",
-           "moe_forward_noalloc"]
+           "moe_forward_noalloc", "moe_forward_with_ids"]
 
 
 class MoeError(RuntimeError):
@@ -69,6 +69,8 @@ def lib():
         L.moe_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.moe_set_wait_limit_ns.restype = ctypes.c_uint64
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(vp), i32]
+        L.moe_forward_with_ids.argtypes = [dp] + [vp] * 9 + [sz, vp]
+        L.moe_forward_with_ids.restype = i32
         L.moe_forward_noalloc.argtypes = [dp] + [vp] * 11
         L.moe_forward_noalloc.restype = i32
         for name in ("moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn", "moe_combine",
@@ -166,3 +168,10 @@ def moe_forward_noalloc(desc, x, Wr, bias, W_gate_up, W_down, Wsh_gate_up, Wsh_d
     _check("moe_forward_noalloc", lib().moe_forward_noalloc(
         ctypes.byref(desc), _p(x), _p(Wr), _p(bias), _p(W_gate_up), _p(W_down), _p(Wsh_gate_up), _p(Wsh_down),
         _p(y), _p(topk_idx_out), _p(topk_w_out), _stream(stream)))
+
+
+def moe_forward_with_ids(desc, x, topk_idx, topk_w, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y, ws, stream=None):
+    """The layer with caller-supplied routing (routing replay / static benchmark routing)."""
+    _check("moe_forward_with_ids", lib().moe_forward_with_ids(
+        ctypes.byref(desc), _p(x), _p(topk_idx), _p(topk_w), _p(W_gate_up), _p(W_down), _p(Wsh_gate_up),
+        _p(Wsh_down), _p(y), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))

@@ -108,13 +108,23 @@ __device__ __forceinline__ void pair_teardown(uint32_t tmem)
     }
 }
 
-// Leader only: the loads of the last S stages (both CTAs' bytes count on the leader's
-// full barriers) have landed.
+// On the way out the loads this CTA issued must have landed. The leader waits on its full
+// barriers (both CTAs' bytes count there) for the last S stages it armed. The peer cannot
+// wait on the leader's barriers; after a normal run its loads are the same stages the
+// leader drains, but after an aborted run it may have issued stages the leader never
+// armed, so it then waits 200 us (TMA latency is microseconds) before the final cluster
+// barrier, behind which neither CTA exits.
 template <int S>
-__device__ __forceinline__ void pair_producer_drain(const PairRing &r, int issued, const WaitCfg &wc)
+__device__ __forceinline__ void pair_producer_drain(const PairRing &r, int issued, bool aborted, const WaitCfg &wc)
 {
-    if (r.rank != 0)
+    if (r.rank != 0) {
+        if (aborted) {
+            const unsigned long long t0 = global_ns();
+            while (global_ns() - t0 < 200000ull) {
+            }
+        }
         return;
+    }
     for (int it = issued > S ? issued - S : 0; it < issued; ++it)
         mbar_wait_drain(&r.full[it % S], (it / S) & 1, wc);
 }
@@ -248,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d_pair(A + G::kABytes, mb, bar, kb * kBK, brow);
                 }
             }
-            pair_producer_drain<S>(r, it, wc);
+            pair_producer_drain<S>(r, it, stop || *r.abort_flag, wc);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -371,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d_pair(A + G::kABytes, mb, bar, kb * kBK, brow);
                 }
             }
-            pair_producer_drain<S>(r, it, wc);
+            pair_producer_drain<S>(r, it, stop || *r.abort_flag, wc);
         }
     } else if (warp == 1) {
         if (lane == 0) {

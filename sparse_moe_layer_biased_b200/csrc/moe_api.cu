@@ -253,6 +253,35 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     return MOE_OK;
 }
 
+// Everything after routing: permutation -> expert FFNs (-> fixed-order combine).
+moe_status_t forward_routed(const moe_layer_desc &d, const DeviceInfo &di, const uint16_t *x, const int32_t *idx,
+                            const float *w, const uint16_t *W_gate_up, const uint16_t *W_down,
+                            const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y, void *ws, cudaStream_t s)
+{
+    const WsLayout L = ws_layout(d);
+    int32_t *counts = at<int32_t>(ws, L.counts);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *perm_token = at<int32_t>(ws, L.perm_token);
+    int32_t *slot_of = at<int32_t>(ws, L.slot_of);
+    if (!stage_mark(1, s))
+        return MOE_ERR_CUDA;
+    const moe::PermuteArgs pa{idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, nullptr, nullptr, nullptr,
+                              nullptr, 0};
+    if (moe::launch_permute(pa, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    float *out = d.deterministic ? at<float>(ws, L.o_perm) : y;
+    moe_status_t st = run_expert_ffn(d, di, x, w, offsets, perm_token, slot_of, W_gate_up, W_down, Wsh_gate_up,
+                                     Wsh_down, out, ws, s);
+    if (st != MOE_OK)
+        return st;
+    if (d.deterministic) {
+        st = cuda_status(moe::launch_combine(out, slot_of, d.T, d.k, d.H, y, s));
+        if (st == MOE_OK && !stage_mark(6, s))
+            st = MOE_ERR_CUDA;
+    }
+    return st;
+}
+
 }  // namespace
 
 extern "C" {
@@ -387,34 +416,39 @@ moe_status_t moe_forward(const moe_layer_desc *desc, const uint16_t *x, const ui
     if ((st = device_info(di)) != MOE_OK)
         return st;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const moe_layer_desc &d = *desc;
     int32_t *idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
     float *w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
-    int32_t *counts = at<int32_t>(ws, L.counts);
-    int32_t *offsets = at<int32_t>(ws, L.offsets);
-    int32_t *perm_token = at<int32_t>(ws, L.perm_token);
-    int32_t *slot_of = at<int32_t>(ws, L.slot_of);
     if (!stage_mark(0, s))
         return MOE_ERR_CUDA;
-    if ((st = run_router(d, di, x, Wr, bias, idx, w, nullptr, s)) != MOE_OK)
+    if ((st = run_router(*desc, di, x, Wr, bias, idx, w, nullptr, s)) != MOE_OK)
         return st;
-    if (!stage_mark(1, s))
+    return forward_routed(*desc, di, x, idx, w, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y, ws, s);
+}
+
+moe_status_t moe_forward_with_ids(const moe_layer_desc *desc, const uint16_t *x, const int32_t *topk_idx,
+                                  const float *topk_w, const uint16_t *W_gate_up, const uint16_t *W_down,
+                                  const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y, void *ws,
+                                  size_t ws_bytes, void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->T == 0)
+        return MOE_OK;
+    if (!x || !topk_idx || !topk_w || !W_gate_up || !W_down || !Wsh_gate_up || !Wsh_down || !y || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W_gate_up) || !aligned16(W_down) || !aligned16(Wsh_gate_up) ||
+        !aligned16(Wsh_down) || !aligned16(y) || !aligned16(ws))
+        return MOE_ERR_UNSUPPORTED;
+    if (ws_bytes < ws_layout(*desc).total)
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!stage_mark(0, s))
         return MOE_ERR_CUDA;
-    const moe::PermuteArgs pa{idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, nullptr, nullptr, nullptr,
-                              nullptr, 0};
-    if (moe::launch_permute(pa, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    float *out = d.deterministic ? at<float>(ws, L.o_perm) : y;
-    if ((st = run_expert_ffn(d, di, x, w, offsets, perm_token, slot_of, W_gate_up, W_down, Wsh_gate_up, Wsh_down,
-                             out, ws, s)) != MOE_OK)
-        return st;
-    if (d.deterministic) {
-        st = cuda_status(moe::launch_combine(out, slot_of, d.T, d.k, d.H, y, s));
-        if (st == MOE_OK && !stage_mark(6, s))
-            st = MOE_ERR_CUDA;
-        return st;
-    }
-    return MOE_OK;
+    return forward_routed(*desc, di, x, topk_idx, topk_w, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y, ws, s);
 }
 
 moe_status_t moe_check_device(void)

@@ -114,3 +114,17 @@ def test_stage_events_validation():
     assert L.moe_set_stage_events(None, 1) == 1
     assert L.moe_set_stage_events(arr, 8) == 1
     assert L.moe_set_stage_events(None, 0) == 0
+
+
+def test_with_ids_validation():
+    L = moe.lib()
+    d = _desc()
+    need = moe.moe_workspace_size(d)
+    args = [FAKE] * 8
+    assert L.moe_forward_with_ids(ctypes.byref(d), *args, FAKE, need - 1, None) == 3
+    args[1] = None
+    assert L.moe_forward_with_ids(ctypes.byref(d), *args, FAKE, need, None) == 1
+    args = [FAKE] * 8
+    args[0] = FAKE + 2
+    assert L.moe_forward_with_ids(ctypes.byref(d), *args, FAKE, need, None) == 2
+    assert L.moe_forward_with_ids(ctypes.byref(_desc(T=0)), *([None] * 9), 0, None) == 0

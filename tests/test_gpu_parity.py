@@ -261,3 +261,54 @@ def test_full_size_output_sampled(full):
     keep = ref["margin"] >= 1e-6
     y = full["y"][torch.from_numpy(rows).cuda()].cpu().numpy()
     check_output(y[keep], ref["y"][keep], sh.name)
+
+
+def _with_ids(sh, inp, idx, w, det=False):
+    d = _abi.desc_of(sh, deterministic=det)
+    ws = torch.empty(_abi.moe_workspace_size(d), dtype=torch.uint8, device="cuda")
+    y = torch.empty((sh.T, sh.H), dtype=torch.float32, device="cuda")
+    _abi.moe_forward_with_ids(d, inp["x"], idx, w, inp["W_gate_up"], inp["W_down"], inp["Wsh_gate_up"],
+                              inp["Wsh_down"], y, ws)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["ragged", "pair", "decode"])
+def test_with_ids_replays_the_router(name):
+    sh = SMALL[name]
+    inp = _to(draw(sh))
+    y, idx, w = _forward(sh, inp, det=True)
+    y2 = _with_ids(sh, inp, torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), det=True)
+    np.testing.assert_array_equal(y2, y)
+
+
+@pytest.mark.parametrize("name", ["mt2", "pair", "decode"])
+def test_with_ids_balanced_static_routing(name):
+    """Round-robin ids with weight scale/k (the fake balanced static expert routing of the
+    Step-5-Preview benchmark setup) against the oracle's given-routing forward."""
+    sh = SMALL[name]
+    inp = draw(sh)
+    t = np.arange(sh.T)[:, None]
+    j = np.arange(sh.k)[None, :]
+    idx = ((t * sh.k + j) % sh.E).astype(np.int32)
+    w = np.full((sh.T, sh.k), sh.scale / sh.k, np.float32)
+    y = _with_ids(sh, _to(inp), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda())
+    gu, d = bf16_bits(inp["W_gate_up"]), bf16_bits(inp["W_down"])
+    ref = oracle.forward_given_routing(bf16_bits(inp["x"]), idx, w, {e: (gu[e], d[e]) for e in range(sh.E)},
+                                       bf16_bits(inp["Wsh_gate_up"]), bf16_bits(inp["Wsh_down"]), E=sh.E,
+                                       limit_routed=sh.limit_routed, limit_shared=sh.limit_shared)
+    check_output(y, ref, name)
+
+
+def test_with_ids_duplicates_and_out_of_range_ids():
+    sh = SMALL["ragged"]
+    inp = draw(sh)
+    rng = np.random.default_rng(5)
+    idx = rng.integers(-3, sh.E + 3, size=(sh.T, sh.k)).astype(np.int32)  # repeats and out-of-range ids
+    w = rng.random((sh.T, sh.k)).astype(np.float32)
+    y = _with_ids(sh, _to(inp), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda())
+    gu, d = bf16_bits(inp["W_gate_up"]), bf16_bits(inp["W_down"])
+    ref = oracle.forward_given_routing(bf16_bits(inp["x"]), idx, w, {e: (gu[e], d[e]) for e in range(sh.E)},
+                                       bf16_bits(inp["Wsh_gate_up"]), bf16_bits(inp["Wsh_down"]), E=sh.E,
+                                       limit_routed=sh.limit_routed, limit_shared=sh.limit_shared)
+    check_output(y, ref, "duplicates")

@@ -300,3 +300,27 @@ def test_zipf_recipe_reaches_target_share(oracle_mod):
     share = counts[:8].sum() / counts.sum()
     assert 0.26 <= share <= 0.34
     assert counts[0] / counts.sum() <= 1.0 / sh.k
+
+
+def test_given_routing_reproduces_the_router_path(oracle_mod):
+    """With the oracle router's own ids and weights, the given-routing forward is the
+    routed forward; with duplicated ids the expert output is added once per slot."""
+    sh = LayerShape("gr", T=21, H=128, E=9, k=3, I=64, Is=128, seed=31, limit_routed=0.25, weight_std=0.05)
+    inp = draw(sh)
+    full = oracle_mod.forward_full(inp, sh)
+    gu, d = bf16_bits(inp["W_gate_up"]), bf16_bits(inp["W_down"])
+    experts = {e: (gu[e], d[e]) for e in range(sh.E)}
+    y = oracle_mod.forward_given_routing(bf16_bits(inp["x"]), full["idx"], full["w"].astype(np.float32), experts,
+                                         bf16_bits(inp["Wsh_gate_up"]), bf16_bits(inp["Wsh_down"]), E=sh.E,
+                                         limit_routed=sh.limit_routed, limit_shared=sh.limit_shared)
+    # weights pass through fp32 here (the replay interface is fp32): relative 6e-8 per weight
+    np.testing.assert_allclose(y, full["y"], rtol=1e-6, atol=1e-7 * np.abs(full["y"]).max())
+    dup = np.full((sh.T, 2), 4, np.int32)
+    w = np.full((sh.T, 2), 0.5, np.float32)
+    y2 = oracle_mod.forward_given_routing(bf16_bits(inp["x"]), dup, w, experts, bf16_bits(inp["Wsh_gate_up"]),
+                                          bf16_bits(inp["Wsh_down"]), E=sh.E, limit_routed=sh.limit_routed,
+                                          limit_shared=sh.limit_shared)
+    one = oracle_mod.forward_given_routing(bf16_bits(inp["x"]), dup[:, :1], np.ones((sh.T, 1), np.float32), experts,
+                                           bf16_bits(inp["Wsh_gate_up"]), bf16_bits(inp["Wsh_down"]), E=sh.E,
+                                           limit_routed=sh.limit_routed, limit_shared=sh.limit_shared)
+    np.testing.assert_allclose(y2, one, rtol=1e-12, atol=1e-15)
