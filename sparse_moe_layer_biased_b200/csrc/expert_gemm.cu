@@ -464,9 +464,9 @@ cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, co
 {
     if (c.pair)
         return launch_down_pair(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
-    if (c.cap == 32)
+    if (c.cap_d == 32)
         return down_impl<32, 10, 1>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
-    if (c.mt == 2)
+    if (c.mt_d == 2)
         return down_impl<128, 4, 2>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
     return down_impl<256, 4, 1>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
 }

@@ -28,6 +28,10 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kBK = 64;
 constexpr uint32_t kATileBytes = 128 * 128;  // 128 weight rows x 64 bf16
+// Token rows reach shared memory in boxes of 64 rows (8 KB per K slice); a stage loads only
+// the boxes that hold rows of its chunk, so a short chunk in a wide tile costs no extra bytes.
+constexpr int kTokBoxRows = 64;
+constexpr uint32_t kTokBoxBytes = kTokBoxRows * 128;
 
 // BN = token rows per pair tile (N of the pair MMA); each CTA holds BN/2 of them.
 // NB = accumulator buffers in TMEM (2: the epilogue of one tile overlaps the next tile's
@@ -47,6 +51,7 @@ struct PairGeo {
     static_assert(kSmemBytes <= kMaxDynSmem, "ring exceeds shared memory");
 
     static_assert(BN % 32 == 0 && BN <= 256, "pair token tile");
+    static_assert((BN / 2) % kTokBoxRows == 0, "token rows per CTA are whole boxes");
 };
 
 struct PairRing {
@@ -237,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_gate_up_pair<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
                 const bool sh = g == a.E;
                 const int half = ((ntok + 15) & ~15) >> 1;  // token rows used from each CTA
+                const int nbox = (half + kTokBoxRows - 1) / kTokBoxRows;
                 const CUtensorMap *mw = sh ? &tm_wsh : &tm_w;
                 const CUtensorMap *mb = sh ? &tm_x : &tm_xp;
                 const int ge = sh ? 0 : g;
@@ -249,13 +255,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (r.rank == 0)
-                        mbar_arrive_expect_tx(&r.full[s], 2 * G::kStageBytes);
+                        mbar_arrive_expect_tx(&r.full[s], 2 * (G::kABytes + nbox * kTokBoxBytes));
                     const uint32_t bar = r.full_leader + 8 * s;
                     uint8_t *A = smem + s * G::kStageBytes;
-                    // one box with this CTA's MT weight tiles, one box of BN/2 token rows
-                    // starting at its half (rows past it are loaded and ignored)
+                    // one box with this CTA's MT weight tiles, then the token boxes that
+                    // cover its half of the chunk (rows past the half are loaded and ignored)
                     tma_load_4d_pair(A, mw, bar, kb * kBK, 0, wt0 * 64, ge);
-                    tma_load_2d_pair(A + G::kABytes, mb, bar, kb * kBK, brow);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d_pair(A + G::kABytes + b * kTokBoxBytes, mb, bar, kb * kBK, brow + b * kTokBoxRows);
                 }
             }
             pair_producer_drain<S>(r, it, stop || *r.abort_flag, wc);
@@ -363,6 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool sh = g == a.E;
                 const int nkb = (sh ? a.Is : a.I) / kBK;
                 const int half = ((ntok + 15) & ~15) >> 1;
+                const int nbox = (half + kTokBoxRows - 1) / kTokBoxRows;
                 const CUtensorMap *mw = sh ? &tm_wdsh : &tm_wd;
                 const CUtensorMap *mb = sh ? &tm_hsh : &tm_h;
                 const int wrow = (sh ? 0 : g * a.H) + (fb * 2 + static_cast<int>(r.rank)) * MT * 128;
@@ -374,11 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (r.rank == 0)
-                        mbar_arrive_expect_tx(&r.full[s], 2 * G::kStageBytes);
+                        mbar_arrive_expect_tx(&r.full[s], 2 * (G::kABytes + nbox * kTokBoxBytes));
                     const uint32_t bar = r.full_leader + 8 * s;
                     uint8_t *A = smem + s * G::kStageBytes;
                     tma_load_2d_pair(A, mw, bar, kb * kBK, wrow);
-                    tma_load_2d_pair(A + G::kABytes, mb, bar, kb * kBK, brow);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d_pair(A + G::kABytes + b * kTokBoxBytes, mb, bar, kb * kBK, brow + b * kTokBoxRows);
                 }
             }
             pair_producer_drain<S>(r, it, stop || *r.abort_flag, wc);
@@ -471,9 +480,12 @@ cudaError_t launch_pairs(Kernel kernel, int smem, int grid, cudaStream_t stream,
     return cudaGetLastError();
 }
 
-// Pair configuration: 128 token rows per pair tile (64 per CTA), two weight tiles per
-// CTA and stage (40 KB stages, 5 deep), two TMEM accumulator buffers.
-constexpr int kPairBN = 128, kPairStages = 5, kPairMT = 2, kPairNB = 2;
+// gate_up: pair tiles of up to 256 token rows (128 per CTA) x 128 features, one weight
+// tile per CTA and stage (32 KB stages, 6 deep). Most experts of a prefill batch then need
+// one pass over their weights. down: 128 token rows x 512 output features, two weight
+// tiles per CTA and stage (40 KB stages, 5 deep). Both keep two TMEM accumulators.
+using GateUpPair = PairGeo<kPairCapGateUp, 6, kPairMtGateUp, 2>;
+using DownPair = PairGeo<kPairCapDown, 5, kPairMtDown, 2>;
 
 }  // namespace
 
@@ -481,18 +493,16 @@ cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_w
                                 const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
                                 cudaStream_t stream)
 {
-    using G = PairGeo<kPairBN, kPairStages, kPairMT, kPairNB>;
-    return launch_pairs(gate_up_pair_kernel<kPairBN, kPairStages, kPairMT, kPairNB>, static_cast<int>(G::kSmemBytes), grid,
-                        stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
+    return launch_pairs(gate_up_pair_kernel<kPairCapGateUp, 6, kPairMtGateUp, 2>,
+                        static_cast<int>(GateUpPair::kSmemBytes), grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
 }
 
 cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
                              const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
                              cudaStream_t stream)
 {
-    using G = PairGeo<kPairBN, kPairStages, kPairMT, kPairNB>;
-    return launch_pairs(down_pair_kernel<kPairBN, kPairStages, kPairMT, kPairNB>, static_cast<int>(G::kSmemBytes), grid,
-                        stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
+    return launch_pairs(down_pair_kernel<kPairCapDown, 5, kPairMtDown, 2>, static_cast<int>(DownPair::kSmemBytes),
+                        grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
 }
 
 }  // namespace moe

@@ -49,36 +49,44 @@ cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream);
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
                           uint16_t *x_perm, float *w_perm, int num_sms, cudaStream_t stream);
 
-// Grouped-GEMM configuration: `cap` = token rows per chunk (the N side of one tile),
-// `mt` = 128-row weight tiles per pipeline stage and CTA, `pair` = tiles run on CTA pairs
-// (cta_group::2). Decode-sized calls (at most 16 tokens per expert on average) use 32-row
-// chunks with one weight tile and a deep ring. Larger calls run on CTA pairs with
-// 128-row chunks when I and Is split into 256-feature and H into 512-feature pair tiles,
-// else on single CTAs with two weight tiles per stage (I, Is multiples of 128, H of 256),
-// else with one weight tile and 256-row chunks.
+// Grouped-GEMM configuration. gate_up and down each split every group into chunks of at
+// most `cap` / `cap_d` token rows (the N side of one tile) and stage `mt` / `mt_d` 128-row
+// weight tiles per pipeline stage and CTA; `pair` = tiles run on CTA pairs (cta_group::2).
+// Decode-sized calls (at most 16 tokens per expert on average) use 32-row chunks with one
+// weight tile and a deep ring. Larger calls run on CTA pairs when I and Is split into
+// 128-feature gate_up pair tiles and H into 512-feature down pair tiles: gate_up on chunks
+// of up to 256 rows (so most experts of a prefill batch stream their weights once), down on
+// 128-row chunks with two weight tiles. Otherwise single CTAs take two weight tiles per
+// stage (I, Is multiples of 128, H of 256), else one weight tile and 256-row chunks.
+constexpr int kPairCapGateUp = 256, kPairMtGateUp = 1, kPairCapDown = 128, kPairMtDown = 2;
 struct GemmConfig {
     int cap;
     int mt;
+    int cap_d;
+    int mt_d;
     int pair;
 };
 inline GemmConfig gemm_config(int64_t T, int64_t k, int64_t E, int64_t H, int64_t I, int64_t Is)
 {
     if (T * k <= 16 * E)
-        return {32, 1, 0};
-    if (I % 256 == 0 && Is % 256 == 0 && H % 512 == 0)
-        return {128, 2, 1};
+        return {32, 1, 32, 1, 0};
+    if (I % 128 == 0 && Is % 128 == 0 && H % 512 == 0)
+        return {kPairCapGateUp, kPairMtGateUp, kPairCapDown, kPairMtDown, 1};
     if (I % 128 == 0 && Is % 128 == 0 && H % 256 == 0)
-        return {128, 2, 0};
-    return {256, 1, 0};
+        return {128, 2, 128, 2, 0};
+    return {256, 1, 256, 1, 0};
 }
 
 // Splits every group (E routed experts, then the shared expert) into chunks of at most
-// `cap` rows. hdr[0] = routed chunk count, hdr[1] = total chunk count.
-cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr,
-                          cudaStream_t stream);
-inline int64_t max_chunks(int64_t T, int64_t k, int64_t E, int64_t H, int64_t I, int64_t Is)
+// `cap` rows. hdr[0] = routed chunk count, hdr[1] = total chunk count. When `chunks_d` is
+// not NULL the same launch also builds a second table of at most `cap_d` rows per chunk
+// (header hdr_d).
+cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr, int cap_d,
+                          int4 *chunks_d, int32_t *hdr_d, cudaStream_t stream);
+// Upper bound on the chunk count of one table: ceil(n / cap) <= n / cap + 1 per group.
+inline int64_t max_chunks(int64_t T, int64_t k, int64_t E, int64_t cap)
 {
-    return (T * k + T) / gemm_config(T, k, E, H, I, Is).cap + E + 2;
+    return (T * k + T) / cap + E + 2;
 }
 
 struct GateUpArgs {

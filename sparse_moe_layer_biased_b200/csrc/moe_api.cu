@@ -85,7 +85,7 @@ moe::WaitCfg wait_cfg(const DeviceInfo &d)
 bool encode_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
                  const cuuint32_t *box)
 {
-    cuuint32_t estr[4] = {1, 1, 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
                                 const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -141,7 +141,7 @@ moe_status_t check_desc(const moe_layer_desc *d)
 }
 
 struct WsLayout {
-    size_t x_perm, w_perm, h, h_sh, chunks, hdr, o_perm, idx, w, counts, offsets, perm_token, slot_of, total;
+    size_t x_perm, w_perm, h, h_sh, chunks, chunks_d, hdr, o_perm, idx, w, counts, offsets, perm_token, slot_of, total;
 };
 
 size_t up256(size_t v)
@@ -163,7 +163,10 @@ WsLayout ws_layout(const moe_layer_desc &d)
     L.w_perm = take(T * k * 4);
     L.h = take(T * k * I * 2);
     L.h_sh = take(T * Is * 2);
-    L.chunks = take(static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, d.H, d.I, d.Is)) * 16);
+    // chunk tables of gate_up and (when its cap differs) of down; hdr holds both headers
+    const moe::GemmConfig cfg = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
+    L.chunks = take(static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, cfg.cap)) * 16);
+    L.chunks_d = take(cfg.cap_d != cfg.cap ? static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, cfg.cap_d)) * 16 : 0);
     L.hdr = take(64);
     L.o_perm = take(d.deterministic ? (T * k + T) * H * 4 : 0);
     L.idx = take(T * k * 4);
@@ -208,17 +211,20 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     float *w_perm = at<float>(ws, L.w_perm);
     uint16_t *h = at<uint16_t>(ws, L.h);
     uint16_t *h_sh = at<uint16_t>(ws, L.h_sh);
+    const moe::GemmConfig cfg = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
     int4 *chunks = at<int4>(ws, L.chunks);
     int32_t *hdr = at<int32_t>(ws, L.hdr);
+    // down reads the gate_up table unless its cap differs
+    int4 *chunks_d = cfg.cap_d != cfg.cap ? at<int4>(ws, L.chunks_d) : chunks;
+    int32_t *hdr_d = cfg.cap_d != cfg.cap ? hdr + 4 : hdr;
     const int64_t Tk = static_cast<int64_t>(d.T) * d.k;
 
-    // One TMA box per operand and pipeline stage: all weight tiles of a stage (64 * mt
-    // gate/up feature pairs, or 128 * mt down rows) and the stage's token rows (the chunk
-    // cap, halved on CTA pairs).
-    const moe::GemmConfig cfg = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
-    const uint32_t brows = static_cast<uint32_t>(cfg.pair ? cfg.cap / 2 : cfg.cap);
+    // One TMA box per weight operand and pipeline stage: all weight tiles of a stage (64 * mt
+    // gate/up feature pairs, or 128 * mt_d down rows). Token rows come in one box of the
+    // chunk cap on single CTAs, in 64-row boxes on CTA pairs.
+    const uint32_t brows = static_cast<uint32_t>(cfg.pair ? 64 : cfg.cap);
     const uint32_t feats = static_cast<uint32_t>(64 * cfg.mt);
-    const uint32_t drows = static_cast<uint32_t>(128 * cfg.mt);
+    const uint32_t drows = static_cast<uint32_t>(128 * cfg.mt_d);
     CUtensorMap tm_w, tm_wsh, tm_xp, tm_x, tm_wd, tm_wdsh, tm_h, tm_hsh;
     bool ok = map_gate_up(&tm_w, Wgu, d.H, d.I, d.E, feats) && map_gate_up(&tm_wsh, Wsh_gu, d.H, d.Is, 1, feats) &&
               map_rows(&tm_xp, x_perm, d.H, Tk, brows) && map_rows(&tm_x, x, d.H, d.T, brows) &&
@@ -232,7 +238,8 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
         return MOE_ERR_CUDA;
     cudaError_t e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, s);
     if (e == cudaSuccess)
-        e = moe::launch_chunks(offsets, d.E, d.T, cfg.cap, chunks, hdr, s);
+        e = moe::launch_chunks(offsets, d.E, d.T, cfg.cap, chunks, hdr, cfg.cap_d,
+                               cfg.cap_d != cfg.cap ? chunks_d : nullptr, hdr_d, s);
     if (e == cudaSuccess && !d.deterministic)
         e = cudaMemsetAsync(out, 0, static_cast<size_t>(d.T) * d.H * 4, s);
     if (e != cudaSuccess)
@@ -244,7 +251,7 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     e = moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s);
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
-    moe::DownArgs da{chunks, hdr, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic};
+    moe::DownArgs da{chunks_d, hdr_d, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic};
     if (!stage_mark(4, s))
         return MOE_ERR_CUDA;
     e = moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s);

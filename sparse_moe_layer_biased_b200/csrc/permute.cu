@@ -242,9 +242,11 @@ __global__ void __launch_bounds__(256)
 // Tile table from an offsets array in global memory (the moe_expert_ffn entry point).
 __global__ void __launch_bounds__(kPermThreads)
     chunks_kernel(const int32_t *__restrict__ offsets, int E, int T, int cap, int4 *__restrict__ chunks,
-                  int32_t *__restrict__ hdr)
+                  int32_t *__restrict__ hdr, int cap_d, int4 *__restrict__ chunks_d, int32_t *__restrict__ hdr_d)
 {
     build_chunk_table(offsets, E, T, cap, chunks, hdr);
+    if (chunks_d)
+        build_chunk_table(offsets, E, T, cap_d, chunks_d, hdr_d);
 }
 
 // y[t] = sum_{j<k} o_perm[slot_of[t, j]] + o_perm[T*k + t], in that order.
@@ -314,10 +316,10 @@ cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t 
     return cudaGetLastError();
 }
 
-cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr,
-                          cudaStream_t stream)
+cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr, int cap_d,
+                          int4 *chunks_d, int32_t *hdr_d, cudaStream_t stream)
 {
-    chunks_kernel<<<1, kPermThreads, 0, stream>>>(offsets, E, T, cap, chunks, hdr);
+    chunks_kernel<<<1, kPermThreads, 0, stream>>>(offsets, E, T, cap, chunks, hdr, cap_d, chunks_d, hdr_d);
     return cudaGetLastError();
 }
 

@@ -29,14 +29,22 @@ SMALL = {
     "wideE": LayerShape("wideE", T=700, H=256, E=300, k=8, I=64, Is=64, seed=24),
     "k32": LayerShape("k32", T=129, H=256, E=64, k=32, I=128, Is=64, seed=25),
     "nonorm": WORKLOADS["tiny"].replace(name="nonorm", norm_expert_weight=False, scale=2.5),
-    # two weight tiles per stage (I, Is multiples of 128, H of 256; > 16 tokens per expert)
-    "mt2": LayerShape("mt2", T=300, H=512, E=12, k=4, I=256, Is=128, limit_routed=0.25, limit_shared=0.125,
+    # two weight tiles per stage on single CTAs (I, Is multiples of 128, H of 256 but not
+    # of 512; > 16 tokens per expert)
+    "mt2": LayerShape("mt2", T=300, H=768, E=12, k=4, I=256, Is=128, limit_routed=0.25, limit_shared=0.125,
                       seed=27, weight_std=0.03),
-    # CTA pairs (I, Is multiples of 256, H of 512)
+    # CTA pairs (I, Is multiples of 128, H of 512)
     "pair": LayerShape("pair", T=300, H=512, E=12, k=4, I=256, Is=256, limit_routed=0.25, limit_shared=0.125,
                        seed=29, weight_std=0.03),
     "pair_ragged": LayerShape("pair_ragged", T=173, H=1024, E=7, k=3, I=512, Is=256, limit_routed=0.0,
                               limit_shared=0.0, seed=30, weight_std=0.03),
+    # odd number of 128-feature gate_up pair tiles (I = 3 * 128)
+    "pair_i384": LayerShape("pair_i384", T=300, H=512, E=12, k=4, I=384, Is=128, limit_routed=0.25,
+                            limit_shared=0.125, seed=31, weight_std=0.03),
+    # ~230 tokens per expert: gate_up tiles with two 64-row token boxes per CTA, experts split
+    # into two gate_up chunks, and down chunks of 128 rows from the same groups
+    "pair_big": LayerShape("pair_big", T=700, H=512, E=6, k=2, I=128, Is=128, limit_routed=0.25,
+                           limit_shared=0.0, seed=32, weight_std=0.03),
     # decode-sized: <= 16 tokens per expert on average
     "decode": LayerShape("decode", T=24, H=512, E=40, k=8, I=192, Is=128, limit_routed=0.25, seed=28,
                          weight_std=0.03),

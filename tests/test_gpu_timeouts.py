@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 
 SHAPES = {
     "decode_config": WORKLOADS["tiny"],
-    "single_cta": LayerShape("mt2", T=300, H=512, E=12, k=4, I=256, Is=128, limit_routed=0.25, seed=27,
+    "single_cta": LayerShape("mt2", T=300, H=768, E=12, k=4, I=256, Is=128, limit_routed=0.25, seed=27,
                              weight_std=0.03),
     "cta_pairs": LayerShape("pair", T=300, H=512, E=12, k=4, I=256, Is=256, limit_routed=0.25, seed=29,
                             weight_std=0.03),
