@@ -15,6 +15,7 @@ from . import build as _build
 _lib = None
 
 _u16p = np.ctypeslib.ndpointer(np.uint16, flags="C_CONTIGUOUS")
+_u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
 _f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
@@ -47,6 +48,13 @@ def lib():
                                                    _u16p, _i32p, _f32p, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                                                    _u16p, _u16p, _f64p]
         L.oracle_forward_given_routing.restype = ctypes.c_int
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_dequant_block128.argtypes = [ctypes.c_int64, ctypes.c_int64, _u8p, _f32p, _f32p]
+        L.oracle_experts_f32w.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_float, ctypes.c_float, _u16p, _i32p, _f64p,
+                                          ctypes.POINTER(_vp), ctypes.POINTER(_vp), _u16p, _u16p, _f64p]
+        L.oracle_experts_f32w.restype = ctypes.c_int
         L.oracle_forward_dense.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                            ctypes.c_float, ctypes.c_float, _u16p, _u16p, _f32p, _u16p,
@@ -232,5 +240,71 @@ def forward_full(inp: dict, shape, *, limit_routed=None, limit_shared=None, scal
         limit_shared=shape.limit_shared if limit_shared is None else limit_shared)
 
 
+def e4m3_values():
+    """Value of every E4M3 code 0..255 (float64; NaN for the two NaN codes)."""
+    return np.array([lib().oracle_e4m3_value(c) for c in range(256)], np.float64)
+
+
+def dequant_block128(q, scale):
+    """FP8 E4M3 matrix q [rows, cols] (uint8 codes) with 128x128 block scales
+    scale [ceil(rows/128), ceil(cols/128)] -> fp32 weights."""
+    q = np.ascontiguousarray(q, np.uint8)
+    scale = np.ascontiguousarray(scale, np.float32)
+    rows, cols = q.shape
+    assert scale.shape == ((rows + 127) // 128, (cols + 127) // 128)
+    out = np.empty((rows, cols), np.float32)
+    lib().oracle_dequant_block128(rows, cols, q, scale, out)
+    return out
+
+
+def experts_f32w(x_rows, idx, w, experts, Wsh_gu, Wsh_d, *, E, limit_routed=0.0, limit_shared=0.0):
+    """Expert part of the layer for a given routing (ids [n, k], weights [n, k] float64)
+    with fp32 routed-expert weights: experts maps id -> (W_gate_up [2I, H] f32,
+    W_down [H, I] f32); the shared expert is BF16 (uint16 bits)."""
+    x_rows = _u16(x_rows)
+    idx = np.ascontiguousarray(idx, np.int32)
+    w = np.ascontiguousarray(w, np.float64)
+    n, H = x_rows.shape
+    k = idx.shape[1]
+    keep = {}
+    gu_ptrs = (_vp * E)()
+    d_ptrs = (_vp * E)()
+    I = None
+    for e, (gu, d) in experts.items():
+        gu = np.ascontiguousarray(gu, np.float32)
+        d = np.ascontiguousarray(d, np.float32)
+        keep[e] = (gu, d)
+        gu_ptrs[e] = gu.ctypes.data
+        d_ptrs[e] = d.ctypes.data
+        I = gu.shape[0] // 2
+    Wsh_gu, Wsh_d = _u16(Wsh_gu), _u16(Wsh_d)
+    Is = Wsh_gu.shape[0] // 2
+    if I is None:
+        I = Is
+    y = np.empty((n, H), np.float64)
+    rc = lib().oracle_experts_f32w(n, H, E, k, I, Is, limit_routed, limit_shared, x_rows, idx, w, gu_ptrs,
+                                   d_ptrs, Wsh_gu, Wsh_d, y)
+    del keep
+    if rc != 0:
+        raise ValueError("a used expert's weights were not supplied")
+    return y
+
+
+def forward_fp8_tokens(x_rows, Wr, bias, Wgu_q, Wgu_s, Wd_q, Wd_s, Wsh_gu, Wsh_d, *, k, scale=3.0, norm=True,
+                       limit_routed=0.0, limit_shared=0.0):
+    """Layer output for the given token rows with FP8 E4M3 routed experts: routing as in
+    router(), then the selected experts dequantized (dequant_block128) and applied with
+    the BF16 shared expert. Wgu_q [E, 2I, H] / Wd_q [E, H, I] uint8 codes with block
+    scales Wgu_s [E, 2I/128, H/128] / Wd_s [E, H/128, I/128]. Returns dict(y, idx, w, margin)."""
+    r = router(x_rows, Wr, bias, k, scale, norm)
+    E = Wgu_q.shape[0]
+    experts = {int(e): (dequant_block128(Wgu_q[e], Wgu_s[e]), dequant_block128(Wd_q[e], Wd_s[e]))
+               for e in np.unique(r["idx"])}
+    y = experts_f32w(x_rows, r["idx"], r["w"], experts, Wsh_gu, Wsh_d, E=E, limit_routed=limit_routed,
+                     limit_shared=limit_shared)
+    return {"y": y, "idx": r["idx"], "w": r["w"], "margin": r["margin"]}
+
+
 __all__ = ["lib", "num_threads", "router_logits", "router_select", "router", "permute", "swiglu_hidden",
-           "swiglu_mlp", "forward_tokens", "forward_given_routing", "forward_dense", "forward_full"]
+           "swiglu_mlp", "forward_tokens", "forward_given_routing", "forward_dense", "forward_full", "e4m3_values",
+           "dequant_block128", "experts_f32w", "forward_fp8_tokens"]

@@ -21,6 +21,8 @@
  *               stacked [num_experts, ...], router_bias kept in float32.
  *  [miles-5.3]  miles Step-5-Preview recipe page, section 5.3: 24 MiB and 12 MiB BF16
  *               expert tensors, i.e. a fused [2I, H] gate_up and a [H, I] down matrix.
+ *  [miles-5.1]  same page, section 1: the checkpoint's routed experts are FP8 E4M3 with
+ *               128x128 block scales, dequantized on load (the FP8 functions at the end).
  *
  * Readings where the pages leave a step open (all restated in the design notes):
  *  - clip form: a = min(silu(g), L), u = clamp(u, -L, L), h = a*u; L = 0 means no clip;
@@ -391,4 +393,114 @@ void oracle_forward_dense(int64_t T, int H, int E, int k, int I, int Is, float s
     free(idx);
     free(w);
     free(mask);
+}
+
+/* ------------------------------------------------------------------------------------
+ * FP8 routed experts. [miles-5.1] miles Step-5-Preview recipe page, section 1 ("FP8
+ * checkpoint"): the routed experts are stored in FP8 E4M3 with one scale per 128x128
+ * block and are dequantized on load; the shared expert is not among them and stays BF16.
+ * Reading taken: the dequantized weight is w[r][c] = e4m3(q[r][c]) * scale[r/128][c/128],
+ * the product rounded once to fp32, the scale an fp32 value.
+ */
+
+/* Value of one E4M3 code (OCP 8-bit floating point, E4M3 variant): sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits; exponent field 0 encodes subnormals m/8 * 2^-6;
+ * exponent field 15 with mantissa 7 is NaN (the variant has no infinities), so the
+ * largest finite magnitude is 1.75 * 2^8 = 448. */
+double oracle_e4m3_value(uint8_t q)
+{
+    const int sign = q >> 7, ex = (q >> 3) & 15, man = q & 7;
+    double v;
+    if (ex == 15 && man == 7)
+        return NAN;
+    if (ex == 0)
+        v = ldexp((double)man / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)man / 8.0, ex - 7);
+    return sign ? -v : v;
+}
+
+/* Dequantize a [rows, cols] E4M3 matrix with 128x128 block scales
+ * (scale [ceil(rows/128), ceil(cols/128)], row-major) to fp32. */
+void oracle_dequant_block128(int64_t rows, int64_t cols, const uint8_t *q, const float *scale, float *out)
+{
+    const int64_t bc = (cols + 127) / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            out[r * cols + c] = (float)(oracle_e4m3_value(q[r * cols + c]) * (double)scale[(r / 128) * bc + c / 128]);
+}
+
+/* The SwiGLU hidden activation and expert MLP of oracle_swiglu_hidden / oracle_swiglu_mlp
+ * for fp32 weights (dequantized FP8 experts): the same sums, clip and product. */
+static void swiglu_mlp_f32w(int H, int Iw, const uint16_t *x_row, const float *Wgu, const float *Wd,
+                            double limit, double *out, double *hid)
+{
+    for (int i = 0; i < Iw; ++i) {
+        const float *wg = Wgu + (int64_t)i * H;
+        const float *wu = Wgu + (int64_t)(Iw + i) * H;
+        double g = 0.0, u = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double xv = bf(x_row[h]);
+            g += (double)wg[h] * xv;
+            u += (double)wu[h] * xv;
+        }
+        double a = g / (1.0 + exp(-g));
+        if (limit > 0.0) {
+            if (a > limit)
+                a = limit;
+            if (u > limit)
+                u = limit;
+            if (u < -limit)
+                u = -limit;
+        }
+        hid[i] = a * u;
+    }
+    for (int f = 0; f < H; ++f) {
+        const float *wd = Wd + (int64_t)f * Iw;
+        double acc = 0.0;
+        for (int i = 0; i < Iw; ++i)
+            acc += (double)wd[i] * hid[i];
+        out[f] = acc;
+    }
+}
+
+/* Expert part of the layer for a given routing with fp32 routed-expert weights (the
+ * dequantized FP8 experts, Wgu_by_e[e] -> [2I, H], Wd_by_e[e] -> [H, I]) and the BF16
+ * shared expert: y = sum_j w[t,j] * MLP_{idx[t,j]}(x; L_routed) + MLP_shared(x; L_shared),
+ * routed terms in the given order, in double. Returns -1 if a used expert's pointer is
+ * NULL or an id is out of range. */
+int oracle_experts_f32w(int64_t ntok, int H, int E, int k, int I, int Is, float limit_routed,
+                        float limit_shared, const uint16_t *x_rows, const int32_t *idx, const double *w,
+                        const float *const *Wgu_by_e, const float *const *Wd_by_e, const uint16_t *Wsh_gu,
+                        const uint16_t *Wsh_d, double *y)
+{
+    for (int64_t n = 0; n < ntok * k; ++n)
+        if (idx[n] < 0 || idx[n] >= E || !Wgu_by_e[idx[n]] || !Wd_by_e[idx[n]])
+            return -1;
+#pragma omp parallel
+    {
+        int Imax = I > Is ? I : Is;
+        double *hid = (double *)malloc(sizeof(double) * (size_t)Imax);
+        double *o = (double *)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < ntok; ++t) {
+            const uint16_t *xr = x_rows + t * (int64_t)H;
+            double *yr = y + t * (int64_t)H;
+            for (int f = 0; f < H; ++f)
+                yr[f] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int e = idx[t * k + j];
+                swiglu_mlp_f32w(H, I, xr, Wgu_by_e[e], Wd_by_e[e], limit_routed, o, hid);
+                for (int f = 0; f < H; ++f)
+                    yr[f] += w[t * k + j] * o[f];
+            }
+            oracle_swiglu_mlp(H, Is, xr, Wsh_gu, Wsh_d, limit_shared, o, hid);
+            for (int f = 0; f < H; ++f)
+                yr[f] += o[f];
+        }
+        free(hid);
+        free(o);
+    }
+    return 0;
 }

@@ -26,6 +26,10 @@ Layouts (row-major, K innermost, PyTorch [out, in] convention):
   x [T, H] bf16; Wr [E, H] bf16; bias [E] fp32;
   W_gate_up [E, 2I, H] bf16 (rows [0, I) gate, rows [I, 2I) up);
   W_down [E, H, I] bf16; Wsh_gate_up [2Is, H] bf16; Wsh_down [H, Is] bf16.
+
+FP8 variant (draw_fp8): the routed experts as FP8 E4M3 codes with one fp32 scale per
+128x128 block, the format of the Step-5-Preview checkpoint (miles Step-5-Preview page,
+section 1); x, Wr, bias and the BF16 shared expert as above.
 """
 from __future__ import annotations
 
@@ -37,6 +41,8 @@ ZIPF_S = 1.1
 # Written by oracle/calibrate_zipf.py (CPU oracle router, 4096 tokens drawn like
 # the skewed workload): hottest-8 share of assignments = 0.30 at this gamma.
 ZIPF_GAMMA = 0.081537
+# Spread of the drawn FP8 E4M3 codes (draw_fp8): most of the format's range below 448.
+FP8_CODE_STD = 64.0
 
 
 @dataclasses.dataclass(frozen=True)
@@ -122,6 +128,54 @@ def draw(shape: LayerShape, device="cpu", gamma: float | None = None) -> dict:
     out["W_down"] = wd
     out["Wsh_gate_up"] = _normal_bf16((2 * Is, H), shape.weight_std, gen, dev)
     out["Wsh_down"] = _normal_bf16((H, Is), shape.weight_std, gen, dev)
+    if shape.bias_kind == "zipf":
+        g = ZIPF_GAMMA if gamma is None else gamma
+        bias = zipf_bias(E, shape.seed, g).to(dev)
+    out["bias"] = bias
+    return out
+
+
+def _e4m3_codes(shape, gen, device):
+    """FP8 E4M3 codes (uint8) of N(0, 64^2) draws, clamped to the format's +-448 range and
+    rounded to nearest even by torch's float8_e4m3fn cast."""
+    t = torch.randn(shape, generator=gen, device=device, dtype=torch.float32).mul_(FP8_CODE_STD)
+    return t.clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def draw_fp8(shape: LayerShape, device="cpu", gamma: float | None = None) -> dict:
+    """Inputs of one layer call with FP8 E4M3 routed experts (128x128 block scales).
+
+    x, Wr, bias and the BF16 shared expert are drawn exactly as draw() draws them; the
+    routed experts are drawn as E4M3 codes ~ N(0, 64^2) (W_gate_up_q [E, 2I, H],
+    W_down_q [E, H, I], uint8) with one fp32 scale per 128x128 block,
+    scale ~ (weight_std / 64) * U(0.5, 1.5) (W_gate_up_s [E, ceil(2I/128), ceil(H/128)],
+    W_down_s [E, ceil(H/128), ceil(I/128)]), so a dequantized weight has about the
+    BF16 draw's spread. Draw order: x, Wr, bias, W_gate_up_q (expert by expert),
+    W_down_q (expert by expert), Wsh_gate_up, Wsh_down, W_gate_up_s, W_down_s.
+    """
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev).manual_seed(shape.seed)
+    T, H, E, I, Is = shape.T, shape.H, shape.E, shape.I, shape.Is
+    out = {}
+    out["x"] = _normal_bf16((T, H), shape.x_std, gen, dev)
+    out["Wr"] = _normal_bf16((E, H), shape.weight_std, gen, dev)
+    bias = torch.rand((E,), generator=gen, device=dev, dtype=torch.float32).mul_(0.2).sub_(0.1)
+    qgu = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=dev)
+    for e in range(E):
+        qgu[e] = _e4m3_codes((2 * I, H), gen, dev)
+    qd = torch.empty((E, H, I), dtype=torch.uint8, device=dev)
+    for e in range(E):
+        qd[e] = _e4m3_codes((H, I), gen, dev)
+    out["W_gate_up_q"] = qgu
+    out["W_down_q"] = qd
+    out["Wsh_gate_up"] = _normal_bf16((2 * Is, H), shape.weight_std, gen, dev)
+    out["Wsh_down"] = _normal_bf16((H, Is), shape.weight_std, gen, dev)
+    blk = lambda n: (n + 127) // 128  # noqa: E731
+    unit = shape.weight_std / FP8_CODE_STD
+    out["W_gate_up_s"] = torch.rand((E, blk(2 * I), blk(H)), generator=gen, device=dev,
+                                    dtype=torch.float32).add_(0.5).mul_(unit)
+    out["W_down_s"] = torch.rand((E, blk(H), blk(I)), generator=gen, device=dev,
+                                 dtype=torch.float32).add_(0.5).mul_(unit)
     if shape.bias_kind == "zipf":
         g = ZIPF_GAMMA if gamma is None else gamma
         bias = zipf_bias(E, shape.seed, g).to(dev)
