@@ -155,6 +155,25 @@ MOE_API moe_status_t moe_forward_with_ids(const moe_layer_desc *desc, const uint
                                   const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y, void *ws,
                                   size_t ws_bytes, void *stream);
 
+/* moe_forward with FP8 E4M3 routed experts: the checkpoint format of the miles
+ * Step-5-Preview page, section 1 ("FP8 checkpoint"), routed experts in FP8 E4M3 with one
+ * scale per 128x128 block, dequantized on load; the shared expert stays BF16.
+ *   W_gate_up_q [E, 2I, H] uint8 E4M3 codes (rows [0, I) gate, [I, 2I) up),
+ *   W_gate_up_scale [E, 2I/128, H/128] fp32, W_down_q [E, H, I] uint8,
+ *   W_down_scale [E, H/128, I/128] fp32: weight[r][c] = e4m3(q[r][c]) * scale[r/128][c/128].
+ * The kernels stream the codes (half the weight bytes of BF16) and turn them into
+ * bf16(e4m3 * scale) in shared memory for the BF16 tensor-core MMA, so a dequantized weight
+ * carries one bf16 rounding (relative 2^-9) besides the BF16 path's arithmetic. Every other
+ * argument, the workspace (moe_workspace_size covers both formats) and the results are
+ * those of moe_forward. Requires I % 128 == 0 (MOE_ERR_UNSUPPORTED otherwise); code arrays
+ * 16-byte aligned, scale arrays 4-byte aligned; the library reads the weights only. */
+MOE_API moe_status_t moe_forward_fp8(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr,
+                                     const float *bias, const uint8_t *W_gate_up_q, const float *W_gate_up_scale,
+                                     const uint8_t *W_down_q, const float *W_down_scale,
+                                     const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y,
+                                     int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                                     void *stream);
+
 /* moe_forward without a caller-provided workspace. The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory at call time, such
  * as a serving runtime whose device memory is already handed to a fixed pool, a

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 # Every exported entry point; the header include/moe_b200.h declares exactly these.
 EXPORTS = ["moe_status_string", "moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events",
-           "moe_forward_noalloc", "moe_forward_with_ids"]
+           "moe_forward_noalloc", "moe_forward_with_ids", "moe_forward_fp8"]
 
 
 class MoeError(RuntimeError):
@@ -70,6 +70,7 @@ def lib():
         L.moe_set_wait_limit_ns.restype = ctypes.c_uint64
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(vp), i32]
         L.moe_forward_with_ids.argtypes = [dp] + [vp] * 9 + [sz, vp]
+        L.moe_forward_fp8.argtypes = [dp] + [vp] * 13 + [sz, vp]
         L.moe_forward_with_ids.restype = i32
         L.moe_forward_noalloc.argtypes = [dp] + [vp] * 11
         L.moe_forward_noalloc.restype = i32
@@ -138,6 +139,15 @@ def moe_forward(desc, x, Wr, bias, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y, 
     _check("moe_forward", lib().moe_forward(
         ctypes.byref(desc), _p(x), _p(Wr), _p(bias), _p(W_gate_up), _p(W_down), _p(Wsh_gate_up), _p(Wsh_down),
         _p(y), _p(topk_idx_out), _p(topk_w_out), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_forward_fp8(desc, x, Wr, bias, W_gate_up_q, W_gate_up_scale, W_down_q, W_down_scale, Wsh_gate_up,
+                    Wsh_down, y, ws, topk_idx_out=None, topk_w_out=None, stream=None):
+    """The layer with FP8 E4M3 routed experts (uint8 codes + fp32 128x128 block scales)."""
+    _check("moe_forward_fp8", lib().moe_forward_fp8(
+        ctypes.byref(desc), _p(x), _p(Wr), _p(bias), _p(W_gate_up_q), _p(W_gate_up_scale), _p(W_down_q),
+        _p(W_down_scale), _p(Wsh_gate_up), _p(Wsh_down), _p(y), _p(topk_idx_out), _p(topk_w_out), _p(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_check_device():

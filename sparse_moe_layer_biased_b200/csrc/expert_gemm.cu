@@ -22,8 +22,7 @@
 //   warps 2..5  epilogue: TMEM -> registers -> activation / weighting -> global
 // Every wait is bounded (mbar_wait); on expiry the CTA drains its own copies and MMAs,
 // frees TMEM and returns with the device error word set.
-#include "gemm_common.cuh"
-#include "internal.h"
+#include "epilogue.cuh"
 
 namespace moe {
 namespace {
@@ -141,27 +140,6 @@ __device__ __forceinline__ bool mma_tile(const Ring &r, uint8_t *smem, uint32_t 
 // map (H, half, row, expert) so TMEM lane 2i holds gate row i and lane 2i+1 its up row;
 // the epilogue pairs them with one shuffle. A tile covers MT * 64 features. Routed
 // chunks read x_perm; the shared expert's chunks read x directly (identity permutation).
-template <int MT>
-__device__ __forceinline__ void decode_gate_up(const GateUpArgs &a, int nrc, int tiles_r, int tile, int &g,
-                                               int &row0, int &ntok, int &fb)
-{
-    int ci;
-    if (tile < tiles_r) {
-        const int nfb = a.I / (64 * MT);
-        ci = tile / nfb;
-        fb = tile - ci * nfb;
-    } else {
-        const int nfb = a.Is / (64 * MT);
-        const int tt = tile - tiles_r;
-        ci = nrc + tt / nfb;
-        fb = tt - (tt / nfb) * nfb;
-    }
-    const int4 c = a.chunks[ci];
-    g = c.x;
-    row0 = c.y;
-    ntok = c.z;
-}
-
 template <int BN, int S, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
     gate_up_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_wsh,
@@ -231,9 +209,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const int pair = row >> 1;
-        const bool is_up = row & 1;
         int tc = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
             int g, row0, ntok, fb;
@@ -243,32 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             tc_fence_after();
             const bool sh = g == a.E;
-            const float L = sh ? a.lim_s : a.lim_r;
-            uint16_t *out = sh ? a.h_sh : a.h;
-            const int64_t ld = sh ? a.Is : a.I;
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                const int64_t feat = (fb * MT + m) * 64 + pair;
-                const uint32_t tb =
-                    tmem + buf * G::kBufCols + m * BN + (static_cast<uint32_t>(q * 32) << 16);
-                for (int cb = 0; cb < ntok; cb += 32) {
-                    float v[32];
-                    tmem_load32(tb + cb, v);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        // even lane finishes column cb+i (needs the up value), odd lane
-                        // column cb+16+i (needs the gate value)
-                        const float send = is_up ? v[i] : v[16 + i];
-                        const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-                        const float gv = is_up ? recv : v[i];
-                        const float uv = is_up ? v[16 + i] : recv;
-                        const int col = cb + (is_up ? 16 + i : i);
-                        const float hv = swiglu_clip(gv, uv, L);
-                        if (col < ntok)
-                            out[(row0 + col) * ld + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
-                    }
-                }
-            }
+            gate_up_epilogue<MT>(tmem + buf * G::kBufCols, BN, static_cast<int64_t>(fb) * MT * 64, ntok, row0,
+                                 sh ? a.h_sh : a.h, sh ? a.Is : a.I, sh ? a.lim_s : a.lim_r, q, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -282,18 +233,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // down: o[f, slot] = Wd_e[f]·h[slot]; routed slots add w_slot * o into y[token] (fp32
 // atomics) or store it in o_perm[slot] (deterministic mode); shared rows add o (weight 1).
 // A tile covers MT * 128 output features.
-template <int MT>
-__device__ __forceinline__ void decode_down(const DownArgs &a, int tile, int &g, int &row0, int &ntok, int &fb)
-{
-    const int nfb = a.H / (128 * MT);
-    const int ci = tile / nfb;
-    fb = tile - ci * nfb;
-    const int4 c = a.chunks[ci];
-    g = c.x;
-    row0 = c.y;
-    ntok = c.z;
-}
-
 template <int BN, int S, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
     down_kernel(const __grid_constant__ CUtensorMap tm_wd, const __grid_constant__ CUtensorMap tm_wdsh,
@@ -360,9 +299,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         const int q = warp & 3;
-        const int64_t f = q * 32 + lane;
-        const int64_t H = a.H;
-        const int64_t shared_base = static_cast<int64_t>(a.T) * a.k;
         int tc = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
             int g, row0, ntok, fb;
@@ -371,39 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(&r.accf[buf], (tc >> 1) & 1, wc, r.abort_flag))
                 break;
             tc_fence_after();
-            const bool sh = g == a.E;
-            for (int cb = 0; cb < ntok; cb += 32) {
-                // lane l fetches the destination row and weight of column cb + l
-                const int mycol = cb + lane;
-                int64_t dst_row = 0;
-                float wgt = 0.0f;
-                if (mycol < ntok) {
-                    const int64_t rr = row0 + mycol;
-                    if (a.deterministic)
-                        dst_row = sh ? shared_base + rr : rr;
-                    else
-                        dst_row = sh ? rr : a.perm_token[rr];
-                    wgt = sh ? 1.0f : a.w_perm[rr];
-                }
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    const int64_t feat = (fb * MT + m) * 128 + f;
-                    float v[32];
-                    tmem_load32(tmem + buf * G::kBufCols + m * BN + (static_cast<uint32_t>(q * 32) << 16) + cb, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int64_t drow = __shfl_sync(0xFFFFFFFFu, dst_row, i);
-                        const float w = __shfl_sync(0xFFFFFFFFu, wgt, i);
-                        if (cb + i < ntok) {
-                            float *p = a.out + drow * H + feat;
-                            if (a.deterministic)
-                                *p = w * v[i];
-                            else
-                                atomicAdd(p, w * v[i]);
-                        }
-                    }
-                }
-            }
+            down_epilogue<MT>(tmem + buf * G::kBufCols, BN, static_cast<int64_t>(fb) * MT * 128, ntok, row0,
+                              g == a.E, a, q, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)

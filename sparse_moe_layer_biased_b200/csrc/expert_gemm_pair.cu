@@ -19,8 +19,7 @@
 //   - TMEM is allocated and freed by warp 1 of both CTAs together (cta_group::2).
 // Every mbarrier wait is bounded; the cluster barriers at the start and end are reached
 // by every thread of both CTAs on every path.
-#include "gemm_common.cuh"
-#include "internal.h"
+#include "epilogue.cuh"
 
 namespace moe {
 namespace {
@@ -278,9 +277,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const int pair = row >> 1;
-        const bool is_up = row & 1;
         int tc = 0;
         for (int tile = first; tile < tiles; tile += stride, ++tc) {
             int g, row0, ntok, fb;
@@ -290,31 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             tc_fence_after();
             const bool sh = g == a.E;
-            const float L = sh ? a.lim_s : a.lim_r;
-            uint16_t *out = sh ? a.h_sh : a.h;
-            const int64_t ld = sh ? a.Is : a.I;
             const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                const int64_t feat = (wt0 + m) * 64 + pair;
-                const uint32_t tb =
-                    tmem + buf * G::kBufCols + m * BN + (static_cast<uint32_t>(q * 32) << 16);
-                for (int cb = 0; cb < ntok; cb += 32) {
-                    float v[32];
-                    tmem_load32(tb + cb, v);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float send = is_up ? v[i] : v[16 + i];
-                        const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-                        const float gv = is_up ? recv : v[i];
-                        const float uv = is_up ? v[16 + i] : recv;
-                        const int col = cb + (is_up ? 16 + i : i);
-                        const float hv = swiglu_clip(gv, uv, L);
-                        if (col < ntok)
-                            out[(row0 + col) * ld + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
-                    }
-                }
-            }
+            gate_up_epilogue<MT>(tmem + buf * G::kBufCols, BN, static_cast<int64_t>(wt0) * 64, ntok, row0,
+                                 sh ? a.h_sh : a.h, sh ? a.Is : a.I, sh ? a.lim_s : a.lim_r, q, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -403,9 +377,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         const int q = warp & 3;
-        const int64_t f = q * 32 + lane;
-        const int64_t H = a.H;
-        const int64_t shared_base = static_cast<int64_t>(a.T) * a.k;
         int tc = 0;
         for (int tile = first; tile < tiles; tile += stride, ++tc) {
             int g, row0, ntok, fb;
@@ -414,39 +385,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(&r.accf[buf], (tc / NB) & 1, wc, r.abort_flag))
                 break;
             tc_fence_after();
-            const bool sh = g == a.E;
             const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
-            for (int cb = 0; cb < ntok; cb += 32) {
-                const int mycol = cb + lane;
-                int64_t dst_row = 0;
-                float wgt = 0.0f;
-                if (mycol < ntok) {
-                    const int64_t rr = row0 + mycol;
-                    if (a.deterministic)
-                        dst_row = sh ? shared_base + rr : rr;
-                    else
-                        dst_row = sh ? rr : a.perm_token[rr];
-                    wgt = sh ? 1.0f : a.w_perm[rr];
-                }
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    const int64_t feat = (wt0 + m) * 128 + f;
-                    float v[32];
-                    tmem_load32(tmem + buf * G::kBufCols + m * BN + (static_cast<uint32_t>(q * 32) << 16) + cb, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int64_t drow = __shfl_sync(0xFFFFFFFFu, dst_row, i);
-                        const float w = __shfl_sync(0xFFFFFFFFu, wgt, i);
-                        if (cb + i < ntok) {
-                            float *p = a.out + drow * H + feat;
-                            if (a.deterministic)
-                                *p = w * v[i];
-                            else
-                                atomicAdd(p, w * v[i]);
-                        }
-                    }
-                }
-            }
+            down_epilogue<MT>(tmem + buf * G::kBufCols, BN, static_cast<int64_t>(wt0) * 128, ntok, row0, g == a.E,
+                              a, q, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)

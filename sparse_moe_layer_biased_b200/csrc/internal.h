@@ -83,6 +83,14 @@ inline GemmConfig gemm_config(int64_t T, int64_t k, int64_t E, int64_t H, int64_
 // (header hdr_d).
 cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr, int cap_d,
                           int4 *chunks_d, int32_t *hdr_d, cudaStream_t stream);
+// FP8-weight configuration (single CTAs, one weight tile per stage): 32-row chunks for
+// decode-sized calls, else 128-row chunks.
+inline GemmConfig gemm_config_fp8(int64_t T, int64_t k, int64_t E)
+{
+    if (T * k <= 16 * E)
+        return {32, 1, 32, 1, 0};
+    return {128, 1, 128, 1, 0};
+}
 // Upper bound on the chunk count of one table: ceil(n / cap) <= n / cap + 1 per group.
 inline int64_t max_chunks(int64_t T, int64_t k, int64_t E, int64_t cap)
 {
@@ -96,6 +104,7 @@ struct GateUpArgs {
     uint16_t *h_sh;  // [T, Is] bf16
     int E, H, I, Is;
     float lim_r, lim_s;
+    const float *w_scale;  // FP8 kernels: block scales [E, 2I/128, H/128]; else unused
 };
 cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
                            const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
@@ -109,6 +118,7 @@ struct DownArgs {
     float *out;  // y [T, H] (atomic) or o_perm [T*k + T, H] (deterministic)
     int E, H, I, Is, T, k;
     int deterministic;
+    const float *w_scale;  // FP8 kernels: block scales [E, H/128, I/128]; else unused
 };
 cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
                         const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
@@ -120,6 +130,15 @@ cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_w
 cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
                              const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
                              cudaStream_t stream);
+
+// FP8 E4M3 routed experts (128x128 block scales, shared expert BF16): tm_w / tm_wd map
+// the E4M3 codes (gate_up: 4-D (H, half, row, expert) bytes; down: 2-D (I, E*H) bytes).
+cudaError_t launch_gate_up_fp8(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
+                               const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
+                               const GemmConfig &c, cudaStream_t stream);
+cudaError_t launch_down_fp8(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
+                            const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
+                            const GemmConfig &c, cudaStream_t stream);
 
 cudaError_t launch_combine(const float *o_perm, const int32_t *slot_of, int T, int k, int H, float *y,
                            cudaStream_t stream);

@@ -113,6 +113,38 @@ bool map_gate_up(CUtensorMap *m, const void *base, int64_t H, int64_t Iw, int64_
     return encode_bf16(m, base, 4, dims, strides, box);
 }
 
+// E4M3 code tensor maps (one byte per element, no swizzle: the converter warps re-lay the
+// tile out), 64-byte inner box.
+bool encode_u8(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
+               const cuuint32_t *box)
+{
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank),
+                                const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// E4M3 gate_up codes [E, 2*Iw, H] viewed as (H, half, row, expert) like map_gate_up.
+bool map_gate_up_u8(CUtensorMap *m, const void *base, int64_t H, int64_t Iw, int64_t G, uint32_t feats)
+{
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(H), 2, static_cast<cuuint64_t>(Iw),
+                                static_cast<cuuint64_t>(G)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(Iw * H), static_cast<cuuint64_t>(H),
+                                   static_cast<cuuint64_t>(2 * Iw * H)};
+    const cuuint32_t box[4] = {64, 2, feats, 1};
+    return encode_u8(m, base, 4, dims, strides, box);
+}
+
+bool map_rows_u8(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, uint32_t box_rows)
+{
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+    const cuuint32_t box[2] = {64, box_rows};
+    return encode_u8(m, base, 2, dims, strides, box);
+}
+
 bool aligned16(const void *p)
 {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
@@ -163,9 +195,12 @@ WsLayout ws_layout(const moe_layer_desc &d)
     L.w_perm = take(T * k * 4);
     L.h = take(T * k * I * 2);
     L.h_sh = take(T * Is * 2);
-    // chunk tables of gate_up and (when its cap differs) of down; hdr holds both headers
+    // chunk tables of gate_up and (when its cap differs) of down, sized for both weight
+    // formats; hdr holds both headers
     const moe::GemmConfig cfg = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
-    L.chunks = take(static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, cfg.cap)) * 16);
+    const moe::GemmConfig cfg8 = moe::gemm_config_fp8(d.T, d.k, d.E);
+    const int cap_min = cfg.cap < cfg8.cap ? cfg.cap : cfg8.cap;
+    L.chunks = take(static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, cap_min)) * 16);
     L.chunks_d = take(cfg.cap_d != cfg.cap ? static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, cfg.cap_d)) * 16 : 0);
     L.hdr = take(64);
     L.o_perm = take(d.deterministic ? (T * k + T) * H * 4 : 0);
@@ -201,17 +236,26 @@ moe_status_t run_router(const moe_layer_desc &d, const DeviceInfo &di, const uin
     return cuda_status(moe::launch_router(tm_x, tm_wr, a, wait_cfg(di), s));
 }
 
+// Expert weights of one call: BF16 routed experts, or FP8 E4M3 codes with 128x128 block
+// scales (gu_scale / d_scale non-NULL); the shared expert is BF16 in both.
+struct ExpertWeights {
+    const void *gu, *d;
+    const float *gu_scale, *d_scale;
+    const uint16_t *sh_gu, *sh_d;
+    bool fp8() const { return gu_scale != nullptr; }
+};
+
 moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const uint16_t *x, const float *topk_w,
                             const int32_t *offsets, const int32_t *perm_token, const int32_t *slot_of,
-                            const uint16_t *Wgu, const uint16_t *Wd, const uint16_t *Wsh_gu, const uint16_t *Wsh_d,
-                            float *out, void *ws, cudaStream_t s)
+                            const ExpertWeights &W, float *out, void *ws, cudaStream_t s)
 {
+    const bool fp8 = W.fp8();
     const WsLayout L = ws_layout(d);
     uint16_t *x_perm = at<uint16_t>(ws, L.x_perm);
     float *w_perm = at<float>(ws, L.w_perm);
     uint16_t *h = at<uint16_t>(ws, L.h);
     uint16_t *h_sh = at<uint16_t>(ws, L.h_sh);
-    const moe::GemmConfig cfg = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
+    const moe::GemmConfig cfg = fp8 ? moe::gemm_config_fp8(d.T, d.k, d.E) : moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
     int4 *chunks = at<int4>(ws, L.chunks);
     int32_t *hdr = at<int32_t>(ws, L.hdr);
     // down reads the gate_up table unless its cap differs
@@ -226,11 +270,12 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     const uint32_t feats = static_cast<uint32_t>(64 * cfg.mt);
     const uint32_t drows = static_cast<uint32_t>(128 * cfg.mt_d);
     CUtensorMap tm_w, tm_wsh, tm_xp, tm_x, tm_wd, tm_wdsh, tm_h, tm_hsh;
-    bool ok = map_gate_up(&tm_w, Wgu, d.H, d.I, d.E, feats) && map_gate_up(&tm_wsh, Wsh_gu, d.H, d.Is, 1, feats) &&
-              map_rows(&tm_xp, x_perm, d.H, Tk, brows) && map_rows(&tm_x, x, d.H, d.T, brows) &&
-              map_rows(&tm_wd, Wd, d.I, static_cast<int64_t>(d.E) * d.H, drows) &&
-              map_rows(&tm_wdsh, Wsh_d, d.Is, d.H, drows) && map_rows(&tm_h, h, d.I, Tk, brows) &&
-              map_rows(&tm_hsh, h_sh, d.Is, d.T, brows);
+    const int64_t EH = static_cast<int64_t>(d.E) * d.H;
+    bool ok = (fp8 ? map_gate_up_u8(&tm_w, W.gu, d.H, d.I, d.E, feats) : map_gate_up(&tm_w, W.gu, d.H, d.I, d.E, feats)) &&
+              (fp8 ? map_rows_u8(&tm_wd, W.d, d.I, EH, drows) : map_rows(&tm_wd, W.d, d.I, EH, drows)) &&
+              map_gate_up(&tm_wsh, W.sh_gu, d.H, d.Is, 1, feats) && map_rows(&tm_xp, x_perm, d.H, Tk, brows) &&
+              map_rows(&tm_x, x, d.H, d.T, brows) && map_rows(&tm_wdsh, W.sh_d, d.Is, d.H, drows) &&
+              map_rows(&tm_h, h, d.I, Tk, brows) && map_rows(&tm_hsh, h_sh, d.Is, d.T, brows);
     if (!ok)
         return MOE_ERR_CUDA;
 
@@ -245,16 +290,19 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
     const moe::WaitCfg wc = wait_cfg(di);
-    moe::GateUpArgs ga{chunks, hdr, h, h_sh, d.E, d.H, d.I, d.Is, d.limit_routed, d.limit_shared};
+    moe::GateUpArgs ga{chunks, hdr, h, h_sh, d.E, d.H, d.I, d.Is, d.limit_routed, d.limit_shared, W.gu_scale};
     if (!stage_mark(3, s))
         return MOE_ERR_CUDA;
-    e = moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s);
+    e = fp8 ? moe::launch_gate_up_fp8(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s)
+            : moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s);
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
-    moe::DownArgs da{chunks_d, hdr_d, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic};
+    moe::DownArgs da{chunks_d, hdr_d, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic,
+                     W.d_scale};
     if (!stage_mark(4, s))
         return MOE_ERR_CUDA;
-    e = moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s);
+    e = fp8 ? moe::launch_down_fp8(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s)
+            : moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s);
     if (e != cudaSuccess || !stage_mark(5, s))
         return MOE_ERR_CUDA;
     return MOE_OK;
@@ -262,8 +310,7 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
 
 // Everything after routing: permutation -> expert FFNs (-> fixed-order combine).
 moe_status_t forward_routed(const moe_layer_desc &d, const DeviceInfo &di, const uint16_t *x, const int32_t *idx,
-                            const float *w, const uint16_t *W_gate_up, const uint16_t *W_down,
-                            const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y, void *ws, cudaStream_t s)
+                            const float *w, const ExpertWeights &W, float *y, void *ws, cudaStream_t s)
 {
     const WsLayout L = ws_layout(d);
     int32_t *counts = at<int32_t>(ws, L.counts);
@@ -277,8 +324,7 @@ moe_status_t forward_routed(const moe_layer_desc &d, const DeviceInfo &di, const
     if (moe::launch_permute(pa, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     float *out = d.deterministic ? at<float>(ws, L.o_perm) : y;
-    moe_status_t st = run_expert_ffn(d, di, x, w, offsets, perm_token, slot_of, W_gate_up, W_down, Wsh_gate_up,
-                                     Wsh_down, out, ws, s);
+    moe_status_t st = run_expert_ffn(d, di, x, w, offsets, perm_token, slot_of, W, out, ws, s);
     if (st != MOE_OK)
         return st;
     if (d.deterministic) {
@@ -381,8 +427,9 @@ moe_status_t moe_expert_ffn(const moe_layer_desc *desc, const uint16_t *x, const
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK)
         return st;
-    return run_expert_ffn(*desc, di, x, topk_w, offsets, perm_token, slot_of, W_gate_up, W_down, Wsh_gate_up,
-                          Wsh_down, out, ws, static_cast<cudaStream_t>(stream));
+    const ExpertWeights W{W_gate_up, W_down, nullptr, nullptr, Wsh_gate_up, Wsh_down};
+    return run_expert_ffn(*desc, di, x, topk_w, offsets, perm_token, slot_of, W, out, ws,
+                          static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_combine(const moe_layer_desc *desc, const float *o_perm, const int32_t *slot_of, float *y,
@@ -429,7 +476,8 @@ moe_status_t moe_forward(const moe_layer_desc *desc, const uint16_t *x, const ui
         return MOE_ERR_CUDA;
     if ((st = run_router(*desc, di, x, Wr, bias, idx, w, nullptr, s)) != MOE_OK)
         return st;
-    return forward_routed(*desc, di, x, idx, w, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y, ws, s);
+    const ExpertWeights W{W_gate_up, W_down, nullptr, nullptr, Wsh_gate_up, Wsh_down};
+    return forward_routed(*desc, di, x, idx, w, W, y, ws, s);
 }
 
 moe_status_t moe_forward_with_ids(const moe_layer_desc *desc, const uint16_t *x, const int32_t *topk_idx,
@@ -455,7 +503,45 @@ moe_status_t moe_forward_with_ids(const moe_layer_desc *desc, const uint16_t *x,
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (!stage_mark(0, s))
         return MOE_ERR_CUDA;
-    return forward_routed(*desc, di, x, topk_idx, topk_w, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y, ws, s);
+    const ExpertWeights W{W_gate_up, W_down, nullptr, nullptr, Wsh_gate_up, Wsh_down};
+    return forward_routed(*desc, di, x, topk_idx, topk_w, W, y, ws, s);
+}
+
+moe_status_t moe_forward_fp8(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr, const float *bias,
+                             const uint8_t *W_gate_up_q, const float *W_gate_up_scale, const uint8_t *W_down_q,
+                             const float *W_down_scale, const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down,
+                             float *y, int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                             void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->I % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;  // gate and up rows must start 128-row scale blocks
+    if (desc->T == 0)
+        return MOE_OK;  // nothing to do; array pointers may be NULL
+    if (!x || !Wr || !bias || !W_gate_up_q || !W_gate_up_scale || !W_down_q || !W_down_scale || !Wsh_gate_up ||
+        !Wsh_down || !y || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wr) || !aligned16(W_gate_up_q) || !aligned16(W_down_q) ||
+        !aligned16(Wsh_gate_up) || !aligned16(Wsh_down) || !aligned16(y) || !aligned16(ws) ||
+        (reinterpret_cast<uintptr_t>(W_gate_up_scale) & 3u) || (reinterpret_cast<uintptr_t>(W_down_scale) & 3u))
+        return MOE_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(*desc);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t *idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+    float *w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
+    if (!stage_mark(0, s))
+        return MOE_ERR_CUDA;
+    if ((st = run_router(*desc, di, x, Wr, bias, idx, w, nullptr, s)) != MOE_OK)
+        return st;
+    const ExpertWeights W{W_gate_up_q, W_down_q, W_gate_up_scale, W_down_scale, Wsh_gate_up, Wsh_down};
+    return forward_routed(*desc, di, x, idx, w, W, y, ws, s);
 }
 
 moe_status_t moe_check_device(void)

@@ -14,13 +14,17 @@ class MoeLayer:
     """One MoE layer call shape (inputs.LayerShape) with its weights on a CUDA device.
 
     weights: dict with Wr [E, H] bf16, bias [E] fp32, W_gate_up [E, 2I, H] bf16,
-    W_down [E, H, I] bf16, Wsh_gate_up [2Is, H] bf16, Wsh_down [H, Is] bf16.
+    W_down [E, H, I] bf16, Wsh_gate_up [2Is, H] bf16, Wsh_down [H, Is] bf16. With FP8 E4M3
+    routed experts the dict holds W_gate_up_q [E, 2I, H] / W_down_q [E, H, I] uint8 codes
+    and their 128x128 block scales W_gate_up_s / W_down_s (fp32) instead of W_gate_up /
+    W_down, and forward runs moe_forward_fp8.
     """
 
     def __init__(self, shape, weights: dict, deterministic: bool = False, max_tokens: int | None = None):
         self.shape = shape
         self.deterministic = deterministic
         self.w = weights
+        self.fp8 = "W_gate_up_q" in weights
         dev = weights["Wr"].device
         self.max_tokens = shape.T if max_tokens is None else max_tokens
         nbytes = _abi.moe_workspace_size(_abi.desc_of(shape, T=self.max_tokens, deterministic=deterministic))
@@ -38,6 +42,10 @@ class MoeLayer:
             idx = torch.empty((T, self.shape.k), dtype=torch.int32, device=x.device)
             w = torch.empty((T, self.shape.k), dtype=torch.float32, device=x.device)
         W = self.w
-        _abi.moe_forward(desc, x, W["Wr"], W["bias"], W["W_gate_up"], W["W_down"], W["Wsh_gate_up"],
-                         W["Wsh_down"], y, self.ws, idx, w, stream=stream)
+        if self.fp8:
+            _abi.moe_forward_fp8(desc, x, W["Wr"], W["bias"], W["W_gate_up_q"], W["W_gate_up_s"], W["W_down_q"],
+                                 W["W_down_s"], W["Wsh_gate_up"], W["Wsh_down"], y, self.ws, idx, w, stream=stream)
+        else:
+            _abi.moe_forward(desc, x, W["Wr"], W["bias"], W["W_gate_up"], W["W_down"], W["Wsh_gate_up"],
+                             W["Wsh_down"], y, self.ws, idx, w, stream=stream)
         return (y, idx, w) if routing else y

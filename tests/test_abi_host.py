@@ -128,3 +128,25 @@ def test_with_ids_validation():
     args[0] = FAKE + 2
     assert L.moe_forward_with_ids(ctypes.byref(d), *args, FAKE, need, None) == 2
     assert L.moe_forward_with_ids(ctypes.byref(_desc(T=0)), *([None] * 9), 0, None) == 0
+
+
+def test_fp8_validation():
+    L = moe.lib()
+    d = _desc()
+    assert d.I % 128 == 0
+    need = moe.moe_workspace_size(d)
+    args = [FAKE] * 10  # x, Wr, bias, codes / scales (gate_up, down), shared gate_up, shared down, y
+    tail = [None, None, FAKE]
+    assert L.moe_forward_fp8(ctypes.byref(d), *args, *tail, need - 1, None) == 3
+    a = list(args)
+    a[4] = None  # gate_up scales
+    assert L.moe_forward_fp8(ctypes.byref(d), *a, *tail, need, None) == 1
+    a = list(args)
+    a[5] = FAKE + 8  # down codes not 16-byte aligned
+    assert L.moe_forward_fp8(ctypes.byref(d), *a, *tail, need, None) == 2
+    a = list(args)
+    a[6] = FAKE + 2  # down scales not 4-byte aligned
+    assert L.moe_forward_fp8(ctypes.byref(d), *a, *tail, need, None) == 2
+    # I must be a multiple of 128 (gate and up rows start scale blocks), even with T = 0
+    assert L.moe_forward_fp8(ctypes.byref(_desc(I=192)), *args, *tail, need, None) == 2
+    assert L.moe_forward_fp8(ctypes.byref(_desc(T=0)), *([None] * 13), 0, None) == 0

@@ -1,0 +1,138 @@
+"""GPU parity of the FP8 E4M3 routed-expert path (moe_forward_fp8) against the oracle.
+
+The oracle dequantizes the selected experts (e4m3 code * 128x128 block scale, fp32) and
+runs the layer in double; the GPU streams the codes and multiplies by bf16(e4m3 *
+scale) on the tensor cores. The extra bf16 rounding of each dequantized weight
+(relative <= 2^-9, independent across weights) adds about 2^-9 / sqrt(3) ~ 1.1e-3
+relative error to a dot product whose terms have random signs, inside the layer's
+1e-2 relative-Frobenius / 3e-2 max-abs bar, which the tests keep.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _parity import check_output, check_routing, rel_fro
+from sparse_moe_layer_biased_b200 import _abi
+from sparse_moe_layer_biased_b200.inputs import WORKLOADS, LayerShape, bf16_bits, draw_fp8, token_sample
+from sparse_moe_layer_biased_b200.layer import MoeLayer
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = {
+    # decode-sized (<= 16 tokens per expert on average): 32-row chunks
+    "tiny": WORKLOADS["tiny"],
+    "decode": LayerShape("fp8_decode", T=24, H=512, E=40, k=8, I=256, Is=128, limit_routed=0.25, seed=51,
+                         weight_std=0.03),
+    # prefill-sized: 128-row chunks, several K blocks, ragged chunk tails, Is not a multiple of 128
+    "prefill": LayerShape("fp8_prefill", T=300, H=512, E=12, k=4, I=256, Is=192, limit_routed=0.25,
+                          limit_shared=0.125, seed=52, weight_std=0.03),
+    "ragged": LayerShape("fp8_ragged", T=333, H=384, E=40, k=6, I=128, Is=320, limit_routed=0.0,
+                         limit_shared=0.0, seed=53, weight_std=0.03),
+    # pre-activations of std ~1 against routed limit 0.5: the up clamp binds on ~60% and
+    # the silu cap on ~20% of routed units (outputs stay at the workloads' scale, where
+    # the absolute bar applies)
+    "clip": LayerShape("fp8_clip", T=200, H=256, E=8, k=2, I=384, Is=128, limit_routed=0.5, limit_shared=0.25,
+                       seed=54, weight_std=0.06),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    _abi.lib()
+    yield
+    _abi.moe_check_device()
+
+
+def _oracle(sh, inp, rows=None):
+    """Oracle layer output (fp64) for the listed rows of a host-resident FP8 draw."""
+    x = inp["x"] if rows is None else inp["x"][rows]
+    return oracle.forward_fp8_tokens(
+        bf16_bits(x), bf16_bits(inp["Wr"]), inp["bias"].numpy(), inp["W_gate_up_q"].numpy(),
+        inp["W_gate_up_s"].numpy(), inp["W_down_q"].numpy(), inp["W_down_s"].numpy(),
+        bf16_bits(inp["Wsh_gate_up"]), bf16_bits(inp["Wsh_down"]), k=sh.k, scale=sh.scale,
+        norm=sh.norm_expert_weight, limit_routed=sh.limit_routed, limit_shared=sh.limit_shared)
+
+
+def _forward(sh, inp_dev, det=False):
+    layer = MoeLayer(sh, inp_dev, deterministic=det)
+    assert layer.fp8
+    y, idx, w = layer.forward(inp_dev["x"], routing=True)
+    torch.cuda.synchronize()
+    _abi.moe_check_device()
+    return y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("det", [False, True])
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_fp8_forward_small(name, det):
+    sh = SHAPES[name]
+    inp = draw_fp8(sh)
+    y, idx, w = _forward(sh, {k: v.cuda() for k, v in inp.items()}, det)
+    ref = _oracle(sh, inp)
+    keep = check_routing(idx, w, ref, sh.E, sh.k)
+    rf, ma = check_output(y[keep], ref["y"][keep], name)
+    print(f"{name} det={det}: rel_fro {rf:.2e} max_abs {ma:.2e}")
+
+
+def test_fp8_deterministic_matches_atomic():
+    sh = SHAPES["prefill"]
+    inp = {k: v.cuda() for k, v in draw_fp8(sh).items()}
+    ya, _, _ = _forward(sh, inp, det=False)
+    yd, _, _ = _forward(sh, inp, det=True)
+    yd2, _, _ = _forward(sh, inp, det=True)
+    np.testing.assert_array_equal(yd, yd2)
+    assert rel_fro(ya, yd) < 1e-6
+
+
+def test_fp8_scales_are_applied_per_block():
+    """Doubling every scale of one expert's down projection doubles that expert's
+    contribution: y(2s) - y(s) equals the difference the oracle predicts."""
+    sh = SHAPES["prefill"]
+    inp = draw_fp8(sh)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    y1, idx, _ = _forward(sh, dev, det=True)
+    e = int(np.bincount(idx.ravel(), minlength=sh.E).argmax())
+    inp2 = dict(inp)
+    s2 = inp["W_down_s"].clone()
+    s2[e] *= 2.0
+    inp2["W_down_s"] = s2
+    dev["W_down_s"] = s2.cuda()
+    y2, _, _ = _forward(sh, dev, det=True)
+    r1, r2 = _oracle(sh, inp), _oracle(sh, inp2)
+    check_output(y2 - y1, r2["y"] - r1["y"], "scale delta")
+
+
+@pytest.fixture(scope="module", params=["step35_decode", "step35_prefill"])
+def full(request):
+    sh = WORKLOADS[request.param]
+    inp = draw_fp8(sh, device="cuda")
+    y, idx, w = _forward(sh, inp)
+    yield {"shape": sh, "inp": inp, "y": y, "idx": idx, "w": w}
+    del inp
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+def test_fp8_full_size_output_sampled(full):
+    """Full-size shapes in the benchmark's launch configuration: routing of the sampled
+    tokens and their outputs against the oracle (only their experts are dequantized)."""
+    sh = full["shape"]
+    rows = token_sample(sh.T, 4, sh.seed).numpy()
+    inp = full["inp"]
+    x_rows = inp["x"][torch.from_numpy(rows).cuda()]
+    r = oracle.router(bf16_bits(x_rows), bf16_bits(inp["Wr"]), inp["bias"].cpu().numpy(), sh.k)
+    ids = sorted(set(int(e) for e in r["idx"].ravel()))
+    experts = {e: (oracle.dequant_block128(inp["W_gate_up_q"][e].cpu().numpy(), inp["W_gate_up_s"][e].cpu().numpy()),
+                   oracle.dequant_block128(inp["W_down_q"][e].cpu().numpy(), inp["W_down_s"][e].cpu().numpy()))
+               for e in ids}
+    y_ref = oracle.experts_f32w(bf16_bits(x_rows), r["idx"], r["w"], experts, bf16_bits(inp["Wsh_gate_up"]),
+                                bf16_bits(inp["Wsh_down"]), E=sh.E, limit_routed=sh.limit_routed,
+                                limit_shared=sh.limit_shared)
+    keep = r["margin"] >= 1e-6
+    np.testing.assert_array_equal(np.sort(full["idx"][rows][keep], 1), np.sort(r["idx"][keep], 1))
+    rf, ma = check_output(full["y"][rows][keep], y_ref[keep], sh.name)
+    print(f"{sh.name} fp8 sampled: rel_fro {rf:.2e} max_abs {ma:.2e}")
