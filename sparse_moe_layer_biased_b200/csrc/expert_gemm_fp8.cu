@@ -5,76 +5,72 @@
 // on load; the shared expert stays BF16. The layer steps are those of expert_gemm.cu
 // ("MAX 中 Step-3.5-Flash 架构解析", section "MoE共享专家、sigmoid 路由与激活裁剪").
 //
-// Dequantization happens on the way from HBM to the tensor cores. A deep staging ring
-// receives, per K slice, the E4M3 weight tile (64 bytes per row, half the bytes of
-// BF16) and the token rows; four converter warps turn the weight tile into
-// bf16(e4m3 * block_scale) in the 128-byte-swizzled K-major layout the MMA reads, in a
-// shallow ring of converted tiles; the MMA (the BF16 tcgen05 MMA of the BF16 path) reads
-// the converted tile and the token rows straight from the staging slot, then frees both
-// slots. Loads therefore run a whole staging ring ahead of the MMA, and the converted
-// ring's turnaround holds no memory latency. Shared-expert tiles are BF16: their weight
-// tile lands directly in the converted ring.
+// Dequantization happens on the way from HBM to the tensor cores without a second trip
+// through shared memory. A staging ring receives, per pipeline stage, the weight tile of
+// 128 rows and the token rows: a routed stage spans one 128-wide scale block (E4M3 codes,
+// 128 bytes per row: half the bytes of BF16), a shared-expert stage 64 K elements of its
+// BF16 weights (also 128 bytes per row). Converter warps each take one weight row (one
+// TMEM lane), turn it into bf16(e4m3 * block_scale) and store it into a TMEM operand
+// slot; the BF16 tcgen05 MMA reads A from TMEM and the token rows (B) from the staging
+// slot. Shared memory then carries each weight byte once in and once out, fewer bytes
+// per weight element than the BF16 kernels move. Two groups of four converter warps take
+// alternate stages, so one group's conversion overlaps the other's waits; a tile's block
+// scales are read once per tile into registers.
 //
 // Roles per CTA (persistent, one CTA per SM, static round-robin over tiles):
-//   warp 0      staging producer: E4M3 weight tile (routed experts) + token rows
-//   warp 1      MMA issuer and TMEM owner (2 accumulator buffers)
-//   warps 2..5  epilogue (TMEM -> activation / weighting -> global)
-//   warps 6..9  converters: staged E4M3 tile -> converted bf16 tile, one block scale per
-//               128-row weight group and 128-wide K block
-//   warp 10     shared-expert producer: BF16 weight tiles of the shared expert -> converted ring
+//   warp 0       staging producer: weight tile (E4M3 routed / BF16 shared) + token rows
+//   warp 1       MMA issuer and TMEM owner (2 accumulator buffers, SA operand slots)
+//   warps 2..5   epilogue (TMEM -> activation / weighting -> global)
+//   warps 6..13  converters, group 0 (warps 6..9) on even stages, group 1 on odd ones;
+//                warp w handles weight rows / TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31
 // Every wait is bounded; on expiry the CTA drains its own copies and MMAs, frees TMEM
 // and returns with the device error word set.
-#include <cuda_fp8.h>
+#include <cuda_bf16.h>
 
 #include "epilogue.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads8 = 352;
+constexpr int kThreads8 = 448;
 constexpr int kBK = 64;
-constexpr uint32_t kATileBytes = 128 * 128;  // 128 weight rows x 64 bf16 (converted)
-constexpr uint32_t kQTileBytes = 128 * 64;   // 128 weight rows x 64 E4M3 codes (staged)
+constexpr uint32_t kWBytes = 128 * 128;  // weight part of a staging slot: 128 rows x 128 bytes
+constexpr uint32_t kACols = 64;          // TMEM columns of one operand slot: 128 bf16 per row
 
-// BN token rows per chunk, SW staging slots (MT E4M3 weight tiles + BN token rows),
-// SA converted slots (MT bf16 weight tiles).
-template <int BN, int SA, int SW, int MT>
+// BN token rows per chunk, SW staging slots, SA TMEM operand slots.
+template <int BN, int SW, int SA>
 struct Geo8 {
-    static constexpr uint32_t kABytes = MT * kATileBytes;  // converted slot
-    static constexpr uint32_t kQBytes = MT * kQTileBytes;  // staged E4M3 part of a staging slot
-    static constexpr uint32_t kBBytes = BN * 128;          // token part of a staging slot
-    static constexpr uint32_t kQSlotBytes = kQBytes + kBBytes;
-    static constexpr uint32_t kQOff = SA * kABytes;
-    static constexpr uint32_t kBarOff = kQOff + SW * kQSlotBytes;
-    static constexpr uint32_t kNumBars = 2 * SW + 3 * SA + 5;
+    static constexpr uint32_t kBSlice = BN * 128;  // token rows of one 64-wide K slice
+    static constexpr uint32_t kSlotBytes = kWBytes + 2 * kBSlice;
+    static constexpr uint32_t kBarOff = SW * kSlotBytes;
+    static constexpr uint32_t kNumBars = 2 * SW + 2 * SA + 5;
     static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
     static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
-    static constexpr uint32_t kBufCols = MT * BN;
-    static constexpr uint32_t kTmemCols = 2 * kBufCols < 32 ? 32 : 2 * kBufCols;
-    static_assert(kABytes % 1024 == 0 && kQSlotBytes % 1024 == 0 && kQBytes % 1024 == 0,
-                  "slots stay 1024-byte aligned");
-    static_assert(kSmemBytes <= kMaxDynSmem, "rings exceed shared memory");
-    static_assert((kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512, "TMEM allocation");
+    static constexpr uint32_t kBufCols = BN;             // one accumulator buffer
+    static constexpr uint32_t kAOff = 2 * kBufCols;      // first operand slot column
+    static constexpr uint32_t kUsedCols = kAOff + SA * kACols;
+    static constexpr uint32_t kTmemCols = kUsedCols <= 128 ? 128 : (kUsedCols <= 256 ? 256 : 512);
+    static_assert(kSlotBytes % 1024 == 0, "slots stay 1024-byte aligned");
+    static_assert(kSmemBytes <= kMaxDynSmem, "ring exceeds shared memory");
+    static_assert(kUsedCols <= 512, "accumulators and operand slots exceed TMEM");
 };
 
 struct Ring8 {
-    uint64_t *qfull, *qempty;        // staging ring: bytes landed / MMA done with the slot
-    uint64_t *afull, *conv, *aempty;  // converted ring: shared-expert weights landed (or a
-                                      // plain arrival) / converted / MMA done with the slot
+    uint64_t *qfull, *qempty;  // staging ring: bytes landed / MMA done with the slot
+    uint64_t *conv, *aempty;   // TMEM operand slots: converted / MMA done with the slot
     uint64_t *accf, *acce, *drain;
     uint32_t *holder;
     volatile int *abort_flag;
 };
 
-template <class G, int SA, int SW>
+template <class G, int SW, int SA>
 __device__ __forceinline__ uint8_t *ring8_setup(uint8_t *smem_raw, Ring8 &r)
 {
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *smem = smem_raw + pad;
     r.qfull = reinterpret_cast<uint64_t *>(smem + G::kBarOff);
     r.qempty = r.qfull + SW;
-    r.afull = r.qempty + SW;
-    r.conv = r.afull + SA;
+    r.conv = r.qempty + SW;
     r.aempty = r.conv + SA;
     r.accf = r.aempty + SA;
     r.acce = r.accf + 2;
@@ -87,8 +83,7 @@ __device__ __forceinline__ uint8_t *ring8_setup(uint8_t *smem_raw, Ring8 &r)
             mbar_init(&r.qempty[s], 1);
         }
         for (int s = 0; s < SA; ++s) {
-            mbar_init(&r.afull[s], 1);
-            mbar_init(&r.conv[s], 4);  // one arrival per converter warp
+            mbar_init(&r.conv[s], 4);  // one arrival per warp of the converting group
             mbar_init(&r.aempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -127,275 +122,298 @@ __device__ __forceinline__ void drain_ring(uint64_t *bars, int depth, int issued
         mbar_wait_drain(&bars[it % depth], (it / depth) & 1, wc);
 }
 
-// bf16 pair (lo, hi) of e4m3 codes b0 (lower K) and b1, each times `scale`.
-__device__ __forceinline__ uint32_t dequant2(uint32_t codes16, float scale)
+// Dequantization on the integer and FMA pipes. An E4M3 code s.eeee.mmm placed in a bf16
+// word as s.0000eeee.mmm0000 (sign at bit 15, exponent field e, fraction m/8) is a bf16
+// number whose value is exactly the code's value times 2^-120: normal codes map to bf16
+// normals 2^(e-127)(1 + m/8) = 2^-120 * 2^(e-7)(1 + m/8), subnormal codes to bf16
+// subnormals 2^-126 * m/8 = 2^-120 * 2^-6 * m/8. The block scale then multiplies as
+// S = scale * 2^120 (exact in fp32 for |scale| < 2^8), split into bf16 parts
+// S = S_hi + S_lo: the weight is fma(q, S_hi, q * S_lo), within one bf16 ulp of
+// bf16(code value * scale) (equal to it except near rounding ties: the S_lo product
+// carries a relative error of 2^-18). The two E4M3 NaN codes are not decoded as NaN
+// (checkpoints hold none).
+struct Scale2 {
+    __nv_bfloat162 hi, lo;
+};
+
+__device__ __forceinline__ Scale2 split_scale(float scale)
 {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes16), __NV_E4M3);
-    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
-    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
-    return *reinterpret_cast<const uint32_t *>(&b);
+    const float S = scale * 0x1p120f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(S);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(S - __bfloat162float(hi));
+    return Scale2{__bfloat162bfloat162(hi), __bfloat162bfloat162(lo)};
 }
 
-// Converts one staged weight tile (128 rows x 64 E4M3 codes, row j at j * 64 bytes) into
-// the 128-byte-swizzled K-major bf16 tile the MMA reads (row j at (j / 8) * 1024 +
-// (j % 8) * 128, 16-byte chunk c stored at chunk c ^ (j % 8)). Row j takes scale
-// s_odd when j is odd, else s_even (gate_up tiles interleave gate and up rows, which
-// sit in different 128-row scale blocks). The 128 converter threads each take 4 units
-// of 16 codes; a warp reads 512 contiguous staged bytes per step.
-__device__ __forceinline__ void convert_tile(const uint8_t *q, uint8_t *a, float s_even, float s_odd, int ct)
+// Codes (b0, b1) of the 16-bit half `sel` selects (0x1404: bytes 0, 1; 0x3424: bytes 2, 3)
+// -> bf16x2 (low half = lower K) of code value * scale.
+__device__ __forceinline__ uint32_t dequant2(uint32_t codes4, uint32_t sel, const Scale2 &sc)
+{
+    const uint32_t y = __byte_perm(codes4, 0u, sel);  // code k in bits 8..15 of its 16-bit half
+    const uint32_t bits = (y & 0x80008000u) | ((y >> 4) & 0x07F007F0u);
+    const __nv_bfloat162 q = *reinterpret_cast<const __nv_bfloat162 *>(&bits);
+    const __nv_bfloat162 w = __hfma2(q, sc.hi, __hmul2(q, sc.lo));
+    return *reinterpret_cast<const uint32_t *>(&w);
+}
+
+// Byte offset of 16-byte chunk c of row j in a 128-byte-swizzled tile of 128-byte rows
+// (the TMA SWIZZLE_128B layout: chunk c of row j stored at chunk c ^ (j % 8)).
+__device__ __forceinline__ uint32_t sw128_chunk(int j, int c)
+{
+    return static_cast<uint32_t>((j >> 3) * 1024 + (j & 7) * 128 + ((c ^ (j & 7)) << 4));
+}
+
+// Routed stage: converts row j (128 E4M3 codes) of the staged tile and stores the 64
+// bf16 pairs into TMEM lane j, columns taddr .. taddr + 63 (taddr carries the lane).
+__device__ __forceinline__ void convert_row_e4m3(const uint8_t *w, int j, uint32_t taddr, const Scale2 &s)
 {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int u = ct + 128 * i;
-        const int j = u >> 2, c = u & 3;
-        const uint4 v = *reinterpret_cast<const uint4 *>(q + j * 64 + c * 16);
-        const float s = (j & 1) ? s_odd : s_even;
-        uint4 lo, hi;
-        lo.x = dequant2(v.x & 0xFFFFu, s);
-        lo.y = dequant2(v.x >> 16, s);
-        lo.z = dequant2(v.y & 0xFFFFu, s);
-        lo.w = dequant2(v.y >> 16, s);
-        hi.x = dequant2(v.z & 0xFFFFu, s);
-        hi.y = dequant2(v.z >> 16, s);
-        hi.z = dequant2(v.w & 0xFFFFu, s);
-        hi.w = dequant2(v.w >> 16, s);
-        uint8_t *row = a + (j >> 3) * 1024 + (j & 7) * 128;
-        *reinterpret_cast<uint4 *>(row + (((2 * c) ^ (j & 7)) << 4)) = lo;
-        *reinterpret_cast<uint4 *>(row + (((2 * c + 1) ^ (j & 7)) << 4)) = hi;
+    for (int h = 0; h < 4; ++h) {  // 32 codes -> 16 columns per store
+        uint32_t out[16];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(w + sw128_chunk(j, 2 * h + cc));
+            out[8 * cc + 0] = dequant2(v.x, 0x1404u, s);
+            out[8 * cc + 1] = dequant2(v.x, 0x3424u, s);
+            out[8 * cc + 2] = dequant2(v.y, 0x1404u, s);
+            out[8 * cc + 3] = dequant2(v.y, 0x3424u, s);
+            out[8 * cc + 4] = dequant2(v.z, 0x1404u, s);
+            out[8 * cc + 5] = dequant2(v.z, 0x3424u, s);
+            out[8 * cc + 6] = dequant2(v.w, 0x1404u, s);
+            out[8 * cc + 7] = dequant2(v.w, 0x3424u, s);
+        }
+        tmem_store16(taddr + 16 * h, out);
     }
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem()
+// Shared-expert stage: copies row j (64 bf16) of the staged BF16 tile into TMEM lane j,
+// columns taddr .. taddr + 31.
+__device__ __forceinline__ void copy_row_bf16(const uint8_t *w, int j, uint32_t taddr)
 {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t out[16];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(w + sw128_chunk(j, 4 * h + cc));
+            out[4 * cc + 0] = v.x;
+            out[4 * cc + 1] = v.y;
+            out[4 * cc + 2] = v.z;
+            out[4 * cc + 3] = v.w;
+        }
+        tmem_store16(taddr + 16 * h, out);
+    }
 }
 
 // One tile of either GEMM: group g (E = shared expert), chunk rows [row0, row0 + ntok),
-// feature block fb, nkb K slices.
+// weight block fb (64 gate/up feature pairs, or 128 down rows), K extent K.
 struct Tile8 {
-    int g, row0, ntok, fb, nkb;
+    int g, row0, ntok, fb, K;
     bool sh;
+    // a routed stage spans one 128-wide scale block (E4M3), a shared stage 64 K (BF16)
+    __device__ __forceinline__ int stage_k() const { return sh ? 64 : 128; }
+    __device__ __forceinline__ int stages() const { return (K + stage_k() - 1) / stage_k(); }
 };
 
-template <int MT>
 __device__ __forceinline__ Tile8 tile_of(const GateUpArgs &a, int tile)
 {
     const int nrc = a.hdr[0];
-    const int tiles_r = nrc * (a.I / (64 * MT));
     Tile8 t;
-    decode_gate_up<MT>(a, nrc, tiles_r, tile, t.g, t.row0, t.ntok, t.fb);
+    decode_gate_up<1>(a, nrc, nrc * (a.I / 64), tile, t.g, t.row0, t.ntok, t.fb);
     t.sh = t.g == a.E;
-    t.nkb = a.H / kBK;
+    t.K = a.H;
     return t;
 }
 
-template <int MT>
 __device__ __forceinline__ Tile8 tile_of(const DownArgs &a, int tile)
 {
     Tile8 t;
-    decode_down<MT>(a, tile, t.g, t.row0, t.ntok, t.fb);
+    decode_down<1>(a, tile, t.g, t.row0, t.ntok, t.fb);
     t.sh = t.g == a.E;
-    t.nkb = (t.sh ? a.Is : a.I) / kBK;
+    t.K = t.sh ? a.Is : a.I;
     return t;
 }
 
-template <int MT>
 __device__ __forceinline__ int tile_count(const GateUpArgs &a)
 {
     const int nrc = a.hdr[0];
-    return nrc * (a.I / (64 * MT)) + (a.hdr[1] - nrc) * (a.Is / (64 * MT));
+    return nrc * (a.I / 64) + (a.hdr[1] - nrc) * (a.Is / 64);
 }
 
-template <int MT>
 __device__ __forceinline__ int tile_count(const DownArgs &a)
 {
-    return a.hdr[1] * (a.H / (128 * MT));
+    return a.hdr[1] * (a.H / 128);
 }
 
-// Weight tile(s) of K slice kb: gate_up maps are (H, half, row, expert) with boxes of
-// MT*64 (gate, up) row pairs; down maps are (I, rows) with boxes of MT*128 rows.
-template <int MT>
+// Weight box of one tile at K element k0 (128 rows x 128 bytes). gate_up maps are (K,
+// half, row, expert) with boxes of 64 (gate, up) row pairs; down maps are (K, rows).
 __device__ __forceinline__ void load_weights(const GateUpArgs &a, const CUtensorMap *m, void *dst, uint64_t *bar,
-                                             const Tile8 &t, int kb)
+                                             const Tile8 &t, int k0)
 {
-    tma_load_4d(dst, m, bar, kb * kBK, 0, t.fb * MT * 64, t.sh ? 0 : t.g);
+    tma_load_4d(dst, m, bar, k0, 0, t.fb * 64, t.sh ? 0 : t.g);
 }
 
-template <int MT>
 __device__ __forceinline__ void load_weights(const DownArgs &a, const CUtensorMap *m, void *dst, uint64_t *bar,
-                                             const Tile8 &t, int kb)
+                                             const Tile8 &t, int k0)
 {
-    tma_load_2d(dst, m, bar, kb * kBK, (t.sh ? 0 : t.g * a.H) + t.fb * MT * 128);
+    tma_load_2d(dst, m, bar, k0, (t.sh ? 0 : t.g * a.H) + t.fb * 128);
 }
 
-// Block scales of weight tile m at K slice kb (even rows, odd rows). gate_up tile m holds
-// gate rows f0 .. f0+63 (scale row block f0/128) interleaved with up rows I+f0 .. (block
-// (I+f0)/128), f0 = (fb*MT + m)*64; scales [E, 2I/128, H/128].
-template <int MT>
-__device__ __forceinline__ float2 tile_scales(const GateUpArgs &a, const Tile8 &t, int m, int kb)
+// Block scales of a routed tile at 128-wide K block kblk: (even rows, odd rows). gate_up
+// tile fb holds gate rows f0 .. f0+63 (scale row block f0/128) interleaved with up rows
+// I+f0 .. (block (I+f0)/128), f0 = 64 fb; scales [E, 2I/128, H/128]. down tile fb holds
+// rows 128 fb .. +127, one scale row block; scales [E, H/128, I/128].
+__device__ __forceinline__ float2 tile_scales(const GateUpArgs &a, const Tile8 &t, int kblk)
 {
     const int nbr = a.I / 64, nbc = a.H / 128;
-    const float *srow = a.w_scale + static_cast<int64_t>(t.g) * nbr * nbc + kb / 2;
-    const int f0 = (t.fb * MT + m) * 64;
+    const float *srow = a.w_scale + static_cast<int64_t>(t.g) * nbr * nbc + kblk;
+    const int f0 = t.fb * 64;
     return make_float2(__ldg(srow + static_cast<int64_t>(f0 / 128) * nbc),
                        __ldg(srow + static_cast<int64_t>((a.I + f0) / 128) * nbc));
 }
 
-// down tile m holds output rows (fb*MT + m)*128 .. +127, one scale row block; scales
-// [E, H/128, I/128].
-template <int MT>
-__device__ __forceinline__ float2 tile_scales(const DownArgs &a, const Tile8 &t, int m, int kb)
+__device__ __forceinline__ float2 tile_scales(const DownArgs &a, const Tile8 &t, int kblk)
 {
     const int nbr = a.H / 128, nbc = a.I / 128;
-    const float v = __ldg(a.w_scale + (static_cast<int64_t>(t.g) * nbr + t.fb * MT + m) * nbc + kb / 2);
+    const float v = __ldg(a.w_scale + (static_cast<int64_t>(t.g) * nbr + t.fb) * nbc + kblk);
     return make_float2(v, v);
 }
 
-template <int MT>
 __device__ __forceinline__ void epilogue8(const GateUpArgs &a, uint32_t tmem_tile, int bn, const Tile8 &t, int q,
                                           int lane)
 {
-    gate_up_epilogue<MT>(tmem_tile, bn, static_cast<int64_t>(t.fb) * MT * 64, t.ntok, t.row0, t.sh ? a.h_sh : a.h,
-                         t.sh ? a.Is : a.I, t.sh ? a.lim_s : a.lim_r, q, lane);
+    gate_up_epilogue<1>(tmem_tile, bn, static_cast<int64_t>(t.fb) * 64, t.ntok, t.row0, t.sh ? a.h_sh : a.h,
+                        t.sh ? a.Is : a.I, t.sh ? a.lim_s : a.lim_r, q, lane);
 }
 
-template <int MT>
 __device__ __forceinline__ void epilogue8(const DownArgs &a, uint32_t tmem_tile, int bn, const Tile8 &t, int q,
                                           int lane)
 {
-    down_epilogue<MT>(tmem_tile, bn, static_cast<int64_t>(t.fb) * MT * 128, t.ntok, t.row0, t.sh, a, q, lane);
+    down_epilogue<1>(tmem_tile, bn, static_cast<int64_t>(t.fb) * 128, t.ntok, t.row0, t.sh, a, q, lane);
 }
 
 // ------------------------------------------------------------------------------------
-// Both GEMMs with E4M3 routed weights. Maps: m_w (E4M3 codes), m_wsh (BF16 shared
-// weights), m_tok (routed token rows: x_perm or h), m_tok_sh (shared token rows: x or
-// h_sh). Stage `it` uses staging slot it % SW and converted slot it % SA.
-template <class Args, int BN, int SA, int SW, int MT>
+// Both GEMMs with E4M3 routed weights. Maps: m_w (E4M3 codes, 128-byte swizzled boxes of
+// 128 K), m_wsh (BF16 shared weights, 64 K), m_tok (routed token rows: x_perm or h),
+// m_tok_sh (shared token rows: x or h_sh). Stage `it` uses staging slot it % SW and TMEM
+// operand slot it % SA; K elements past a tile's extent are zero-filled by TMA for both
+// operands.
+template <class Args, int BN, int SW, int SA>
 __global__ void __launch_bounds__(kThreads8, 1)
     gemm_fp8_kernel(const __grid_constant__ CUtensorMap m_w, const __grid_constant__ CUtensorMap m_wsh,
                     const __grid_constant__ CUtensorMap m_tok, const __grid_constant__ CUtensorMap m_tok_sh,
                     const Args a, const WaitCfg wc)
 {
-    using G = Geo8<BN, SA, SW, MT>;
+    using G = Geo8<BN, SW, SA>;
     extern __shared__ uint8_t smem_raw[];
     Ring8 r;
-    uint8_t *smem = ring8_setup<G, SA, SW>(smem_raw, r);
+    uint8_t *smem = ring8_setup<G, SW, SA>(smem_raw, r);
     const uint32_t tmem = *r.holder;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int tiles = tile_count<MT>(a);
-    uint8_t *const conv_ring = smem;
-    uint8_t *const stage_ring = smem + G::kQOff;
+    const int tiles = tile_count(a);
 
     if (warp == 0) {
-        // staging producer: E4M3 weights (routed) and token rows, one slot per K slice
+        // staging producer: one weight box and one (shared) or two (routed) token slices
         if (lane == 0) {
             tma_prefetch_map(&m_w);
+            tma_prefetch_map(&m_wsh);
             tma_prefetch_map(&m_tok);
             tma_prefetch_map(&m_tok_sh);
             int it = 0;
             bool stop = false;
             for (int tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x) {
-                const Tile8 t = tile_of<MT>(a, tile);
-                for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+                const Tile8 t = tile_of(a, tile);
+                const int nsl = t.sh ? 1 : 2;
+                for (int st = 0; st < t.stages(); ++st, ++it) {
                     const int s = it % SW;
                     if (!mbar_wait(&r.qempty[s], ((it / SW) & 1) ^ 1, wc, r.abort_flag)) {
                         stop = true;
                         break;
                     }
-                    uint8_t *slot = stage_ring + s * G::kQSlotBytes;
-                    mbar_arrive_expect_tx(&r.qfull[s], G::kBBytes + (t.sh ? 0u : G::kQBytes));
-                    if (!t.sh)
-                        load_weights<MT>(a, &m_w, slot, &r.qfull[s], t, kb);
-                    tma_load_2d(slot + G::kQBytes, t.sh ? &m_tok_sh : &m_tok, &r.qfull[s], kb * kBK, t.row0);
+                    uint8_t *slot = smem + s * G::kSlotBytes;
+                    const int k0 = st * t.stage_k();
+                    mbar_arrive_expect_tx(&r.qfull[s], kWBytes + nsl * G::kBSlice);
+                    load_weights(a, t.sh ? &m_wsh : &m_w, slot, &r.qfull[s], t, k0);
+                    for (int kc = 0; kc < nsl; ++kc)
+                        tma_load_2d(slot + kWBytes + kc * G::kBSlice, t.sh ? &m_tok_sh : &m_tok, &r.qfull[s],
+                                    k0 + kc * kBK, t.row0);
                 }
             }
             drain_ring(r.qfull, SW, it, wc);
         }
-    } else if (warp == 10) {
-        // shared-expert BF16 weights straight into the converted ring; routed slots get a
-        // plain arrival so every converted slot completes one afull phase per stage
-        if (lane == 0) {
-            tma_prefetch_map(&m_wsh);
-            int it = 0;
-            bool stop = false;
-            for (int tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x) {
-                const Tile8 t = tile_of<MT>(a, tile);
-                for (int kb = 0; kb < t.nkb; ++kb, ++it) {
-                    const int s = it % SA;
-                    if (!mbar_wait(&r.aempty[s], ((it / SA) & 1) ^ 1, wc, r.abort_flag)) {
-                        stop = true;
-                        break;
-                    }
-                    if (t.sh) {
-                        mbar_arrive_expect_tx(&r.afull[s], G::kABytes);
-                        load_weights<MT>(a, &m_wsh, conv_ring + s * G::kABytes, &r.afull[s], t, kb);
-                    } else {
-                        mbar_arrive(&r.afull[s]);
-                    }
-                }
-            }
-            drain_ring(r.afull, SA, it, wc);
-        }
     } else if (warp >= 6) {
-        // converters: stage `it` is ready for the MMA once its staged bytes landed and
-        // (routed) its weight tile is converted or (shared) its BF16 tile landed
-        const int ct = threadIdx.x - 192;
+        // converters: group gi takes the stages with it % 2 == gi; thread = weight row j
+        const int gi = (warp - 6) >> 2;
+        const int j = 32 * (warp & 3) + lane;
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
         int it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-            const Tile8 t = tile_of<MT>(a, tile);
-            for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+            const Tile8 t = tile_of(a, tile);
+            const int nkblk = t.K / 128;
+            // lane l caches the scales of K block base + l (reloaded every 32 blocks)
+            int base = -32;
+            float se = 0.0f, so = 0.0f;
+            for (int st = 0; st < t.stages(); ++st, ++it) {
+                if ((it & 1) != gi)
+                    continue;
                 const int sa = it % SA, sq = it % SW;
+                if (!t.sh && st - base >= 32) {
+                    base = st;
+                    if (base + lane < nkblk) {
+                        const float2 sc = tile_scales(a, t, base + lane);
+                        se = sc.x;
+                        so = sc.y;
+                    }
+                }
                 ok = warp_wait(&r.aempty[sa], ((it / SA) & 1) ^ 1, wc, r.abort_flag) &&
-                     warp_wait(&r.qfull[sq], (it / SW) & 1, wc, r.abort_flag) &&
-                     warp_wait(&r.afull[sa], (it / SA) & 1, wc, r.abort_flag);
+                     warp_wait(&r.qfull[sq], (it / SW) & 1, wc, r.abort_flag);
                 if (!ok)
                     break;
-                if (!t.sh) {
-                    const uint8_t *q = stage_ring + sq * G::kQSlotBytes;
-                    uint8_t *dst = conv_ring + sa * G::kABytes;
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        const float2 sc = tile_scales<MT>(a, t, m, kb);
-                        convert_tile(q + m * kQTileBytes, dst + m * kATileBytes, sc.x, sc.y, ct);
-                    }
-                    fence_proxy_async_smem();  // generic-proxy stores -> the MMA's async-proxy reads
+                tc_fence_after();  // the MMA that read this operand slot has completed
+                const uint8_t *w = smem + sq * G::kSlotBytes;
+                const uint32_t taddr = lane_addr + G::kAOff + sa * kACols;
+                if (t.sh) {
+                    copy_row_bf16(w, j, taddr);
+                } else {
+                    const float s_even = __shfl_sync(0xFFFFFFFFu, se, st - base);
+                    const float s_odd = __shfl_sync(0xFFFFFFFFu, so, st - base);
+                    convert_row_e4m3(w, j, taddr, split_scale((j & 1) ? s_odd : s_even));
                 }
+                tmem_store_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&r.conv[sa]);
             }
         }
     } else if (warp == 1) {
-        // MMA: converted weights (A) x staged token rows (B); one commit frees both slots
+        // MMA: A (weights) from the TMEM operand slot, B (token rows) from the staging slot
         if (lane == 0) {
             int it = 0, tc = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
-                const Tile8 t = tile_of<MT>(a, tile);
+                const Tile8 t = tile_of(a, tile);
                 const int buf = tc & 1;
                 if (!mbar_wait(&r.acce[buf], ((tc >> 1) & 1) ^ 1, wc, r.abort_flag))
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem + buf * G::kBufCols;
                 const uint32_t idesc = idesc_bf16_f32(128, (t.ntok + 15) & ~15);
-                for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+                const int nks = t.stage_k() / 16;
+                for (int st = 0; st < t.stages(); ++st, ++it) {
                     const int sa = it % SA, sq = it % SW;
-                    if (!mbar_wait(&r.conv[sa], (it / SA) & 1, wc, r.abort_flag)) {
+                    if (!mbar_wait(&r.conv[sa], (it / SA) & 1, wc, r.abort_flag) ||
+                        !mbar_wait(&r.qfull[sq], (it / SW) & 1, wc, r.abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(conv_ring + sa * G::kABytes);
-                    const uint64_t bd = sdesc_kmajor_sw128(smem_u32(stage_ring + sq * G::kQSlotBytes) + G::kQBytes);
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) {
-                            const uint64_t ad = sdesc_kmajor_sw128(a_addr + m * kATileBytes);
-                            umma_bf16(d + m * BN, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
-                        }
+                    const uint32_t a_col = tmem + G::kAOff + sa * kACols;
+                    const uint32_t b_addr = smem_u32(smem + sq * G::kSlotBytes) + kWBytes;
+                    for (int ks = 0; ks < nks; ++ks) {
+                        const uint64_t bd = sdesc_kmajor_sw128(b_addr + (ks >> 2) * G::kBSlice) + 2 * (ks & 3);
+                        umma_bf16_ta(d, a_col + 8 * ks, bd, idesc, (st | ks) != 0);
                     }
                     umma_commit(&r.aempty[sa]);
                     umma_commit(&r.qempty[sq]);
@@ -406,17 +424,17 @@ __global__ void __launch_bounds__(kThreads8, 1)
             umma_commit(r.drain);
             mbar_wait_drain(r.drain, 0, wc);
         }
-    } else {
+    } else if (warp >= 2) {
         // warps 2..5: epilogue
         const int q = warp & 3;
         int tc = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
-            const Tile8 t = tile_of<MT>(a, tile);
+            const Tile8 t = tile_of(a, tile);
             const int buf = tc & 1;
             if (!warp_wait(&r.accf[buf], (tc >> 1) & 1, wc, r.abort_flag))
                 break;
             tc_fence_after();
-            epilogue8<MT>(a, tmem + buf * G::kBufCols, BN, t, q, lane);
+            epilogue8(a, tmem + buf * G::kBufCols, BN, t, q, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -426,12 +444,12 @@ __global__ void __launch_bounds__(kThreads8, 1)
     ring8_teardown<G>(tmem);
 }
 
-template <class Args, int BN, int SA, int SW, int MT>
+template <class Args, int BN, int SW, int SA>
 cudaError_t launch8(int grid, cudaStream_t stream, const CUtensorMap &m0, const CUtensorMap &m1,
                     const CUtensorMap &m2, const CUtensorMap &m3, const Args &a, const WaitCfg &wc)
 {
-    constexpr int smem = static_cast<int>(Geo8<BN, SA, SW, MT>::kSmemBytes);
-    auto kernel = gemm_fp8_kernel<Args, BN, SA, SW, MT>;
+    constexpr int smem = static_cast<int>(Geo8<BN, SW, SA>::kSmemBytes);
+    auto kernel = gemm_fp8_kernel<Args, BN, SW, SA>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
@@ -441,16 +459,16 @@ cudaError_t launch8(int grid, cudaStream_t stream, const CUtensorMap &m0, const 
 
 }  // namespace
 
-// Decode-sized calls: 32-row chunks; 12 KB staging slots (8 KB E4M3 + 4 KB tokens), 12
-// deep (96 KB of weight bytes in flight per SM), 4 converted slots of 16 KB. Prefill:
-// 128-row chunks; 24 KB staging slots, 7 deep; 3 converted slots.
+// Decode-sized calls: 32-row chunks; staging slots of 24 KB (16 KB weights + two 4 KB
+// token slices), 9 deep (144 KB of E4M3 bytes in flight per SM); 4 TMEM operand slots.
+// Prefill: 128-row chunks; 48 KB staging slots, 4 deep; 4 TMEM operand slots.
 cudaError_t launch_gate_up_fp8(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
                                const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
                                const GemmConfig &c, cudaStream_t stream)
 {
     if (c.cap == 32)
-        return launch8<GateUpArgs, 32, 4, 12, 1>(grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
-    return launch8<GateUpArgs, 128, 3, 7, 1>(grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
+        return launch8<GateUpArgs, 32, 9, 4>(grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
+    return launch8<GateUpArgs, 128, 4, 4>(grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
 }
 
 cudaError_t launch_down_fp8(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
@@ -458,8 +476,8 @@ cudaError_t launch_down_fp8(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh
                             const GemmConfig &c, cudaStream_t stream)
 {
     if (c.cap_d == 32)
-        return launch8<DownArgs, 32, 4, 12, 1>(grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
-    return launch8<DownArgs, 128, 3, 7, 1>(grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
+        return launch8<DownArgs, 32, 9, 4>(grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
+    return launch8<DownArgs, 128, 4, 4>(grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
 }
 
 }  // namespace moe

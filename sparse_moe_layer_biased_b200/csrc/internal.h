@@ -91,6 +91,7 @@ inline GemmConfig gemm_config_fp8(int64_t T, int64_t k, int64_t E)
         return {32, 1, 32, 1, 0};
     return {128, 1, 128, 1, 0};
 }
+
 // Upper bound on the chunk count of one table: ceil(n / cap) <= n / cap + 1 per group.
 inline int64_t max_chunks(int64_t T, int64_t k, int64_t E, int64_t cap)
 {

@@ -113,35 +113,36 @@ bool map_gate_up(CUtensorMap *m, const void *base, int64_t H, int64_t Iw, int64_
     return encode_bf16(m, base, 4, dims, strides, box);
 }
 
-// E4M3 code tensor maps (one byte per element, no swizzle: the converter warps re-lay the
-// tile out), 64-byte inner box.
+// E4M3 code tensor maps (one byte per element), inner box of `inner` = 128 bytes, 128-byte
+// swizzle (converter threads read one row each without bank conflicts).
 bool encode_u8(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
                const cuuint32_t *box)
 {
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank),
                                 const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 // E4M3 gate_up codes [E, 2*Iw, H] viewed as (H, half, row, expert) like map_gate_up.
-bool map_gate_up_u8(CUtensorMap *m, const void *base, int64_t H, int64_t Iw, int64_t G, uint32_t feats)
+bool map_gate_up_u8(CUtensorMap *m, const void *base, int64_t H, int64_t Iw, int64_t G, uint32_t feats,
+                    uint32_t inner)
 {
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(H), 2, static_cast<cuuint64_t>(Iw),
                                 static_cast<cuuint64_t>(G)};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(Iw * H), static_cast<cuuint64_t>(H),
                                    static_cast<cuuint64_t>(2 * Iw * H)};
-    const cuuint32_t box[4] = {64, 2, feats, 1};
+    const cuuint32_t box[4] = {inner, 2, feats, 1};
     return encode_u8(m, base, 4, dims, strides, box);
 }
 
-bool map_rows_u8(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, uint32_t box_rows)
+bool map_rows_u8(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, uint32_t box_rows, uint32_t inner)
 {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
-    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t box[2] = {inner, box_rows};
     return encode_u8(m, base, 2, dims, strides, box);
 }
 
@@ -271,8 +272,10 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     const uint32_t drows = static_cast<uint32_t>(128 * cfg.mt_d);
     CUtensorMap tm_w, tm_wsh, tm_xp, tm_x, tm_wd, tm_wdsh, tm_h, tm_hsh;
     const int64_t EH = static_cast<int64_t>(d.E) * d.H;
-    bool ok = (fp8 ? map_gate_up_u8(&tm_w, W.gu, d.H, d.I, d.E, feats) : map_gate_up(&tm_w, W.gu, d.H, d.I, d.E, feats)) &&
-              (fp8 ? map_rows_u8(&tm_wd, W.d, d.I, EH, drows) : map_rows(&tm_wd, W.d, d.I, EH, drows)) &&
+    const uint32_t inner8 = 128;  // one 128-wide scale block of E4M3 codes per stage
+    bool ok = (fp8 ? map_gate_up_u8(&tm_w, W.gu, d.H, d.I, d.E, feats, inner8)
+                   : map_gate_up(&tm_w, W.gu, d.H, d.I, d.E, feats)) &&
+              (fp8 ? map_rows_u8(&tm_wd, W.d, d.I, EH, drows, inner8) : map_rows(&tm_wd, W.d, d.I, EH, drows)) &&
               map_gate_up(&tm_wsh, W.sh_gu, d.H, d.Is, 1, feats) && map_rows(&tm_xp, x_perm, d.H, Tk, brows) &&
               map_rows(&tm_x, x, d.H, d.T, brows) && map_rows(&tm_wdsh, W.sh_d, d.Is, d.H, drows) &&
               map_rows(&tm_h, h, d.I, Tk, brows) && map_rows(&tm_hsh, h_sh, d.Is, d.T, brows);

@@ -24,6 +24,10 @@ SHAPES = {
     "tiny": WORKLOADS["tiny"],
     "decode": LayerShape("fp8_decode", T=24, H=512, E=40, k=8, I=256, Is=128, limit_routed=0.25, seed=51,
                          weight_std=0.03),
+    # decode stages span 128 K elements: the shared expert's down GEMM (K = Is = 192) ends
+    # in a half-empty stage that TMA fills with zeros for both operands
+    "decode_is192": LayerShape("fp8_decode_is192", T=24, H=512, E=40, k=8, I=256, Is=192, limit_shared=0.25,
+                               seed=55, weight_std=0.03),
     # prefill-sized: 128-row chunks, several K blocks, ragged chunk tails, Is not a multiple of 128
     "prefill": LayerShape("fp8_prefill", T=300, H=512, E=12, k=4, I=256, Is=192, limit_routed=0.25,
                           limit_shared=0.125, seed=52, weight_std=0.03),
