@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--routing", default="router", choices=["router", "balanced"],
                     help="router: full layer; balanced: fixed round-robin routing through moe_forward_with_ids "
                          "(fake balanced static expert routing)")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
+                    help="routed expert weights: bf16, or FP8 E4M3 with 128x128 block scales (moe_forward_fp8)")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling runs)")
     return ap.parse_args()
@@ -217,13 +219,42 @@ def run_reference(args, shape):
     print(json.dumps(line), flush=True)
 
 
-def gate_up_bytes(shape, counts):
+# DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu capture
+# (profiles/dram_gate_up_down_step35_prefill.md). A figure holds only for the kernel sources
+# it was taken from: the lookup returns None once any file under csrc/ changes.
+PROFILED_TRAFFIC = {
+    ("step35_prefill", "bf16"): {"bytes": 5615333888 + 86790144,
+                                 "csrc_sha256": "a95344f822829ab2f8dd440a746a3cd056fea661d4dbd6c9428dce9038cec81b",
+                                 "source": "profiles/dram_gate_up_down_step35_prefill.md"},
+}
+
+
+def csrc_digest() -> str:
+    import hashlib
+    d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "sparse_moe_layer_biased_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(shape_name: str, weights: str):
+    e = PROFILED_TRAFFIC.get((shape_name, weights))
+    if e is None or e["csrc_sha256"] != csrc_digest():
+        return None
+    return e["bytes"]
+
+
+def gate_up_bytes(shape, counts, fp8=False):
     """Algorithmic HBM bytes of one gate_up launch: weights of every expert that received
-    tokens (2I x H bf16 each) + shared gate_up + permuted token rows + shared token rows +
-    hidden activations written."""
+    tokens (2I x H, bf16 or E4M3 codes plus one fp32 scale per 128x128 block) + shared
+    gate_up (bf16) + permuted token rows + shared token rows + hidden activations written."""
     touched = int((counts[: shape.E] > 0).sum())
     T, H, k, I, Is = shape.T, shape.H, shape.k, shape.I, shape.Is
-    w = touched * 2 * I * H * 2 + 2 * Is * H * 2
+    per_expert = 2 * I * H + (2 * I // 128) * (H // 128) * 4 if fp8 else 2 * I * H * 2
+    w = touched * per_expert + 2 * Is * H * 2
     acts = T * k * H * 2 + T * H * 2
     out = T * k * I * 2 + T * Is * 2
     return w + acts + out, touched
@@ -235,9 +266,12 @@ def run_b200(args, shape):
     import torch.distributed as dist
 
     from sparse_moe_layer_biased_b200 import _abi
-    from sparse_moe_layer_biased_b200.inputs import draw
+    from sparse_moe_layer_biased_b200.inputs import draw, draw_fp8
     from sparse_moe_layer_biased_b200.layer import MoeLayer
 
+    fp8 = args.weights == "fp8"
+    if fp8 and args.routing == "balanced":
+        raise SystemExit("--routing balanced replays routing through the BF16 entry point only")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -252,7 +286,7 @@ def run_b200(args, shape):
         if world > 1:
             dist.barrier()
 
-    inp = draw(shape, device="cuda")
+    inp = (draw_fp8 if fp8 else draw)(shape, device="cuda")
     layer = MoeLayer(shape, inp, deterministic=args.deterministic)
     x = inp["x"]
     y = torch.empty((shape.T, shape.H), dtype=torch.float32, device="cuda")
@@ -332,11 +366,13 @@ def run_b200(args, shape):
                "h2d_bytes_per_step": shape.T * shape.H * 2, "d2h_bytes_per_step": shape.T * shape.H * 4}
 
     peaks, peak_kind = load_peaks()
-    gbytes, touched = gate_up_bytes(shape, counts)
+    gbytes, touched = gate_up_bytes(shape, counts, fp8)
     gate_ms = stage_ms["gate_up"]
     achieved = gbytes / (gate_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "gate_up_kernel", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+    kernel = "gemm_fp8_kernel<GateUpArgs>" if fp8 else "gate_up_kernel"
+    roofline = {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": profiled_traffic(shape.name, args.weights),
                 "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": gbytes, "launch_ms": gate_ms,
                 "touched_experts": touched}
     flops = shape.flops_per_token * shape.T
@@ -349,6 +385,7 @@ def run_b200(args, shape):
         "config": workload_config(shape, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                                           "l2": "inputs larger than L2 (expert weights streamed every step)",
                                           "routing": args.routing,
+                                          "weights": "fp8_e4m3_block128x128" if fp8 else "bf16",
                                           "deterministic": bool(args.deterministic)}),
         "roofline": roofline,
         "tensor": {"achieved_tflops": flops / (step_ms / 1e3) / 1e12,
@@ -358,7 +395,7 @@ def run_b200(args, shape):
         "e2e": e2e,
         "gpu_launches": (nstage - (1 if args.routing == "balanced" else 0)) * args.steps,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         rate, n, dt, threads = cpu_oracle_sample(shape, inp, target_s=15.0)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": f"{n} tokens of {shape.name} through the CPU oracle forward "
