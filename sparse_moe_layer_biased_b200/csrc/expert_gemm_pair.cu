@@ -35,14 +35,16 @@ constexpr uint32_t kTokBoxBytes = kTokBoxRows * 128;
 // BN = token rows per pair tile (N of the pair MMA); each CTA holds BN/2 of them.
 // NB = accumulator buffers in TMEM (2: the epilogue of one tile overlaps the next tile's
 // mainloop; 1: larger tiles, the MMA waits for the epilogue between tiles).
-template <int BN, int S, int MT, int NB>
+// OUT = bytes of output staging after the ring (the down epilogue's bulk-reduction buffers).
+template <int BN, int S, int MT, int NB, int OUT = 0>
 struct PairGeo {
     static constexpr uint32_t kABytes = MT * kATileBytes;
     static constexpr uint32_t kBBytes = (BN / 2) * 128;
     static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-    static constexpr uint32_t kBarOff = S * kStageBytes;
-    static constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * S + 5);
-    static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
+    static constexpr uint32_t kOutOff = S * kStageBytes;
+    static constexpr uint32_t kBarOff = kOutOff + OUT;
+    static constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * S + 5);  // holder, abort flag, epilogue flags
+    static constexpr uint32_t kSmemBytes = kMiscOff + 48 + 1024;
     static constexpr uint32_t kBufCols = MT * BN;
     static constexpr uint32_t kTmemCols = NB * kBufCols <= 32 ? 32 : (NB * kBufCols <= 64 ? 64 : (NB * kBufCols <= 128 ? 128 : (NB * kBufCols <= 256 ? 256 : 512)));
     static_assert(NB * kBufCols <= 512, "accumulators exceed TMEM");
@@ -300,6 +302,64 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------------------------
 // down on pairs: a pair tile covers 2 * MT * 128 output features.
+//
+// Epilogue through shared memory and TMA bulk reductions: per block of 16 token columns,
+// the four epilogue warps write the weighted outputs of this CTA's MT * 128 features as 16
+// rows of MT * 512 bytes (one row per token) into a staging buffer; then one lane per token
+// issues a bulk reduce-add of its row into y[token] (or, in deterministic mode, a bulk store
+// into o_perm[slot]). Each output row thus takes one MT * 512-byte reduction at L2 instead
+// of MT * 4 reductions of 128 bytes. NOB staging buffers rotate so a block's reductions
+// overlap the next block's TMEM loads; a buffer is rewritten only after its bulk reads are
+// done. Named barrier 1 joins the 4 epilogue warps.
+constexpr int kOutTok = 16;
+
+template <int MT, int NOB>
+__device__ __forceinline__ void down_epilogue_bulk(uint32_t tmem_tile, int bn, int64_t feat0, int ntok, int64_t row0,
+                                                   bool sh, const DownArgs &a, int q, int lane, uint8_t *stage,
+                                                   int &ob)
+{
+    constexpr uint32_t kRowBytes = MT * 128 * 4;
+    constexpr uint32_t kBufBytes = kOutTok * kRowBytes;
+    const int64_t shared_base = static_cast<int64_t>(a.T) * a.k;
+    for (int cb = 0; cb < ntok; cb += kOutTok, ++ob) {
+        uint8_t *buf = stage + (ob % NOB) * kBufBytes;
+        // lane l (and l + 16) fetch the destination row and weight of column cb + l % 16
+        const int mycol = cb + (lane & (kOutTok - 1));
+        int64_t dst_row = 0;
+        float wgt = 0.0f;
+        if (mycol < ntok) {
+            const int64_t rr = row0 + mycol;
+            if (a.deterministic)
+                dst_row = sh ? shared_base + rr : rr;
+            else
+                dst_row = sh ? rr : a.perm_token[rr];
+            wgt = sh ? 1.0f : a.w_perm[rr];
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            float v[kOutTok];
+            tmem_load16(tmem_tile + m * bn + (static_cast<uint32_t>(q * 32) << 16) + cb, v);
+            float *col = reinterpret_cast<float *>(buf) + m * 128 + q * 32 + lane;
+#pragma unroll
+            for (int i = 0; i < kOutTok; ++i)
+                col[i * (kRowBytes / 4)] = __shfl_sync(0xFFFFFFFFu, wgt, i) * v[i];
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (q == 0 && lane < kOutTok) {
+            if (mycol < ntok) {
+                float *dst = a.out + dst_row * a.H + feat0;
+                if (a.deterministic)
+                    bulk_store(dst, buf + lane * kRowBytes, kRowBytes);
+                else
+                    bulk_reduce_add_f32(dst, buf + lane * kRowBytes, kRowBytes);
+                bulk_commit();
+            }
+            bulk_wait_read<NOB - 1>();  // the buffer written next is no longer being read
+        }
+        named_bar_sync(1, 128);
+    }
+}
 template <int MT>
 __device__ __forceinline__ void decode_down_pair(const DownArgs &a, int tile, int &g, int &row0, int &ntok, int &fb)
 {
@@ -312,13 +372,13 @@ __device__ __forceinline__ void decode_down_pair(const DownArgs &a, int tile, in
     ntok = c.z;
 }
 
-template <int BN, int S, int MT, int NB>
+template <int BN, int S, int MT, int NB, int NOB>
 __global__ void __launch_bounds__(kThreads, 1)
     down_pair_kernel(const __grid_constant__ CUtensorMap tm_wd, const __grid_constant__ CUtensorMap tm_wdsh,
                      const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_hsh,
                      const DownArgs a, const WaitCfg wc)
 {
-    using G = PairGeo<BN, S, MT, NB>;
+    using G = PairGeo<BN, S, MT, NB, NOB * kOutTok * MT * 512>;
     extern __shared__ uint8_t smem_raw[];
     PairRing r;
     uint8_t *smem = pair_setup<G, S>(smem_raw, r);
@@ -377,22 +437,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         const int q = warp & 3;
-        int tc = 0;
+        int tc = 0, ob = 0;
+        volatile int *epi_ok = reinterpret_cast<volatile int *>(smem + G::kMiscOff + 16);
         for (int tile = first; tile < tiles; tile += stride, ++tc) {
             int g, row0, ntok, fb;
             decode_down_pair<MT>(a, tile, g, row0, ntok, fb);
             const int buf = tc % NB;
-            if (!warp_wait(&r.accf[buf], (tc / NB) & 1, wc, r.abort_flag))
+            // The four warps agree on the wait's outcome before the barrier-synchronised
+            // epilogue, so a wait that expires in one warp cannot strand the others at a
+            // named barrier (flags double-buffered by tile parity).
+            const bool ok = warp_wait(&r.accf[buf], (tc / NB) & 1, wc, r.abort_flag);
+            if (lane == 0)
+                epi_ok[(tc & 1) * 4 + q] = ok ? 1 : 0;
+            named_bar_sync(1, 128);
+            const volatile int *f = epi_ok + (tc & 1) * 4;
+            if (!(f[0] && f[1] && f[2] && f[3]))
                 break;
             tc_fence_after();
             const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
-            down_epilogue<MT>(tmem + buf * G::kBufCols, BN, static_cast<int64_t>(wt0) * 128, ntok, row0, g == a.E,
-                              a, q, lane);
+            down_epilogue_bulk<MT, NOB>(tmem + buf * G::kBufCols, BN, static_cast<int64_t>(wt0) * 128, ntok, row0,
+                                        g == a.E, a, q, lane, smem + G::kOutOff, ob);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive_cluster(r.acce_leader + 8 * buf);
         }
+        if (q == 0 && lane < kOutTok)
+            bulk_wait<0>();  // this lane's reductions have landed before the CTA exits
     }
     pair_teardown<G>(tmem);
 }
@@ -424,9 +495,11 @@ cudaError_t launch_pairs(Kernel kernel, int smem, int grid, cudaStream_t stream,
 // gate_up: pair tiles of up to 256 token rows (128 per CTA) x 128 features, one weight
 // tile per CTA and stage (32 KB stages, 6 deep). Most experts of a prefill batch then need
 // one pass over their weights. down: 128 token rows x 512 output features, two weight
-// tiles per CTA and stage (40 KB stages, 5 deep). Both keep two TMEM accumulators.
+// tiles per CTA and stage (40 KB stages, 4 deep) and two 16 KB output staging buffers for
+// the bulk reductions. Both keep two TMEM accumulators.
 using GateUpPair = PairGeo<kPairCapGateUp, 6, kPairMtGateUp, 2>;
-using DownPair = PairGeo<kPairCapDown, 5, kPairMtDown, 2>;
+constexpr int kDownStages = 4, kDownOutBufs = 2;  // 4 x 40 KB ring + 2 x 16 KB output staging
+using DownPair = PairGeo<kPairCapDown, kDownStages, kPairMtDown, 2, kDownOutBufs * kOutTok * kPairMtDown * 512>;
 
 }  // namespace
 
@@ -442,7 +515,8 @@ cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wds
                              const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
                              cudaStream_t stream)
 {
-    return launch_pairs(down_pair_kernel<kPairCapDown, 5, kPairMtDown, 2>, static_cast<int>(DownPair::kSmemBytes),
+    return launch_pairs(down_pair_kernel<kPairCapDown, kDownStages, kPairMtDown, 2, kDownOutBufs>,
+                        static_cast<int>(DownPair::kSmemBytes),
                         grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
 }
 
