@@ -55,6 +55,11 @@ def lib():
                                           ctypes.c_int, ctypes.c_float, ctypes.c_float, _u16p, _i32p, _f64p,
                                           ctypes.POINTER(_vp), ctypes.POINTER(_vp), _u16p, _u16p, _f64p]
         L.oracle_experts_f32w.restype = ctypes.c_int
+        L.oracle_backward.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                      _u16p, _u16p, _f32p, _u16p, _u16p, _u16p, _u16p, _f32p, _f64p, _f64p, _f64p,
+                                      _f64p, _f64p, _f64p, _i32p, _f64p, _f64p]
+        L.oracle_backward.restype = ctypes.c_int
         L.oracle_forward_dense.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                            ctypes.c_float, ctypes.c_float, _u16p, _u16p, _f32p, _u16p,
@@ -305,6 +310,29 @@ def forward_fp8_tokens(x_rows, Wr, bias, Wgu_q, Wgu_s, Wd_q, Wd_s, Wsh_gu, Wsh_d
     return {"y": y, "idx": r["idx"], "w": r["w"], "margin": r["margin"]}
 
 
+def backward(x, Wr, bias, W_gate_up, W_down, Wsh_gu, Wsh_d, dy, *, k, scale=3.0, norm=True, limit_routed=0.0,
+             limit_shared=0.0):
+    """Gradients of the layer for upstream gradient dy [T, H] (fp32): dict(dx [T, H], dWr [E, H],
+    dW_gate_up [E, 2I, H], dW_down [E, H, I], dWsh_gate_up [2Is, H], dWsh_down [H, Is]) in
+    float64, plus the forward's idx, w and dw = dLoss/dw [T, k]. The router bias gets no
+    gradient (selection only). Stacked weights; small shapes only (one pass over all tokens)."""
+    x, Wr, W_gate_up, W_down = _u16(x), _u16(Wr), _u16(W_gate_up), _u16(W_down)
+    Wsh_gu, Wsh_d = _u16(Wsh_gu), _u16(Wsh_d)
+    bias = np.ascontiguousarray(bias, np.float32)
+    dy = np.ascontiguousarray(dy, np.float32)
+    T, H = x.shape
+    E = Wr.shape[0]
+    I = W_gate_up.shape[1] // 2
+    Is = Wsh_gu.shape[0] // 2
+    out = {"dx": np.empty((T, H)), "dWr": np.empty((E, H)), "dW_gate_up": np.empty((E, 2 * I, H)),
+           "dW_down": np.empty((E, H, I)), "dWsh_gate_up": np.empty((2 * Is, H)), "dWsh_down": np.empty((H, Is)),
+           "idx": np.empty((T, k), np.int32), "w": np.empty((T, k)), "dw": np.empty((T, k))}
+    lib().oracle_backward(T, H, E, k, I, Is, scale, int(bool(norm)), limit_routed, limit_shared, x, Wr, bias,
+                          W_gate_up, W_down, Wsh_gu, Wsh_d, dy, out["dx"], out["dWr"], out["dW_gate_up"],
+                          out["dW_down"], out["dWsh_gate_up"], out["dWsh_down"], out["idx"], out["w"], out["dw"])
+    return out
+
+
 __all__ = ["lib", "num_threads", "router_logits", "router_select", "router", "permute", "swiglu_hidden",
            "swiglu_mlp", "forward_tokens", "forward_given_routing", "forward_dense", "forward_full", "e4m3_values",
-           "dequant_block128", "experts_f32w", "forward_fp8_tokens"]
+           "dequant_block128", "experts_f32w", "forward_fp8_tokens", "backward"]

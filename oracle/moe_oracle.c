@@ -31,7 +31,9 @@
  *    biased score below every number (ties among NaNs by index), -0.0 equal to +0.0;
  *  - normalisation has no epsilon; if the selected scores sum to 0 every selected
  *    weight is scale/k; without normalisation the weight is scale*s;
- *  - margin = (k-th biased score) - ((k+1)-th biased score) in fp32, +inf when k = E.
+ *  - margin = (k-th biased score) - ((k+1)-th biased score) in fp32, +inf when k = E;
+ *  - backward (oracle_backward): no gradient through the top-k selection (the bias gets
+ *    none), clips pass the gradient at their boundary.
  *
  * Precision: inputs are bf16 bit patterns (decoded exactly). The router logit is the
  * dot product accumulated in double and rounded once to fp32 (the FP32 gate); the
@@ -502,5 +504,183 @@ int oracle_experts_f32w(int64_t ntok, int H, int E, int k, int I, int Is, float 
         free(hid);
         free(o);
     }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------
+ * Backward pass of the layer (the layer is trained: NeMo AutoModel Step-5-Preview page,
+ * benchmark recipe runs forward, backward and optimizer steps; miles page: BF16 training).
+ * The pages give no formulas; this is the chain rule on the forward above, with two
+ * readings: no gradient flows through the top-k selection (the selected set is a step
+ * function of the biased scores, so the router bias receives none and the logits only
+ * through the selected experts' weights), and a clip passes the gradient at its boundary
+ * (a == L, |u| == L), as an inclusive clamp does.
+ *
+ * Given dy = dLoss/dy [ntok, H] (fp32), with the forward's selection (ids e_j, scores s):
+ *   per selected (t, j), expert e = e_j, weight w_j:
+ *     g = Wg_e x, u = Wu_e x, a = silu(g), clipped a_c, u_c, h = a_c u_c, o = Wd_e h
+ *     dW_down_e += (w_j dy) h^T;  dh = w_j Wd_e^T dy;  dw_j = dy . o
+ *     da = dh u_c [a <= L],  du = dh a_c [-L <= u <= L]   (masks only when L > 0)
+ *     dg = da silu'(g),  silu'(g) = sig(g) (1 + g (1 - sig(g)))
+ *     dWg_e += dg x^T, dWu_e += du x^T,  dx += Wg_e^T dg + Wu_e^T du
+ *   the shared expert the same with weight 1 and no dw;
+ *   router, normalised (Z = sum of the k selected scores, c = scale): w_j = c s_j / Z,
+ *     ds_i = (c / Z) dw_i - (c / Z^2) sum_j dw_j s_j;  otherwise w_j = c s_j, ds_i = c dw_i;
+ *     dlogit_i = ds_i s_i (1 - s_i) for the selected experts, 0 for the others;
+ *     dWr[e] += dlogit_e x,  dx += sum_e dlogit_e Wr[e].
+ * Everything in double; weights stacked: W_gate_up [E, 2I, H] (gate rows first),
+ * W_down [E, H, I]. Outputs are overwritten. Returns 0.
+ */
+static void mlp_backward(int H, int Iw, const uint16_t *x_row, const uint16_t *Wgu, const uint16_t *Wd,
+                         double limit, double wgt, const float *dy_row, double *dWgu, double *dWd, double *dx_row,
+                         double *dw_out, double *hid, double *gpre, double *upre, double *dh)
+{
+    for (int i = 0; i < Iw; ++i) {
+        const uint16_t *wg = Wgu + (int64_t)i * H;
+        const uint16_t *wu = Wgu + (int64_t)(Iw + i) * H;
+        double g = 0.0, u = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double xv = bf(x_row[h]);
+            g += bf(wg[h]) * xv;
+            u += bf(wu[h]) * xv;
+        }
+        gpre[i] = g;
+        upre[i] = u;
+        double a = g / (1.0 + exp(-g)), uc = u;
+        if (limit > 0.0) {
+            if (a > limit)
+                a = limit;
+            if (uc > limit)
+                uc = limit;
+            if (uc < -limit)
+                uc = -limit;
+        }
+        hid[i] = a * uc;
+    }
+    /* dw = dy . (Wd h); dh = w Wd^T dy; dWd += (w dy) h^T */
+    double dw = 0.0;
+    for (int i = 0; i < Iw; ++i)
+        dh[i] = 0.0;
+    for (int f = 0; f < H; ++f) {
+        const uint16_t *wd = Wd + (int64_t)f * Iw;
+        const double d = (double)dy_row[f];
+        double o = 0.0;
+        for (int i = 0; i < Iw; ++i) {
+            o += bf(wd[i]) * hid[i];
+            dh[i] += bf(wd[i]) * d;
+        }
+        dw += d * o;
+        double *dwd = dWd + (int64_t)f * Iw;
+        for (int i = 0; i < Iw; ++i)
+            dwd[i] += wgt * d * hid[i];
+    }
+    if (dw_out)
+        *dw_out = dw;
+    for (int i = 0; i < Iw; ++i) {
+        const double g = gpre[i], u = upre[i];
+        const double sg = 1.0 / (1.0 + exp(-g));
+        const double a = g * sg;
+        double ac = a, uc = u, ma = 1.0, mu = 1.0;
+        if (limit > 0.0) {
+            if (a > limit) {
+                ac = limit;
+                ma = 0.0;
+            }
+            if (u > limit) {
+                uc = limit;
+                mu = 0.0;
+            } else if (u < -limit) {
+                uc = -limit;
+                mu = 0.0;
+            }
+        }
+        const double dhi = wgt * dh[i];
+        const double dg = dhi * uc * ma * sg * (1.0 + g * (1.0 - sg));
+        const double du = dhi * ac * mu;
+        const uint16_t *wg = Wgu + (int64_t)i * H;
+        const uint16_t *wu = Wgu + (int64_t)(Iw + i) * H;
+        double *dwg = dWgu + (int64_t)i * H;
+        double *dwu = dWgu + (int64_t)(Iw + i) * H;
+        for (int h = 0; h < H; ++h) {
+            const double xv = bf(x_row[h]);
+            dwg[h] += dg * xv;
+            dwu[h] += du * xv;
+            dx_row[h] += bf(wg[h]) * dg + bf(wu[h]) * du;
+        }
+    }
+}
+
+int oracle_backward(int64_t T, int H, int E, int k, int I, int Is, float scale, int norm, float limit_routed,
+                    float limit_shared, const uint16_t *x, const uint16_t *Wr, const float *bias,
+                    const uint16_t *W_gate_up, const uint16_t *W_down, const uint16_t *Wsh_gu,
+                    const uint16_t *Wsh_d, const float *dy, double *dx, double *dWr, double *dWgu, double *dWd,
+                    double *dWsh_gu, double *dWsh_d, int32_t *idx_out, double *w_out, double *dw_out)
+{
+    float *logits = (float *)malloc(sizeof(float) * (size_t)(T * E));
+    float *scores = (float *)malloc(sizeof(float) * (size_t)(T * E));
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T * k));
+    double *w = (double *)malloc(sizeof(double) * (size_t)(T * k));
+    double *dw = (double *)malloc(sizeof(double) * (size_t)(T * k));
+    oracle_router_logits(T, H, E, x, Wr, logits);
+    oracle_router_select(T, E, k, logits, bias, scale, norm, idx, NULL, w, NULL, scores);
+    memset(dx, 0, sizeof(double) * (size_t)(T * H));
+    memset(dWr, 0, sizeof(double) * (size_t)E * H);
+    memset(dWgu, 0, sizeof(double) * (size_t)E * 2 * I * H);
+    memset(dWd, 0, sizeof(double) * (size_t)E * H * I);
+    memset(dWsh_gu, 0, sizeof(double) * (size_t)2 * Is * H);
+    memset(dWsh_d, 0, sizeof(double) * (size_t)H * Is);
+    int Imax = I > Is ? I : Is;
+    double *buf = (double *)malloc(sizeof(double) * (size_t)4 * Imax);
+    /* experts, token by token in order (weight gradients accumulate in token order) */
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *xr = x + t * (int64_t)H;
+        const float *dyr = dy + t * (int64_t)H;
+        double *dxr = dx + t * (int64_t)H;
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[t * k + j];
+            mlp_backward(H, I, xr, W_gate_up + (int64_t)e * 2 * I * H, W_down + (int64_t)e * H * I, limit_routed,
+                         w[t * k + j], dyr, dWgu + (int64_t)e * 2 * I * H, dWd + (int64_t)e * H * I, dxr,
+                         &dw[t * k + j], buf, buf + Imax, buf + 2 * Imax, buf + 3 * Imax);
+        }
+        mlp_backward(H, Is, xr, Wsh_gu, Wsh_d, limit_shared, 1.0, dyr, dWsh_gu, dWsh_d, dxr, NULL, buf,
+                     buf + Imax, buf + 2 * Imax, buf + 3 * Imax);
+        /* router: selected experts only */
+        double Z = 0.0, sdw = 0.0;
+        for (int j = 0; j < k; ++j) {
+            const double s = scores[t * E + idx[t * k + j]];
+            Z += s;
+            sdw += dw[t * k + j] * s;
+        }
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[t * k + j];
+            const double s = scores[t * E + e];
+            double ds;
+            if (norm && Z > 0.0)
+                ds = (double)scale / Z * dw[t * k + j] - (double)scale / (Z * Z) * sdw;
+            else if (norm)
+                ds = 0.0; /* all selected scores underflowed: the weights are constant scale/k */
+            else
+                ds = (double)scale * dw[t * k + j];
+            const double dl = ds * s * (1.0 - s);
+            const uint16_t *wr = Wr + (int64_t)e * H;
+            double *dwr = dWr + (int64_t)e * H;
+            for (int h = 0; h < H; ++h) {
+                dwr[h] += dl * bf(xr[h]);
+                dxr[h] += dl * bf(wr[h]);
+            }
+        }
+    }
+    if (idx_out)
+        memcpy(idx_out, idx, sizeof(int32_t) * (size_t)(T * k));
+    if (w_out)
+        memcpy(w_out, w, sizeof(double) * (size_t)(T * k));
+    if (dw_out)
+        memcpy(dw_out, dw, sizeof(double) * (size_t)(T * k));
+    free(buf);
+    free(logits);
+    free(scores);
+    free(idx);
+    free(w);
+    free(dw);
     return 0;
 }
