@@ -174,6 +174,26 @@ MOE_API moe_status_t moe_forward_fp8(const moe_layer_desc *desc, const uint16_t 
                                      int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
                                      void *stream);
 
+/* Backward pass of the layer (the layer is trained: NeMo AutoModel Step-5-Preview page,
+ * benchmark recipe with forward, backward and optimizer steps; miles page: BF16 training).
+ * Given the forward's routing (topk_idx [T,k] int32, topk_w [T,k] fp32, e.g. the outputs of
+ * moe_forward) and dy = dLoss/dy [T,H] fp32, overwrites
+ *   dx [T,H], dWr [E,H], dW_gate_up [E,2I,H], dW_down [E,H,I], dWsh_gate_up [2Is,H],
+ *   dWsh_down [H,Is]   (all fp32, layouts of the corresponding forward tensors).
+ * Chain rule on the forward; no gradient flows through the top-k selection (the router
+ * bias gets none, so no dbias is produced), clips pass the gradient at their boundary.
+ * The router logits of the selected experts are recomputed in fp32. GEMM operands are bf16
+ * (dy, the pre-activation gradients and w*h are rounded to bf16), accumulation fp32.
+ * Requires I % 128 == 0 and Is % 128 == 0 (MOE_ERR_UNSUPPORTED), every pointer 16-byte
+ * aligned; workspace of moe_backward_workspace_size() bytes (about (T*k + 64*E + T) * (4*H
+ * + 14*I) bytes). T = 0 returns MOE_OK and writes nothing. */
+MOE_API moe_status_t moe_backward_workspace_size(const moe_layer_desc *desc, size_t *bytes);
+MOE_API moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr,
+                                  const uint16_t *W_gate_up, const uint16_t *W_down, const uint16_t *Wsh_gate_up,
+                                  const uint16_t *Wsh_down, const int32_t *topk_idx, const float *topk_w,
+                                  const float *dy, float *dx, float *dWr, float *dW_gate_up, float *dW_down,
+                                  float *dWsh_gate_up, float *dWsh_down, void *ws, size_t ws_bytes, void *stream);
+
 /* moe_forward without a caller-provided workspace. The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory at call time, such
  * as a serving runtime whose device memory is already handed to a fixed pool, a

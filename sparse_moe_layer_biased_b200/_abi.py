@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 # Every exported entry point; the header include/moe_b200.h declares exactly these.
 EXPORTS = ["moe_status_string", "moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events",
-           "moe_forward_noalloc", "moe_forward_with_ids", "moe_forward_fp8"]
+           "moe_forward_noalloc", "moe_forward_with_ids", "moe_forward_fp8", "moe_backward",
+           "moe_backward_workspace_size"]
 
 
 class MoeError(RuntimeError):
@@ -71,6 +72,8 @@ def lib():
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(vp), i32]
         L.moe_forward_with_ids.argtypes = [dp] + [vp] * 9 + [sz, vp]
         L.moe_forward_fp8.argtypes = [dp] + [vp] * 13 + [sz, vp]
+        L.moe_backward_workspace_size.argtypes = [dp, ctypes.POINTER(sz)]
+        L.moe_backward.argtypes = [dp] + [vp] * 16 + [sz, vp]
         L.moe_forward_with_ids.restype = i32
         L.moe_forward_noalloc.argtypes = [dp] + [vp] * 11
         L.moe_forward_noalloc.restype = i32
@@ -147,6 +150,21 @@ def moe_forward_fp8(desc, x, Wr, bias, W_gate_up_q, W_gate_up_scale, W_down_q, W
     _check("moe_forward_fp8", lib().moe_forward_fp8(
         ctypes.byref(desc), _p(x), _p(Wr), _p(bias), _p(W_gate_up_q), _p(W_gate_up_scale), _p(W_down_q),
         _p(W_down_scale), _p(Wsh_gate_up), _p(Wsh_down), _p(y), _p(topk_idx_out), _p(topk_w_out), _p(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_backward_workspace_size(desc) -> int:
+    out = ctypes.c_size_t(0)
+    _check("moe_backward_workspace_size", lib().moe_backward_workspace_size(ctypes.byref(desc), ctypes.byref(out)))
+    return int(out.value)
+
+
+def moe_backward(desc, x, Wr, W_gate_up, W_down, Wsh_gate_up, Wsh_down, topk_idx, topk_w, dy, dx, dWr, dW_gate_up,
+                 dW_down, dWsh_gate_up, dWsh_down, ws, stream=None):
+    """Gradients of the layer for the forward's routing and dy (all outputs overwritten)."""
+    _check("moe_backward", lib().moe_backward(
+        ctypes.byref(desc), _p(x), _p(Wr), _p(W_gate_up), _p(W_down), _p(Wsh_gate_up), _p(Wsh_down), _p(topk_idx),
+        _p(topk_w), _p(dy), _p(dx), _p(dWr), _p(dW_gate_up), _p(dW_down), _p(dWsh_gate_up), _p(dWsh_down), _p(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
 
 

@@ -141,6 +141,61 @@ cudaError_t launch_down_fp8(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh
                             const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
                             const GemmConfig &c, cudaStream_t stream);
 
+// ------------------------------------------------------------------------------------
+// Backward pass. Rows live in a padded permuted space: the shared group takes rows [0, T)
+// of a span of P_s = T rounded up to 64 rows, then routed group e occupies rows
+// [poff[e], poff[e] + count[e]) of a span rounded up to 64 rows; padding rows are zero in
+// x_pad / dy_pad, so the weight-gradient GEMMs reduce over whole 64-row K slices. chunks: tiles of <= kBwdCap valid rows (group, first
+// row, rows); wgroups: (group, first row, padded rows). hdr: [0] routed chunks, [1] all
+// chunks, [2] routed wgroups, [3] all wgroups.
+constexpr int kBwdCap = 128;
+constexpr int kBwdPad = 64;
+struct BwdArgs {
+    int T, H, E, k, I, Is;
+    float lim_r, lim_s;
+    int P_s;  // rows of the shared group's span = first routed row
+    const int4 *chunks;
+    const int4 *wgroups;
+    const int32_t *hdr;
+    const float *w_pad;      // [P] routing weight of the row (1 for shared rows, 0 for padding)
+    const int32_t *tok_pad;  // [P] token of the row (-1 for padding)
+    float *gu_r, *gu_s;      // pre-activations [rows - P_s, 2I] / [P_s, 2Is] fp32 (gate columns, then up)
+    uint16_t *dgu_r, *dgu_s;  // gradients of the pre-activations, same shapes, bf16
+    uint16_t *hw_r, *hw_s;    // w * h [rows - P_s, I] / [P_s, Is] bf16
+    float *dw_pad;            // [P] dLoss/dw of routed rows (accumulated)
+    float *dx;                // [T, H]
+    float *dWd, *dWgu, *dWsh_d, *dWsh_gu;
+};
+enum BwdMode { kBwdGU = 0, kBwdDH = 1, kBwdDX = 2, kBwdWD = 3, kBwdWGU = 4 };
+// Maps per mode (routed A, shared A, routed B, shared B):
+//   GU : W_gate_up / Wsh_gate_up (4-D gate/up interleave, K-major), x_pad, x_pad
+//   DH : W_down / Wsh_down as (I, rows) MN-major, dy_pad, dy_pad
+//   DX : W_gate_up / Wsh_gate_up as (H, rows) MN-major, dgu_r, dgu_s (K-major)
+//   WD : dy_pad (H, rows) MN-major (both), hw_r / hw_s (I, rows) MN-major
+//   WGU: dgu_r / dgu_s (2I, rows) MN-major, x_pad (H, rows) MN-major (both)
+cudaError_t launch_bwd_gemm(int mode, const CUtensorMap &a_r, const CUtensorMap &a_s, const CUtensorMap &b_r,
+                            const CUtensorMap &b_s, const BwdArgs &a, const WaitCfg &wc, int grid,
+                            cudaStream_t stream);
+// Padded layout + tile tables from the permutation's counts (one CTA).
+cudaError_t launch_bwd_layout(const int32_t *counts, int E, int T, int32_t *poff, int4 *chunks, int4 *wgroups,
+                              int32_t *hdr, cudaStream_t stream);
+// x_pad, dy_pad (bf16 of dy), w_pad, tok_pad from the forward's routing; padding rows zero.
+cudaError_t launch_bwd_gather(const uint16_t *x, const float *dy, const int32_t *topk_idx, const float *topk_w,
+                              const int32_t *slot_of, const int32_t *offsets, const int32_t *counts,
+                              const int32_t *poff, int T, int k, int E, int H, uint16_t *x_pad, uint16_t *dy_pad,
+                              float *w_pad, int32_t *tok_pad, cudaStream_t stream);
+// Router part: logits of the selected experts, dLoss/dlogit, dx = sum_j dlogit_j Wr[e_j]
+// (overwrites dx) and dlogit per padded row (dl_pad).
+cudaError_t launch_bwd_router(const uint16_t *x, const uint16_t *Wr, const int32_t *topk_idx, const int32_t *slot_of,
+                              const int32_t *offsets, const int32_t *poff, const float *dw_pad, int T, int k, int E,
+                              int H, float scale, int norm, float *dx, float *dl_pad, cudaStream_t stream);
+// Zeroes dW_gate_up[e] and dW_down[e] of routed experts with no tokens.
+cudaError_t launch_bwd_zero_untouched(const int32_t *counts, int E, int H, int I, float *dWgu, float *dWd,
+                                      cudaStream_t stream);
+// dWr[e] = sum of dl_pad[row] * x_pad[row] over group e's rows.
+cudaError_t launch_bwd_dwr(const uint16_t *x_pad, const float *dl_pad, const int32_t *poff, const int32_t *counts,
+                           int E, int H, float *dWr, cudaStream_t stream);
+
 cudaError_t launch_combine(const float *o_perm, const int32_t *slot_of, int T, int k, int H, float *y,
                            cudaStream_t stream);
 

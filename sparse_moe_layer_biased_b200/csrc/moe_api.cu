@@ -338,6 +338,62 @@ moe_status_t forward_routed(const moe_layer_desc &d, const DeviceInfo &di, const
     return st;
 }
 
+// ---------------------------------------------------------------- backward
+struct BwdLayout {
+    size_t counts, offsets, perm_token, slot_of, poff, chunks, wgroups, hdr, x_pad, dy_pad, w_pad, tok_pad, gu_r,
+        gu_s, dgu_r, dgu_s, hw_r, hw_s, dw_pad, dl_pad, total;
+    int64_t P_s, P_r_max, P_max;
+};
+
+// Sizes are upper bounds: each routed group pads fewer than 64 rows.
+BwdLayout bwd_layout(const moe_layer_desc &d)
+{
+    const size_t T = d.T, H = d.H, E = d.E, k = d.k, I = d.I, Is = d.Is;
+    BwdLayout L{};
+    L.P_s = (static_cast<int64_t>(T) + moe::kBwdPad - 1) / moe::kBwdPad * moe::kBwdPad;
+    L.P_r_max = static_cast<int64_t>(T * k + moe::kBwdPad * E);
+    L.P_max = L.P_s + L.P_r_max;
+    const size_t P = L.P_max, Pr = L.P_r_max, Ps = L.P_s;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += up256(bytes);
+        return o;
+    };
+    L.counts = take((E + 1) * 4);
+    L.offsets = take((E + 2) * 4);
+    L.perm_token = take((T * k + T) * 4);
+    L.slot_of = take(T * k * 4);
+    L.poff = take((E + 2) * 4);
+    L.chunks = take(((T * k + T) / moe::kBwdCap + E + 2) * 16);
+    L.wgroups = take((E + 1) * 16);
+    L.hdr = take(64);
+    L.x_pad = take(P * H * 2);
+    L.dy_pad = take(P * H * 2);
+    L.w_pad = take(P * 4);
+    L.tok_pad = take(P * 4);
+    L.gu_r = take(Pr * 2 * I * 4);
+    L.gu_s = take(Ps * 2 * Is * 4);
+    L.dgu_r = take(Pr * 2 * I * 2);
+    L.dgu_s = take(Ps * 2 * Is * 2);
+    L.hw_r = take(Pr * I * 2);
+    L.hw_s = take(Ps * Is * 2);
+    L.dw_pad = take(P * 4);
+    L.dl_pad = take(P * 4);
+    L.total = off;
+    return L;
+}
+
+moe_status_t check_bwd_desc(const moe_layer_desc *d)
+{
+    const moe_status_t st = check_desc(d);
+    if (st != MOE_OK)
+        return st;
+    if (d->I % 128 != 0 || d->Is % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -545,6 +601,104 @@ moe_status_t moe_forward_fp8(const moe_layer_desc *desc, const uint16_t *x, cons
         return st;
     const ExpertWeights W{W_gate_up_q, W_down_q, W_gate_up_scale, W_down_scale, Wsh_gate_up, Wsh_down};
     return forward_routed(*desc, di, x, idx, w, W, y, ws, s);
+}
+
+moe_status_t moe_backward_workspace_size(const moe_layer_desc *desc, size_t *bytes)
+{
+    if (!bytes)
+        return MOE_ERR_INVALID_ARG;
+    const moe_status_t st = check_bwd_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    *bytes = bwd_layout(*desc).total;
+    return MOE_OK;
+}
+
+moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr,
+                          const uint16_t *W_gate_up, const uint16_t *W_down, const uint16_t *Wsh_gate_up,
+                          const uint16_t *Wsh_down, const int32_t *topk_idx, const float *topk_w, const float *dy,
+                          float *dx, float *dWr, float *dW_gate_up, float *dW_down, float *dWsh_gate_up,
+                          float *dWsh_down, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status_t st = check_bwd_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->T == 0)
+        return MOE_OK;  // nothing to do (the weight gradients of an empty batch are not written)
+    const void *ptrs[] = {x, Wr, W_gate_up, W_down, Wsh_gate_up, Wsh_down, topk_idx, topk_w, dy, dx, dWr,
+                          dW_gate_up, dW_down, dWsh_gate_up, dWsh_down, ws};
+    for (const void *p : ptrs)
+        if (!p)
+            return MOE_ERR_INVALID_ARG;
+    for (const void *p : ptrs)
+        if (!aligned16(p))
+            return MOE_ERR_UNSUPPORTED;
+    const moe_layer_desc &d = *desc;
+    const BwdLayout L = bwd_layout(d);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t *counts = at<int32_t>(ws, L.counts), *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *perm_token = at<int32_t>(ws, L.perm_token), *slot_of = at<int32_t>(ws, L.slot_of);
+    int32_t *poff = at<int32_t>(ws, L.poff), *hdr = at<int32_t>(ws, L.hdr);
+    int4 *chunks = at<int4>(ws, L.chunks), *wgroups = at<int4>(ws, L.wgroups);
+    uint16_t *x_pad = at<uint16_t>(ws, L.x_pad), *dy_pad = at<uint16_t>(ws, L.dy_pad);
+    float *w_pad = at<float>(ws, L.w_pad), *dw_pad = at<float>(ws, L.dw_pad), *dl_pad = at<float>(ws, L.dl_pad);
+    int32_t *tok_pad = at<int32_t>(ws, L.tok_pad);
+    float *gu_r = at<float>(ws, L.gu_r), *gu_s = at<float>(ws, L.gu_s);
+    uint16_t *dgu_r = at<uint16_t>(ws, L.dgu_r), *dgu_s = at<uint16_t>(ws, L.dgu_s);
+    uint16_t *hw_r = at<uint16_t>(ws, L.hw_r), *hw_s = at<uint16_t>(ws, L.hw_s);
+    const int64_t E = d.E, H = d.H, I = d.I, Is = d.Is, P = L.P_max, Pr = L.P_r_max, Ps = L.P_s;
+
+    // tensor maps (rows of the padded buffers are upper bounds; tiles only touch filled rows)
+    CUtensorMap gu_a_r, gu_a_s, gu_b, dh_a_r, dh_a_s, dh_b, dx_a_r, dx_a_s, dx_b_r, dx_b_s, wd_a, wd_b_r, wd_b_s,
+        wg_a_r, wg_a_s, wg_b;
+    const bool ok = map_gate_up(&gu_a_r, W_gate_up, H, I, E, 64) && map_gate_up(&gu_a_s, Wsh_gate_up, H, Is, 1, 64) &&
+                    map_rows(&gu_b, x_pad, H, P, moe::kBwdCap) && map_rows(&dh_a_r, W_down, I, E * H, 64) &&
+                    map_rows(&dh_a_s, Wsh_down, Is, H, 64) && map_rows(&dh_b, dy_pad, H, P, moe::kBwdCap) &&
+                    map_rows(&dx_a_r, W_gate_up, H, E * 2 * I, 64) && map_rows(&dx_a_s, Wsh_gate_up, H, 2 * Is, 64) &&
+                    map_rows(&dx_b_r, dgu_r, 2 * I, Pr, moe::kBwdCap) &&
+                    map_rows(&dx_b_s, dgu_s, 2 * Is, Ps, moe::kBwdCap) && map_rows(&wd_a, dy_pad, H, P, 64) &&
+                    map_rows(&wd_b_r, hw_r, I, Pr, 64) && map_rows(&wd_b_s, hw_s, Is, Ps, 64) &&
+                    map_rows(&wg_a_r, dgu_r, 2 * I, Pr, 64) && map_rows(&wg_a_s, dgu_s, 2 * Is, Ps, 64) &&
+                    map_rows(&wg_b, x_pad, H, P, 64);
+    if (!ok)
+        return MOE_ERR_CUDA;
+    const moe::WaitCfg wc = wait_cfg(di);
+    moe::BwdArgs ba{d.T, d.H, d.E, d.k, d.I, d.Is, d.limit_routed, d.limit_shared, static_cast<int>(Ps), chunks,
+                    wgroups, hdr, w_pad, tok_pad, gu_r, gu_s, dgu_r, dgu_s, hw_r, hw_s, dw_pad, dx, dW_down,
+                    dW_gate_up, dWsh_down, dWsh_gate_up};
+    const moe::PermuteArgs pa{topk_idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, nullptr, nullptr,
+                              nullptr, nullptr, 0};
+    cudaError_t e = moe::launch_permute(pa, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_layout(counts, d.E, d.T, poff, chunks, wgroups, hdr, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_gather(x, dy, topk_idx, topk_w, slot_of, offsets, counts, poff, d.T, d.k, d.E, d.H,
+                                   x_pad, dy_pad, w_pad, tok_pad, s);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(dw_pad, 0, static_cast<size_t>(P) * 4, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_gemm(moe::kBwdGU, gu_a_r, gu_a_s, gu_b, gu_b, ba, wc, di.num_sms, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_gemm(moe::kBwdDH, dh_a_r, dh_a_s, dh_b, dh_b, ba, wc, di.num_sms, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_router(x, Wr, topk_idx, slot_of, offsets, poff, dw_pad, d.T, d.k, d.E, d.H, d.scale,
+                                   d.norm_expert_weight, dx, dl_pad, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_gemm(moe::kBwdDX, dx_a_r, dx_a_s, dx_b_r, dx_b_s, ba, wc, di.num_sms, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_zero_untouched(counts, d.E, d.H, d.I, dW_gate_up, dW_down, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_gemm(moe::kBwdWD, wd_a, wd_a, wd_b_r, wd_b_s, ba, wc, di.num_sms, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_gemm(moe::kBwdWGU, wg_a_r, wg_a_s, wg_b, wg_b, ba, wc, di.num_sms, s);
+    if (e == cudaSuccess)
+        e = moe::launch_bwd_dwr(x_pad, dl_pad, poff, counts, d.E, d.H, dWr, s);
+    return cuda_status(e);
 }
 
 moe_status_t moe_check_device(void)

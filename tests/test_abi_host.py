@@ -150,3 +150,21 @@ def test_fp8_validation():
     # I must be a multiple of 128 (gate and up rows start scale blocks), even with T = 0
     assert L.moe_forward_fp8(ctypes.byref(_desc(I=192)), *args, *tail, need, None) == 2
     assert L.moe_forward_fp8(ctypes.byref(_desc(T=0)), *([None] * 13), 0, None) == 0
+
+
+def test_backward_validation():
+    L = moe.lib()
+    d = _desc()
+    assert d.I % 128 == 0 and d.Is % 128 == 0
+    need = moe.moe_backward_workspace_size(d)
+    assert need > 0
+    args = [FAKE] * 15  # x .. dWsh_down
+    assert L.moe_backward(ctypes.byref(d), *args, FAKE, need - 1, None) == 3
+    a = list(args)
+    a[8] = None  # dy
+    assert L.moe_backward(ctypes.byref(d), *a, FAKE, need, None) == 1
+    a = list(args)
+    a[9] = FAKE + 4  # dx misaligned
+    assert L.moe_backward(ctypes.byref(d), *a, FAKE, need, None) == 2
+    assert L.moe_backward(ctypes.byref(_desc(I=192)), *args, FAKE, need, None) == 2
+    assert L.moe_backward(ctypes.byref(_desc(T=0)), *([None] * 16), 0, None) == 0
