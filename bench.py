@@ -48,6 +48,8 @@ def parse():
                          "(fake balanced static expert routing)")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
                     help="routed expert weights: bf16, or FP8 E4M3 with 128x128 block scales (moe_forward_fp8)")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                    help="backward: time moe_backward (all gradients) for the forward's routing")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling runs)")
     return ap.parse_args()
@@ -407,6 +409,61 @@ def run_b200(args, shape):
         print(json.dumps(line), flush=True)
 
 
+def run_backward(args, shape):
+    """Times moe_backward (dx, dWr, dW_gate_up, dW_down and the shared expert's gradients) on
+    device-resident inputs for the forward's routing; one GPU. Algorithmic FLOPs per routed
+    (token, expert) row: recompute 4HI + dgrad 2HI + 4HI + wgrad 2HI + 4HI = 16HI (shared
+    rows 16H*Is) + router 4HE-level work not counted."""
+    import torch
+
+    from sparse_moe_layer_biased_b200 import _abi
+    from sparse_moe_layer_biased_b200.inputs import draw
+    from sparse_moe_layer_biased_b200.layer import MoeLayer
+
+    torch.cuda.set_device(0)
+    inp = draw(shape, device="cuda")
+    _, idx, w = MoeLayer(shape, inp).forward(inp["x"], routing=True)
+    dy = torch.randn((shape.T, shape.H), generator=torch.Generator(device="cuda").manual_seed(5), device="cuda")
+    d = _abi.desc_of(shape)
+    ws = torch.empty(_abi.moe_backward_workspace_size(d), dtype=torch.uint8, device="cuda")
+    E, H, I, Is, T = shape.E, shape.H, shape.I, shape.Is, shape.T
+    outs = [torch.empty((T, H), device="cuda"), torch.empty((E, H), device="cuda"),
+            torch.empty((E, 2 * I, H), device="cuda"), torch.empty((E, H, I), device="cuda"),
+            torch.empty((2 * Is, H), device="cuda"), torch.empty((H, Is), device="cuda")]
+
+    def step():
+        _abi.moe_backward(d, inp["x"], inp["Wr"], inp["W_gate_up"], inp["W_down"], inp["Wsh_gate_up"],
+                          inp["Wsh_down"], idx, w, dy, *outs, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    _abi.moe_check_device()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(str(torch.cuda.get_device_properties(0).uuid))
+    sampler.start()
+    time.sleep(0.3)
+    s0.record()
+    for _ in range(args.steps):
+        step()
+    s1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    _abi.moe_check_device()
+    ms = s0.elapsed_time(s1) / args.steps
+    flops = 16.0 * H * (I * T * shape.k + Is * T)
+    wbytes = 4.0 * (E * 3 * I * H + 3 * Is * H)  # fp32 weight gradients written
+    peaks, _ = load_peaks()
+    line = {"metric": "MoE layer backward tokens/s on 1 B200", "value": T / (ms / 1e3), "unit": UNIT,
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic (seeded draw on device; random-init weights)",
+            "config": workload_config(shape, {"pass": "backward", "routing": "router"}),
+            "tensor": {"achieved_tflops": flops / (ms / 1e3) / 1e12,
+                       "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+            "weight_grad_bytes": wbytes, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     from sparse_moe_layer_biased_b200.inputs import WORKLOADS
@@ -417,6 +474,8 @@ def main():
                               T=args.tokens or shape.T, E=args.experts or shape.E)
     if args.impl == "reference":
         run_reference(args, shape)
+    elif args.which == "backward":
+        run_backward(args, shape)
     else:
         run_b200(args, shape)
 

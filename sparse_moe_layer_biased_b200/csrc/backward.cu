@@ -332,7 +332,9 @@ constexpr uint32_t kBwdTile = 16384;  // one operand per stage
 constexpr uint32_t kBwdStage = 2 * kBwdTile;
 constexpr uint32_t kBwdBarOff = kBwdStages * kBwdStage;
 constexpr uint32_t kBwdMiscOff = kBwdBarOff + 8 * (2 * kBwdStages + 5);
-constexpr uint32_t kBwdSmem = kBwdMiscOff + 16 + 1024;
+constexpr uint32_t kBwdEpiOff = kBwdMiscOff + 16;       // per epilogue warp: a 32 x 33 fp32 transpose
+constexpr uint32_t kBwdEpiWarp = 32 * 33 * 4;
+constexpr uint32_t kBwdSmem = kBwdEpiOff + 4 * kBwdEpiWarp + 1024;
 static_assert(kBwdSmem <= kMaxDynSmem, "backward ring exceeds shared memory");
 
 // MN-major operand in 128-byte swizzle: 64-element MN chunks lbo bytes apart, 8-row K
@@ -456,7 +458,8 @@ __device__ __forceinline__ void bwd_load(const BwdArgs &a, const CUtensorMap *ma
 
 // Epilogue of one tile for one warp (TMEM lane quarter q; lane row = q*32 + lane of M).
 template <int MODE>
-__device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, const BTile &t, int q, int lane)
+__device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, const BTile &t, int q, int lane,
+                                             float *tr)
 {
     const int row = q * 32 + lane;
     const uint32_t tq = tacc + (static_cast<uint32_t>(q * 32) << 16);
@@ -495,15 +498,22 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
         uint16_t *dgu = t.sh ? a.dgu_s : a.dgu_r;
         const float L = t.sh ? a.lim_s : a.lim_r;
         for (int cb = 0; cb < t.ntok; cb += 32) {
-            float v[32];
+            float v[32], gg[32], uu[32];
             tmem_load32(tq + cb, v);
-#pragma unroll 4
+            const int ncol = t.ntok - cb < 32 ? t.ntok - cb : 32;
+            // all 64 pre-activation loads of the block in flight before any use
+#pragma unroll
             for (int c = 0; c < 32; ++c) {
-                const bool valid = cb + c < t.ntok;  // uniform across the warp
-                if (!valid)
+                const int64_t rr = rs + cb + (c < ncol ? c : 0);
+                gg[c] = gu[rr * 2 * Iw + i];
+                uu[c] = gu[rr * 2 * Iw + Iw + i];
+            }
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                if (c >= ncol)  // uniform across the warp
                     break;
                 const int64_t rr = rs + cb + c;
-                const float g = gu[rr * 2 * Iw + i], u = gu[rr * 2 * Iw + Iw + i];
+                const float g = gg[c], u = uu[c];
                 const float sg = 1.0f / (1.0f + expf(-g));
                 const float act = g * sg;
                 float ac = act, uc = u, ma = 1.0f, mu = 1.0f;
@@ -558,12 +568,20 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
         else
             out = t.sh ? a.dWsh_gu + m * a.H : a.dWgu + (static_cast<int64_t>(t.g) * 2 * a.I + m) * a.H;
         out += t.nb * kBwdBN;
+        // through a 32 x 33 transpose so each store writes 128 contiguous bytes of one row
+        const int64_t ld = MODE == kBwdWD ? (t.sh ? a.Is : a.I) : a.H;
+        float *rowbase = out - static_cast<int64_t>(lane) * ld;  // row q*32 of the tile
         for (int cb = 0; cb < kBwdBN; cb += 32) {
             float v[32];
             tmem_load32(tq + cb, v);
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4 *>(out + cb + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            for (int c = 0; c < 32; ++c)
+                tr[lane * 33 + c] = v[c];
+            __syncwarp();
+#pragma unroll 8
+            for (int r = 0; r < 32; ++r)
+                rowbase[r * ld + cb + lane] = tr[r * 33 + lane];
+            __syncwarp();
         }
     }
 }
@@ -681,7 +699,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!warp_wait(&accf[buf], (tc >> 1) & 1, wc, abort_flag))
                 break;
             tc_fence_after();
-            bwd_epilogue<MODE>(a, tmem + buf * kBwdBN, t, q, lane);
+            bwd_epilogue<MODE>(a, tmem + buf * kBwdBN, t, q, lane,
+                               reinterpret_cast<float *>(smem + kBwdEpiOff + q * kBwdEpiWarp));
             tc_fence_before();
             __syncwarp();
             if (lane == 0)

@@ -84,3 +84,45 @@ def test_backward_matches_oracle(name):
     unused = np.setdiff1d(np.arange(sh.E), used)
     for e in unused:  # experts without tokens get zero weight gradients
         assert not got["dW_gate_up"][e].any() and not got["dW_down"][e].any() and not got["dWr"][e].any()
+
+
+@pytest.mark.slow
+def test_backward_full_size_one_expert():
+    """Step-3.5 prefill shape, forward routing from the GPU: the weight gradients of a
+    touched expert with about 8 tokens and the router row of that expert depend only on
+    the tokens routed to it, so the oracle's backward over just those tokens gives them
+    exactly, with those tokens' dx."""
+    sh = WORKLOADS["step35_prefill"]
+    inp = draw(sh, device="cuda")
+    from sparse_moe_layer_biased_b200.layer import MoeLayer
+    _, idx, w = MoeLayer(sh, inp).forward(inp["x"], routing=True)
+    dy = torch.randn((sh.T, sh.H), generator=torch.Generator(device="cuda").manual_seed(77), device="cuda")
+    d = _abi.desc_of(sh)
+    ws = torch.empty(_abi.moe_backward_workspace_size(d), dtype=torch.uint8, device="cuda")
+    E, H, I, Is, T = sh.E, sh.H, sh.I, sh.Is, sh.T
+    out = {"dx": torch.empty((T, H), device="cuda"), "dWr": torch.empty((E, H), device="cuda"),
+           "dW_gate_up": torch.empty((E, 2 * I, H), device="cuda"), "dW_down": torch.empty((E, H, I), device="cuda"),
+           "dWsh_gate_up": torch.empty((2 * Is, H), device="cuda"), "dWsh_down": torch.empty((H, Is), device="cuda")}
+    _abi.moe_backward(d, inp["x"], inp["Wr"], inp["W_gate_up"], inp["W_down"], inp["Wsh_gate_up"],
+                      inp["Wsh_down"], idx, w, dy, out["dx"], out["dWr"], out["dW_gate_up"], out["dW_down"],
+                      out["dWsh_gate_up"], out["dWsh_down"], ws)
+    torch.cuda.synchronize()
+    _abi.moe_check_device()
+    idx_h = idx.cpu().numpy()
+    counts = np.bincount(idx_h.ravel(), minlength=E)
+    e = int(np.where(counts > 0, np.abs(counts - 8), 1 << 30).argmin())  # about 8 tokens: cheap for the oracle
+    rows = np.nonzero((idx_h == e).any(1))[0]
+    rsel = torch.from_numpy(rows).cuda()
+    ref = oracle.backward(bf16_bits(inp["x"][rsel]), bf16_bits(inp["Wr"]), inp["bias"].cpu().numpy(),
+                          bf16_bits(inp["W_gate_up"]), bf16_bits(inp["W_down"]), bf16_bits(inp["Wsh_gate_up"]),
+                          bf16_bits(inp["Wsh_down"]), dy[rsel].cpu().numpy(), k=sh.k, scale=sh.scale,
+                          norm=sh.norm_expert_weight, limit_routed=sh.limit_routed, limit_shared=sh.limit_shared)
+    np.testing.assert_array_equal(np.sort(ref["idx"], 1), np.sort(idx_h[rows], 1))
+    pairs = {"dW_gate_up": (out["dW_gate_up"][e], ref["dW_gate_up"][e]), "dW_down": (out["dW_down"][e],
+             ref["dW_down"][e]), "dWr": (out["dWr"][e], ref["dWr"][e]), "dx": (out["dx"][rsel], ref["dx"])}
+    for key, (g, r) in pairs.items():
+        g = g.cpu().numpy()
+        rf = rel_fro(g, r)
+        ma = float(np.abs(g - r).max()) / max(float(np.abs(r).max()), 1e-30)
+        print(f"step35 expert {e} ({len(rows)} tokens) {key}: rel_fro {rf:.2e} max_abs/max {ma:.2e}")
+        assert rf <= 1e-2 and ma <= 2e-2, key
