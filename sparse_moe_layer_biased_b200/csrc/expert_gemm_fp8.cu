@@ -77,6 +77,10 @@ __device__ __forceinline__ uint8_t *ring8_setup(uint8_t *smem_raw, Ring8 &r)
     r.drain = r.acce + 2;
     r.holder = reinterpret_cast<uint32_t *>(smem + G::kMiscOff);
     r.abort_flag = reinterpret_cast<volatile int *>(smem + G::kMiscOff + 4);
+    // equal ring depths: stage it uses staging slot and operand slot it % SW, both freed by
+    // the same MMA completion, so one barrier (one commit per stage) releases both
+    if (SA == SW)
+        r.aempty = r.qempty;
     if (threadIdx.x == 0) {
         for (int s = 0; s < SW; ++s) {
             mbar_init(&r.qfull[s], 1);
@@ -144,12 +148,16 @@ __device__ __forceinline__ Scale2 split_scale(float scale)
     return Scale2{__bfloat162bfloat162(hi), __bfloat162bfloat162(lo)};
 }
 
-// Codes (b0, b1) of the 16-bit half `sel` selects (0x1404: bytes 0, 1; 0x3424: bytes 2, 3)
-// -> bf16x2 (low half = lower K) of code value * scale.
+// Codes (b0, b1) of the byte pair `sel` selects (0x4140: bytes 0, 1; 0x4342: bytes 2, 3)
+// -> bf16x2 (low half = lower K) of code value * scale. Each code lands in bits 0..7 of its
+// 16-bit half; multiplying by 16 moves it to bits 4..11, and adding 240 x (its sign bit)
+// carries the sign from bit 11 to bit 15 (2^11 + 15 * 2^11 = 2^15), so the integer work is
+// one byte permute, one mask and one multiply-add.
 __device__ __forceinline__ uint32_t dequant2(uint32_t codes4, uint32_t sel, const Scale2 &sc)
 {
-    const uint32_t y = __byte_perm(codes4, 0u, sel);  // code k in bits 8..15 of its 16-bit half
-    const uint32_t bits = (y & 0x80008000u) | ((y >> 4) & 0x07F007F0u);
+    const uint32_t pu = __byte_perm(codes4, 0u, sel);
+    const uint32_t sg = pu & 0x00800080u;
+    const uint32_t bits = pu * 16u + sg * 240u;
     const __nv_bfloat162 q = *reinterpret_cast<const __nv_bfloat162 *>(&bits);
     const __nv_bfloat162 w = __hfma2(q, sc.hi, __hmul2(q, sc.lo));
     return *reinterpret_cast<const uint32_t *>(&w);
@@ -172,14 +180,14 @@ __device__ __forceinline__ void convert_row_e4m3(const uint8_t *w, int j, uint32
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
             const uint4 v = *reinterpret_cast<const uint4 *>(w + sw128_chunk(j, 2 * h + cc));
-            out[8 * cc + 0] = dequant2(v.x, 0x1404u, s);
-            out[8 * cc + 1] = dequant2(v.x, 0x3424u, s);
-            out[8 * cc + 2] = dequant2(v.y, 0x1404u, s);
-            out[8 * cc + 3] = dequant2(v.y, 0x3424u, s);
-            out[8 * cc + 4] = dequant2(v.z, 0x1404u, s);
-            out[8 * cc + 5] = dequant2(v.z, 0x3424u, s);
-            out[8 * cc + 6] = dequant2(v.w, 0x1404u, s);
-            out[8 * cc + 7] = dequant2(v.w, 0x3424u, s);
+            out[8 * cc + 0] = dequant2(v.x, 0x4140u, s);
+            out[8 * cc + 1] = dequant2(v.x, 0x4342u, s);
+            out[8 * cc + 2] = dequant2(v.y, 0x4140u, s);
+            out[8 * cc + 3] = dequant2(v.y, 0x4342u, s);
+            out[8 * cc + 4] = dequant2(v.z, 0x4140u, s);
+            out[8 * cc + 5] = dequant2(v.z, 0x4342u, s);
+            out[8 * cc + 6] = dequant2(v.w, 0x4140u, s);
+            out[8 * cc + 7] = dequant2(v.w, 0x4342u, s);
         }
         tmem_store16(taddr + 16 * h, out);
     }
@@ -388,7 +396,10 @@ __global__ void __launch_bounds__(kThreads8, 1)
             }
         }
     } else if (warp == 1) {
-        // MMA: A (weights) from the TMEM operand slot, B (token rows) from the staging slot
+        // MMA: A (weights) from the TMEM operand slot, B (token rows) from the staging slot.
+        // The converter group of a stage waited for the slot's bytes before it arrived on
+        // conv, so conv's completion implies qfull's: the MMA thread waits on conv alone
+        // (each barrier test costs the single issuing thread about 100 cycles per stage).
         if (lane == 0) {
             int it = 0, tc = 0;
             bool ok = true;
@@ -403,8 +414,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 const int nks = t.stage_k() / 16;
                 for (int st = 0; st < t.stages(); ++st, ++it) {
                     const int sa = it % SA, sq = it % SW;
-                    if (!mbar_wait(&r.conv[sa], (it / SA) & 1, wc, r.abort_flag) ||
-                        !mbar_wait(&r.qfull[sq], (it / SW) & 1, wc, r.abort_flag)) {
+                    if (!mbar_wait(&r.conv[sa], (it / SA) & 1, wc, r.abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -415,7 +425,8 @@ __global__ void __launch_bounds__(kThreads8, 1)
                         const uint64_t bd = sdesc_kmajor_sw128(b_addr + (ks >> 2) * G::kBSlice) + 2 * (ks & 3);
                         umma_bf16_ta(d, a_col + 8 * ks, bd, idesc, (st | ks) != 0);
                     }
-                    umma_commit(&r.aempty[sa]);
+                    if (SA != SW)
+                        umma_commit(&r.aempty[sa]);
                     umma_commit(&r.qempty[sq]);
                 }
                 if (ok)

@@ -177,9 +177,12 @@ __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr)
 }
 
 // Arrive on a barrier that may live in another CTA of the cluster (address from dsmem_addr).
+// Default (CTA-scope release) semantics: what the arrival publishes are tensor-memory
+// accesses already completed by tcgen05.wait, and a cluster-scope release would put a
+// cluster-wide memory barrier on every arrival.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // ---------------------------------------------------------------- CTA pairs (cta_group::2)

@@ -31,6 +31,10 @@ SHAPES = {
     # prefill-sized: 128-row chunks, several K blocks, ragged chunk tails, Is not a multiple of 128
     "prefill": LayerShape("fp8_prefill", T=300, H=512, E=12, k=4, I=256, Is=192, limit_routed=0.25,
                           limit_shared=0.125, seed=52, weight_std=0.03),
+    # prefill-sized, wider: 6 K blocks of gate/up, 6 down row blocks, 4 shared-expert
+    # gate/up feature blocks, ragged chunk tails
+    "prefill_h768": LayerShape("fp8_prefill_h768", T=333, H=768, E=10, k=4, I=384, Is=256, limit_routed=0.25,
+                               limit_shared=0.125, seed=56, weight_std=0.03),
     "ragged": LayerShape("fp8_ragged", T=333, H=384, E=40, k=6, I=128, Is=320, limit_routed=0.0,
                          limit_shared=0.0, seed=53, weight_std=0.03),
     # pre-activations of std ~1 against routed limit 0.5: the up clamp binds on ~60% and
