@@ -349,10 +349,12 @@ __device__ __forceinline__ void down_epilogue_bulk(uint32_t tmem_tile, int bn, i
         if (q == 0 && lane < kOutTok) {
             if (mycol < ntok) {
                 float *dst = a.out + dst_row * a.H + feat0;
+                // each output row receives k + 1 reductions spread over the whole launch:
+                // keep its lines in L2 against the weight stream (evict-last policy)
                 if (a.deterministic)
                     bulk_store(dst, buf + lane * kRowBytes, kRowBytes);
                 else
-                    bulk_reduce_add_f32(dst, buf + lane * kRowBytes, kRowBytes);
+                    bulk_reduce_add_f32_hint(dst, buf + lane * kRowBytes, kRowBytes, l2_policy_evict_last());
                 bulk_commit();
             }
             bulk_wait_read<NOB - 1>();  // the buffer written next is no longer being read

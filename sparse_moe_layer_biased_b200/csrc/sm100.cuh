@@ -421,6 +421,24 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float *dst, const void *src,
                  : "memory");
 }
 
+// The same reduction with an L2 eviction-priority policy (from l2_policy_evict_last).
+__device__ __forceinline__ void bulk_reduce_add_f32_hint(float *dst, const void *src, uint32_t bytes, uint64_t policy)
+{
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.L2::cache_hint.add.f32 [%0], [%1], %2, %3;" ::"l"(
+                     dst),
+                 "r"(smem_u32(src)), "r"(bytes), "l"(policy)
+                 : "memory");
+}
+
+// L2 eviction-priority policy for the whole access (fraction 1.0): lines stay in L2 ahead
+// of normally cached traffic.
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 __device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes)
 {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
