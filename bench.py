@@ -65,19 +65,54 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    """SM clock and clock-event reasons of this GPU, read through NVML every 5 ms while the
+    timed region runs (read-only queries; nvidia-smi at its 200 ms minimum if NVML is
+    unavailable)."""
 
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
+        self.samples = []  # (sm_mhz, sm_max_mhz, reasons)
         self.lines = []
         self.proc = None
         self.thread = None
+        self.stop_flag = threading.Event()
+        self.source = None
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            smax = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+            masks = [(name, getattr(pynvml, attr)) for name, attr in self.REASONS]
+        except Exception:
+            self._start_smi()
+            return
+        self.source = "nvml 5 ms"
+
+        def poll():
+            while not self.stop_flag.is_set():
+                try:
+                    sm = float(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM))
+                    bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                    self.samples.append((sm, smax, {n for n, m in masks if bits & m}))
+                except Exception:
+                    pass
+                time.sleep(0.005)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+
+    def _start_smi(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-i", self.gpu_id,
@@ -85,6 +120,7 @@ class ClockSampler:
         except OSError:
             self.proc = None
             return
+        self.source = "nvidia-smi 200 ms"
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
@@ -93,31 +129,32 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+        self.stop_flag.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
         if self.thread:
             self.thread.join(timeout=5)
-        sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
             try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
+                self.samples.append((float(parts[0]), float(parts[1]),
+                                     {n for n, v in zip(names, parts[4:8]) if v.lower() == "active"}))
             except ValueError:
                 continue
-            for name, val in zip(names, parts[4:8]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock samples"], "samples": 0,
+                    "source": self.source}
+        sm = [x[0] for x in self.samples]
+        reasons = set().union(*(x[2] for x in self.samples))
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 def max_over_ranks(value: float, device) -> float:
@@ -326,7 +363,6 @@ def run_b200(args, shape):
     barrier()
     torch.cuda.synchronize()
     sampler.start()
-    time.sleep(0.3)
     start.record(stream)
     for i in range(args.steps):
         _abi.moe_set_stage_events(evs[i])
@@ -439,9 +475,9 @@ def run_backward(args, shape):
     torch.cuda.synchronize()
     _abi.moe_check_device()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(str(torch.cuda.get_device_properties(0).uuid))
+    uuid = str(torch.cuda.get_device_properties(0).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
     sampler.start()
-    time.sleep(0.3)
     s0.record()
     for _ in range(args.steps):
         step()

@@ -1,0 +1,42 @@
+"""Host logic of bench.py that needs no GPU: clock-record summarising and the byte model."""
+import numpy as np
+
+import bench
+from sparse_moe_layer_biased_b200.inputs import WORKLOADS
+
+
+def test_clock_record_from_smi_lines():
+    s = bench.ClockSampler("GPU-fake")
+    s.lines = ["1965, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active",
+               "1950, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active",
+               "1800, 1965, 990.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+               "garbage"]
+    r = s.stop()
+    assert r["samples"] == 3 and r["sm_mhz"] == 1950 and r["sm_min_mhz"] == 1800 and r["sm_max_mhz"] == 1965
+    assert r["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_record_flags_thermal_reason():
+    s = bench.ClockSampler("GPU-fake")
+    s.samples = [(1500.0, 1965.0, {"hw_thermal_slowdown"}), (1965.0, 1965.0, set())]
+    r = s.stop()
+    assert r["reasons"] == ["hw_thermal_slowdown"] and r["samples"] == 2
+
+
+def test_no_samples_is_reported():
+    r = bench.ClockSampler("GPU-fake").stop()
+    assert r["samples"] == 0 and r["sm_mhz"] is None
+
+
+def test_gate_up_byte_model_counts_touched_experts_only():
+    sh = WORKLOADS["step35_prefill"]
+    counts = np.zeros(sh.E + 1, np.int64)
+    counts[:10] = 5
+    b, touched = bench.gate_up_bytes(sh, counts)
+    assert touched == 10
+    w = 10 * 2 * sh.I * sh.H * 2 + 2 * sh.Is * sh.H * 2
+    acts = sh.T * sh.k * sh.H * 2 + sh.T * sh.H * 2
+    out = sh.T * sh.k * sh.I * 2 + sh.T * sh.Is * 2
+    assert b == w + acts + out
+    b8, _ = bench.gate_up_bytes(sh, counts, fp8=True)
+    assert b8 == b - 10 * 2 * sh.I * sh.H + 10 * (2 * sh.I // 128) * (sh.H // 128) * 4
