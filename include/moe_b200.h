@@ -162,7 +162,7 @@ MOE_API moe_status_t moe_forward_with_ids(const moe_layer_desc *desc, const uint
  *   W_gate_up_scale [E, 2I/128, H/128] fp32, W_down_q [E, H, I] uint8,
  *   W_down_scale [E, H/128, I/128] fp32: weight[r][c] = e4m3(q[r][c]) * scale[r/128][c/128].
  * The kernels stream the codes (half the weight bytes of BF16) and turn them into
- * bf16(e4m3 * scale) in shared memory for the BF16 tensor-core MMA, so a dequantized weight
+ * bf16(e4m3 * scale) in tensor memory for the BF16 tensor-core MMA, so a dequantized weight
  * carries one bf16 rounding (relative 2^-9) besides the BF16 path's arithmetic. Every other
  * argument, the workspace (moe_workspace_size covers both formats) and the results are
  * those of moe_forward. Requires I % 128 == 0 (MOE_ERR_UNSUPPORTED otherwise); code arrays
@@ -173,6 +173,49 @@ MOE_API moe_status_t moe_forward_fp8(const moe_layer_desc *desc, const uint16_t 
                                      const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y,
                                      int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
                                      void *stream);
+
+/* ---- Expert parallelism ("MAX 中 Step-3.5-Flash 架构解析", section "并行模式TP_TP / TP_EP /
+ * DP_EP": in DP_EP each rank runs its own batch shard, the routed experts are split across
+ * ranks and an EP combine follows the MoE; NeMo AutoModel Step-5-Preview page, "Model
+ * Architecture" table: expert parallelism, e.g. EP32 with 11 routed experts per rank).
+ * With R ranks, rank r owns the routed experts [r*Er, (r+1)*Er), Er = E / R; the router and
+ * the shared expert are replicated. One forward on each rank:
+ *   moe_router, moe_permute (global E): slots in global expert order = (owner rank, local
+ *   expert) order; moe_ep_pack: the send rows; an all-to-all of the per-(owner, local expert)
+ *   counts and of the rows (NCCL, by the caller); moe_ep_experts on the received rows; the
+ *   reverse all-to-all of their fp32 outputs into rows [0, T*k) of o_perm;
+ *   moe_shared_expert into rows [T*k, T*k + T); moe_combine. */
+
+/* Send buffer of a dispatch: x_send[slot_of[t, j]] = x[t], w_send[slot_of[t, j]] = topk_w[t, j]
+ * for every routed (token, rank); desc, x [T, H] bf16, topk_w [T, k] fp32 and slot_of [T, k]
+ * as in moe_expert_ffn. x_send [T*k, H] bf16 (16-byte aligned), w_send [T*k] fp32. Rows of
+ * owner rank r are the slots [offsets[r*Er], offsets[(r+1)*Er]). */
+MOE_API moe_status_t moe_ep_pack(const moe_layer_desc *desc, const uint16_t *x, const float *topk_w,
+                                 const int32_t *slot_of, uint16_t *x_send, float *w_send, void *stream);
+
+/* Owner side of a dispatch: the routed experts of this rank on the rows it received.
+ *   desc: T = rows received, k = 1, E = local experts Er; H, I, Is, limits as the layer
+ *         (deterministic is ignored: every output row has one contribution).
+ *   ep_ranks R (1..64, R * Er <= 8192); recv_counts [R, Er] int32 on the device: rows that
+ *         source rank s sent for local expert e. Rows arrive source-major: all rows of source
+ *         0 (its expert 0 rows, then expert 1, ...), then source 1, ...
+ *   x_recv [T, H] bf16, w_recv [T] fp32 routing weights of the rows;
+ *   W_gate_up [Er, 2I, H], W_down [Er, H, I] bf16: this rank's experts;
+ *   out [T, H] fp32 (overwritten): out[n] = w_recv[n] * expert(x_recv[n]), in received order;
+ *   ws, ws_bytes: at least moe_workspace_size(desc) bytes.
+ * MOE_ERR_INVALID_ARG for k != 1 or R out of range, MOE_ERR_UNSUPPORTED for a count table
+ * above 8192 entries. The sum of recv_counts must equal T; rows past the sum are not written. */
+MOE_API moe_status_t moe_ep_experts(const moe_layer_desc *desc, int32_t ep_ranks, const int32_t *recv_counts,
+                                    const uint16_t *x_recv, const float *w_recv, const uint16_t *W_gate_up,
+                                    const uint16_t *W_down, float *out, void *ws, size_t ws_bytes, void *stream);
+
+/* The shared expert alone on this rank's tokens: out[t] = shared_expert(x[t]) with the
+ * shared clip limit; x [T, H] bf16, Wsh_gate_up [2Is, H], Wsh_down [H, Is] bf16, out [T, H]
+ * fp32 (overwritten; e.g. rows [T*k, T*k + T) of an o_perm for moe_combine); ws of at least
+ * moe_workspace_size(desc) bytes. */
+MOE_API moe_status_t moe_shared_expert(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wsh_gate_up,
+                                       const uint16_t *Wsh_down, float *out, void *ws, size_t ws_bytes,
+                                       void *stream);
 
 /* Backward pass of the layer (the layer is trained: NeMo AutoModel Step-5-Preview page,
  * benchmark recipe with forward, backward and optimizer steps; miles page: BF16 training).

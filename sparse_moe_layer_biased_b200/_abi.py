@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_status_string", "moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events",
            "moe_forward_noalloc", "moe_forward_with_ids", "moe_forward_fp8", "moe_backward",
-           "moe_backward_workspace_size"]
+           "moe_backward_workspace_size", "moe_ep_pack", "moe_ep_experts", "moe_shared_expert"]
 
 
 class MoeError(RuntimeError):
@@ -77,6 +77,11 @@ def lib():
         L.moe_forward_with_ids.restype = i32
         L.moe_forward_noalloc.argtypes = [dp] + [vp] * 11
         L.moe_forward_noalloc.restype = i32
+        L.moe_ep_pack.argtypes = [dp] + [vp] * 6
+        L.moe_ep_experts.argtypes = [dp, ctypes.c_int32] + [vp] * 7 + [sz, vp]
+        L.moe_shared_expert.argtypes = [dp] + [vp] * 5 + [sz, vp]
+        for name in ("moe_ep_pack", "moe_ep_experts", "moe_shared_expert"):
+            getattr(L, name).restype = i32
         for name in ("moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn", "moe_combine",
                      "moe_forward", "moe_check_device", "moe_set_stage_events"):
             getattr(L, name).restype = i32
@@ -203,3 +208,20 @@ def moe_forward_with_ids(desc, x, topk_idx, topk_w, W_gate_up, W_down, Wsh_gate_
     _check("moe_forward_with_ids", lib().moe_forward_with_ids(
         ctypes.byref(desc), _p(x), _p(topk_idx), _p(topk_w), _p(W_gate_up), _p(W_down), _p(Wsh_gate_up),
         _p(Wsh_down), _p(y), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_ep_pack(desc, x, topk_w, slot_of, x_send, w_send, stream=None):
+    _check("moe_ep_pack", lib().moe_ep_pack(ctypes.byref(desc), _p(x), _p(topk_w), _p(slot_of), _p(x_send),
+                                            _p(w_send), _stream(stream)))
+
+
+def moe_ep_experts(desc, ep_ranks, recv_counts, x_recv, w_recv, W_gate_up, W_down, out, ws, stream=None):
+    _check("moe_ep_experts", lib().moe_ep_experts(
+        ctypes.byref(desc), int(ep_ranks), _p(recv_counts), _p(x_recv), _p(w_recv), _p(W_gate_up), _p(W_down),
+        _p(out), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_shared_expert(desc, x, Wsh_gate_up, Wsh_down, out, ws, stream=None):
+    _check("moe_shared_expert", lib().moe_shared_expert(
+        ctypes.byref(desc), _p(x), _p(Wsh_gate_up), _p(Wsh_down), _p(out), _p(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))

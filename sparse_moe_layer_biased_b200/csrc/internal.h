@@ -46,6 +46,13 @@ struct PermuteArgs {
 };
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream);
 
+// Expert-parallel receive side: rows arrive source-major (counts [R, Er] rows per source and
+// local expert); writes the expert-major offsets [Er + 2], perm_token and slot_of of the
+// received rows. Shared memory of the prefix tables: ep_regroup_smem(R, Er) bytes.
+size_t ep_regroup_smem(int R, int Er);
+cudaError_t launch_ep_regroup(const int32_t *counts, int R, int Er, int64_t nrows, int32_t *offsets,
+                              int32_t *perm_token, int32_t *slot_of, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
                           uint16_t *x_perm, float *w_perm, int num_sms, cudaStream_t stream);
 

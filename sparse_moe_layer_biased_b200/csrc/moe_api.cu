@@ -146,6 +146,11 @@ bool map_rows_u8(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, u
     return encode_u8(m, base, 2, dims, strides, box);
 }
 
+// Expert-parallel limits: ranks of one dispatch, and ranks x local experts of the per-source
+// count table the receive side scans.
+constexpr int kMaxEpRanks = 64;
+constexpr int64_t kMaxEpTable = 8192;
+
 bool aligned16(const void *p)
 {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
@@ -246,10 +251,24 @@ struct ExpertWeights {
     bool fp8() const { return gu_scale != nullptr; }
 };
 
+// Which expert groups one call computes: the layer (routed + shared), the routed experts of
+// dispatched rows only (expert parallelism's owner side), or the shared expert only.
+enum class FfnGroups { kBoth, kRoutedOnly, kSharedOnly };
+
 moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const uint16_t *x, const float *topk_w,
                             const int32_t *offsets, const int32_t *perm_token, const int32_t *slot_of,
-                            const ExpertWeights &W, float *out, void *ws, cudaStream_t s)
+                            const ExpertWeights &Win, float *out, void *ws, cudaStream_t s,
+                            FfnGroups groups = FfnGroups::kBoth)
 {
+    // a group that is not computed has no tiles; its tensor maps only need a valid address
+    ExpertWeights W = Win;
+    if (groups == FfnGroups::kRoutedOnly) {
+        W.sh_gu = static_cast<const uint16_t *>(W.gu);
+        W.sh_d = static_cast<const uint16_t *>(W.d);
+    } else if (groups == FfnGroups::kSharedOnly) {
+        W.gu = W.sh_gu;
+        W.d = W.sh_d;
+    }
     const bool fp8 = W.fp8();
     const WsLayout L = ws_layout(d);
     uint16_t *x_perm = at<uint16_t>(ws, L.x_perm);
@@ -284,9 +303,12 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
 
     if (!stage_mark(2, s))
         return MOE_ERR_CUDA;
-    cudaError_t e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, s);
+    cudaError_t e = cudaSuccess;
+    if (groups != FfnGroups::kSharedOnly)
+        e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, s);
+    const int shared_rows = groups == FfnGroups::kRoutedOnly ? 0 : d.T;
     if (e == cudaSuccess)
-        e = moe::launch_chunks(offsets, d.E, d.T, cfg.cap, chunks, hdr, cfg.cap_d,
+        e = moe::launch_chunks(offsets, d.E, shared_rows, cfg.cap, chunks, hdr, cfg.cap_d,
                                cfg.cap_d != cfg.cap ? chunks_d : nullptr, hdr_d, s);
     if (e == cudaSuccess && !d.deterministic)
         e = cudaMemsetAsync(out, 0, static_cast<size_t>(d.T) * d.H * 4, s);
@@ -505,6 +527,90 @@ moe_status_t moe_combine(const moe_layer_desc *desc, const float *o_perm, const 
         return MOE_ERR_UNSUPPORTED;
     return cuda_status(
         moe::launch_combine(o_perm, slot_of, desc->T, desc->k, desc->H, y, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_pack(const moe_layer_desc *desc, const uint16_t *x, const float *topk_w, const int32_t *slot_of,
+                         uint16_t *x_send, float *w_send, void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->T == 0)
+        return MOE_OK;  // nothing to do; array pointers may be NULL
+    if (!x || !topk_w || !slot_of || !x_send || !w_send)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_send))
+        return MOE_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    return cuda_status(moe::launch_gather(x, topk_w, slot_of, desc->T, desc->k, desc->H, x_send, w_send, di.num_sms,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_experts(const moe_layer_desc *desc, int32_t ep_ranks, const int32_t *recv_counts,
+                            const uint16_t *x_recv, const float *w_recv, const uint16_t *W_gate_up,
+                            const uint16_t *W_down, float *out, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->k != 1 || ep_ranks < 1 || ep_ranks > kMaxEpRanks)
+        return MOE_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(ep_ranks) * desc->E > kMaxEpTable)
+        return MOE_ERR_UNSUPPORTED;
+    if (desc->T == 0)
+        return MOE_OK;  // nothing received; array pointers may be NULL
+    if (!recv_counts || !x_recv || !w_recv || !W_gate_up || !W_down || !out || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_recv) || !aligned16(W_gate_up) || !aligned16(W_down) || !aligned16(out) || !aligned16(ws))
+        return MOE_ERR_UNSUPPORTED;
+    moe_layer_desc d = *desc;
+    d.deterministic = 0;  // one contribution per output row: the sum order is fixed anyway
+    const WsLayout L = ws_layout(d);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *perm_token = at<int32_t>(ws, L.perm_token);
+    int32_t *slot_of = at<int32_t>(ws, L.slot_of);
+    st = cuda_status(moe::launch_ep_regroup(recv_counts, ep_ranks, d.E, d.T, offsets, perm_token, slot_of, di.num_sms, s));
+    if (st != MOE_OK)
+        return st;
+    const ExpertWeights W{W_gate_up, W_down, nullptr, nullptr, nullptr, nullptr};
+    return run_expert_ffn(d, di, x_recv, w_recv, offsets, perm_token, slot_of, W, out, ws, s, FfnGroups::kRoutedOnly);
+}
+
+moe_status_t moe_shared_expert(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wsh_gate_up,
+                               const uint16_t *Wsh_down, float *out, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (desc->T == 0)
+        return MOE_OK;  // nothing to do; array pointers may be NULL
+    if (!x || !Wsh_gate_up || !Wsh_down || !out || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wsh_gate_up) || !aligned16(Wsh_down) || !aligned16(out) || !aligned16(ws))
+        return MOE_ERR_UNSUPPORTED;
+    moe_layer_desc d = *desc;
+    d.deterministic = 0;  // one contribution per output row
+    const WsLayout L = ws_layout(d);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);  // no routed rows: every routed group is empty
+    if (cudaMemsetAsync(offsets, 0, static_cast<size_t>(d.E + 2) * 4, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const ExpertWeights W{nullptr, nullptr, nullptr, nullptr, Wsh_gate_up, Wsh_down};
+    return run_expert_ffn(d, di, x, nullptr, offsets, at<int32_t>(ws, L.perm_token), at<int32_t>(ws, L.slot_of), W,
+                          out, ws, s, FfnGroups::kSharedOnly);
 }
 
 moe_status_t moe_forward(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr, const float *bias,

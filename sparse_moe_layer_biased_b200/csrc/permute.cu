@@ -239,6 +239,93 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Rows received by an expert-parallel dispatch ("MAX 中 Step-3.5-Flash 架构解析", section
+// "并行模式TP_TP / TP_EP / DP_EP": DP_EP, each rank routes its own tokens and the experts are
+// split across ranks) arrive source-major: source s sends, for each of this rank's Er experts
+// in order, counts[s * Er + e] rows. The grouped GEMMs want expert-major order (expert e's
+// rows from all sources contiguous), so received row n of source s at position p of that
+// source's block, belonging to expert e, goes to slot
+//     off[e] + col[s][e] + (p - pre[s][e])
+// with off = exclusive prefix of the expert totals, col[s][e] = rows of e from sources
+// before s, pre[s][e] = rows of source s for experts before e. Writes offsets [Er + 2]
+// (offsets[Er] = offsets[Er + 1] = rows), perm_token[slot] = n and slot_of[n] = slot. Every
+// block builds the prefix tables in shared memory; rows past the received total are skipped.
+__global__ void __launch_bounds__(256)
+    ep_regroup_kernel(const int32_t *__restrict__ counts, int R, int Er, int64_t nrows, int32_t *__restrict__ offsets,
+                      int32_t *__restrict__ perm_token, int32_t *__restrict__ slot_of)
+{
+    extern __shared__ int32_t tab[];
+    int32_t *src_base = tab;                 // [R + 1]
+    int32_t *pre = src_base + (R + 1);       // [R][Er + 1]
+    int32_t *col = pre + R * (Er + 1);       // [R][Er]
+    int32_t *off = col + R * Er;             // [Er + 1]
+    for (int s = threadIdx.x; s < R; s += blockDim.x) {
+        int acc = 0;
+        for (int e = 0; e < Er; ++e) {
+            pre[s * (Er + 1) + e] = acc;
+            acc += counts[s * Er + e];
+        }
+        pre[s * (Er + 1) + Er] = acc;
+    }
+    for (int e = threadIdx.x; e < Er; e += blockDim.x) {
+        int acc = 0;
+        for (int s = 0; s < R; ++s) {
+            col[s * Er + e] = acc;
+            acc += counts[s * Er + e];
+        }
+        off[e] = acc;  // expert total until the scan below
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int s = 0; s < R; ++s) {
+            src_base[s] = acc;
+            acc += pre[s * (Er + 1) + Er];
+        }
+        src_base[R] = acc;
+        int acc2 = 0;
+        for (int e = 0; e < Er; ++e) {
+            const int t = off[e];
+            off[e] = acc2;
+            acc2 += t;
+        }
+        off[Er] = acc2;
+        if (blockIdx.x == 0) {
+            for (int e = 0; e <= Er; ++e)
+                offsets[e] = off[e];
+            offsets[Er + 1] = acc2;
+        }
+    }
+    __syncthreads();
+    const int64_t total = src_base[R] < nrows ? src_base[R] : nrows;
+    for (int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; n < total;
+         n += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        int lo = 0, hi = R - 1;  // last source whose block starts at or before n
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (src_base[mid] <= n)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int p = static_cast<int>(n - src_base[lo]);
+        const int32_t *ps = pre + lo * (Er + 1);
+        int a = 0, b = Er - 1;  // last expert whose rows start at or before p
+        while (a < b) {
+            const int mid = (a + b + 1) >> 1;
+            if (ps[mid] <= p)
+                a = mid;
+            else
+                b = mid - 1;
+        }
+        const int64_t slot = off[a] + col[lo * Er + a] + (p - ps[a]);
+        if (slot < total) {
+            perm_token[slot] = static_cast<int32_t>(n);
+            slot_of[n] = static_cast<int32_t>(slot);
+        }
+    }
+}
+
 // Tile table from an offsets array in global memory (the moe_expert_ffn entry point).
 __global__ void __launch_bounds__(kPermThreads)
     chunks_kernel(const int32_t *__restrict__ offsets, int E, int T, int cap, int4 *__restrict__ chunks,
@@ -313,6 +400,28 @@ cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t 
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
     gather_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(x), topk_w, slot_of, nent, k, H / 8,
                                             reinterpret_cast<uint4 *>(x_perm), w_perm);
+    return cudaGetLastError();
+}
+
+size_t ep_regroup_smem(int R, int Er)
+{
+    return static_cast<size_t>((R + 1) + R * (Er + 1) + R * Er + (Er + 1)) * 4;
+}
+
+cudaError_t launch_ep_regroup(const int32_t *counts, int R, int Er, int64_t nrows, int32_t *offsets,
+                              int32_t *perm_token, int32_t *slot_of, int num_sms, cudaStream_t stream)
+{
+    const size_t smem = ep_regroup_smem(R, Er);
+    if (smem > 48 * 1024) {
+        const cudaError_t err =
+            cudaFuncSetAttribute(ep_regroup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (err != cudaSuccess)
+            return err;
+    }
+    const int64_t need = (nrows + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(num_sms) * 2;
+    const int grid = static_cast<int>(need < 1 ? 1 : (need < cap ? need : cap));
+    ep_regroup_kernel<<<grid, 256, smem, stream>>>(counts, R, Er, nrows, offsets, perm_token, slot_of);
     return cudaGetLastError();
 }
 

@@ -168,3 +168,34 @@ def test_backward_validation():
     assert L.moe_backward(ctypes.byref(d), *a, FAKE, need, None) == 2
     assert L.moe_backward(ctypes.byref(_desc(I=192)), *args, FAKE, need, None) == 2
     assert L.moe_backward(ctypes.byref(_desc(T=0)), *([None] * 16), 0, None) == 0
+
+
+def test_ep_validation():
+    L = moe.lib()
+    d = _desc()
+    # pack: null and misaligned pointers, empty call
+    assert L.moe_ep_pack(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, None) == 1
+    assert L.moe_ep_pack(ctypes.byref(d), FAKE + 2, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert L.moe_ep_pack(ctypes.byref(_desc(T=0)), *([None] * 6)) == 0
+    # owner side: k must be 1, ranks in 1..64, count table at most 8192 entries
+    dl = _desc(k=1)
+    need = moe.moe_workspace_size(dl)
+    args = [FAKE] * 7
+    assert L.moe_ep_experts(ctypes.byref(_desc(k=2)), 2, *args, need, None) == 1
+    assert L.moe_ep_experts(ctypes.byref(dl), 0, *args, need, None) == 1
+    assert L.moe_ep_experts(ctypes.byref(dl), 65, *args, need, None) == 1
+    assert L.moe_ep_experts(ctypes.byref(_desc(k=1, E=512)), 64, *args, need, None) == 2
+    assert L.moe_ep_experts(ctypes.byref(dl), 2, *args, need - 1, None) == 3
+    a = list(args)
+    a[0] = None  # recv_counts
+    assert L.moe_ep_experts(ctypes.byref(dl), 2, *a, need, None) == 1
+    a = list(args)
+    a[1] = FAKE + 4  # x_recv not 16-byte aligned
+    assert L.moe_ep_experts(ctypes.byref(dl), 2, *a, need, None) == 2
+    assert L.moe_ep_experts(ctypes.byref(_desc(T=0, k=1)), 2, *([None] * 7), 0, None) == 0
+    # shared expert alone
+    need = moe.moe_workspace_size(d)
+    assert L.moe_shared_expert(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, None) == 3
+    assert L.moe_shared_expert(ctypes.byref(d), FAKE, None, FAKE, FAKE, FAKE, need, None) == 1
+    assert L.moe_shared_expert(ctypes.byref(d), FAKE, FAKE, FAKE + 8, FAKE, FAKE, need, None) == 2
+    assert L.moe_shared_expert(ctypes.byref(_desc(T=0)), *([None] * 5), 0, None) == 0
