@@ -50,6 +50,8 @@ def parse():
                     help="routed expert weights: bf16, or FP8 E4M3 with 128x128 block scales (moe_forward_fp8)")
     ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
                     help="backward: time moe_backward (all gradients) for the forward's routing")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
+                    help="ep: expert parallelism, E/N routed experts per rank, T tokens per rank")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling runs)")
     return ap.parse_args()
@@ -444,6 +446,82 @@ def run_b200(args, shape):
         print(json.dumps(line), flush=True)
 
 
+def run_ep(args, shape):
+    """Expert-parallel layer (EPMoeLayer): N ranks, rank r owns routed experts
+    [r*E/N, (r+1)*E/N), each rank routes its own T tokens (weak scaling); dispatch, return and
+    combine go through NCCL all-to-alls. At N = 1 the exchanges are copies, which measures
+    the cost of the split path against the fused single-GPU forward. Kernel launches per
+    step: router, permute, pack, regroup, gather, tile table, gate_up, down (owner side),
+    tile table, gate_up, down (shared expert), combine."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from sparse_moe_layer_biased_b200 import _abi
+    from sparse_moe_layer_biased_b200.ep import EPMoeLayer
+    from sparse_moe_layer_biased_b200.inputs import draw
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    kw = {"timeout": datetime.timedelta(seconds=120), "device_id": torch.device("cuda", local)}
+    if world > 1:
+        dist.init_process_group("nccl", **kw)
+    else:
+        dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1, **kw)
+    inp = draw(shape, device="cuda")
+    Er = shape.E // world
+    w = {"Wr": inp["Wr"], "bias": inp["bias"], "Wsh_gate_up": inp["Wsh_gate_up"], "Wsh_down": inp["Wsh_down"],
+         "W_gate_up": inp["W_gate_up"][rank * Er:(rank + 1) * Er].contiguous(),
+         "W_down": inp["W_down"][rank * Er:(rank + 1) * Er].contiguous()}
+    del inp["W_gate_up"], inp["W_down"]
+    if rank == 0:
+        x = inp["x"]
+    else:
+        g = torch.Generator(device="cuda").manual_seed(shape.seed * 1000 + rank)
+        x = (torch.randn((shape.T, shape.H), generator=g, device="cuda") * shape.x_std).to(torch.bfloat16)
+    layer = EPMoeLayer(shape, w)
+    for _ in range(max(1, args.warmup)):
+        layer.forward(x)
+    torch.cuda.synchronize()
+    _abi.moe_check_device()
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = str(torch.cuda.get_device_properties(local).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    start.record(stream)
+    for _ in range(args.steps):
+        layer.forward(x)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    dist.barrier()
+    _abi.moe_check_device()
+    ms = max_over_ranks(start.elapsed_time(end), "cuda")
+    line = {
+        "metric": METRIC, "value": job_tokens_per_s(world, shape.T, args.steps, ms), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded draw on device; random-init weights)",
+        "config": workload_config(shape, {"parallelism": f"ep{world} ({Er} routed experts per rank)",
+                                          "l2": "inputs larger than L2 (expert weights streamed every step)",
+                                          "routing": "router", "weights": "bf16", "deterministic": True}),
+        "roofline": None,
+        "clocks": clocks,
+        "e2e": None,
+        "gpu_launches": 12 * args.steps,
+    }
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_backward(args, shape):
     """Times moe_backward (dx, dWr, dW_gate_up, dW_down and the shared expert's gradients) on
     device-resident inputs for the forward's routing; one GPU. Algorithmic FLOPs per routed
@@ -511,6 +589,8 @@ def main():
         run_reference(args, shape)
     elif args.which == "backward":
         run_backward(args, shape)
+    elif args.parallel == "ep":
+        run_ep(args, shape)
     else:
         run_b200(args, shape)
 
