@@ -174,6 +174,26 @@ MOE_API moe_status_t moe_forward_fp8(const moe_layer_desc *desc, const uint16_t 
                                      int32_t *topk_idx_out, float *topk_w_out, void *ws, size_t ws_bytes,
                                      void *stream);
 
+/* Device workspace of moe_forward_host: moe_workspace_size(desc) plus two [T, H] bf16 input
+ * and two [T, H] fp32 output staging buffers. */
+MOE_API moe_status_t moe_host_workspace_size(const moe_layer_desc *desc, size_t *bytes);
+
+/* moe_forward over n_batches batches of T tokens that live in host memory: the layer of a
+ * serving or inference loop fed from the host.
+ *   x_host [n_batches, T, H] bf16 and y_host [n_batches, T, H] fp32 in host memory (page-
+ *   locked, e.g. cudaHostAlloc, for the copies to overlap; pageable memory works but the
+ *   host then waits for each copy); batch i's layer output is written to y_host[i].
+ *   Weights, desc and the routing as in moe_forward; ws of at least moe_host_workspace_size.
+ * The copies run on two internal streams, double-buffered in ws: batch i+1's input copy
+ * and batch i-1's output copy overlap batch i's forward on `stream`. The call only enqueues
+ * work; when `stream` has completed, every output row is in y_host. n_batches = 0 or T = 0
+ * is a no-op. */
+MOE_API moe_status_t moe_forward_host(const moe_layer_desc *desc, int32_t n_batches, const uint16_t *x_host,
+                                      const uint16_t *Wr, const float *bias, const uint16_t *W_gate_up,
+                                      const uint16_t *W_down, const uint16_t *Wsh_gate_up,
+                                      const uint16_t *Wsh_down, float *y_host, void *ws, size_t ws_bytes,
+                                      void *stream);
+
 /* ---- Expert parallelism ("MAX 中 Step-3.5-Flash 架构解析", section "并行模式TP_TP / TP_EP /
  * DP_EP": in DP_EP each rank runs its own batch shard, the routed experts are split across
  * ranks and an EP combine follows the MoE; NeMo AutoModel Step-5-Preview page, "Model

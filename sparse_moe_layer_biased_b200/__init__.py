@@ -10,7 +10,7 @@ library; the first call does, and raises if it is not built.
 _ABI = {"moe_status_string", "moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn", "moe_combine",
         "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events", "moe_forward_noalloc",
         "moe_forward_with_ids", "moe_forward_fp8", "moe_backward", "moe_backward_workspace_size", "moe_ep_pack",
-        "moe_ep_experts", "moe_shared_expert", "MoeError",
+        "moe_ep_experts", "moe_shared_expert", "moe_host_workspace_size", "moe_forward_host", "MoeError",
         "LayerDesc", "desc_of", "lib", "EXPORTS", "LIB_PATH"}
 
 

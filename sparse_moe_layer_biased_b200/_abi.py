@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_status_string", "moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device", "moe_set_wait_limit_ns", "moe_set_stage_events",
            "moe_forward_noalloc", "moe_forward_with_ids", "moe_forward_fp8", "moe_backward",
-           "moe_backward_workspace_size", "moe_ep_pack", "moe_ep_experts", "moe_shared_expert"]
+           "moe_backward_workspace_size", "moe_ep_pack", "moe_ep_experts", "moe_shared_expert",
+           "moe_host_workspace_size", "moe_forward_host"]
 
 
 class MoeError(RuntimeError):
@@ -80,7 +81,10 @@ def lib():
         L.moe_ep_pack.argtypes = [dp] + [vp] * 6
         L.moe_ep_experts.argtypes = [dp, ctypes.c_int32] + [vp] * 7 + [sz, vp]
         L.moe_shared_expert.argtypes = [dp] + [vp] * 5 + [sz, vp]
-        for name in ("moe_ep_pack", "moe_ep_experts", "moe_shared_expert"):
+        L.moe_host_workspace_size.argtypes = [dp, ctypes.POINTER(sz)]
+        L.moe_forward_host.argtypes = [dp, ctypes.c_int32] + [vp] * 9 + [sz, vp]
+        for name in ("moe_ep_pack", "moe_ep_experts", "moe_shared_expert", "moe_host_workspace_size",
+                     "moe_forward_host"):
             getattr(L, name).restype = i32
         for name in ("moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn", "moe_combine",
                      "moe_forward", "moe_check_device", "moe_set_stage_events"):
@@ -225,3 +229,17 @@ def moe_shared_expert(desc, x, Wsh_gate_up, Wsh_down, out, ws, stream=None):
     _check("moe_shared_expert", lib().moe_shared_expert(
         ctypes.byref(desc), _p(x), _p(Wsh_gate_up), _p(Wsh_down), _p(out), _p(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_host_workspace_size(desc: LayerDesc) -> int:
+    out = ctypes.c_size_t(0)
+    _check("moe_host_workspace_size", lib().moe_host_workspace_size(ctypes.byref(desc), ctypes.byref(out)))
+    return out.value
+
+
+def moe_forward_host(desc, n_batches, x_host, Wr, bias, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y_host, ws,
+                     stream=None):
+    _check("moe_forward_host", lib().moe_forward_host(
+        ctypes.byref(desc), int(n_batches), _p(x_host), _p(Wr), _p(bias), _p(W_gate_up), _p(W_down),
+        _p(Wsh_gate_up), _p(Wsh_down), _p(y_host), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _stream(stream)))

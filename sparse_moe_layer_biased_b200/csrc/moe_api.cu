@@ -529,6 +529,114 @@ moe_status_t moe_combine(const moe_layer_desc *desc, const float *o_perm, const 
         moe::launch_combine(o_perm, slot_of, desc->T, desc->k, desc->H, y, static_cast<cudaStream_t>(stream)));
 }
 
+// Device staging of moe_forward_host after the forward workspace: two input buffers
+// [T, H] bf16 and two output buffers [T, H] fp32, each 256-byte aligned.
+struct HostLayout {
+    size_t fwd, x0, x1, y0, y1, total;
+};
+
+HostLayout host_layout(const moe_layer_desc &d)
+{
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    const size_t xb = up(static_cast<size_t>(d.T) * d.H * 2), yb = up(static_cast<size_t>(d.T) * d.H * 4);
+    HostLayout L;
+    L.fwd = 0;
+    L.x0 = up(ws_layout(d).total);
+    L.x1 = L.x0 + xb;
+    L.y0 = L.x1 + xb;
+    L.y1 = L.y0 + yb;
+    L.total = L.y1 + yb;
+    return L;
+}
+
+moe_status_t moe_host_workspace_size(const moe_layer_desc *desc, size_t *bytes)
+{
+    if (!bytes)
+        return MOE_ERR_INVALID_ARG;
+    const moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    *bytes = host_layout(*desc).total;
+    return MOE_OK;
+}
+
+moe_status_t moe_forward_host(const moe_layer_desc *desc, int32_t n_batches, const uint16_t *x_host,
+                              const uint16_t *Wr, const float *bias, const uint16_t *W_gate_up, const uint16_t *W_down,
+                              const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y_host, void *ws,
+                              size_t ws_bytes, void *stream)
+{
+    moe_status_t st = check_desc(desc);
+    if (st != MOE_OK)
+        return st;
+    if (n_batches < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (desc->T == 0 || n_batches == 0)
+        return MOE_OK;  // nothing to do; array pointers may be NULL
+    if (!x_host || !y_host || !Wr || !bias || !W_gate_up || !W_down || !Wsh_gate_up || !Wsh_down || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(ws))
+        return MOE_ERR_UNSUPPORTED;
+    const HostLayout L = host_layout(*desc);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t xe = static_cast<size_t>(desc->T) * desc->H;  // elements of one batch
+    uint16_t *xd[2] = {at<uint16_t>(ws, L.x0), at<uint16_t>(ws, L.x1)};
+    float *yd[2] = {at<float>(ws, L.y0), at<float>(ws, L.y1)};
+
+    // copy streams and the events that order them against the compute stream s; streams and
+    // events are released by the runtime once their pending work completes
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t ev[7] = {};  // start, h2d done x2, compute done x2, d2h done x2
+    bool ok = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) == cudaSuccess;
+    for (int i = 0; ok && i < 7; ++i)
+        ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+    cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_comp = ev + 3, *ev_out = ev + 5;
+    // the copies start after the work already queued on s
+    ok = ok && cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(h2d, ev_start, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(d2h, ev_start, 0) == cudaSuccess;
+    st = ok ? MOE_OK : MOE_ERR_CUDA;
+    for (int i = 0; st == MOE_OK && i < n_batches; ++i) {
+        const int b = i & 1;
+        // input buffer b was last read by batch i - 2's forward; output buffer b last copied
+        // out by batch i - 2's transfer
+        if (i >= 2 && (cudaStreamWaitEvent(h2d, ev_comp[b], 0) != cudaSuccess ||
+                       cudaStreamWaitEvent(s, ev_out[b], 0) != cudaSuccess)) {
+            st = MOE_ERR_CUDA;
+            break;
+        }
+        if (cudaMemcpyAsync(xd[b], x_host + static_cast<size_t>(i) * xe, xe * 2, cudaMemcpyHostToDevice, h2d) !=
+                cudaSuccess ||
+            cudaEventRecord(ev_in[b], h2d) != cudaSuccess || cudaStreamWaitEvent(s, ev_in[b], 0) != cudaSuccess) {
+            st = MOE_ERR_CUDA;
+            break;
+        }
+        st = moe_forward(desc, xd[b], Wr, bias, W_gate_up, W_down, Wsh_gate_up, Wsh_down, yd[b], nullptr, nullptr,
+                         ws, L.x0, stream);
+        if (st != MOE_OK)
+            break;
+        if (cudaEventRecord(ev_comp[b], s) != cudaSuccess || cudaStreamWaitEvent(d2h, ev_comp[b], 0) != cudaSuccess ||
+            cudaMemcpyAsync(y_host + static_cast<size_t>(i) * xe, yd[b], xe * 4, cudaMemcpyDeviceToHost, d2h) !=
+                cudaSuccess ||
+            cudaEventRecord(ev_out[b], d2h) != cudaSuccess)
+            st = MOE_ERR_CUDA;
+    }
+    // s completes after every transfer issued above (the copy streams are in order)
+    if (d2h && ev[0] && cudaEventRecord(ev_out[0], d2h) == cudaSuccess)
+        cudaStreamWaitEvent(s, ev_out[0], 0);
+    if (h2d && ev[0] && cudaEventRecord(ev_in[0], h2d) == cudaSuccess)
+        cudaStreamWaitEvent(s, ev_in[0], 0);
+    for (cudaEvent_t e : ev)
+        if (e)
+            cudaEventDestroy(e);
+    if (h2d)
+        cudaStreamDestroy(h2d);
+    if (d2h)
+        cudaStreamDestroy(d2h);
+    return st;
+}
+
 moe_status_t moe_ep_pack(const moe_layer_desc *desc, const uint16_t *x, const float *topk_w, const int32_t *slot_of,
                          uint16_t *x_send, float *w_send, void *stream)
 {

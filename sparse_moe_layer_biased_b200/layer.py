@@ -49,3 +49,23 @@ class MoeLayer:
             _abi.moe_forward(desc, x, W["Wr"], W["bias"], W["W_gate_up"], W["W_down"], W["Wsh_gate_up"],
                              W["Wsh_down"], y, self.ws, idx, w, stream=stream)
         return (y, idx, w) if routing else y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor | None = None, stream=None):
+        """The layer over batches in host memory: x_host [n, T, H] bf16 -> y_host [n, T, H]
+        fp32 (page-locked tensors for overlapped copies) through moe_forward_host. Returns
+        y_host once the work is enqueued; synchronize the stream before reading it."""
+        if self.fp8:
+            raise ValueError("forward_host runs BF16 routed experts")
+        n, T, H = x_host.shape
+        if T > self.max_tokens:
+            raise ValueError(f"{T} tokens exceed the workspace size of {self.max_tokens}")
+        desc = _abi.desc_of(self.shape, T=T, deterministic=self.deterministic)
+        need = _abi.moe_host_workspace_size(desc)
+        if getattr(self, "ws_host", None) is None or self.ws_host.numel() < need:
+            self.ws_host = torch.empty(need, dtype=torch.uint8, device=self.w["Wr"].device)
+        if y_host is None:
+            y_host = torch.empty((n, T, H), dtype=torch.float32, pin_memory=True)
+        W = self.w
+        _abi.moe_forward_host(desc, n, x_host, W["Wr"], W["bias"], W["W_gate_up"], W["W_down"], W["Wsh_gate_up"],
+                              W["Wsh_down"], y_host, self.ws_host, stream=stream)
+        return y_host

@@ -199,3 +199,21 @@ def test_ep_validation():
     assert L.moe_shared_expert(ctypes.byref(d), FAKE, None, FAKE, FAKE, FAKE, need, None) == 1
     assert L.moe_shared_expert(ctypes.byref(d), FAKE, FAKE, FAKE + 8, FAKE, FAKE, need, None) == 2
     assert L.moe_shared_expert(ctypes.byref(_desc(T=0)), *([None] * 5), 0, None) == 0
+
+
+def test_forward_host_validation():
+    L = moe.lib()
+    d = _desc()
+    need = moe.moe_host_workspace_size(d)
+    assert need > moe.moe_workspace_size(d)
+    args = [FAKE] * 9  # x_host, Wr, bias, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y_host, ws
+    assert L.moe_forward_host(ctypes.byref(d), -1, *args, need, None) == 1
+    assert L.moe_forward_host(ctypes.byref(d), 2, *args, need - 1, None) == 3
+    a = list(args)
+    a[7] = None  # y_host
+    assert L.moe_forward_host(ctypes.byref(d), 2, *a, need, None) == 1
+    a = list(args)
+    a[8] = FAKE + 8  # workspace not 16-byte aligned
+    assert L.moe_forward_host(ctypes.byref(d), 2, *a, need, None) == 2
+    assert L.moe_forward_host(ctypes.byref(d), 0, *([None] * 9), 0, None) == 0
+    assert L.moe_forward_host(ctypes.byref(_desc(T=0)), 3, *([None] * 9), 0, None) == 0
