@@ -412,16 +412,9 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// dst[0 .. bytes/4) += src[...] (fp32 adds performed at L2, bulk-group completion);
-// dst and src 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_reduce_add_f32(float *dst, const void *src, uint32_t bytes)
-{
-    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
-                 "r"(smem_u32(src)), "r"(bytes)
-                 : "memory");
-}
-
-// The same reduction with an L2 eviction-priority policy (from l2_policy_evict_last).
+// dst[0 .. bytes/4) += src[...] (fp32 adds performed at L2, bulk-group completion) with an
+// L2 eviction-priority policy (from l2_policy_evict_last); dst and src 16-byte aligned,
+// bytes a multiple of 16.
 __device__ __forceinline__ void bulk_reduce_add_f32_hint(float *dst, const void *src, uint32_t bytes, uint64_t policy)
 {
     asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.L2::cache_hint.add.f32 [%0], [%1], %2, %3;" ::"l"(
