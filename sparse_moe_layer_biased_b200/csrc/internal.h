@@ -22,12 +22,12 @@ struct RouterArgs {
     int norm;
     int num_sms;
 };
-// Router launch geometry: sl experts per CTA, ns CTAs per cluster, Wr rows per TMA box
-// (the Wr tensor map must be encoded with this box height).
+// Router launch geometry: e_pad experts per CTA (E rounded up to 16), ks CTAs per cluster
+// splitting K, Wr rows per TMA box (the Wr tensor map must be encoded with this box height).
 struct RouterSplit {
-    int sl, ns, box_rows;
+    int e_pad, ks, box_rows;
 };
-RouterSplit router_split(int E, int T, int num_sms);
+RouterSplit router_split(int E, int T, int H, int num_sms);
 cudaError_t launch_router(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const RouterArgs &a,
                           const WaitCfg &wc, cudaStream_t stream);
 

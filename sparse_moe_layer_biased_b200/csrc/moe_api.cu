@@ -235,7 +235,7 @@ moe_status_t run_router(const moe_layer_desc &d, const DeviceInfo &di, const uin
                         const float *bias, int32_t *idx, float *w, float *margin, cudaStream_t s)
 {
     CUtensorMap tm_x, tm_wr;
-    const moe::RouterSplit sp = moe::router_split(d.E, d.T, di.num_sms);
+    const moe::RouterSplit sp = moe::router_split(d.E, d.T, d.H, di.num_sms);
     if (!map_rows(&tm_x, x, d.H, d.T, 128) || !map_rows(&tm_wr, Wr, d.H, d.E, sp.box_rows))
         return MOE_ERR_CUDA;
     moe::RouterArgs a{bias, idx, w, margin, d.T, d.H, d.E, d.k, d.scale, d.norm_expert_weight, di.num_sms};

@@ -6,45 +6,53 @@
 // sum 1 (norm_expert_weight) and multiplied by moe_router_scaling_factor; indices clamped
 // to [0, E-1].
 //
-// A thread-block cluster of NS CTAs owns 128 tokens; CTA r owns the experts of slice r
-// (SL experts, a multiple of 16, up to 512). Each CTA computes its logits tile
-// [128 tokens x SL] with tcgen05 MMAs (bf16 x bf16 products, fp32 accumulation in TMEM;
-// two MMAs when SL > 256) fed by a TMA ring,
-// then gives each TMEM lane (= token) to one thread, which keeps a sorted top-(k+1) list
-// of its slice in registers. The lists meet in CTA 0 through distributed shared memory,
-// where each thread merges the NS lists of its token and writes ids, weights and margin.
-// No logits reach global memory. NS is chosen so the grid covers the SMs about once:
-// decode-sized calls split the experts over up to 8 CTAs, large calls use NS = 1.
+// A thread-block cluster of S CTAs owns a tile of TOK tokens (128, or 64 when E > 384) and
+// all E experts; CTA s computes the fp32 logits of the tile over its K range
+// [s*H/S, (s+1)*H/S) with tcgen05 MMAs (bf16 x bf16 products, fp32 accumulation in TMEM; two
+// MMAs when E > 256) fed by a TMA ring, then parks the partial tile [TOK x E] in its shared
+// memory (the idle ring). After a cluster barrier each CTA takes a share of the tile's tokens:
+// one warp per token sums the S partials of each expert through distributed shared memory in
+// rank order (a fixed order: the logits do not depend on timing), applies the sigmoid and the
+// bias, and selects the top k by k+1 rounds of a warp-wide maximum over sortable keys (biased
+// score, then lower expert index), which also gives the (k+1)-th for the margin. No logits
+// reach global memory. S (1, 2, 4 or 8) is chosen so the grid covers the SMs about once.
 #include "internal.h"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
+// warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 TMEM -> shared memory; all 16 warps select
+// (the selection is latency-bound per warp: more warps per SM keep more tokens in flight)
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
 constexpr int kTileM = 128;
 constexpr int kBK = 64;                         // bf16 elements per 128-byte swizzled row
 constexpr uint32_t kABytes = kTileM * kBK * 2;  // 16 KB
 constexpr int kMaxStages = 8;
+constexpr int kMaxKeysPerLane = 16;             // E <= 512 experts over 32 lanes
 
-template <int KMAX>
+// Shared-memory layout for E_pad experts (a multiple of 16): a ring of stages (x tile +
+// Wr rows of every expert), its barriers, and after the main loop the partial logits
+// [tok][E_pad + 1] fp32 over the ring (row stride E_pad + 1 floats: conflict-free column
+// writes from the TMEM epilogue).
 struct Layout {
-    uint32_t b_bytes, stage_bytes, list_off, bias_off, bar_off, misc_off, total, tmem_cols;
-    int stages;
-    __host__ __device__ explicit Layout(int sl)
+    uint32_t b_bytes, stage_bytes, bar_off, misc_off, total, tmem_cols, part_stride;
+    int stages, tok;
+    __host__ __device__ explicit Layout(int e_pad)
     {
-        b_bytes = (static_cast<uint32_t>(sl) * 128 + 1023) / 1024 * 1024;
+        b_bytes = static_cast<uint32_t>(e_pad) * 128;
         stage_bytes = kABytes + b_bytes;
-        const uint32_t list_bytes = kTileM * (KMAX + 1) * 12;
-        const uint32_t fixed = list_bytes + static_cast<uint32_t>(sl) * 4 + 8 * (2 * kMaxStages + 2) + 64;
+        const uint32_t fixed = 8 * (2 * kMaxStages + 2) + 64;
         int s = static_cast<int>((kMaxDynSmem - 1024 - fixed) / stage_bytes);
         stages = s > kMaxStages ? kMaxStages : s;
-        list_off = stages * stage_bytes;  // keys [128][KMAX+1] u64, then scores [128][KMAX+1] f32
-        bias_off = list_off + list_bytes;
-        bar_off = (bias_off + static_cast<uint32_t>(sl) * 4 + 7) / 8 * 8;
+        part_stride = static_cast<uint32_t>(e_pad) + 1;
+        const uint32_t ring = static_cast<uint32_t>(stages) * stage_bytes;
+        tok = static_cast<uint32_t>(kTileM) * part_stride * 4 <= ring ? kTileM : kTileM / 2;
+        bar_off = ring;
         misc_off = bar_off + 8 * (2 * kMaxStages + 2);
         total = misc_off + 16;
         uint32_t c = 32;
-        while (c < static_cast<uint32_t>(sl))
+        while (c < static_cast<uint32_t>(e_pad))
             c <<= 1;
         tmem_cols = c;
     }
@@ -76,54 +84,40 @@ __device__ __forceinline__ int key_expert(uint64_t key)
     return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
 }
 
-// Insert (key, s) into the descending register list keys[0..KMAX] (fully unrolled).
-template <int KMAX>
-__device__ __forceinline__ void list_insert(uint64_t (&keys)[KMAX + 1], float (&sv)[KMAX + 1], uint64_t key, float s)
+// Warp-wide maximum of 64-bit rank keys (unique per expert): the larger high word (biased
+// score), then among lanes holding it the larger low word (lower expert index).
+__device__ __forceinline__ uint64_t warp_max_key(uint64_t key)
 {
-    if (key > keys[KMAX]) {
-        keys[KMAX] = key;
-        sv[KMAX] = s;
-#pragma unroll
-        for (int j = KMAX; j > 0; --j) {
-            if (keys[j] > keys[j - 1]) {
-                const uint64_t tk = keys[j];
-                keys[j] = keys[j - 1];
-                keys[j - 1] = tk;
-                const float ts = sv[j];
-                sv[j] = sv[j - 1];
-                sv[j - 1] = ts;
-            }
-        }
-    }
+    const uint32_t hi = static_cast<uint32_t>(key >> 32), lo = static_cast<uint32_t>(key);
+    const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+    const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+    return (static_cast<uint64_t>(mhi) << 32) | mlo;
 }
 
-template <int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     router_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wr,
-                  const RouterArgs a, const int sl, const WaitCfg wc)
+                  const RouterArgs a, const int e_pad, const WaitCfg wc)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *smem = smem_raw + pad;
-    const Layout<KMAX> L(sl);
-    uint64_t *list_keys = reinterpret_cast<uint64_t *>(smem + L.list_off);
-    float *list_s = reinterpret_cast<float *>(smem + L.list_off + kTileM * (KMAX + 1) * 8);
-    float *bias_s = reinterpret_cast<float *>(smem + L.bias_off);
+    const Layout L(e_pad);
+    float *part = reinterpret_cast<float *>(smem);  // [tok][part_stride], over the ring after the main loop
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *empty = full + kMaxStages;
     uint64_t *accf = empty + kMaxStages;
     uint64_t *drain = accf + 1;
     uint32_t *holder = reinterpret_cast<uint32_t *>(smem + L.misc_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc_off + 4);
+    volatile int *ok_flag = reinterpret_cast<volatile int *>(smem + L.misc_off + 8);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();
-    const int ns = static_cast<int>(gridDim.x);
-    const int e0 = static_cast<int>(blockIdx.x) * sl;
-    const int ne = (a.E - e0) < sl ? (a.E - e0) : sl;  // experts of this slice (>= 1)
-    const int m0 = blockIdx.y * kTileM;
-    const int nkb = a.H / kBK;
+    const int S = static_cast<int>(gridDim.x);  // the cluster: the S CTAs of one token tile
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int m0 = static_cast<int>(blockIdx.y) * L.tok;
+    const int nkb = a.H / (kBK * S);  // K stages of this CTA
+    const int kb0 = rank * nkb;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxStages; ++s) {
@@ -133,10 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(accf, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
+        *ok_flag = 1;
         fence_barrier_init();
     }
-    for (int e = threadIdx.x; e < sl; e += kThreads)
-        bias_s[e] = e < ne ? a.bias[e0 + e] : 0.0f;
     if (warp == 1) {
         tmem_alloc(holder, L.tmem_cols);
         tmem_relinquish();
@@ -145,36 +138,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *holder;
-    const int box = sl <= 256 ? sl : sl / 2;  // Wr rows per TMA box (one or two per stage)
-
-    // registers of the epilogue thread's list (kept across the cluster barrier in CTA 0)
-    uint64_t keys[KMAX + 1];
-    float sv[KMAX + 1];
-#pragma unroll
-    for (int j = 0; j <= KMAX; ++j) {
-        keys[j] = 0;
-        sv[j] = 0.0f;
-    }
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
 
     if (warp == 0) {
         if (lane == 0) {
             tma_prefetch_map(&tm_x);
             tma_prefetch_map(&tm_wr);
-            const uint32_t tx = kABytes + static_cast<uint32_t>(sl) * 128;
+            const uint32_t tx = kABytes + L.b_bytes;
+            const int box = e_pad <= 256 ? e_pad : e_pad / 2;  // Wr rows per TMA box
             int issued = 0;
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % L.stages;
-                const uint32_t ph = (kb / L.stages) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, wc, abort_flag))
+                if (!mbar_wait(&empty[s], ((kb / L.stages) & 1) ^ 1, wc, abort_flag))
                     break;
                 mbar_arrive_expect_tx(&full[s], tx);
                 uint8_t *A = smem + s * L.stage_bytes;
                 uint8_t *B = A + kABytes;
-                tma_load_2d(A, &tm_x, &full[s], kb * kBK, m0);
-                for (int r = 0; r < sl; r += box)
-                    tma_load_2d(B + r * 128, &tm_wr, &full[s], kb * kBK, e0 + r);
+                tma_load_2d(A, &tm_x, &full[s], (kb0 + kb) * kBK, m0);
+                for (int r = 0; r < e_pad; r += box)
+                    tma_load_2d(B + r * 128, &tm_wr, &full[s], (kb0 + kb) * kBK, r);
                 ++issued;
             }
             for (int kb = issued > L.stages ? issued - L.stages : 0; kb < issued; ++kb)
@@ -182,16 +163,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // N up to 256 per MMA: a slice of more than 256 experts takes two MMAs
-            const int n0 = sl < 256 ? sl : 256;
-            const int n1 = sl - n0;
+            // N up to 256 per MMA: more than 256 experts take two MMAs
+            const int n0 = e_pad < 256 ? e_pad : 256;
+            const int n1 = e_pad - n0;
             const uint32_t id0 = idesc_bf16_f32(kTileM, n0);
             const uint32_t id1 = idesc_bf16_f32(kTileM, n1 > 0 ? n1 : 16);
             bool ok = true;
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % L.stages;
-                const uint32_t ph = (kb / L.stages) & 1;
-                if (!mbar_wait(&full[s], ph, wc, abort_flag)) {
+                if (!mbar_wait(&full[s], (kb / L.stages) & 1, wc, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -213,92 +193,122 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(drain);
             mbar_wait_drain(drain, 0, wc);
         }
-    } else {
-        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31; one thread per token row
+    } else if (warp < 6) {
+        // warps 2-5: TMEM lane quarter q (token rows 32q .. 32q+31) -> the partial tile. Every
+        // MMA has completed (accf), so every stage of the ring has been consumed.
         bool ok = false;
         if (lane == 0)
             ok = mbar_wait(accf, 0, wc, abort_flag);
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         tc_fence_after();
         if (ok) {
+            const int q = warp & 3;
+            const int row = q * 32 + lane;
             const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
-            for (int c0 = 0; c0 < ne; c0 += 32) {
+            for (int c0 = 0; c0 < e_pad; c0 += 32) {
                 float v[32];
                 tmem_load32(tbase + c0, v);
+                if (row < L.tok) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int e = c0 + i;
-                    if (e < ne) {
-                        const float s = 1.0f / (1.0f + expf(-v[i]));
-                        const float b = s + bias_s[e];
-                        list_insert<KMAX>(keys, sv, rank_key(b, e0 + e), s);
-                    }
+                    for (int i = 0; i < 32; ++i)
+                        if (c0 + i < e_pad)
+                            part[row * L.part_stride + c0 + i] = v[i];
                 }
             }
-        }
-        if (rank != 0) {
-#pragma unroll
-            for (int j = 0; j <= KMAX; ++j) {
-                list_keys[row * (KMAX + 1) + j] = keys[j];
-                list_s[row * (KMAX + 1) + j] = sv[j];
-            }
+        } else if (lane == 0) {
+            *ok_flag = 0;
         }
     }
 
-    // Lists of CTAs 1..ns-1 become visible to CTA 0; every thread of every CTA gets here.
+    // The partial tiles of all S CTAs are complete and visible cluster-wide.
+    tc_fence_before();
     cluster_sync_all();
 
-    if (rank == 0 && warp >= 2) {
-        const uint32_t keys_local = smem_u32(list_keys + row * (KMAX + 1));
-        const uint32_t s_local = smem_u32(list_s + row * (KMAX + 1));
-        for (int p = 1; p < ns; ++p) {
-            const uint32_t kp = dsmem_addr(keys_local, p);
-            const uint32_t sp = dsmem_addr(s_local, p);
-            for (int j = 0; j <= KMAX; ++j) {
-                const uint64_t key = dsmem_ld_u64(kp + 8 * j);
-                if (key <= keys[KMAX])
-                    break;  // peer lists are sorted: nothing further can enter
-                list_insert<KMAX>(keys, sv, key, dsmem_ld_f32(sp + 4 * j));
-            }
-        }
-        const int t = m0 + row;
-        if (t < a.T) {
-            const int k = a.k;
-            float sum = 0.0f;
+    bool all_ok = true;
+    for (int p = 0; p < S; ++p)
+        all_ok = all_ok && dsmem_ld_s32(dsmem_addr(smem_u32(const_cast<int *>(ok_flag)), p)) != 0;
+    if (all_ok) {
+        // this CTA's share of the tile's tokens, one warp per token
+        const int per = (L.tok + S - 1) / S;
+        const int t_hi = (rank + 1) * per < L.tok ? (rank + 1) * per : L.tok;
+        const float *peer[8];
 #pragma unroll
-            for (int j = 0; j < KMAX; ++j)
-                if (j < k)
-                    sum += sv[j];
+        for (int p = 0; p < 8; ++p)
+            peer[p] = peer_ptr(part, static_cast<uint32_t>(p < S ? p : 0));
+        const int rounds = a.k < a.E ? a.k + 1 : a.k;
+        for (int tt = rank * per + warp; tt < t_hi; tt += kWarps) {
+            const int t = m0 + tt;
+            if (t >= a.T)
+                break;
+            // lane l holds experts l, l + 32, ...: logit = sum of the S partials in rank order
+            uint64_t key[kMaxKeysPerLane];
+            float sc[kMaxKeysPerLane];
 #pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-                if (j < k) {
-                    int e = key_expert(keys[j]);
-                    e = e < 0 ? 0 : (e > a.E - 1 ? a.E - 1 : e);
-                    float w;
-                    if (a.norm)
-                        w = sum > 0.0f ? a.scale * (sv[j] / sum) : a.scale / static_cast<float>(k);
-                    else
-                        w = a.scale * sv[j];
-                    a.idx[static_cast<int64_t>(t) * k + j] = e;
-                    a.w[static_cast<int64_t>(t) * k + j] = w;
+            for (int i = 0; i < kMaxKeysPerLane; ++i) {
+                const int e = lane + 32 * i;
+                key[i] = 0;
+                sc[i] = 0.0f;
+                if (e < a.E) {
+                    const int off = tt * static_cast<int>(L.part_stride) + e;
+                    float l = 0.0f;
+#pragma unroll
+                    for (int p = 0; p < 8; ++p)
+                        if (p < S)
+                            l += peer[p][off];
+                    const float s = 1.0f / (1.0f + expf(-l));
+                    key[i] = rank_key(s + a.bias[e], e);
+                    sc[i] = s;
                 }
             }
-            // k-th and (k+1)-th keys picked by a compare-and-select chain (a dynamic
-            // index would move the list to local memory)
-            uint64_t key_k = 0, key_k1 = 0;
+            // k (+1 for the margin) rounds of a warp-wide maximum: lane j keeps round j's
+            // expert and score (lane 0 also round 32's key); the normalisation sum and the
+            // margin keys are warp-uniform, accumulated in rank order
+            const int k = a.k;
+            uint64_t my_key = 0, key_k = 0, key_k1 = 0;
+            float my_s = 0.0f, sum = 0.0f;
+            for (int j = 0; j < rounds; ++j) {
+                uint64_t best = 0;
+                float best_s = 0.0f;
 #pragma unroll
-            for (int j = 0; j <= KMAX; ++j) {
-                const bool at_k = (j + 1 == k), at_k1 = (j == k);
-                key_k = at_k ? keys[j] : key_k;
-                key_k1 = at_k1 ? keys[j] : key_k1;
-                asm volatile("" : "+l"(key_k), "+l"(key_k1));
+                for (int i = 0; i < kMaxKeysPerLane; ++i) {
+                    const bool gt = key[i] > best;
+                    best = gt ? key[i] : best;
+                    best_s = gt ? sc[i] : best_s;
+                }
+                const uint64_t m = warp_max_key(best);
+                const unsigned owner = __ballot_sync(0xFFFFFFFFu, best == m && m != 0);
+                const float ms = __shfl_sync(0xFFFFFFFFu, best_s, owner ? __ffs(owner) - 1 : 0);
+                if (best == m) {
+#pragma unroll
+                    for (int i = 0; i < kMaxKeysPerLane; ++i)
+                        key[i] = key[i] == m ? 0ull : key[i];
+                }
+                if (lane == (j & 31) && j < k) {
+                    my_key = m;
+                    my_s = ms;
+                }
+                if (j < k)
+                    sum += ms;
+                key_k = j + 1 == k ? m : key_k;
+                key_k1 = j == k ? m : key_k1;
             }
-            if (a.margin)
+            if (lane < k) {
+                int e = key_expert(my_key);
+                e = e < 0 ? 0 : (e > a.E - 1 ? a.E - 1 : e);
+                float w;
+                if (a.norm)
+                    w = sum > 0.0f ? a.scale * (my_s / sum) : a.scale / static_cast<float>(k);
+                else
+                    w = a.scale * my_s;
+                a.idx[static_cast<int64_t>(t) * k + lane] = e;
+                a.w[static_cast<int64_t>(t) * k + lane] = w;
+            }
+            if (lane == 0 && a.margin)
                 a.margin[t] = k < a.E ? key_value(key_k) - key_value(key_k1) : __int_as_float(0x7F800000);
         }
     }
 
-    // CTA 0 has finished reading its peers' shared memory before any CTA exits.
+    // Peers have finished reading this CTA's partial tile before any CTA exits.
     cluster_sync_all();
 
     tc_fence_before();
@@ -309,29 +319,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int KMAX>
 cudaError_t launch_impl(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const RouterArgs &a,
                         const WaitCfg &wc, cudaStream_t stream)
 {
-    const RouterSplit sp = router_split(a.E, a.T, a.num_sms);
-    const Layout<KMAX> L(sp.sl);
+    const RouterSplit sp = router_split(a.E, a.T, a.H, a.num_sms);
+    const Layout L(sp.e_pad);
     const int smem = static_cast<int>(L.total) + 1024;
-    cudaError_t err = cudaFuncSetAttribute(router_kernel<KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(sp.ns, (a.T + kTileM - 1) / kTileM, 1);
+    cfg.gridDim = dim3(sp.ks, (a.T + L.tok - 1) / L.tok, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = sp.ns;
+    attr[0].val.clusterDim.x = sp.ks;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, router_kernel<KMAX>, tm_x, tm_wr, a, sp.sl, wc);
+    err = cudaLaunchKernelEx(&cfg, router_kernel, tm_x, tm_wr, a, sp.e_pad, wc);
     if (err != cudaSuccess)
         return err;
     return cudaGetLastError();
@@ -339,36 +348,28 @@ cudaError_t launch_impl(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const
 
 }  // namespace
 
-// Enough CTAs to cover the SMs once: with few token tiles (decode) the experts are split
-// over up to 8 CTAs; with many token tiles each CTA keeps all experts, so x is read once.
-// Slices above 256 experts are a multiple of 32, loaded as two Wr boxes of sl / 2 rows.
-RouterSplit router_split(int E, int T, int num_sms)
+// K split S (a power of two up to 8 that divides H / 64) so that about one CTA runs per SM:
+// token tiles x S ~ num_sms. All experts in every CTA (E padded to a multiple of 16; above
+// 256 experts the Wr rows of a stage come as two boxes of E_pad / 2 rows).
+RouterSplit router_split(int E, int T, int H, int num_sms)
 {
-    const int tiles = (T + kTileM - 1) / kTileM;
     const int e_pad = (E + 15) / 16 * 16;
-    int ns = num_sms / tiles;
-    ns = ns < 1 ? 1 : (ns > 8 ? 8 : ns);
-    ns = ns > e_pad / 16 ? e_pad / 16 : ns;
-    int sl = ((e_pad + ns - 1) / ns + 15) / 16 * 16;
-    if (sl > 256)
-        sl = (sl + 31) / 32 * 32;
+    const Layout L(e_pad);
+    const int tiles = (T + L.tok - 1) / L.tok;
+    int ks = 1;
+    while (ks < 8 && tiles * ks * 2 <= num_sms && (H / kBK) % (ks * 2) == 0)
+        ks *= 2;
     RouterSplit r;
-    r.sl = sl;
-    r.ns = (E + sl - 1) / sl;
-    r.box_rows = sl <= 256 ? sl : sl / 2;
+    r.e_pad = e_pad;
+    r.ks = ks;
+    r.box_rows = e_pad <= 256 ? e_pad : e_pad / 2;
     return r;
 }
 
 cudaError_t launch_router(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const RouterArgs &a,
                           const WaitCfg &wc, cudaStream_t stream)
 {
-    if (a.k <= 4)
-        return launch_impl<4>(tm_x, tm_wr, a, wc, stream);
-    if (a.k <= 8)
-        return launch_impl<8>(tm_x, tm_wr, a, wc, stream);
-    if (a.k <= 16)
-        return launch_impl<16>(tm_x, tm_wr, a, wc, stream);
-    return launch_impl<32>(tm_x, tm_wr, a, wc, stream);
+    return launch_impl(tm_x, tm_wr, a, wc, stream);
 }
 
 }  // namespace moe

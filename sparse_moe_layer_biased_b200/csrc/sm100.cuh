@@ -155,6 +155,16 @@ __device__ __forceinline__ uint32_t dsmem_addr(uint32_t local_saddr, uint32_t ra
     return r;
 }
 
+// Generic pointer to the same shared-memory variable in CTA `rank` of this cluster: ordinary
+// loads through it reach the peer's shared memory and can be scheduled like any other load.
+template <class T>
+__device__ __forceinline__ const T *peer_ptr(const T *local, uint32_t rank)
+{
+    uint64_t out;
+    asm volatile("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"(reinterpret_cast<uint64_t>(local)), "r"(rank));
+    return reinterpret_cast<const T *>(out);
+}
+
 __device__ __forceinline__ uint64_t dsmem_ld_u64(uint32_t addr)
 {
     uint64_t v;
