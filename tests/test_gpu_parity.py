@@ -28,6 +28,11 @@ SMALL = {
     "kE": LayerShape("kE", T=50, H=128, E=8, k=8, I=64, Is=128, seed=23),
     "wideE": LayerShape("wideE", T=700, H=256, E=300, k=8, I=64, Is=64, seed=24),
     "k32": LayerShape("k32", T=129, H=256, E=64, k=32, I=128, Is=64, seed=25),
+    # the most experts (512 > 384: the router keeps 64-token tiles so a tile's partial
+    # logits fit in shared memory), three ragged tiles, K split over the cluster
+    "E512": LayerShape("E512", T=150, H=512, E=512, k=8, I=64, Is=64, seed=33),
+    # E = 392: 64-token tiles from a ring of three 63 KB stages
+    "E392": LayerShape("E392", T=333, H=256, E=392, k=12, I=64, Is=64, seed=34),
     "nonorm": WORKLOADS["tiny"].replace(name="nonorm", norm_expert_weight=False, scale=2.5),
     # two weight tiles per stage on single CTAs (I, Is multiples of 128, H of 256 but not
     # of 512; > 16 tokens per expert)
