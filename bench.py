@@ -48,8 +48,9 @@ def parse():
                          "(fake balanced static expert routing)")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
                     help="routed expert weights: bf16, or FP8 E4M3 with 128x128 block scales (moe_forward_fp8)")
-    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
-                    help="backward: time moe_backward (all gradients) for the forward's routing")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward", "router"],
+                    help="backward: time moe_backward (all gradients) for the forward's routing; "
+                         "router: time moe_router alone (profiling)")
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
                     help="ep: expert parallelism, E/N routed experts per rank, T tokens per rank")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
@@ -547,6 +548,39 @@ def run_ep(args, shape):
         print(json.dumps(line), flush=True)
 
 
+def run_router_only(args, shape):
+    """Times moe_router alone on the workload's x, router weights and bias (the same draw as
+    the layer; the expert tensors are drawn at I = Is = 64 to keep the device footprint
+    small). One GPU; one router_kernel launch per step."""
+    import torch
+
+    from sparse_moe_layer_biased_b200 import _abi
+    from sparse_moe_layer_biased_b200.inputs import draw
+
+    torch.cuda.set_device(0)
+    inp = draw(shape.replace(I=64, Is=64), device="cuda")
+    d = _abi.desc_of(shape)
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((shape.T, shape.k), dtype=torch.float32, device="cuda")
+    for _ in range(max(1, args.warmup)):
+        _abi.moe_router(d, inp["x"], inp["Wr"], inp["bias"], idx, w)
+    torch.cuda.synchronize()
+    _abi.moe_check_device()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(args.steps):
+        _abi.moe_router(d, inp["x"], inp["Wr"], inp["bias"], idx, w)
+    end.record()
+    torch.cuda.synchronize()
+    _abi.moe_check_device()
+    ms = start.elapsed_time(end) / args.steps
+    print(json.dumps({"metric": "MoE router tokens/s on 1 B200", "value": shape.T / (ms / 1e3), "unit": UNIT,
+                      "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                      "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded draw on device)",
+                      "config": workload_config(shape, {"pass": "router"}), "gpu_launches": args.steps}),
+          flush=True)
+
+
 def run_backward(args, shape):
     """Times moe_backward (dx, dWr, dW_gate_up, dW_down and the shared expert's gradients) on
     device-resident inputs for the forward's routing; one GPU. Algorithmic FLOPs per routed
@@ -614,6 +648,8 @@ def main():
         run_reference(args, shape)
     elif args.which == "backward":
         run_backward(args, shape)
+    elif args.which == "router":
+        run_router_only(args, shape)
     elif args.parallel == "ep":
         run_ep(args, shape)
     else:
