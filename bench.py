@@ -384,7 +384,7 @@ def run_b200(args, shape):
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
-    if not args.no_e2e and not fp8 and args.routing == "router":
+    if not args.no_e2e and args.routing == "router":
         # moe_forward_host: every step's batch comes from pinned host memory and its output
         # goes back to it; the copies overlap the forward of the neighbouring batch
         per_batch = shape.T * shape.H * 6

@@ -178,21 +178,25 @@ MOE_API moe_status_t moe_forward_fp8(const moe_layer_desc *desc, const uint16_t 
  * and two [T, H] fp32 output staging buffers. */
 MOE_API moe_status_t moe_host_workspace_size(const moe_layer_desc *desc, size_t *bytes);
 
-/* moe_forward over n_batches batches of T tokens that live in host memory: the layer of a
- * serving or inference loop fed from the host.
+/* moe_forward (or moe_forward_fp8) over n_batches batches of T tokens that live in host
+ * memory: the layer of a serving or inference loop fed from the host.
  *   x_host [n_batches, T, H] bf16 and y_host [n_batches, T, H] fp32 in host memory (page-
  *   locked, e.g. cudaHostAlloc, for the copies to overlap; pageable memory works but the
  *   host then waits for each copy); batch i's layer output is written to y_host[i].
- *   Weights, desc and the routing as in moe_forward; ws of at least moe_host_workspace_size.
+ *   W_gate_up_scale, W_down_scale: NULL for BF16 routed experts (W_gate_up, W_down bf16 as in
+ *   moe_forward), or the 128x128 block scales of FP8 E4M3 routed experts (W_gate_up, W_down
+ *   the E4M3 codes, as in moe_forward_fp8); both NULL or both given.
+ *   Other weights, desc and the routing as in moe_forward; ws of at least
+ *   moe_host_workspace_size.
  * The copies run on two internal streams, double-buffered in ws: batch i+1's input copy
  * and batch i-1's output copy overlap batch i's forward on `stream`. The call only enqueues
  * work; when `stream` has completed, every output row is in y_host. n_batches = 0 or T = 0
  * is a no-op. */
 MOE_API moe_status_t moe_forward_host(const moe_layer_desc *desc, int32_t n_batches, const uint16_t *x_host,
-                                      const uint16_t *Wr, const float *bias, const uint16_t *W_gate_up,
-                                      const uint16_t *W_down, const uint16_t *Wsh_gate_up,
-                                      const uint16_t *Wsh_down, float *y_host, void *ws, size_t ws_bytes,
-                                      void *stream);
+                                      const uint16_t *Wr, const float *bias, const void *W_gate_up,
+                                      const float *W_gate_up_scale, const void *W_down, const float *W_down_scale,
+                                      const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y_host,
+                                      void *ws, size_t ws_bytes, void *stream);
 
 /* ---- Expert parallelism ("MAX 中 Step-3.5-Flash 架构解析", section "并行模式TP_TP / TP_EP /
  * DP_EP": in DP_EP each rank runs its own batch shard, the routed experts are split across

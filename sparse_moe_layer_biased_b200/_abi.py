@@ -82,7 +82,7 @@ def lib():
         L.moe_ep_experts.argtypes = [dp, ctypes.c_int32] + [vp] * 7 + [sz, vp]
         L.moe_shared_expert.argtypes = [dp] + [vp] * 5 + [sz, vp]
         L.moe_host_workspace_size.argtypes = [dp, ctypes.POINTER(sz)]
-        L.moe_forward_host.argtypes = [dp, ctypes.c_int32] + [vp] * 9 + [sz, vp]
+        L.moe_forward_host.argtypes = [dp, ctypes.c_int32] + [vp] * 11 + [sz, vp]
         for name in ("moe_ep_pack", "moe_ep_experts", "moe_shared_expert", "moe_host_workspace_size",
                      "moe_forward_host"):
             getattr(L, name).restype = i32
@@ -238,8 +238,8 @@ def moe_host_workspace_size(desc: LayerDesc) -> int:
 
 
 def moe_forward_host(desc, n_batches, x_host, Wr, bias, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y_host, ws,
-                     stream=None):
+                     stream=None, W_gate_up_scale=None, W_down_scale=None):
     _check("moe_forward_host", lib().moe_forward_host(
-        ctypes.byref(desc), int(n_batches), _p(x_host), _p(Wr), _p(bias), _p(W_gate_up), _p(W_down),
-        _p(Wsh_gate_up), _p(Wsh_down), _p(y_host), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
-        _stream(stream)))
+        ctypes.byref(desc), int(n_batches), _p(x_host), _p(Wr), _p(bias), _p(W_gate_up), _p(W_gate_up_scale),
+        _p(W_down), _p(W_down_scale), _p(Wsh_gate_up), _p(Wsh_down), _p(y_host), _p(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))

@@ -561,14 +561,15 @@ moe_status_t moe_host_workspace_size(const moe_layer_desc *desc, size_t *bytes)
 }
 
 moe_status_t moe_forward_host(const moe_layer_desc *desc, int32_t n_batches, const uint16_t *x_host,
-                              const uint16_t *Wr, const float *bias, const uint16_t *W_gate_up, const uint16_t *W_down,
-                              const uint16_t *Wsh_gate_up, const uint16_t *Wsh_down, float *y_host, void *ws,
-                              size_t ws_bytes, void *stream)
+                              const uint16_t *Wr, const float *bias, const void *W_gate_up, const float *W_gate_up_scale,
+                              const void *W_down, const float *W_down_scale, const uint16_t *Wsh_gate_up,
+                              const uint16_t *Wsh_down, float *y_host, void *ws, size_t ws_bytes, void *stream)
 {
     moe_status_t st = check_desc(desc);
     if (st != MOE_OK)
         return st;
-    if (n_batches < 0)
+    const bool fp8 = W_gate_up_scale != nullptr;
+    if (n_batches < 0 || fp8 != (W_down_scale != nullptr))
         return MOE_ERR_INVALID_ARG;
     if (desc->T == 0 || n_batches == 0)
         return MOE_OK;  // nothing to do; array pointers may be NULL
@@ -612,8 +613,12 @@ moe_status_t moe_forward_host(const moe_layer_desc *desc, int32_t n_batches, con
             st = MOE_ERR_CUDA;
             break;
         }
-        st = moe_forward(desc, xd[b], Wr, bias, W_gate_up, W_down, Wsh_gate_up, Wsh_down, yd[b], nullptr, nullptr,
-                         ws, L.x0, stream);
+        st = fp8 ? moe_forward_fp8(desc, xd[b], Wr, bias, static_cast<const uint8_t *>(W_gate_up), W_gate_up_scale,
+                                   static_cast<const uint8_t *>(W_down), W_down_scale, Wsh_gate_up, Wsh_down, yd[b],
+                                   nullptr, nullptr, ws, L.x0, stream)
+                 : moe_forward(desc, xd[b], Wr, bias, static_cast<const uint16_t *>(W_gate_up),
+                               static_cast<const uint16_t *>(W_down), Wsh_gate_up, Wsh_down, yd[b], nullptr, nullptr,
+                               ws, L.x0, stream);
         if (st != MOE_OK)
             break;
         if (cudaEventRecord(ev_comp[b], s) != cudaSuccess || cudaStreamWaitEvent(d2h, ev_comp[b], 0) != cudaSuccess ||

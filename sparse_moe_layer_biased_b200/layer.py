@@ -52,10 +52,9 @@ class MoeLayer:
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor | None = None, stream=None):
         """The layer over batches in host memory: x_host [n, T, H] bf16 -> y_host [n, T, H]
-        fp32 (page-locked tensors for overlapped copies) through moe_forward_host. Returns
-        y_host once the work is enqueued; synchronize the stream before reading it."""
-        if self.fp8:
-            raise ValueError("forward_host runs BF16 routed experts")
+        fp32 (page-locked tensors for overlapped copies) through moe_forward_host, with BF16
+        or FP8 routed experts. Returns y_host once the work is enqueued; synchronize the
+        stream before reading it."""
         n, T, H = x_host.shape
         if T > self.max_tokens:
             raise ValueError(f"{T} tokens exceed the workspace size of {self.max_tokens}")
@@ -66,6 +65,11 @@ class MoeLayer:
         if y_host is None:
             y_host = torch.empty((n, T, H), dtype=torch.float32, pin_memory=True)
         W = self.w
-        _abi.moe_forward_host(desc, n, x_host, W["Wr"], W["bias"], W["W_gate_up"], W["W_down"], W["Wsh_gate_up"],
-                              W["Wsh_down"], y_host, self.ws_host, stream=stream)
+        if self.fp8:
+            _abi.moe_forward_host(desc, n, x_host, W["Wr"], W["bias"], W["W_gate_up_q"], W["W_down_q"],
+                                  W["Wsh_gate_up"], W["Wsh_down"], y_host, self.ws_host, stream=stream,
+                                  W_gate_up_scale=W["W_gate_up_s"], W_down_scale=W["W_down_s"])
+        else:
+            _abi.moe_forward_host(desc, n, x_host, W["Wr"], W["bias"], W["W_gate_up"], W["W_down"],
+                                  W["Wsh_gate_up"], W["Wsh_down"], y_host, self.ws_host, stream=stream)
         return y_host

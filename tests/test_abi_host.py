@@ -206,14 +206,18 @@ def test_forward_host_validation():
     d = _desc()
     need = moe.moe_host_workspace_size(d)
     assert need > moe.moe_workspace_size(d)
-    args = [FAKE] * 9  # x_host, Wr, bias, W_gate_up, W_down, Wsh_gate_up, Wsh_down, y_host, ws
+    # x_host, Wr, bias, W_gate_up, W_gate_up_scale, W_down, W_down_scale, Wsh_gate_up, Wsh_down, y_host, ws
+    args = [FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, FAKE, FAKE, FAKE]
     assert L.moe_forward_host(ctypes.byref(d), -1, *args, need, None) == 1
     assert L.moe_forward_host(ctypes.byref(d), 2, *args, need - 1, None) == 3
     a = list(args)
-    a[7] = None  # y_host
+    a[9] = None  # y_host
     assert L.moe_forward_host(ctypes.byref(d), 2, *a, need, None) == 1
     a = list(args)
-    a[8] = FAKE + 8  # workspace not 16-byte aligned
+    a[10] = FAKE + 8  # workspace not 16-byte aligned
     assert L.moe_forward_host(ctypes.byref(d), 2, *a, need, None) == 2
-    assert L.moe_forward_host(ctypes.byref(d), 0, *([None] * 9), 0, None) == 0
-    assert L.moe_forward_host(ctypes.byref(_desc(T=0)), 3, *([None] * 9), 0, None) == 0
+    a = list(args)
+    a[4] = FAKE  # one FP8 scale array without the other
+    assert L.moe_forward_host(ctypes.byref(d), 2, *a, need, None) == 1
+    assert L.moe_forward_host(ctypes.byref(d), 0, *([None] * 11), 0, None) == 0
+    assert L.moe_forward_host(ctypes.byref(_desc(T=0)), 3, *([None] * 11), 0, None) == 0

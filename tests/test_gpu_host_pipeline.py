@@ -12,7 +12,7 @@ import torch
 from _parity import check_output
 import oracle
 from sparse_moe_layer_biased_b200 import _abi
-from sparse_moe_layer_biased_b200.inputs import WORKLOADS, LayerShape, draw
+from sparse_moe_layer_biased_b200.inputs import WORKLOADS, LayerShape, draw, draw_fp8
 from sparse_moe_layer_biased_b200.layer import MoeLayer
 
 pytestmark = pytest.mark.gpu
@@ -63,3 +63,17 @@ def test_forward_host_against_oracle():
     ref = oracle.forward_full(inp, sh)
     keep = ref["margin"] >= 1e-6  # near-tied selections are excluded as in the layer's parity tests
     check_output(y[0].numpy()[keep], ref["y"][keep], "tiny host")
+
+
+def test_forward_host_fp8_equals_device_forward():
+    sh = SHAPE.replace(name="host_pipe_fp8", weight_std=0.03)
+    layer = MoeLayer(sh, {k: v.cuda() for k, v in draw_fp8(sh).items()}, deterministic=True)
+    assert layer.fp8
+    xs = _batches(sh, 3)
+    y_host = layer.forward_host(xs.pin_memory())
+    torch.cuda.synchronize()
+    _abi.moe_check_device()
+    for i in range(3):
+        y_dev = layer.forward(xs[i].cuda())
+        torch.cuda.synchronize()
+        assert torch.equal(y_host[i], y_dev.cpu()), f"batch {i}"
