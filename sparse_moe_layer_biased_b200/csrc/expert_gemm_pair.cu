@@ -6,9 +6,11 @@
 // cluster (an SM pair) work on one tile: each holds MT weight tiles of 128 rows and HALF
 // of the token rows of the chunk; the leader CTA issues M = 256 MMAs that read the weight
 // rows of both CTAs and the token rows of both, and each CTA's TMEM receives its own 128
-// weight rows x all N tokens. Per SM, the token bytes per stage halve and the ring gets a
-// fifth stage, so more weight bytes are in flight (the HBM-bound case) and each MMA reads
-// half as many token bytes from this SM's shared memory (the compute-bound case).
+// weight rows x all N tokens. Per SM, the token bytes per stage halve, so more weight bytes
+// are in flight (the HBM-bound case) and each MMA reads half as many token bytes from this
+// SM's shared memory (the compute-bound case). gate_up stages hold two 64-wide K slices:
+// the single MMA-issuing thread then pays its per-stage barrier test and commit once per
+// 8 pair MMAs instead of 4.
 //
 // Pair protocol (leader = cluster rank 0):
 //   - both producers load into their own shared memory; the transaction bytes of both
@@ -36,11 +38,14 @@ constexpr uint32_t kTokBoxBytes = kTokBoxRows * 128;
 // NB = accumulator buffers in TMEM (2: the epilogue of one tile overlaps the next tile's
 // mainloop; 1: larger tiles, the MMA waits for the epilogue between tiles).
 // OUT = bytes of output staging after the ring (the down epilogue's bulk-reduction buffers).
-template <int BN, int S, int MT, int NB, int OUT = 0>
+// NSL = 64-wide K slices per stage, each laid out as [MT weight tiles][token rows]: more MMAs
+// per barrier wait and commit of the single MMA-issuing thread, fewer stages.
+template <int BN, int S, int MT, int NB, int OUT = 0, int NSL = 1>
 struct PairGeo {
     static constexpr uint32_t kABytes = MT * kATileBytes;
     static constexpr uint32_t kBBytes = (BN / 2) * 128;
-    static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+    static constexpr uint32_t kSliceBytes = kABytes + kBBytes;
+    static constexpr uint32_t kStageBytes = NSL * kSliceBytes;
     static constexpr uint32_t kOutOff = S * kStageBytes;
     static constexpr uint32_t kBarOff = kOutOff + OUT;
     static constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * S + 5);  // holder, abort flag, epilogue flags
@@ -48,7 +53,7 @@ struct PairGeo {
     static constexpr uint32_t kBufCols = MT * BN;
     static constexpr uint32_t kTmemCols = NB * kBufCols <= 32 ? 32 : (NB * kBufCols <= 64 ? 64 : (NB * kBufCols <= 128 ? 128 : (NB * kBufCols <= 256 ? 256 : 512)));
     static_assert(NB * kBufCols <= 512, "accumulators exceed TMEM");
-    static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
+    static_assert(kSliceBytes % 1024 == 0, "slices must stay 1024-byte aligned");
     static_assert(kSmemBytes <= kMaxDynSmem, "ring exceeds shared memory");
 
     static_assert(BN % 32 == 0 && BN <= 256, "pair token tile");
@@ -135,9 +140,9 @@ __device__ __forceinline__ void pair_producer_drain(const PairRing &r, int issue
         mbar_wait_drain(&r.full[it % S], (it / S) & 1, wc);
 }
 
-// Leader's MMA issue for one pair tile: nkb K-slices; weight tile m accumulates into
-// columns [d + m*BN, d + m*BN + n) of both CTAs' TMEM.
-template <class G, int S, int BN, int MT>
+// Leader's MMA issue for one pair tile: nkb stages of NSL 64-wide K slices; weight tile m
+// accumulates into columns [d + m*BN, d + m*BN + n) of both CTAs' TMEM.
+template <class G, int S, int BN, int MT, int NSL>
 __device__ __forceinline__ bool pair_mma_tile(const PairRing &r, uint8_t *smem, uint32_t d, int n, int nkb,
                                               int &it, const WaitCfg &wc)
 {
@@ -147,14 +152,17 @@ __device__ __forceinline__ bool pair_mma_tile(const PairRing &r, uint8_t *smem, 
         if (!mbar_wait(&r.full[s], (it / S) & 1, wc, r.abort_flag))
             return false;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * G::kStageBytes);
-        const uint64_t bd = sdesc_kmajor_sw128(a_addr + G::kABytes);
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
+        for (int c = 0; c < NSL; ++c) {
+            const uint32_t a_addr = smem_u32(smem + s * G::kStageBytes + c * G::kSliceBytes);
+            const uint64_t bd = sdesc_kmajor_sw128(a_addr + G::kABytes);
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                const uint64_t ad = sdesc_kmajor_sw128(a_addr + m * kATileBytes);
-                umma_bf16_pair(d + m * BN, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    const uint64_t ad = sdesc_kmajor_sw128(a_addr + m * kATileBytes);
+                    umma_bf16_pair(d + m * BN, ad + 2 * kk, bd + 2 * kk, idesc, (kb | c | kk) != 0);
+                }
             }
         }
         umma_commit_pair_mc(&r.empty[s], 0x3);
@@ -163,7 +171,7 @@ __device__ __forceinline__ bool pair_mma_tile(const PairRing &r, uint8_t *smem, 
 }
 
 // The leader runs the MMA loop; the peer's MMA warp only waits for the final drain.
-template <class G, int S, int BN, int MT, int NB, class NextTile>
+template <class G, int S, int BN, int MT, int NB, int NSL, class NextTile>
 __device__ __forceinline__ void pair_mma_role(const PairRing &r, uint8_t *smem, uint32_t tmem, int first,
                                               int tiles, int stride, NextTile tile_info, const WaitCfg &wc)
 {
@@ -176,7 +184,8 @@ __device__ __forceinline__ void pair_mma_role(const PairRing &r, uint8_t *smem, 
             if (!mbar_wait(&r.acce[buf], ((tc / NB) & 1) ^ 1, wc, r.abort_flag))
                 break;
             tc_fence_after();
-            if (!pair_mma_tile<G, S, BN, MT>(r, smem, tmem + buf * G::kBufCols, (ntok + 15) & ~15, nkb, it, wc))
+            if (!pair_mma_tile<G, S, BN, MT, NSL>(r, smem, tmem + buf * G::kBufCols, (ntok + 15) & ~15, nkb, it,
+                                                  wc))
                 break;
             umma_commit_pair_mc(&r.accf[buf], 0x3);
         }
@@ -209,13 +218,13 @@ __device__ __forceinline__ void decode_gate_up_pair(const GateUpArgs &a, int nrc
     ntok = c.z;
 }
 
-template <int BN, int S, int MT, int NB>
+template <int BN, int S, int MT, int NB, int NSL>
 __global__ void __launch_bounds__(kThreads, 1)
     gate_up_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_wsh,
                         const __grid_constant__ CUtensorMap tm_xp, const __grid_constant__ CUtensorMap tm_x,
                         const GateUpArgs a, const WaitCfg wc)
 {
-    using G = PairGeo<BN, S, MT, NB>;
+    using G = PairGeo<BN, S, MT, NB, 0, NSL>;
     extern __shared__ uint8_t smem_raw[];
     PairRing r;
     uint8_t *smem = pair_setup<G, S>(smem_raw, r);
@@ -226,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ntot = a.hdr[1];
     const int tiles_r = nrc * (a.I / (128 * MT));
     const int tiles = tiles_r + (ntot - nrc) * (a.Is / (128 * MT));
-    const int nkb = a.H / kBK;
+    const int nkb = a.H / (kBK * NSL);  // stages per tile
     const int first = blockIdx.x >> 1;
     const int stride = gridDim.x >> 1;
 
@@ -256,14 +265,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (r.rank == 0)
-                        mbar_arrive_expect_tx(&r.full[s], 2 * (G::kABytes + nbox * kTokBoxBytes));
+                        mbar_arrive_expect_tx(&r.full[s], 2 * NSL * (G::kABytes + nbox * kTokBoxBytes));
                     const uint32_t bar = r.full_leader + 8 * s;
-                    uint8_t *A = smem + s * G::kStageBytes;
-                    // one box with this CTA's MT weight tiles, then the token boxes that
-                    // cover its half of the chunk (rows past the half are loaded and ignored)
-                    tma_load_4d_pair(A, mw, bar, kb * kBK, 0, wt0 * 64, ge);
-                    for (int b = 0; b < nbox; ++b)
-                        tma_load_2d_pair(A + G::kABytes + b * kTokBoxBytes, mb, bar, kb * kBK, brow + b * kTokBoxRows);
+                    // per K slice: one box with this CTA's MT weight tiles, then the token
+                    // boxes that cover its half of the chunk (rows past the half are loaded
+                    // and ignored)
+                    for (int c = 0; c < NSL; ++c) {
+                        uint8_t *A = smem + s * G::kStageBytes + c * G::kSliceBytes;
+                        const int k0 = (kb * NSL + c) * kBK;
+                        tma_load_4d_pair(A, mw, bar, k0, 0, wt0 * 64, ge);
+                        for (int b = 0; b < nbox; ++b)
+                            tma_load_2d_pair(A + G::kABytes + b * kTokBoxBytes, mb, bar, k0, brow + b * kTokBoxRows);
+                    }
                 }
             }
             pair_producer_drain<S>(r, it, stop || *r.abort_flag, wc);
@@ -275,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_gate_up_pair<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
                 nk = nkb;
             };
-            pair_mma_role<G, S, BN, MT, NB>(r, smem, tmem, first, tiles, stride, info, wc);
+            pair_mma_role<G, S, BN, MT, NB, NSL>(r, smem, tmem, first, tiles, stride, info, wc);
         }
     } else {
         const int q = warp & 3;
@@ -435,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_down_pair<MT>(a, tile, g, row0, ntok, fb);
                 nk = (g == a.E ? a.Is : a.I) / kBK;
             };
-            pair_mma_role<G, S, BN, MT, NB>(r, smem, tmem, first, tiles, stride, info, wc);
+            pair_mma_role<G, S, BN, MT, NB, 1>(r, smem, tmem, first, tiles, stride, info, wc);
         }
     } else {
         const int q = warp & 3;
@@ -499,7 +512,10 @@ cudaError_t launch_pairs(Kernel kernel, int smem, int grid, cudaStream_t stream,
 // one pass over their weights. down: 128 token rows x 512 output features, two weight
 // tiles per CTA and stage (40 KB stages, 4 deep) and two 16 KB output staging buffers for
 // the bulk reductions. Both keep two TMEM accumulators.
-using GateUpPair = PairGeo<kPairCapGateUp, 6, kPairMtGateUp, 2>;
+// gate_up: two 64-wide K slices per stage (8 pair MMAs per barrier test and commit of the
+// MMA thread), three 64 KB stages
+constexpr int kGateUpStages = 3, kGateUpSlices = 2;
+using GateUpPair = PairGeo<kPairCapGateUp, kGateUpStages, kPairMtGateUp, 2, 0, kGateUpSlices>;
 constexpr int kDownStages = 4, kDownOutBufs = 2;  // 4 x 40 KB ring + 2 x 16 KB output staging
 using DownPair = PairGeo<kPairCapDown, kDownStages, kPairMtDown, 2, kDownOutBufs * kOutTok * kPairMtDown * 512>;
 
@@ -509,7 +525,7 @@ cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_w
                                 const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
                                 cudaStream_t stream)
 {
-    return launch_pairs(gate_up_pair_kernel<kPairCapGateUp, 6, kPairMtGateUp, 2>,
+    return launch_pairs(gate_up_pair_kernel<kPairCapGateUp, kGateUpStages, kPairMtGateUp, 2, kGateUpSlices>,
                         static_cast<int>(GateUpPair::kSmemBytes), grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
 }
 
