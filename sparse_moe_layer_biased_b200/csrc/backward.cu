@@ -595,7 +595,9 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
     }
 }
 
-template <int MODE>
+// NSL = 64-wide K slices per stage (2: half as many stages of twice the size, so the MMA
+// thread's barrier test and commit cover 8 MMAs; the tile's K must be a multiple of 128).
+template <int MODE, int NSL>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap a_r, const __grid_constant__ CUtensorMap a_s,
                     const __grid_constant__ CUtensorMap b_r, const __grid_constant__ CUtensorMap b_s,
@@ -603,7 +605,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 {
     constexpr bool kAmn = MODE != kBwdGU;
     constexpr bool kBmn = MODE == kBwdWD || MODE == kBwdWGU;
-    constexpr int S = kBwdStages;
+    constexpr int S = kBwdStages / NSL;
+    constexpr uint32_t kStage = NSL * kBwdStage;
+    static_assert(S * kStage <= kBwdBarOff, "ring exceeds its region");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *smem = smem_raw + pad;
@@ -649,15 +653,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bool stop = false;
             for (int tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x) {
                 const BTile t = bwd_tile<MODE>(a, tile);
-                for (int k0 = 0; k0 < t.K; k0 += 64, ++it) {
+                for (int k0 = 0; k0 < t.K; k0 += 64 * NSL, ++it) {
                     const int s = it % S;
                     if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, wc, abort_flag)) {
                         stop = true;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], kBwdStage);
-                    uint8_t *A = smem + s * kBwdStage;
-                    bwd_load<MODE>(a, t.sh ? &a_s : &a_r, t.sh ? &b_s : &b_r, A, A + kBwdTile, &full[s], t, k0);
+                    mbar_arrive_expect_tx(&full[s], kStage);
+                    for (int c = 0; c < NSL; ++c) {
+                        uint8_t *A = smem + s * kStage + c * kBwdStage;
+                        bwd_load<MODE>(a, t.sh ? &a_s : &a_r, t.sh ? &b_s : &b_r, A, A + kBwdTile, &full[s], t,
+                                       k0 + 64 * c);
+                    }
                 }
             }
             for (int i = it > S ? it - S : 0; i < it; ++i)
@@ -676,20 +683,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const uint32_t d = tmem + buf * kBwdBN;
                 const uint32_t idesc = idesc_bf16_f32(128, (t.ntok + 15) & ~15) | (kAmn ? 1u << 15 : 0u) |
                                        (kBmn ? 1u << 16 : 0u);
-                for (int k0 = 0; k0 < t.K; k0 += 64, ++it) {
+                for (int k0 = 0; k0 < t.K; k0 += 64 * NSL, ++it) {
                     const int s = it % S;
                     if (!mbar_wait(&full[s], (it / S) & 1, wc, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + s * kBwdStage);
-                    const uint32_t sb = sa + kBwdTile;
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = kAmn ? sdesc_mn_sw128(sa + ks * 2048, 8192) : sdesc_kmajor_sw128(sa) + 2 * ks;
-                        const uint64_t bd = kBmn ? sdesc_mn_sw128(sb + ks * 2048, 8192) : sdesc_kmajor_sw128(sb) + 2 * ks;
-                        umma_bf16(d, ad, bd, idesc, (k0 | ks) != 0);
+                    for (int c = 0; c < NSL; ++c) {
+                        const uint32_t sa = smem_u32(smem + s * kStage + c * kBwdStage);
+                        const uint32_t sb = sa + kBwdTile;
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t ad =
+                                kAmn ? sdesc_mn_sw128(sa + ks * 2048, 8192) : sdesc_kmajor_sw128(sa) + 2 * ks;
+                            const uint64_t bd =
+                                kBmn ? sdesc_mn_sw128(sb + ks * 2048, 8192) : sdesc_kmajor_sw128(sb) + 2 * ks;
+                            umma_bf16(d, ad, bd, idesc, (k0 | c | ks) != 0);
+                        }
                     }
                     umma_commit(&empty[s]);
                 }
@@ -724,15 +736,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
 }
 
-template <int MODE>
+template <int MODE, int NSL>
 cudaError_t launch_mode(const CUtensorMap &a_r, const CUtensorMap &a_s, const CUtensorMap &b_r, const CUtensorMap &b_s,
                         const BwdArgs &a, const WaitCfg &wc, int grid, cudaStream_t stream)
 {
-    cudaError_t err = cudaFuncSetAttribute(bwd_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t err = cudaFuncSetAttribute(bwd_gemm_kernel<MODE, NSL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(kBwdSmem));
     if (err != cudaSuccess)
         return err;
-    bwd_gemm_kernel<MODE><<<grid, kBwdThreads, kBwdSmem, stream>>>(a_r, a_s, b_r, b_s, a, wc);
+    bwd_gemm_kernel<MODE, NSL><<<grid, kBwdThreads, kBwdSmem, stream>>>(a_r, a_s, b_r, b_s, a, wc);
     return cudaGetLastError();
 }
 
@@ -742,17 +754,22 @@ cudaError_t launch_bwd_gemm(int mode, const CUtensorMap &a_r, const CUtensorMap 
                             const CUtensorMap &b_s, const BwdArgs &a, const WaitCfg &wc, int grid,
                             cudaStream_t stream)
 {
+    // weight-streaming modes take two K slices per stage when K (H for GU and DH, 2 I for
+    // DX) is a multiple of 128; the weight-gradient modes reduce over 64-row padded groups
+    const bool h2 = a.H % 128 == 0;
     switch (mode) {
     case kBwdGU:
-        return launch_mode<kBwdGU>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return h2 ? launch_mode<kBwdGU, 2>(a_r, a_s, b_r, b_s, a, wc, grid, stream)
+                  : launch_mode<kBwdGU, 1>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
     case kBwdDH:
-        return launch_mode<kBwdDH>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return h2 ? launch_mode<kBwdDH, 2>(a_r, a_s, b_r, b_s, a, wc, grid, stream)
+                  : launch_mode<kBwdDH, 1>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
     case kBwdDX:
-        return launch_mode<kBwdDX>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return launch_mode<kBwdDX, 2>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
     case kBwdWD:
-        return launch_mode<kBwdWD>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return launch_mode<kBwdWD, 1>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
     case kBwdWGU:
-        return launch_mode<kBwdWGU>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return launch_mode<kBwdWGU, 1>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
     default:
         return cudaErrorInvalidValue;
     }
