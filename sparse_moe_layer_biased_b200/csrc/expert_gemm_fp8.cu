@@ -37,18 +37,21 @@ constexpr int kBK = 64;
 constexpr uint32_t kWBytes = 128 * 128;  // weight part of a staging slot: 128 rows x 128 bytes
 constexpr uint32_t kACols = 64;          // TMEM columns of one operand slot: 128 bf16 per row
 
-// BN token rows per chunk, SW staging slots, SA TMEM operand slots.
-template <int BN, int SW, int SA>
+// BN token rows per chunk, SW staging slots, SA TMEM operand slots, KS 128-wide scale
+// blocks per stage (a routed stage spans 128 KS of K, a shared-expert stage 64 KS).
+template <int BN, int SW, int SA, int KS>
 struct Geo8 {
     static constexpr uint32_t kBSlice = BN * 128;  // token rows of one 64-wide K slice
-    static constexpr uint32_t kSlotBytes = kWBytes + 2 * kBSlice;
+    static constexpr uint32_t kWStage = KS * kWBytes;
+    static constexpr uint32_t kSlotBytes = kWStage + 2 * KS * kBSlice;
+    static constexpr uint32_t kSlotCols = KS * kACols;  // TMEM columns of one operand slot
     static constexpr uint32_t kBarOff = SW * kSlotBytes;
     static constexpr uint32_t kNumBars = 2 * SW + 2 * SA + 5;
     static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
     static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
     static constexpr uint32_t kBufCols = BN;             // one accumulator buffer
     static constexpr uint32_t kAOff = 2 * kBufCols;      // first operand slot column
-    static constexpr uint32_t kUsedCols = kAOff + SA * kACols;
+    static constexpr uint32_t kUsedCols = kAOff + SA * kSlotCols;
     static constexpr uint32_t kTmemCols = kUsedCols <= 128 ? 128 : (kUsedCols <= 256 ? 256 : 512);
     static_assert(kSlotBytes % 1024 == 0, "slots stay 1024-byte aligned");
     static_assert(kSmemBytes <= kMaxDynSmem, "ring exceeds shared memory");
@@ -217,9 +220,10 @@ __device__ __forceinline__ void copy_row_bf16(const uint8_t *w, int j, uint32_t 
 struct Tile8 {
     int g, row0, ntok, fb, K;
     bool sh;
-    // a routed stage spans one 128-wide scale block (E4M3), a shared stage 64 K (BF16)
-    __device__ __forceinline__ int stage_k() const { return sh ? 64 : 128; }
-    __device__ __forceinline__ int stages() const { return (K + stage_k() - 1) / stage_k(); }
+    // K of one 128-byte weight box: a 128-wide scale block of E4M3 codes, or 64 K of the
+    // BF16 shared expert; a stage holds KS boxes
+    __device__ __forceinline__ int box_k() const { return sh ? 64 : 128; }
+    __device__ __forceinline__ int stages(int ks) const { return (K + ks * box_k() - 1) / (ks * box_k()); }
 };
 
 __device__ __forceinline__ Tile8 tile_of(const GateUpArgs &a, int tile)
@@ -305,13 +309,13 @@ __device__ __forceinline__ void epilogue8(const DownArgs &a, uint32_t tmem_tile,
 // m_tok_sh (shared token rows: x or h_sh). Stage `it` uses staging slot it % SW and TMEM
 // operand slot it % SA; K elements past a tile's extent are zero-filled by TMA for both
 // operands.
-template <class Args, int BN, int SW, int SA>
+template <class Args, int BN, int SW, int SA, int KS>
 __global__ void __launch_bounds__(kThreads8, 1)
     gemm_fp8_kernel(const __grid_constant__ CUtensorMap m_w, const __grid_constant__ CUtensorMap m_wsh,
                     const __grid_constant__ CUtensorMap m_tok, const __grid_constant__ CUtensorMap m_tok_sh,
                     const Args a, const WaitCfg wc)
 {
-    using G = Geo8<BN, SW, SA>;
+    using G = Geo8<BN, SW, SA, KS>;
     extern __shared__ uint8_t smem_raw[];
     Ring8 r;
     uint8_t *smem = ring8_setup<G, SW, SA>(smem_raw, r);
@@ -331,19 +335,21 @@ __global__ void __launch_bounds__(kThreads8, 1)
             bool stop = false;
             for (int tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x) {
                 const Tile8 t = tile_of(a, tile);
-                const int nsl = t.sh ? 1 : 2;
-                for (int st = 0; st < t.stages(); ++st, ++it) {
+                const int nsl = (t.sh ? 1 : 2) * KS;  // 64-wide token slices per stage
+                const int nst = t.stages(KS);
+                for (int st = 0; st < nst; ++st, ++it) {
                     const int s = it % SW;
                     if (!mbar_wait(&r.qempty[s], ((it / SW) & 1) ^ 1, wc, r.abort_flag)) {
                         stop = true;
                         break;
                     }
                     uint8_t *slot = smem + s * G::kSlotBytes;
-                    const int k0 = st * t.stage_k();
-                    mbar_arrive_expect_tx(&r.qfull[s], kWBytes + nsl * G::kBSlice);
-                    load_weights(a, t.sh ? &m_wsh : &m_w, slot, &r.qfull[s], t, k0);
+                    const int k0 = st * KS * t.box_k();
+                    mbar_arrive_expect_tx(&r.qfull[s], G::kWStage + nsl * G::kBSlice);
+                    for (int c = 0; c < KS; ++c)
+                        load_weights(a, t.sh ? &m_wsh : &m_w, slot + c * kWBytes, &r.qfull[s], t, k0 + c * t.box_k());
                     for (int kc = 0; kc < nsl; ++kc)
-                        tma_load_2d(slot + kWBytes + kc * G::kBSlice, t.sh ? &m_tok_sh : &m_tok, &r.qfull[s],
+                        tma_load_2d(slot + G::kWStage + kc * G::kBSlice, t.sh ? &m_tok_sh : &m_tok, &r.qfull[s],
                                     k0 + kc * kBK, t.row0);
                 }
             }
@@ -358,16 +364,18 @@ __global__ void __launch_bounds__(kThreads8, 1)
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
             const Tile8 t = tile_of(a, tile);
-            const int nkblk = t.K / 128;
+            const int nkblk = (t.K + 127) / 128;
+            const int nst = t.stages(KS);
             // lane l caches the scales of K block base + l (reloaded every 32 blocks)
             int base = -32;
             float se = 0.0f, so = 0.0f;
-            for (int st = 0; st < t.stages(); ++st, ++it) {
+            for (int st = 0; st < nst; ++st, ++it) {
                 if ((it & 1) != gi)
                     continue;
                 const int sa = it % SA, sq = it % SW;
-                if (!t.sh && st - base >= 32) {
-                    base = st;
+                if (!t.sh && st * KS + KS - 1 - base >= 32) {
+                    base = st * KS;
+                    se = so = 0.0f;
                     if (base + lane < nkblk) {
                         const float2 sc = tile_scales(a, t, base + lane);
                         se = sc.x;
@@ -379,14 +387,17 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 if (!ok)
                     break;
                 tc_fence_after();  // the MMA that read this operand slot has completed
-                const uint8_t *w = smem + sq * G::kSlotBytes;
-                const uint32_t taddr = lane_addr + G::kAOff + sa * kACols;
-                if (t.sh) {
-                    copy_row_bf16(w, j, taddr);
-                } else {
-                    const float s_even = __shfl_sync(0xFFFFFFFFu, se, st - base);
-                    const float s_odd = __shfl_sync(0xFFFFFFFFu, so, st - base);
-                    convert_row_e4m3(w, j, taddr, split_scale((j & 1) ? s_odd : s_even));
+#pragma unroll
+                for (int c = 0; c < KS; ++c) {
+                    const uint8_t *w = smem + sq * G::kSlotBytes + c * kWBytes;
+                    const uint32_t taddr = lane_addr + G::kAOff + sa * G::kSlotCols;
+                    if (t.sh) {
+                        copy_row_bf16(w, j, taddr + c * (kACols / 2));
+                    } else {
+                        const float s_even = __shfl_sync(0xFFFFFFFFu, se, st * KS + c - base);
+                        const float s_odd = __shfl_sync(0xFFFFFFFFu, so, st * KS + c - base);
+                        convert_row_e4m3(w, j, taddr + c * kACols, split_scale((j & 1) ? s_odd : s_even));
+                    }
                 }
                 tmem_store_wait();
                 tc_fence_before();
@@ -411,16 +422,17 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 tc_fence_after();
                 const uint32_t d = tmem + buf * G::kBufCols;
                 const uint32_t idesc = idesc_bf16_f32(128, (t.ntok + 15) & ~15);
-                const int nks = t.stage_k() / 16;
-                for (int st = 0; st < t.stages(); ++st, ++it) {
+                const int nks = KS * t.box_k() / 16;  // K=16 MMAs per stage
+                const int nst = t.stages(KS);
+                for (int st = 0; st < nst; ++st, ++it) {
                     const int sa = it % SA, sq = it % SW;
                     if (!mbar_wait(&r.conv[sa], (it / SA) & 1, wc, r.abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_col = tmem + G::kAOff + sa * kACols;
-                    const uint32_t b_addr = smem_u32(smem + sq * G::kSlotBytes) + kWBytes;
+                    const uint32_t a_col = tmem + G::kAOff + sa * G::kSlotCols;
+                    const uint32_t b_addr = smem_u32(smem + sq * G::kSlotBytes) + G::kWStage;
                     for (int ks = 0; ks < nks; ++ks) {
                         const uint64_t bd = sdesc_kmajor_sw128(b_addr + (ks >> 2) * G::kBSlice) + 2 * (ks & 3);
                         umma_bf16_ta(d, a_col + 8 * ks, bd, idesc, (st | ks) != 0);
@@ -455,12 +467,12 @@ __global__ void __launch_bounds__(kThreads8, 1)
     ring8_teardown<G>(tmem);
 }
 
-template <class Args, int BN, int SW, int SA>
+template <class Args, int BN, int SW, int SA, int KS>
 cudaError_t launch8(int grid, cudaStream_t stream, const CUtensorMap &m0, const CUtensorMap &m1,
                     const CUtensorMap &m2, const CUtensorMap &m3, const Args &a, const WaitCfg &wc)
 {
-    constexpr int smem = static_cast<int>(Geo8<BN, SW, SA>::kSmemBytes);
-    auto kernel = gemm_fp8_kernel<Args, BN, SW, SA>;
+    constexpr int smem = static_cast<int>(Geo8<BN, SW, SA, KS>::kSmemBytes);
+    auto kernel = gemm_fp8_kernel<Args, BN, SW, SA, KS>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
@@ -470,16 +482,18 @@ cudaError_t launch8(int grid, cudaStream_t stream, const CUtensorMap &m0, const 
 
 }  // namespace
 
-// Decode-sized calls: 32-row chunks; staging slots of 24 KB (16 KB weights + two 4 KB
-// token slices), 9 deep (144 KB of E4M3 bytes in flight per SM); 4 TMEM operand slots.
-// Prefill: 128-row chunks; 48 KB staging slots, 4 deep; 4 TMEM operand slots.
+// Decode-sized calls: 32-row chunks; stages of two scale blocks (256 K: 16 MMAs per barrier
+// test and commit of the MMA thread), staging slots of 48 KB (32 KB weights + four 4 KB token
+// slices), 4 deep; 3 TMEM operand slots of 128 columns.
+// Prefill: 128-row chunks; stages of one scale block, 48 KB staging slots, 4 deep; 4 TMEM
+// operand slots.
 cudaError_t launch_gate_up_fp8(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
                                const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
                                const GemmConfig &c, cudaStream_t stream)
 {
     if (c.cap == 32)
-        return launch8<GateUpArgs, 32, 9, 4>(grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
-    return launch8<GateUpArgs, 128, 4, 4>(grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
+        return launch8<GateUpArgs, 32, 4, 3, 2>(grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
+    return launch8<GateUpArgs, 128, 4, 4, 1>(grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
 }
 
 cudaError_t launch_down_fp8(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
@@ -487,8 +501,8 @@ cudaError_t launch_down_fp8(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh
                             const GemmConfig &c, cudaStream_t stream)
 {
     if (c.cap_d == 32)
-        return launch8<DownArgs, 32, 9, 4>(grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
-    return launch8<DownArgs, 128, 4, 4>(grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
+        return launch8<DownArgs, 32, 4, 3, 2>(grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
+    return launch8<DownArgs, 128, 4, 4, 1>(grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
 }
 
 }  // namespace moe
