@@ -266,19 +266,44 @@ def run_reference(args, shape):
 # it was taken from: the lookup returns None once any file under csrc/ changes.
 PROFILED_TRAFFIC = {
     ("step35_prefill", "bf16"): {"bytes": 5590671360 + 86992128,
-                                 "csrc_sha256": "899d4b775c82b3a466824431bbc848e09316e689966cf31847bac64a970b3609",
+                                 "csrc_sha256": "1e91803dc29b3a44ed62a0a4f539f08c3c2186d6b856d0f770923b1d5dfea99b",
                                  "source": "profiles/dram_gate_up_down_step35_prefill.md"},
 }
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without its comments and blank lines (string and character literals kept)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "\n".join(l.strip() for l in "".join(out).splitlines() if l.strip())
+
+
 def csrc_digest() -> str:
+    """Digest of the kernel sources' code (comments excluded), which the profiled traffic
+    figures are tied to."""
     import hashlib
     d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "sparse_moe_layer_biased_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(d)):
         if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(d, name), encoding="utf-8") as f:
+                h.update(name.encode() + b"\0" + _strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

@@ -508,12 +508,11 @@ cudaError_t launch_pairs(Kernel kernel, int smem, int grid, cudaStream_t stream,
 }
 
 // gate_up: pair tiles of up to 256 token rows (128 per CTA) x 128 features, one weight
-// tile per CTA and stage (32 KB stages, 6 deep). Most experts of a prefill batch then need
-// one pass over their weights. down: 128 token rows x 512 output features, two weight
+// tile per CTA and K slice, two 64-wide K slices per stage (8 pair MMAs per barrier test
+// and commit of the MMA thread), three 64 KB stages. Most experts of a prefill batch then
+// need one pass over their weights. down: 128 token rows x 512 output features, two weight
 // tiles per CTA and stage (40 KB stages, 4 deep) and two 16 KB output staging buffers for
 // the bulk reductions. Both keep two TMEM accumulators.
-// gate_up: two 64-wide K slices per stage (8 pair MMAs per barrier test and commit of the
-// MMA thread), three 64 KB stages
 constexpr int kGateUpStages = 3, kGateUpSlices = 2;
 using GateUpPair = PairGeo<kPairCapGateUp, kGateUpStages, kPairMtGateUp, 2, 0, kGateUpSlices>;
 constexpr int kDownStages = 4, kDownOutBufs = 2;  // 4 x 40 KB ring + 2 x 16 KB output staging

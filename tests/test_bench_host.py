@@ -40,3 +40,18 @@ def test_gate_up_byte_model_counts_touched_experts_only():
     assert b == w + acts + out
     b8, _ = bench.gate_up_bytes(sh, counts, fp8=True)
     assert b8 == b - 10 * 2 * sh.I * sh.H + 10 * (2 * sh.I // 128) * (sh.H // 128) * 4
+
+
+def test_source_digest_ignores_comments_only():
+    src = 'asm("mov.u32 %0, 1; // not a comment inside the string" : "=r"(x));\n'
+    a = bench._strip_comments("// header\n" + src + "/* block\n comment */ int y = '/';\n")
+    b = bench._strip_comments(src + "int y = '/';  // trailing\n\n")
+    assert a == b and "not a comment" in a and "header" not in a
+    assert bench._strip_comments("int a;") != bench._strip_comments("int b;")
+
+
+def test_profiled_traffic_is_tied_to_the_current_sources():
+    for (shape, weights), e in bench.PROFILED_TRAFFIC.items():
+        assert shape in WORKLOADS
+        got = bench.profiled_traffic(shape, weights)
+        assert got is None or got == e["bytes"]
