@@ -26,6 +26,8 @@ SMALL = {
     "clip": WORKLOADS["tiny"].replace(name="clip", weight_std=0.2, limit_routed=0.5, limit_shared=0.25),
     "k1": LayerShape("k1", T=77, H=256, E=3, k=1, I=64, Is=64, seed=22),
     "kE": LayerShape("kE", T=50, H=128, E=8, k=8, I=64, Is=128, seed=23),
+    # a single routed expert: every token selects it with weight scale (after normalising)
+    "E1": LayerShape("E1", T=77, H=256, E=1, k=1, I=64, Is=64, limit_routed=0.25, seed=35, weight_std=0.05),
     "wideE": LayerShape("wideE", T=700, H=256, E=300, k=8, I=64, Is=64, seed=24),
     "k32": LayerShape("k32", T=129, H=256, E=64, k=32, I=128, Is=64, seed=25),
     # the most experts (512 > 384: the router keeps 64-token tiles so a tile's partial
