@@ -332,8 +332,12 @@ constexpr uint32_t kBwdTile = 16384;  // one operand per stage
 constexpr uint32_t kBwdStage = 2 * kBwdTile;
 constexpr uint32_t kBwdBarOff = kBwdStages * kBwdStage;
 constexpr uint32_t kBwdMiscOff = kBwdBarOff + 8 * (2 * kBwdStages + 5);
-constexpr uint32_t kBwdEpiOff = kBwdMiscOff + 16;       // per epilogue warp: a 32 x 33 fp32 transpose
-constexpr uint32_t kBwdEpiWarp = 32 * 33 * 4;
+// per epilogue warp: two 4 KB staging boxes of the weight-gradient stores (1024-byte aligned
+// for the 128-byte swizzle), or the DH mode's 32 x 33 fp32 transpose
+constexpr uint32_t kBwdEpiOff = (kBwdMiscOff + 16 + 1023) / 1024 * 1024;
+constexpr uint32_t kBwdEpiBox = 32 * 32 * 4;
+constexpr uint32_t kBwdEpiWarp = 2 * kBwdEpiBox;
+static_assert(32 * 33 * 4 <= kBwdEpiWarp, "transpose buffer");
 constexpr uint32_t kBwdSmem = kBwdEpiOff + 4 * kBwdEpiWarp + 1024;
 static_assert(kBwdSmem <= kMaxDynSmem, "backward ring exceeds shared memory");
 
@@ -457,9 +461,11 @@ __device__ __forceinline__ void bwd_load(const BwdArgs &a, const CUtensorMap *ma
 }
 
 // Epilogue of one tile for one warp (TMEM lane quarter q; lane row = q*32 + lane of M).
+// om = tensor map of the tile's weight-gradient output (WD / WGU), 32 x 32 fp32 boxes with
+// 128-byte swizzle; tr = this warp's staging area (kBwdEpiWarp bytes, 1024-byte aligned).
 template <int MODE>
 __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, const BTile &t, int q, int lane,
-                                             float *tr)
+                                             float *tr, const CUtensorMap *om)
 {
     const int row = q * 32 + lane;
     const uint32_t tq = tacc + (static_cast<uint32_t>(q * 32) << 16);
@@ -569,28 +575,33 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
             }
         }
     } else {
-        // weight gradients: row m of the output tile, columns nb*BN .. +BN, plain stores
-        const int64_t m = t.mb * 128 + row;
-        float *out;
-        if (MODE == kBwdWD)
-            out = t.sh ? a.dWsh_d + m * a.Is : a.dWd + (static_cast<int64_t>(t.g) * a.H + m) * a.I;
-        else
-            out = t.sh ? a.dWsh_gu + m * a.H : a.dWgu + (static_cast<int64_t>(t.g) * 2 * a.I + m) * a.H;
-        out += t.nb * kBwdBN;
-        // through a 32 x 33 transpose so each store writes 128 contiguous bytes of one row
-        const int64_t ld = MODE == kBwdWD ? (t.sh ? a.Is : a.I) : a.H;
-        float *rowbase = out - static_cast<int64_t>(lane) * ld;  // row q*32 of the tile
+        // weight gradients: rows mb*128 + q*32 .. +32 of the output, columns nb*BN .. +BN, as
+        // four 32 x 32 boxes. Lane l holds row l of a box: it writes its eight 16-byte pieces
+        // in the 128-byte swizzle (piece j at j ^ (l % 8), conflict-free), and lane 0 stores
+        // the box with one TMA copy. Two boxes alternate: a box is rewritten only after the
+        // copy issued from it two boxes earlier has read it.
+        const int64_t row0 = (MODE == kBwdWD ? (t.sh ? 0 : static_cast<int64_t>(t.g) * a.H)
+                                             : (t.sh ? 0 : static_cast<int64_t>(t.g) * 2 * a.I)) +
+                             t.mb * 128 + q * 32;
+        uint8_t *stage = reinterpret_cast<uint8_t *>(tr);
         for (int cb = 0; cb < kBwdBN; cb += 32) {
             float v[32];
             tmem_load32(tq + cb, v);
+            uint8_t *box = stage + ((cb >> 5) & 1) * kBwdEpiBox;
+            if (lane == 0)
+                bulk_wait_read<1>();
+            __syncwarp();
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-                tr[lane * 33 + c] = v[c];
+            for (int j = 0; j < 8; ++j) {
+                float4 *dst = reinterpret_cast<float4 *>(box + lane * 128 + ((j ^ (lane & 7)) << 4));
+                *dst = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            }
+            fence_proxy_async_smem();
             __syncwarp();
-#pragma unroll 8
-            for (int r = 0; r < 32; ++r)
-                rowbase[r * ld + cb + lane] = tr[r * 33 + lane];
-            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(om, box, t.nb * kBwdBN + cb, static_cast<int32_t>(row0));
+                bulk_commit();
+            }
         }
     }
 }
@@ -601,6 +612,7 @@ template <int MODE, int NSL>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap a_r, const __grid_constant__ CUtensorMap a_s,
                     const __grid_constant__ CUtensorMap b_r, const __grid_constant__ CUtensorMap b_s,
+                    const __grid_constant__ CUtensorMap o_r, const __grid_constant__ CUtensorMap o_s,
                     const BwdArgs a, const WaitCfg wc)
 {
     constexpr bool kAmn = MODE != kBwdGU;
@@ -721,12 +733,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             tc_fence_after();
             bwd_epilogue<MODE>(a, tmem + buf * kBwdBN, t, q, lane,
-                               reinterpret_cast<float *>(smem + kBwdEpiOff + q * kBwdEpiWarp));
+                               reinterpret_cast<float *>(smem + kBwdEpiOff + q * kBwdEpiWarp), t.sh ? &o_s : &o_r);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&acce[buf]);
         }
+        if (lane == 0)
+            bulk_wait<0>();  // this warp's gradient stores have completed before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -738,38 +752,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 template <int MODE, int NSL>
 cudaError_t launch_mode(const CUtensorMap &a_r, const CUtensorMap &a_s, const CUtensorMap &b_r, const CUtensorMap &b_s,
-                        const BwdArgs &a, const WaitCfg &wc, int grid, cudaStream_t stream)
+                        const CUtensorMap &o_r, const CUtensorMap &o_s, const BwdArgs &a, const WaitCfg &wc, int grid,
+                        cudaStream_t stream)
 {
     cudaError_t err = cudaFuncSetAttribute(bwd_gemm_kernel<MODE, NSL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(kBwdSmem));
     if (err != cudaSuccess)
         return err;
-    bwd_gemm_kernel<MODE, NSL><<<grid, kBwdThreads, kBwdSmem, stream>>>(a_r, a_s, b_r, b_s, a, wc);
+    bwd_gemm_kernel<MODE, NSL><<<grid, kBwdThreads, kBwdSmem, stream>>>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_bwd_gemm(int mode, const CUtensorMap &a_r, const CUtensorMap &a_s, const CUtensorMap &b_r,
-                            const CUtensorMap &b_s, const BwdArgs &a, const WaitCfg &wc, int grid,
-                            cudaStream_t stream)
+                            const CUtensorMap &b_s, const CUtensorMap &o_r, const CUtensorMap &o_s, const BwdArgs &a,
+                            const WaitCfg &wc, int grid, cudaStream_t stream)
 {
     // weight-streaming modes take two K slices per stage when K (H for GU and DH, 2 I for
     // DX) is a multiple of 128; the weight-gradient modes reduce over 64-row padded groups
     const bool h2 = a.H % 128 == 0;
     switch (mode) {
     case kBwdGU:
-        return h2 ? launch_mode<kBwdGU, 2>(a_r, a_s, b_r, b_s, a, wc, grid, stream)
-                  : launch_mode<kBwdGU, 1>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return h2 ? launch_mode<kBwdGU, 2>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream)
+                  : launch_mode<kBwdGU, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
     case kBwdDH:
-        return h2 ? launch_mode<kBwdDH, 2>(a_r, a_s, b_r, b_s, a, wc, grid, stream)
-                  : launch_mode<kBwdDH, 1>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return h2 ? launch_mode<kBwdDH, 2>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream)
+                  : launch_mode<kBwdDH, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
     case kBwdDX:
-        return launch_mode<kBwdDX, 2>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return launch_mode<kBwdDX, 2>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
     case kBwdWD:
-        return launch_mode<kBwdWD, 1>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return launch_mode<kBwdWD, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
     case kBwdWGU:
-        return launch_mode<kBwdWGU, 1>(a_r, a_s, b_r, b_s, a, wc, grid, stream);
+        return launch_mode<kBwdWGU, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
     default:
         return cudaErrorInvalidValue;
     }

@@ -180,9 +180,12 @@ enum BwdMode { kBwdGU = 0, kBwdDH = 1, kBwdDX = 2, kBwdWD = 3, kBwdWGU = 4 };
 //   DX : W_gate_up / Wsh_gate_up as (H, rows) MN-major, dgu_r, dgu_s (K-major)
 //   WD : dy_pad (H, rows) MN-major (both), hw_r / hw_s (I, rows) MN-major
 //   WGU: dgu_r / dgu_s (2I, rows) MN-major, x_pad (H, rows) MN-major (both)
+// and output maps (routed, shared) of the weight-gradient modes, fp32 32 x 32 boxes with
+// 128-byte swizzle: WD dW_down (I, E*H) / dWsh_down (Is, H), WGU dW_gate_up (H, E*2I) /
+// dWsh_gate_up (H, 2Is); the other modes ignore them.
 cudaError_t launch_bwd_gemm(int mode, const CUtensorMap &a_r, const CUtensorMap &a_s, const CUtensorMap &b_r,
-                            const CUtensorMap &b_s, const BwdArgs &a, const WaitCfg &wc, int grid,
-                            cudaStream_t stream);
+                            const CUtensorMap &b_s, const CUtensorMap &o_r, const CUtensorMap &o_s, const BwdArgs &a,
+                            const WaitCfg &wc, int grid, cudaStream_t stream);
 // Padded layout + tile tables from the permutation's counts (one CTA).
 cudaError_t launch_bwd_layout(const int32_t *counts, int E, int T, int32_t *poff, int4 *chunks, int4 *wgroups,
                               int32_t *hdr, cudaStream_t stream);

@@ -93,6 +93,20 @@ bool encode_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *d
     return r == CUDA_SUCCESS;
 }
 
+// fp32 [rows, cols] row-major as the destination of 32 x 32 boxes (128 bytes wide, 128-byte
+// swizzle), for tiled stores
+bool map_rows_f32_store(CUtensorMap *m, const void *base, int64_t cols, int64_t rows)
+{
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool map_rows(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, uint32_t box_rows)
 {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -874,7 +888,7 @@ moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const u
 
     // tensor maps (rows of the padded buffers are upper bounds; tiles only touch filled rows)
     CUtensorMap gu_a_r, gu_a_s, gu_b, dh_a_r, dh_a_s, dh_b, dx_a_r, dx_a_s, dx_b_r, dx_b_s, wd_a, wd_b_r, wd_b_s,
-        wg_a_r, wg_a_s, wg_b;
+        wg_a_r, wg_a_s, wg_b, wd_o_r, wd_o_s, wg_o_r, wg_o_s;
     const bool ok = map_gate_up(&gu_a_r, W_gate_up, H, I, E, 64) && map_gate_up(&gu_a_s, Wsh_gate_up, H, Is, 1, 64) &&
                     map_rows(&gu_b, x_pad, H, P, moe::kBwdCap) && map_rows(&dh_a_r, W_down, I, E * H, 64) &&
                     map_rows(&dh_a_s, Wsh_down, Is, H, 64) && map_rows(&dh_b, dy_pad, H, P, moe::kBwdCap) &&
@@ -883,7 +897,10 @@ moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const u
                     map_rows(&dx_b_s, dgu_s, 2 * Is, Ps, moe::kBwdCap) && map_rows(&wd_a, dy_pad, H, P, 64) &&
                     map_rows(&wd_b_r, hw_r, I, Pr, 64) && map_rows(&wd_b_s, hw_s, Is, Ps, 64) &&
                     map_rows(&wg_a_r, dgu_r, 2 * I, Pr, 64) && map_rows(&wg_a_s, dgu_s, 2 * Is, Ps, 64) &&
-                    map_rows(&wg_b, x_pad, H, P, 64);
+                    map_rows(&wg_b, x_pad, H, P, 64) && map_rows_f32_store(&wd_o_r, dW_down, I, E * H) &&
+                    map_rows_f32_store(&wd_o_s, dWsh_down, Is, H) &&
+                    map_rows_f32_store(&wg_o_r, dW_gate_up, H, E * 2 * I) &&
+                    map_rows_f32_store(&wg_o_s, dWsh_gate_up, H, 2 * Is);
     if (!ok)
         return MOE_ERR_CUDA;
     const moe::WaitCfg wc = wait_cfg(di);
@@ -901,20 +918,20 @@ moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const u
     if (e == cudaSuccess)
         e = cudaMemsetAsync(dw_pad, 0, static_cast<size_t>(P) * 4, s);
     if (e == cudaSuccess)
-        e = moe::launch_bwd_gemm(moe::kBwdGU, gu_a_r, gu_a_s, gu_b, gu_b, ba, wc, di.num_sms, s);
+        e = moe::launch_bwd_gemm(moe::kBwdGU, gu_a_r, gu_a_s, gu_b, gu_b, gu_b, gu_b, ba, wc, di.num_sms, s);
     if (e == cudaSuccess)
-        e = moe::launch_bwd_gemm(moe::kBwdDH, dh_a_r, dh_a_s, dh_b, dh_b, ba, wc, di.num_sms, s);
+        e = moe::launch_bwd_gemm(moe::kBwdDH, dh_a_r, dh_a_s, dh_b, dh_b, dh_b, dh_b, ba, wc, di.num_sms, s);
     if (e == cudaSuccess)
         e = moe::launch_bwd_router(x, Wr, topk_idx, slot_of, offsets, poff, dw_pad, d.T, d.k, d.E, d.H, d.scale,
                                    d.norm_expert_weight, dx, dl_pad, s);
     if (e == cudaSuccess)
-        e = moe::launch_bwd_gemm(moe::kBwdDX, dx_a_r, dx_a_s, dx_b_r, dx_b_s, ba, wc, di.num_sms, s);
+        e = moe::launch_bwd_gemm(moe::kBwdDX, dx_a_r, dx_a_s, dx_b_r, dx_b_s, dx_b_r, dx_b_s, ba, wc, di.num_sms, s);
     if (e == cudaSuccess)
         e = moe::launch_bwd_zero_untouched(counts, d.E, d.H, d.I, dW_gate_up, dW_down, s);
     if (e == cudaSuccess)
-        e = moe::launch_bwd_gemm(moe::kBwdWD, wd_a, wd_a, wd_b_r, wd_b_s, ba, wc, di.num_sms, s);
+        e = moe::launch_bwd_gemm(moe::kBwdWD, wd_a, wd_a, wd_b_r, wd_b_s, wd_o_r, wd_o_s, ba, wc, di.num_sms, s);
     if (e == cudaSuccess)
-        e = moe::launch_bwd_gemm(moe::kBwdWGU, wg_a_r, wg_a_s, wg_b, wg_b, ba, wc, di.num_sms, s);
+        e = moe::launch_bwd_gemm(moe::kBwdWGU, wg_a_r, wg_a_s, wg_b, wg_b, wg_o_r, wg_o_s, ba, wc, di.num_sms, s);
     if (e == cudaSuccess)
         e = moe::launch_bwd_dwr(x_pad, dl_pad, poff, counts, d.E, d.H, dWr, s);
     return cuda_status(e);

@@ -416,6 +416,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N)
 }
 
 // ---------------------------------------------------------------- bulk copies to global
+// Tiled store of one box from shared memory (laid out as the map's swizzle says) to global
+// memory, tracked by this thread's bulk groups; c0 (innermost) must be a multiple of 16 bytes
+// and neither coordinate negative. Parts of the box outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *src, int32_t c0, int32_t c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 // Generic-proxy shared-memory writes made visible to the async proxy (bulk copies, MMA).
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
