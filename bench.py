@@ -314,6 +314,18 @@ def profiled_traffic(shape_name: str, weights: str):
     return e["bytes"]
 
 
+def kernels_per_step(shape, fp8=False, deterministic=False, router=True):
+    """Kernels one forward call launches: router, permute, gather, tile tables, gate_up and
+    down (+ combine in deterministic mode; no router with given ids). With FP8 routed experts
+    on a prefill-sized call the BF16 shared expert runs on the CTA-pair kernels with its own
+    tile tables, gate_up and down."""
+    n = 6 + (1 if deterministic else 0) - (0 if router else 1)
+    if (fp8 and shape.T * shape.k > 16 * shape.E and shape.I % 128 == 0 and shape.Is % 128 == 0
+            and shape.H % 512 == 0):
+        n += 3
+    return n
+
+
 def gate_up_bytes(shape, counts, fp8=False):
     """Algorithmic HBM bytes of one gate_up launch: weights of every expert that received
     tokens (2I x H, bf16 or E4M3 codes plus one fp32 scale per 128x128 block) + shared
@@ -483,7 +495,7 @@ def run_b200(args, shape):
         "stages_ms": stage_ms,
         "clocks": clocks,
         "e2e": e2e,
-        "gpu_launches": (nstage - (1 if args.routing == "balanced" else 0)) * args.steps,
+        "gpu_launches": kernels_per_step(shape, fp8, args.deterministic, args.routing != "balanced") * args.steps,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         rate, n, dt, threads = cpu_oracle_sample(shape, inp, target_s=15.0)

@@ -315,15 +315,40 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     if (!ok)
         return MOE_ERR_CUDA;
 
+    // FP8 prefill: the routed experts run on the FP8 kernels and the BF16 shared expert on
+    // the BF16 CTA-pair kernels (full 128-wide K stages, no conversion), as a group of its
+    // own (expert count 0, so its chunks are the shared group) with tile tables in the
+    // second table region, which the FP8 configuration leaves unused (one table, cap ==
+    // cap_d), and headers at hdr + 4 / hdr + 8.
+    const moe::GemmConfig cfg_sh = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
+    const bool split = fp8 && groups == FfnGroups::kBoth && cfg.cap > 32 && cfg_sh.pair;
+    CUtensorMap tm_wsh2, tm_x2, tm_wdsh2, tm_hsh2;
+    int4 *chunks_s = nullptr, *chunks_sd = nullptr;
+    if (split) {
+        const int64_t n_gu = (d.T + cfg_sh.cap - 1) / cfg_sh.cap + 1;
+        const int64_t n_d = (d.T + cfg_sh.cap_d - 1) / cfg_sh.cap_d + 1;
+        if (cfg_sh.cap_d == cfg_sh.cap || n_gu + n_d > moe::max_chunks(d.T, d.k, d.E, cfg_sh.cap_d))
+            return MOE_ERR_WORKSPACE;
+        chunks_s = at<int4>(ws, L.chunks_d);
+        chunks_sd = chunks_s + n_gu;
+        if (!(map_gate_up(&tm_wsh2, W.sh_gu, d.H, d.Is, 1, static_cast<uint32_t>(64 * cfg_sh.mt)) &&
+              map_rows(&tm_x2, x, d.H, d.T, 64) &&
+              map_rows(&tm_wdsh2, W.sh_d, d.Is, d.H, static_cast<uint32_t>(128 * cfg_sh.mt_d)) &&
+              map_rows(&tm_hsh2, h_sh, d.Is, d.T, 64)))
+            return MOE_ERR_CUDA;
+    }
+
     if (!stage_mark(2, s))
         return MOE_ERR_CUDA;
     cudaError_t e = cudaSuccess;
     if (groups != FfnGroups::kSharedOnly)
         e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, s);
-    const int shared_rows = groups == FfnGroups::kRoutedOnly ? 0 : d.T;
+    const int shared_rows = groups == FfnGroups::kRoutedOnly || split ? 0 : d.T;
     if (e == cudaSuccess)
         e = moe::launch_chunks(offsets, d.E, shared_rows, cfg.cap, chunks, hdr, cfg.cap_d,
                                cfg.cap_d != cfg.cap ? chunks_d : nullptr, hdr_d, s);
+    if (e == cudaSuccess && split)
+        e = moe::launch_chunks(offsets, 0, d.T, cfg_sh.cap, chunks_s, hdr + 4, cfg_sh.cap_d, chunks_sd, hdr + 8, s);
     if (e == cudaSuccess && !d.deterministic)
         e = cudaMemsetAsync(out, 0, static_cast<size_t>(d.T) * d.H * 4, s);
     if (e != cudaSuccess)
@@ -334,6 +359,11 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
         return MOE_ERR_CUDA;
     e = fp8 ? moe::launch_gate_up_fp8(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s)
             : moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s);
+    if (e == cudaSuccess && split) {
+        const moe::GateUpArgs gs{chunks_s, hdr + 4, h, h_sh, 0, d.H, d.I, d.Is, d.limit_routed, d.limit_shared,
+                                 nullptr};
+        e = moe::launch_gate_up(tm_wsh2, tm_wsh2, tm_x2, tm_x2, gs, wc, di.num_sms, cfg_sh, s);
+    }
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
     moe::DownArgs da{chunks_d, hdr_d, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic,
@@ -342,6 +372,11 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
         return MOE_ERR_CUDA;
     e = fp8 ? moe::launch_down_fp8(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s)
             : moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s);
+    if (e == cudaSuccess && split) {
+        const moe::DownArgs ds{chunks_sd, hdr + 8, perm_token, w_perm, out, 0, d.H, d.I, d.Is, d.T, d.k,
+                               d.deterministic, nullptr};
+        e = moe::launch_down(tm_wdsh2, tm_wdsh2, tm_hsh2, tm_hsh2, ds, wc, di.num_sms, cfg_sh, s);
+    }
     if (e != cudaSuccess || !stage_mark(5, s))
         return MOE_ERR_CUDA;
     return MOE_OK;

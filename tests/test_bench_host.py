@@ -55,3 +55,12 @@ def test_profiled_traffic_is_tied_to_the_current_sources():
         assert shape in WORKLOADS
         got = bench.profiled_traffic(shape, weights)
         assert got is None or got == e["bytes"]
+
+
+def test_kernels_per_step():
+    s35, dec = WORKLOADS["step35_prefill"], WORKLOADS["step35_decode"]
+    assert bench.kernels_per_step(s35) == 6
+    assert bench.kernels_per_step(s35, deterministic=True) == 7
+    assert bench.kernels_per_step(s35, router=False) == 5
+    assert bench.kernels_per_step(s35, fp8=True) == 9  # shared expert on the BF16 pair kernels
+    assert bench.kernels_per_step(dec, fp8=True) == 6

@@ -35,6 +35,10 @@ SHAPES = {
     # gate/up feature blocks, ragged chunk tails
     "prefill_h768": LayerShape("fp8_prefill_h768", T=333, H=768, E=10, k=4, I=384, Is=256, limit_routed=0.25,
                                limit_shared=0.125, seed=56, weight_std=0.03),
+    # prefill-sized with I, Is multiples of 128 and H of 512: the BF16 shared expert runs on
+    # the CTA-pair kernels (its own tile tables), the routed experts on the FP8 kernels
+    "prefill_pair": LayerShape("fp8_prefill_pair", T=300, H=512, E=12, k=4, I=256, Is=256, limit_routed=0.25,
+                               limit_shared=0.125, seed=57, weight_std=0.03),
     "ragged": LayerShape("fp8_ragged", T=333, H=384, E=40, k=6, I=128, Is=320, limit_routed=0.0,
                          limit_shared=0.0, seed=53, weight_std=0.03),
     # pre-activations of std ~1 against routed limit 0.5: the up clamp binds on ~60% and
