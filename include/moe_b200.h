@@ -266,17 +266,21 @@ MOE_API moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x,
  * as a serving runtime whose device memory is already handed to a fixed pool, a
  * latency-bound decode loop that must avoid cudaMalloc / cudaFree (they can synchronise
  * the device), or a plugin without access to its host framework's allocator.
- * The library keeps one 16 MiB scratch array in device memory on every device that loads
- * it, until the process exits, and uses it as the workspace; nothing is allocated per
- * call. Arguments and results are those of moe_forward (inputs and y are still the
- * caller's). A call whose moe_workspace_size() exceeds 16 MiB (16777216 bytes) returns
- * MOE_ERR_WORKSPACE before enqueueing anything; at H = 4096, k = 8, I = Is = 1280 the
- * limit is 188 tokens in the default mode. The first call on a device looks up the
- * array's device address (a runtime query, no allocation); make that first call before
- * any stream capture. All calls on a device share the one array: calls whose work
- * overlaps on the GPU (for example on two streams) race and give wrong results; calls on
- * one stream are ordered and safe. Nothing from a previous call needs clearing: every
- * scratch byte read is written first in the same call. */
+ * The library keeps one 16 MiB scratch array in device memory and uses it as the
+ * workspace; nothing is allocated per call. Under CUDA's default lazy module loading a
+ * device gets the array at the first moe_forward_noalloc call made on it (under eager
+ * loading, when the library's device code loads), and keeps it until the process exits.
+ * Make that first call on each device before any stream capture. Every call looks up the
+ * array's device address in the current context (a runtime query, no allocation), so no
+ * address outlives its context. Arguments and results are those of moe_forward (inputs
+ * and y are still the caller's). A call whose moe_workspace_size() exceeds 16 MiB
+ * (16777216 bytes) returns MOE_ERR_WORKSPACE before enqueueing anything; at H = 4096,
+ * E = 288, k = 8, I = Is = 1280 the limit is 188 tokens in the default mode and 70 tokens
+ * in the deterministic mode (which adds the (T*k + T) x H fp32 per-slot outputs). All
+ * calls on a device share the one array: calls whose work overlaps on the GPU (for
+ * example on two streams) race and give wrong results; calls on one stream are ordered
+ * and safe. Nothing from a previous call needs clearing: every scratch byte read is
+ * written first in the same call. */
 MOE_API moe_status_t moe_forward_noalloc(const moe_layer_desc *desc, const uint16_t *x, const uint16_t *Wr,
                                  const float *bias, const uint16_t *W_gate_up,
                                  const uint16_t *W_down, const uint16_t *Wsh_gate_up,

@@ -40,7 +40,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
     bool ready = false;
     int num_sms = 0;
-    uint32_t *err = nullptr;
+    uint32_t *err = nullptr;  // device address of g_moe_err in the current context (looked up per call)
 };
 
 std::mutex g_mu;
@@ -65,13 +65,16 @@ moe_status_t device_info(DeviceInfo &out)
     if (!d.ready) {
         if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_moe_err) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        d.err = static_cast<uint32_t *>(p);
         d.ready = true;
     }
+    // The error word's address belongs to the current context's copy of this module: a
+    // runtime query on every call, so no saved address outlives its context (after
+    // cudaDeviceReset the module may load at another address).
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_err) != cudaSuccess || p == nullptr)
+        return MOE_ERR_CUDA;
     out = d;
+    out.err = static_cast<uint32_t *>(p);
     return MOE_OK;
 }
 

@@ -10,40 +10,30 @@
 // caller-provided workspace of moe_forward.
 //
 // How: the workspace lives in one file-scope device array of kScratchBytes (16 MiB).
-// The CUDA runtime creates it when the library's device code is loaded on a device, and
-// every device that loads the library keeps it until the process exits. Host code cannot
-// use the array's name as a device address (on the host it names a host-side stand-in),
-// so the first call on each device looks up its device address with
-// cudaGetSymbolAddress, with that device current, and caches it.
-#include <mutex>
-
+// Under CUDA's default lazy module loading the array is created on a device by the first
+// moe_forward_noalloc call there (the address lookup below loads this file's module);
+// under eager loading it is created when the library's device code is loaded. Either way
+// the device keeps it until the process exits. Host code cannot use the array's name as
+// a device address (on the host it names a host-side stand-in), so every call looks up
+// the device address with cudaGetSymbolAddress, with the caller's device current. The
+// lookup is a runtime query that allocates nothing; doing it on every call means no
+// saved address can outlive the context it belongs to (after cudaDeviceReset, or under
+// another context bound to the same device, the module and its array may move).
 #include "../../include/moe_b200.h"
 #include "internal.h"
 
 namespace {
 
 constexpr size_t kScratchBytes = size_t(16) << 20;
-constexpr int kMaxDevices = 64;
-
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-std::mutex g_scratch_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (looked up once per device).
+// Device address of the scratch array in the current context.
 moe_status_t scratch_on_current_device(void **out)
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
         return MOE_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-            return MOE_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return MOE_OK;
 }
 

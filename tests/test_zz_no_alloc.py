@@ -38,6 +38,19 @@ def test_noalloc_rejects_calls_larger_than_its_scratch():
                                  None, None) == 0
 
 
+def test_noalloc_token_limits_fit_the_scratch():
+    """The documented limits at H = 4096, E = 288, k = 8, I = Is = 1280: 188 tokens fit the
+    16 MiB scratch and 189 do not in the default mode; 70 and 71 in the deterministic mode."""
+    sh = WORKLOADS["step35_decode"]
+    for det, last in ((False, 188), (True, 70)):
+        assert _abi.moe_workspace_size(_abi.desc_of(sh, T=last, deterministic=det)) <= 16 << 20
+        assert _abi.moe_workspace_size(_abi.desc_of(sh, T=last + 1, deterministic=det)) > 16 << 20
+    L = _abi.lib()
+    args = [FAKE] * 8
+    over = _abi.desc_of(sh, T=71, deterministic=True)
+    assert L.moe_forward_noalloc(ctypes.byref(over), *args, None, None, None) == 3
+
+
 def _forward_with_workspace(d, inp, x):
     T, H, k = x.shape[0], inp["Wr"].shape[1], d.k
     ws = torch.empty(_abi.moe_workspace_size(d), dtype=torch.uint8, device="cuda")
