@@ -4,9 +4,12 @@ experts, shared expert) through the C ABI.
 
 One step = one moe_forward over one batch: router -> permutation -> gather / tile table ->
 grouped gate_up GEMM + clipped SwiGLU -> grouped down GEMM + weighted scatter-add.
-Default workload: Step-3.5-Flash-shaped prefill layer (T=4096, H=4096, E=288, top-8,
-I=Is=1280). Inputs are seeded synthetic tensors drawn on the device; the expert weights
-(9.1 GB) are larger than L2, so every step streams them from HBM.
+Default workload: the largest single-GPU configuration, the Step-5-Preview-shaped layer
+with skewed routing (T=16384, H=4096, E=352, top-8, I=Is=1536, Zipf-shaped router bias).
+Inputs are seeded synthetic tensors drawn on the device; the expert weights (13 GB) are
+larger than L2, so every step streams them from HBM. Decode-sized workloads (at most 16
+routed rows per expert) also write a 512 MiB buffer between timed steps, outside the
+timed intervals, so no step starts with the previous step's weights in L2.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl b200|reference]
 
@@ -38,7 +41,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="step35_prefill")
+    ap.add_argument("--workload", default="step5_skewed")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -210,20 +213,22 @@ def cpu_oracle_sample(shape, inp, target_s: float, max_tokens: int = 4096, start
                 cache[int(e)] = (bf16_bits(gu[int(e)]), bf16_bits(wd[int(e)]))
         experts = {int(e): cache[int(e)] for e in np.unique(r["idx"])}
         t0 = time.perf_counter()
-        oracle.forward_tokens(x_rows, Wr, bias, experts, Wsh_gu, Wsh_d, k=shape.k, scale=shape.scale,
-                              norm=shape.norm_expert_weight, limit_routed=shape.limit_routed,
-                              limit_shared=shape.limit_shared)
-        return time.perf_counter() - t0
+        ref = oracle.forward_tokens(x_rows, Wr, bias, experts, Wsh_gu, Wsh_d, k=shape.k, scale=shape.scale,
+                                    norm=shape.norm_expert_weight, limit_routed=shape.limit_routed,
+                                    limit_shared=shape.limit_shared)
+        return time.perf_counter() - t0, ref
 
     nthreads = oracle.num_threads()
     n0 = max(1, min(nthreads, shape.T))
     rows = [(start + i) % shape.T for i in range(n0)]
-    dt = run(rows)
+    dt, _ = run(rows)
     per_tok = dt / n0
     n = int(min(max_tokens, shape.T, max(n0, target_s / max(per_tok, 1e-9))))
-    rows = [(start + n0 + i) % shape.T for i in range(n)]
-    dt = run(rows)
-    return n / dt, n, dt, nthreads
+    # spread the timed sample over the whole batch (every region of the permuted rows)
+    step = max(1, shape.T // n)
+    rows = sorted({(start + n0 + i * step) % shape.T for i in range(n)})
+    dt, ref = run(rows)
+    return len(rows) / dt, len(rows), dt, nthreads, rows, ref
 
 
 def run_reference(args, shape):
@@ -241,7 +246,7 @@ def run_reference(args, shape):
     n_used = None
     threads = None
     for i in range(args.warmup + args.steps):
-        rate, n, dt, threads = cpu_oracle_sample(shape, inp, target_s=budget, start=i * 97)
+        rate, n, dt, threads, _, _ = cpu_oracle_sample(shape, inp, target_s=budget, start=i * 97)
         if i >= args.warmup:
             rates.append(rate)
             times.append(dt * 1e3)
@@ -329,14 +334,77 @@ def kernels_per_step(shape, fp8=False, deterministic=False, router=True):
 def gate_up_bytes(shape, counts, fp8=False):
     """Algorithmic HBM bytes of one gate_up launch: weights of every expert that received
     tokens (2I x H, bf16 or E4M3 codes plus one fp32 scale per 128x128 block) + shared
-    gate_up (bf16) + permuted token rows + shared token rows + hidden activations written."""
+    gate_up (bf16) + the token rows x, counted once (the method reads each token once;
+    the implementation's permuted copy of x is not algorithmic) + the hidden activations
+    written (routed and shared rows, bf16)."""
     touched = int((counts[: shape.E] > 0).sum())
     T, H, k, I, Is = shape.T, shape.H, shape.k, shape.I, shape.Is
     per_expert = 2 * I * H + (2 * I // 128) * (H // 128) * 4 if fp8 else 2 * I * H * 2
     w = touched * per_expert + 2 * Is * H * 2
-    acts = T * k * H * 2 + T * H * 2
+    acts = T * H * 2
     out = T * k * I * 2 + T * Is * 2
     return w + acts + out, touched
+
+
+def gate_up_flops(shape):
+    """Algorithmic FLOPs of one gate_up launch: 2 x (2I x H) per routed row, 2 x (2Is x H) per
+    shared row."""
+    return 4.0 * shape.H * (shape.I * shape.T * shape.k + shape.Is * shape.T)
+
+
+def gate_up_roofline(shape, counts, launch_ms, peaks, peak_kind, fp8=False, traffic=None):
+    """Roofline block of the dominant kernel (gate_up). The bound is the resource whose
+    time floor is longer at the measured peaks: algorithmic bytes / HBM copy bandwidth
+    against algorithmic FLOPs / bf16 dense peak (burst). achieved / frac are reported on
+    that bound; the other figure is kept beside it for context."""
+    nbytes, touched = gate_up_bytes(shape, counts, fp8)
+    flops = gate_up_flops(shape)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    gbs = nbytes / (launch_ms / 1e3) / 1e9
+    tfs = flops / (launch_ms / 1e3) / 1e12
+    kernel = "gemm_fp8_kernel<GateUpArgs>" if fp8 else "gate_up_pair_kernel"
+    common = {"kernel": kernel, "traffic": traffic, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+              "intensity_flop_per_byte": flops / nbytes,
+              "ridge_flop_per_byte": peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9),
+              "launch_ms": launch_ms, "touched_experts": touched,
+              "hbm": {"achieved": gbs, "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"]},
+              "tensor": {"achieved": tfs, "peak": peaks["bf16_tflops"], "frac": tfs / peaks["bf16_tflops"],
+                         "frac_of_sustained": tfs / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])}}
+    if t_tc >= t_hbm and not fp8:
+        head = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tfs / peaks["bf16_tflops"], "peak_source": f"{peak_kind} bf16_tflops (burst)"}
+    else:
+        head = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs"}
+    head.update(common)
+    return head
+
+
+def decode_sized(shape) -> bool:
+    """At most 16 routed rows per expert on average (the decode tiling of the kernels)."""
+    return shape.T * shape.k <= 16 * shape.E
+
+
+def sample_parity(y, idx, w, rows, ref, near_tie=1e-6):
+    """Parity of the timed path on the oracle's token sample: expert-id sets equal outside
+    near-ties (oracle margin < 1e-6, counted), and the output's relative Frobenius and max
+    abs errors against the fp64 oracle over the sampled tokens whose id sets agree (a
+    near-tie token routed to another valid set is counted, not compared)."""
+    import numpy as np
+    import torch
+
+    r = torch.as_tensor(rows, device=y.device)
+    yg = y[r].double().cpu().numpy()
+    ig = idx[r].cpu().numpy()
+    keep = ref["margin"] >= near_tie
+    same = (np.sort(ig, 1) == np.sort(ref["idx"], 1)).all(1)
+    d = yg[same] - ref["y"][same]
+    return {"tokens": int(len(rows)), "near_ties": int((~keep).sum()),
+            "ids_equal_outside_near_ties": bool(same[keep].all()),
+            "near_tie_tokens_routed_differently": int((~same & ~keep).sum()),
+            "rel_fro": float(np.linalg.norm(d) / np.linalg.norm(ref["y"][same])),
+            "max_abs": float(np.abs(d).max()), "bar": {"rel_fro": 1e-2, "max_abs": 3e-2}}
 
 
 def run_b200(args, shape):
@@ -401,11 +469,15 @@ def run_b200(args, shape):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     gpu_name = str(torch.cuda.get_device_properties(local).uuid)
     sampler = ClockSampler("GPU-" + gpu_name if not gpu_name.startswith("GPU-") else gpu_name)
+    flush = decode_sized(shape)
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device="cuda") if flush else None
     barrier()
     torch.cuda.synchronize()
     sampler.start()
     start.record(stream)
     for i in range(args.steps):
+        if flush:
+            flush_buf.fill_(i & 0xFF)  # evicts L2 between steps, outside the step's events
         _abi.moe_set_stage_events(evs[i])
         step(x, y)
     end.record(stream)
@@ -413,7 +485,11 @@ def run_b200(args, shape):
     clocks = sampler.stop()
     _abi.moe_set_stage_events([])
     barrier()
-    ms = max_over_ranks(start.elapsed_time(end), "cuda")
+    if flush:  # the steps' own intervals, first to last stage event, flushes excluded
+        total = sum(evs[i][0].elapsed_time(evs[i][nstage - 1]) for i in range(args.steps))
+    else:
+        total = start.elapsed_time(end)
+    ms = max_over_ranks(total, "cuda")
     names = ["router", "permute", "gather_tiles", "gate_up", "down", "combine"][: nstage - 1]
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
                 for j, n in enumerate(names)}
@@ -468,15 +544,8 @@ def run_b200(args, shape):
                "h2d_bytes_per_step": shape.T * shape.H * 2, "d2h_bytes_per_step": shape.T * shape.H * 4}
 
     peaks, peak_kind = load_peaks()
-    gbytes, touched = gate_up_bytes(shape, counts, fp8)
-    gate_ms = stage_ms["gate_up"]
-    achieved = gbytes / (gate_ms / 1e3) / 1e9
-    kernel = "gemm_fp8_kernel<GateUpArgs>" if fp8 else "gate_up_kernel"
-    roofline = {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                "traffic": profiled_traffic(shape.name, args.weights),
-                "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": gbytes, "launch_ms": gate_ms,
-                "touched_experts": touched}
+    roofline = gate_up_roofline(shape, counts, stage_ms["gate_up"], peaks, peak_kind, fp8,
+                                profiled_traffic(shape.name, args.weights))
     flops = shape.flops_per_token * shape.T
     step_ms = ms / args.steps
     value = job_tokens_per_s(world, shape.T, args.steps, ms)
@@ -485,7 +554,9 @@ def run_b200(args, shape):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded draw on device; random-init weights)",
         "config": workload_config(shape, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                                          "l2": "inputs larger than L2 (expert weights streamed every step)",
+                                          "l2": ("512 MiB written between timed steps (decode-sized); "
+                                                 "expert weights larger than L2") if flush else
+                                                "inputs larger than L2 (expert weights streamed every step)",
                                           "routing": args.routing,
                                           "weights": "fp8_e4m3_block128x128" if fp8 else "bf16",
                                           "deterministic": bool(args.deterministic)}),
@@ -498,10 +569,15 @@ def run_b200(args, shape):
         "gpu_launches": kernels_per_step(shape, fp8, args.deterministic, args.routing != "balanced") * args.steps,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
-        rate, n, dt, threads = cpu_oracle_sample(shape, inp, target_s=15.0)
+        # one more forward in the timed launch configuration: the oracle's sample doubles
+        # as a parity check of the timed path
+        _, idx_now, w_now = layer.forward(x, y=y, routing=True)
+        torch.cuda.synchronize()
+        rate, n, dt, threads, rows, ref = cpu_oracle_sample(shape, inp, target_s=15.0)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": f"{n} tokens of {shape.name} through the CPU oracle forward "
-                                          f"({dt:.1f} s, fp64)"}
+                                "sample": f"{n} tokens of {shape.name} spread over the batch, through the CPU "
+                                          f"oracle forward ({dt:.1f} s, fp64)"}
+        line["parity"] = sample_parity(y, idx_now, w_now, rows, ref)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -29,6 +29,12 @@
  *    is left for cudaGetLastError()).
  *  - Device-side waits are bounded; a wait that expires sets a device error word that
  *    moe_check_device() reports as MOE_ERR_TIMEOUT. Kernels never trap.
+ *  - Debug build (libmoe_b200_debug.so, compiled with MOE_DEBUG): every index the kernels
+ *    read from device data (expert ids, slots, tile-table entries, destination rows) is
+ *    range-checked before use; a failed check sets a bit of the device error word, the
+ *    access is clamped into range or skipped (no fault, results then meaningless), and
+ *    moe_check_device() reports MOE_ERR_DEVICE_BOUNDS. The release build compiles the
+ *    checks out.
  *  - T = 0 is valid: after the descriptor check the call returns MOE_OK without
  *    enqueueing anything, and the array pointers may then be NULL.
  */
@@ -54,7 +60,8 @@ typedef enum {
     MOE_ERR_UNSUPPORTED = 2,
     MOE_ERR_WORKSPACE = 3,
     MOE_ERR_CUDA = 4,
-    MOE_ERR_TIMEOUT = 5
+    MOE_ERR_TIMEOUT = 5,
+    MOE_ERR_DEVICE_BOUNDS = 6
 } moe_status_t;
 
 /* One MoE layer call. Field names follow Step3p5Config ("Step3p5Config配置项全解"):
@@ -288,7 +295,8 @@ MOE_API moe_status_t moe_forward_noalloc(const moe_layer_desc *desc, const uint1
                                  float *topk_w_out, void *stream);
 
 /* Waits for the current device, then reports and clears the device error word:
- * MOE_ERR_TIMEOUT if a bounded device wait expired since the last call, MOE_ERR_CUDA if
+ * MOE_ERR_TIMEOUT if a bounded device wait expired since the last call,
+ * MOE_ERR_DEVICE_BOUNDS if a range check of the debug build failed, MOE_ERR_CUDA if
  * the device reports an error, else MOE_OK. This call synchronises the device. */
 MOE_API moe_status_t moe_check_device(void);
 

@@ -13,11 +13,13 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+# MOE_B200_DEBUG=1 loads the debug build (device-side range checks, MOE_ERR_DEVICE_BOUNDS)
+DEBUG = os.environ.get("MOE_B200_DEBUG", "0") == "1"
+LIB_PATH = os.path.join(_HERE, "libmoe_b200_debug.so" if DEBUG else "libmoe_b200.so")
 
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
-                4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
+                4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_DEVICE_BOUNDS"}
 
 # Every exported entry point; the header include/moe_b200.h declares exactly these.
 EXPORTS = ["moe_status_string", "moe_workspace_size", "moe_router", "moe_permute", "moe_expert_ffn",

@@ -3,7 +3,10 @@
 Each .cu under csrc/ compiles to an object in _build/; the objects link into
 sparse_moe_layer_biased_b200/libmoe_b200.so with the CUDA runtime linked statically
 (the library then loads on a host without a driver; it needs one only to run).
-`python -m sparse_moe_layer_biased_b200.build [--force] [--verbose-ptxas]`.
+The debug variant (`--debug`) compiles the same sources with MOE_DEBUG into _build/debug/
+and links libmoe_b200_debug.so: device-side range checks of every index read from device
+data, reported through moe_check_device() as MOE_ERR_DEVICE_BOUNDS.
+`python -m sparse_moe_layer_biased_b200.build [--force] [--debug] [--verbose-ptxas]`.
 """
 from __future__ import annotations
 
@@ -17,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
+LIB_DEBUG = os.path.join(PKG, "libmoe_b200_debug.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -34,9 +38,9 @@ def _deps():
     return max(os.path.getmtime(f) for f in files)
 
 
-def _compile(src, verbose_ptxas):
-    obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+def _compile(src, verbose_ptxas, debug=False):
+    obj = os.path.join(OBJ, "debug" if debug else "", os.path.basename(src)[:-3] + ".o")
+    cmd = [NVCC, *ARCH, *FLAGS, *(["-DMOE_DEBUG"] if debug else []), "-c", src, "-o", obj]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -45,24 +49,26 @@ def _compile(src, verbose_ptxas):
     return obj, r.stderr
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps():
-        return LIB
-    os.makedirs(OBJ, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= _deps():
+        return lib
+    os.makedirs(os.path.join(OBJ, "debug") if debug else OBJ, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose_ptxas), sources()))
+        results = list(ex.map(lambda s: _compile(s, verbose_ptxas, debug), sources()))
     if verbose_ptxas:
         for obj, log in results:
             print(f"== {os.path.basename(obj)}\n{log}", file=sys.stderr)
     objs = [o for o, _ in results]
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose_ptxas="--verbose-ptxas" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose_ptxas="--verbose-ptxas" in sys.argv,
+                debug="--debug" in sys.argv))

@@ -15,6 +15,70 @@
 
 namespace moe {
 
+// Tile-table header (routed chunks, all chunks); the debug build checks it against the
+// table's capacity and clamps a bad header.
+__device__ __forceinline__ void table_counts(const int32_t *hdr, int max_chunks, uint32_t *err, int &nrc, int &ntot)
+{
+    nrc = hdr[0];
+    ntot = hdr[1];
+    if (!dbg_ok(nrc >= 0 && nrc <= ntot && ntot <= max_chunks, err)) {
+        ntot = ntot < 0 ? 0 : (ntot > max_chunks ? max_chunks : ntot);
+        nrc = nrc < 0 ? 0 : (nrc > ntot ? ntot : nrc);
+    }
+}
+
+// Tile-table entry ci = (group, first row, rows, -). The debug build checks it against
+// the table's capacity, the row capacities of the routed (rows_r) and shared (rows_s)
+// groups and the rows of one tile (cap), and clamps a bad entry into range.
+__device__ __forceinline__ int4 chunk_at(const int4 *chunks, int ci, int E, int64_t rows_r, int64_t rows_s,
+                                         int max_chunks, int cap, uint32_t *err)
+{
+    if (!dbg_ok(ci >= 0 && ci < max_chunks, err))
+        ci = 0;
+    int4 c = chunks[ci];
+    if (kDebugChecks) {
+        const int64_t span = c.x == E ? rows_s : rows_r;
+        const bool ok = c.x >= 0 && c.x <= E && c.z >= 1 && c.z <= cap && c.y >= 0 &&
+                        c.y + static_cast<int64_t>(c.z) <= span;
+        if (!dbg_ok(ok, err)) {
+            c.x = c.x < 0 ? 0 : (c.x > E ? E : c.x);
+            const int64_t sp = c.x == E ? rows_s : rows_r;
+            c.z = c.z < 1 ? 1 : (c.z > cap ? cap : c.z);
+            if (c.z > sp)
+                c.z = static_cast<int>(sp);
+            if (c.y < 0)
+                c.y = 0;
+            if (c.y + static_cast<int64_t>(c.z) > sp)
+                c.y = static_cast<int>(sp - c.z);
+        }
+    }
+    return c;
+}
+
+__device__ __forceinline__ int4 chunk_at(const GateUpArgs &a, int ci)
+{
+    return chunk_at(a.chunks, ci, a.E, a.rows_r, a.rows_s, a.max_chunks, a.cap, a.err);
+}
+
+__device__ __forceinline__ int4 chunk_at(const DownArgs &a, int ci)
+{
+    return chunk_at(a.chunks, ci, a.E, static_cast<int64_t>(a.T) * a.k, a.T, a.max_chunks, a.cap, a.err);
+}
+
+// Destination row of a down-GEMM column (slot rr of group sh ? shared : routed): the token's
+// row of y, or the slot's row of o_perm in the deterministic mode. Returns false (and the
+// debug build records it) when the row is out of range; the caller skips the column.
+__device__ __forceinline__ bool down_dst_row(const DownArgs &a, bool sh, int64_t rr, int64_t &dst_row)
+{
+    const int64_t shared_base = static_cast<int64_t>(a.T) * a.k;
+    if (a.deterministic)
+        dst_row = sh ? shared_base + rr : rr;
+    else
+        dst_row = sh ? rr : a.perm_token[rr];
+    return dbg_ok(dst_row >= 0 && dst_row < (a.deterministic ? shared_base + a.T : static_cast<int64_t>(a.T)),
+                  a.err);
+}
+
 // Tile decoding of the single-CTA grouped GEMMs. gate_up tiles enumerate (routed chunk,
 // 64*MT-feature block), then (shared chunk, feature block); down tiles (chunk,
 // 128*MT-output-feature block). chunks[ci] = (group, first row, rows).
@@ -33,7 +97,7 @@ __device__ __forceinline__ void decode_gate_up(const GateUpArgs &a, int nrc, int
         ci = nrc + tt / nfb;
         fb = tt - (tt / nfb) * nfb;
     }
-    const int4 c = a.chunks[ci];
+    const int4 c = chunk_at(a, ci);
     g = c.x;
     row0 = c.y;
     ntok = c.z;
@@ -45,7 +109,7 @@ __device__ __forceinline__ void decode_down(const DownArgs &a, int tile, int &g,
     const int nfb = a.H / (128 * MT);
     const int ci = tile / nfb;
     fb = tile - ci * nfb;
-    const int4 c = a.chunks[ci];
+    const int4 c = chunk_at(a, ci);
     g = c.x;
     row0 = c.y;
     ntok = c.z;
@@ -94,18 +158,15 @@ __device__ __forceinline__ void down_epilogue(uint32_t tmem_tile, int bn, int64_
 {
     const int64_t f = q * 32 + lane;
     const int64_t H = a.H;
-    const int64_t shared_base = static_cast<int64_t>(a.T) * a.k;
     for (int cb = 0; cb < ntok; cb += 32) {
-        // lane l fetches the destination row and weight of column cb + l
+        // lane l fetches the destination row and weight of column cb + l (-1: no column)
         const int mycol = cb + lane;
-        int64_t dst_row = 0;
+        int64_t dst_row = -1;
         float wgt = 0.0f;
         if (mycol < ntok) {
             const int64_t rr = row0 + mycol;
-            if (a.deterministic)
-                dst_row = sh ? shared_base + rr : rr;
-            else
-                dst_row = sh ? rr : a.perm_token[rr];
+            if (!down_dst_row(a, sh, rr, dst_row))
+                dst_row = -1;
             wgt = sh ? 1.0f : a.w_perm[rr];
         }
 #pragma unroll
@@ -117,7 +178,7 @@ __device__ __forceinline__ void down_epilogue(uint32_t tmem_tile, int bn, int64_
             for (int i = 0; i < 32; ++i) {
                 const int64_t drow = __shfl_sync(0xFFFFFFFFu, dst_row, i);
                 const float w = __shfl_sync(0xFFFFFFFFu, wgt, i);
-                if (cb + i < ntok) {
+                if (drow >= 0) {
                     float *p = a.out + drow * H + feat;
                     if (a.deterministic)
                         *p = w * v[i];

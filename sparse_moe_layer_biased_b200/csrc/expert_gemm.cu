@@ -153,8 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *r.holder;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int nrc = a.hdr[0];
-    const int ntot = a.hdr[1];
+    int nrc, ntot;
+    table_counts(a.hdr, a.max_chunks, a.err, nrc, ntot);
     const int tiles_r = nrc * (a.I / (64 * MT));
     const int tiles = tiles_r + (ntot - nrc) * (a.Is / (64 * MT));
     const int nkb = a.H / kBK;
@@ -246,7 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *r.holder;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int ntot = a.hdr[1];
+    int nrc, ntot;
+    table_counts(a.hdr, a.max_chunks, a.err, nrc, ntot);
     const int tiles = ntot * (a.H / (128 * MT));
 
     if (warp == 0) {

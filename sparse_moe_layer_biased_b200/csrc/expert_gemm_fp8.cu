@@ -228,7 +228,8 @@ struct Tile8 {
 
 __device__ __forceinline__ Tile8 tile_of(const GateUpArgs &a, int tile)
 {
-    const int nrc = a.hdr[0];
+    int nrc, ntot;
+    table_counts(a.hdr, a.max_chunks, a.err, nrc, ntot);
     Tile8 t;
     decode_gate_up<1>(a, nrc, nrc * (a.I / 64), tile, t.g, t.row0, t.ntok, t.fb);
     t.sh = t.g == a.E;
@@ -247,13 +248,16 @@ __device__ __forceinline__ Tile8 tile_of(const DownArgs &a, int tile)
 
 __device__ __forceinline__ int tile_count(const GateUpArgs &a)
 {
-    const int nrc = a.hdr[0];
-    return nrc * (a.I / 64) + (a.hdr[1] - nrc) * (a.Is / 64);
+    int nrc, ntot;
+    table_counts(a.hdr, a.max_chunks, a.err, nrc, ntot);
+    return nrc * (a.I / 64) + (ntot - nrc) * (a.Is / 64);
 }
 
 __device__ __forceinline__ int tile_count(const DownArgs &a)
 {
-    return a.hdr[1] * (a.H / 128);
+    int nrc, ntot;
+    table_counts(a.hdr, a.max_chunks, a.err, nrc, ntot);
+    return ntot * (a.H / 128);
 }
 
 // Weight box of one tile at K element k0 (128 rows x 128 bytes). gate_up maps are (K,

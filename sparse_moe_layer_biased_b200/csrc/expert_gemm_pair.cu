@@ -212,7 +212,7 @@ __device__ __forceinline__ void decode_gate_up_pair(const GateUpArgs &a, int nrc
         ci = nrc + tt / nfb;
         fb = tt - (tt / nfb) * nfb;
     }
-    const int4 c = a.chunks[ci];
+    const int4 c = chunk_at(a, ci);
     g = c.x;
     row0 = c.y;
     ntok = c.z;
@@ -231,8 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *r.holder;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int nrc = a.hdr[0];
-    const int ntot = a.hdr[1];
+    int nrc, ntot;
+    table_counts(a.hdr, a.max_chunks, a.err, nrc, ntot);
     const int tiles_r = nrc * (a.I / (128 * MT));
     const int tiles = tiles_r + (ntot - nrc) * (a.Is / (128 * MT));
     const int nkb = a.H / (kBK * NSL);  // stages per tile
@@ -333,19 +333,17 @@ __device__ __forceinline__ void down_epilogue_bulk(uint32_t tmem_tile, int bn, i
 {
     constexpr uint32_t kRowBytes = MT * 128 * 4;
     constexpr uint32_t kBufBytes = kOutTok * kRowBytes;
-    const int64_t shared_base = static_cast<int64_t>(a.T) * a.k;
     for (int cb = 0; cb < ntok; cb += kOutTok, ++ob) {
         uint8_t *buf = stage + (ob % NOB) * kBufBytes;
         // lane l (and l + 16) fetch the destination row and weight of column cb + l % 16
+        // (-1: no column)
         const int mycol = cb + (lane & (kOutTok - 1));
-        int64_t dst_row = 0;
+        int64_t dst_row = -1;
         float wgt = 0.0f;
         if (mycol < ntok) {
             const int64_t rr = row0 + mycol;
-            if (a.deterministic)
-                dst_row = sh ? shared_base + rr : rr;
-            else
-                dst_row = sh ? rr : a.perm_token[rr];
+            if (!down_dst_row(a, sh, rr, dst_row))
+                dst_row = -1;
             wgt = sh ? 1.0f : a.w_perm[rr];
         }
 #pragma unroll
@@ -360,7 +358,7 @@ __device__ __forceinline__ void down_epilogue_bulk(uint32_t tmem_tile, int bn, i
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (q == 0 && lane < kOutTok) {
-            if (mycol < ntok) {
+            if (dst_row >= 0) {
                 float *dst = a.out + dst_row * a.H + feat0;
                 // each output row receives k + 1 reductions spread over the whole launch:
                 // keep its lines in L2 against the weight stream (evict-last policy)
@@ -381,7 +379,7 @@ __device__ __forceinline__ void decode_down_pair(const DownArgs &a, int tile, in
     const int nfb = a.H / (256 * MT);
     const int ci = tile / nfb;
     fb = tile - ci * nfb;
-    const int4 c = a.chunks[ci];
+    const int4 c = chunk_at(a, ci);
     g = c.x;
     row0 = c.y;
     ntok = c.z;
@@ -400,7 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *r.holder;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int ntot = a.hdr[1];
+    int nrc, ntot;
+    table_counts(a.hdr, a.max_chunks, a.err, nrc, ntot);
     const int tiles = ntot * (a.H / (256 * MT));
     const int first = blockIdx.x >> 1;
     const int stride = gridDim.x >> 1;

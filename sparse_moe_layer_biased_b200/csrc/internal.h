@@ -43,6 +43,8 @@ struct PermuteArgs {
     int4 *chunks;         // optional tile table of the grouped GEMMs (with hdr, cap)
     int32_t *hdr;
     int cap;
+    uint32_t *err;        // device error word (range checks of the debug build)
+    int max_chunks;       // capacity of `chunks` (entries)
 };
 cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream);
 
@@ -54,7 +56,7 @@ cudaError_t launch_ep_regroup(const int32_t *counts, int R, int Er, int64_t nrow
                               int32_t *perm_token, int32_t *slot_of, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
-                          uint16_t *x_perm, float *w_perm, int num_sms, cudaStream_t stream);
+                          uint16_t *x_perm, float *w_perm, int num_sms, uint32_t *err, cudaStream_t stream);
 
 // Grouped-GEMM configuration. gate_up and down each split every group into chunks of at
 // most `cap` / `cap_d` token rows (the N side of one tile) and stage `mt` / `mt_d` 128-row
@@ -87,9 +89,11 @@ inline GemmConfig gemm_config(int64_t T, int64_t k, int64_t E, int64_t H, int64_
 // Splits every group (E routed experts, then the shared expert) into chunks of at most
 // `cap` rows. hdr[0] = routed chunk count, hdr[1] = total chunk count. When `chunks_d` is
 // not NULL the same launch also builds a second table of at most `cap_d` rows per chunk
-// (header hdr_d).
+// (header hdr_d). max_chunks / max_chunks_d: table capacities (range checks of the debug
+// build, which also check the offsets against `rows`, the permuted rows' capacity).
 cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr, int cap_d,
-                          int4 *chunks_d, int32_t *hdr_d, cudaStream_t stream);
+                          int4 *chunks_d, int32_t *hdr_d, int max_chunks, int max_chunks_d, int64_t rows,
+                          uint32_t *err, cudaStream_t stream);
 // FP8-weight configuration (single CTAs, one weight tile per stage): 32-row chunks for
 // decode-sized calls, else 128-row chunks.
 inline GemmConfig gemm_config_fp8(int64_t T, int64_t k, int64_t E)
@@ -113,6 +117,11 @@ struct GateUpArgs {
     int E, H, I, Is;
     float lim_r, lim_s;
     const float *w_scale;  // FP8 kernels: block scales [E, 2I/128, H/128]; else unused
+    // capacities checked by the debug build: routed rows of x_perm / h, shared rows of
+    // h_sh, tile-table entries, rows per tile
+    int64_t rows_r, rows_s;
+    int max_chunks, cap;
+    uint32_t *err;  // device error word
 };
 cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
                            const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
@@ -127,6 +136,8 @@ struct DownArgs {
     int E, H, I, Is, T, k;
     int deterministic;
     const float *w_scale;  // FP8 kernels: block scales [E, H/128, I/128]; else unused
+    int max_chunks, cap;   // tile-table capacity and rows per tile (debug-build range checks)
+    uint32_t *err;         // device error word
 };
 cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
                         const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
@@ -207,6 +218,6 @@ cudaError_t launch_bwd_dwr(const uint16_t *x_pad, const float *dl_pad, const int
                            int E, int H, float *dWr, cudaStream_t stream);
 
 cudaError_t launch_combine(const float *o_perm, const int32_t *slot_of, int T, int k, int H, float *y,
-                           cudaStream_t stream);
+                           uint32_t *err, cudaStream_t stream);
 
 }  // namespace moe

@@ -345,39 +345,48 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
         return MOE_ERR_CUDA;
     cudaError_t e = cudaSuccess;
     if (groups != FfnGroups::kSharedOnly)
-        e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, s);
+        e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, di.err, s);
     const int shared_rows = groups == FfnGroups::kRoutedOnly || split ? 0 : d.T;
+    const int nch = static_cast<int>(moe::max_chunks(d.T, d.k, d.E, cfg.cap));
+    const int nch_d = static_cast<int>(moe::max_chunks(d.T, d.k, d.E, cfg.cap_d));
+    int nch_s = 0, nch_sd = 0;  // shared-expert tables of the FP8 split (see above)
+    if (split) {
+        nch_s = static_cast<int>(chunks_sd - chunks_s);
+        nch_sd = static_cast<int>(moe::max_chunks(d.T, d.k, d.E, cfg_sh.cap_d)) - nch_s;
+    }
     if (e == cudaSuccess)
         e = moe::launch_chunks(offsets, d.E, shared_rows, cfg.cap, chunks, hdr, cfg.cap_d,
-                               cfg.cap_d != cfg.cap ? chunks_d : nullptr, hdr_d, s);
+                               cfg.cap_d != cfg.cap ? chunks_d : nullptr, hdr_d, nch, nch_d, Tk, di.err, s);
     if (e == cudaSuccess && split)
-        e = moe::launch_chunks(offsets, 0, d.T, cfg_sh.cap, chunks_s, hdr + 4, cfg_sh.cap_d, chunks_sd, hdr + 8, s);
+        e = moe::launch_chunks(offsets, 0, d.T, cfg_sh.cap, chunks_s, hdr + 4, cfg_sh.cap_d, chunks_sd, hdr + 8,
+                               nch_s, nch_sd, Tk, di.err, s);
     if (e == cudaSuccess && !d.deterministic)
         e = cudaMemsetAsync(out, 0, static_cast<size_t>(d.T) * d.H * 4, s);
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
     const moe::WaitCfg wc = wait_cfg(di);
-    moe::GateUpArgs ga{chunks, hdr, h, h_sh, d.E, d.H, d.I, d.Is, d.limit_routed, d.limit_shared, W.gu_scale};
+    moe::GateUpArgs ga{chunks, hdr, h, h_sh, d.E, d.H, d.I, d.Is, d.limit_routed, d.limit_shared, W.gu_scale,
+                       Tk, d.T, nch, cfg.cap, di.err};
     if (!stage_mark(3, s))
         return MOE_ERR_CUDA;
     e = fp8 ? moe::launch_gate_up_fp8(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s)
             : moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s);
     if (e == cudaSuccess && split) {
         const moe::GateUpArgs gs{chunks_s, hdr + 4, h, h_sh, 0, d.H, d.I, d.Is, d.limit_routed, d.limit_shared,
-                                 nullptr};
+                                 nullptr, Tk, d.T, nch_s, cfg_sh.cap, di.err};
         e = moe::launch_gate_up(tm_wsh2, tm_wsh2, tm_x2, tm_x2, gs, wc, di.num_sms, cfg_sh, s);
     }
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
     moe::DownArgs da{chunks_d, hdr_d, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic,
-                     W.d_scale};
+                     W.d_scale, cfg.cap_d != cfg.cap ? nch_d : nch, cfg.cap_d, di.err};
     if (!stage_mark(4, s))
         return MOE_ERR_CUDA;
     e = fp8 ? moe::launch_down_fp8(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s)
             : moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s);
     if (e == cudaSuccess && split) {
         const moe::DownArgs ds{chunks_sd, hdr + 8, perm_token, w_perm, out, 0, d.H, d.I, d.Is, d.T, d.k,
-                               d.deterministic, nullptr};
+                               d.deterministic, nullptr, nch_sd, cfg_sh.cap_d, di.err};
         e = moe::launch_down(tm_wdsh2, tm_wdsh2, tm_hsh2, tm_hsh2, ds, wc, di.num_sms, cfg_sh, s);
     }
     if (e != cudaSuccess || !stage_mark(5, s))
@@ -397,7 +406,7 @@ moe_status_t forward_routed(const moe_layer_desc &d, const DeviceInfo &di, const
     if (!stage_mark(1, s))
         return MOE_ERR_CUDA;
     const moe::PermuteArgs pa{idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, nullptr, nullptr, nullptr,
-                              nullptr, 0};
+                              nullptr, 0, di.err, 0};
     if (moe::launch_permute(pa, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     float *out = d.deterministic ? at<float>(ws, L.o_perm) : y;
@@ -405,7 +414,7 @@ moe_status_t forward_routed(const moe_layer_desc &d, const DeviceInfo &di, const
     if (st != MOE_OK)
         return st;
     if (d.deterministic) {
-        st = cuda_status(moe::launch_combine(out, slot_of, d.T, d.k, d.H, y, s));
+        st = cuda_status(moe::launch_combine(out, slot_of, d.T, d.k, d.H, y, di.err, s));
         if (st == MOE_OK && !stage_mark(6, s))
             st = MOE_ERR_CUDA;
     }
@@ -487,6 +496,8 @@ const char *moe_status_string(int status)
         return "CUDA error";
     case MOE_ERR_TIMEOUT:
         return "device wait timed out";
+    case MOE_ERR_DEVICE_BOUNDS:
+        return "device range check failed (debug build)";
     default:
         return "unknown status";
     }
@@ -535,7 +546,7 @@ moe_status_t moe_permute(const moe_layer_desc *desc, const int32_t *topk_idx, in
     if ((st = device_info(di)) != MOE_OK)
         return st;
     const moe::PermuteArgs pa{topk_idx, desc->T, desc->k, desc->E, counts, offsets, perm_token, slot_of,
-                              nullptr, nullptr, nullptr, nullptr, 0};
+                              nullptr, nullptr, nullptr, nullptr, 0, di.err, 0};
     return cuda_status(moe::launch_permute(pa, static_cast<cudaStream_t>(stream)));
 }
 
@@ -577,8 +588,11 @@ moe_status_t moe_combine(const moe_layer_desc *desc, const float *o_perm, const 
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(o_perm) || !aligned16(y))
         return MOE_ERR_UNSUPPORTED;
-    return cuda_status(
-        moe::launch_combine(o_perm, slot_of, desc->T, desc->k, desc->H, y, static_cast<cudaStream_t>(stream)));
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK)
+        return st;
+    return cuda_status(moe::launch_combine(o_perm, slot_of, desc->T, desc->k, desc->H, y, di.err,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 // Device staging of moe_forward_host after the forward workspace: two input buffers
@@ -710,7 +724,7 @@ moe_status_t moe_ep_pack(const moe_layer_desc *desc, const uint16_t *x, const fl
     if ((st = device_info(di)) != MOE_OK)
         return st;
     return cuda_status(moe::launch_gather(x, topk_w, slot_of, desc->T, desc->k, desc->H, x_send, w_send, di.num_sms,
-                                          static_cast<cudaStream_t>(stream)));
+                                          di.err, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_ep_experts(const moe_layer_desc *desc, int32_t ep_ranks, const int32_t *recv_counts,
@@ -946,7 +960,7 @@ moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const u
                     wgroups, hdr, w_pad, tok_pad, gu_r, gu_s, dgu_r, dgu_s, hw_r, hw_s, dw_pad, dx, dW_down,
                     dW_gate_up, dWsh_down, dWsh_gate_up};
     const moe::PermuteArgs pa{topk_idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, nullptr, nullptr,
-                              nullptr, nullptr, 0};
+                              nullptr, nullptr, 0, di.err, 0};
     cudaError_t e = moe::launch_permute(pa, s);
     if (e == cudaSuccess)
         e = moe::launch_bwd_layout(counts, d.E, d.T, poff, chunks, wgroups, hdr, s);
@@ -991,7 +1005,9 @@ moe_status_t moe_check_device(void)
         if (cudaMemcpyToSymbol(g_moe_err, &zero, sizeof zero) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
-    return (v & moe::kDevErrTimeout) ? MOE_ERR_TIMEOUT : MOE_OK;
+    if (v & moe::kDevErrTimeout)
+        return MOE_ERR_TIMEOUT;
+    return (v & moe::kDevErrBounds) ? MOE_ERR_DEVICE_BOUNDS : MOE_OK;
 }
 
 moe_status_t moe_set_stage_events(void *const *events, int n)

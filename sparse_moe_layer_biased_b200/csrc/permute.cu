@@ -18,7 +18,10 @@ constexpr int kPermThreads = 1024;  // 32 warps per CTA; warp w owns a contiguou
 // scan `offs` (E + 1 entries in shared or global memory): group g in [0, E] (E = shared
 // expert, T rows) of n rows becomes ceil(n / cap) chunks of equal size rounded up to 16
 // rows (the last one shorter). hdr[0] = routed chunk count, hdr[1] = total.
-__device__ void build_chunk_table(const int32_t *offs, int E, int T, int cap, int4 *chunks, int32_t *hdr)
+// The debug build checks every group's rows against `rows` (capacity of the permuted rows
+// of the group's kind: T*k routed, T shared) and every entry against the table capacity.
+__device__ void build_chunk_table(const int32_t *offs, int E, int T, int cap, int4 *chunks, int32_t *hdr,
+                                  int max_chunks, int64_t rows, uint32_t *err)
 {
     __shared__ int warp_sums[32];
     for (int g0 = 0; g0 <= E; g0 += kPermThreads) {
@@ -29,6 +32,8 @@ __device__ void build_chunk_table(const int32_t *offs, int E, int T, int cap, in
         if (g < E) {
             base = offs[g];
             n = offs[g + 1] - base;
+            if (!dbg_ok(base >= 0 && n >= 0 && base + static_cast<int64_t>(n) <= rows, err))
+                n = 0;
         } else if (g == E) {
             n = T;
         }
@@ -58,7 +63,8 @@ __device__ void build_chunk_table(const int32_t *offs, int E, int T, int cap, in
         for (int c = 0; c < nch; ++c) {
             const int r = c * csz;
             const int len = n - r < csz ? n - r : csz;
-            chunks[start + c] = make_int4(g, base + r, len, 0);
+            if (dbg_ok(start + c < max_chunks, err))
+                chunks[start + c] = make_int4(g, base + r, len, 0);
         }
         if (g == E) {
             hdr[0] = start;
@@ -198,9 +204,11 @@ __global__ void __launch_bounds__(kPermThreads)
         if (valid) {
             const int slot = mine[e] + __popc(m & ((1u << lane) - 1u));
             a.slot_of[n] = slot;
-            a.perm_token[slot] = static_cast<int32_t>(n / k);
-            if (a.w_perm)
-                a.w_perm[slot] = a.topk_w[n];
+            if (dbg_ok(slot >= 0 && slot < static_cast<int64_t>(T) * k, a.err)) {
+                a.perm_token[slot] = static_cast<int32_t>(n / k);
+                if (a.w_perm)
+                    a.w_perm[slot] = a.topk_w[n];
+            }
         }
         __syncwarp();
         if (valid && lane == 31 - __clz(m))
@@ -211,7 +219,7 @@ __global__ void __launch_bounds__(kPermThreads)
     for (int t = c0 + threadIdx.x; t < c1; t += kPermThreads)
         a.perm_token[shared_base + t] = t;
     if (rank == 0 && a.chunks)
-        build_chunk_table(offs, E, T, a.cap, a.chunks, a.hdr);
+        build_chunk_table(offs, E, T, a.cap, a.chunks, a.hdr, a.max_chunks, static_cast<int64_t>(T) * k, a.err);
 
     cluster_sync_all();  // no CTA leaves while a peer may still read its totals
 }
@@ -221,13 +229,15 @@ __global__ void __launch_bounds__(kPermThreads)
 __global__ void __launch_bounds__(256)
     gather_kernel(const uint4 *__restrict__ x, const float *__restrict__ topk_w,
                   const int32_t *__restrict__ slot_of, int64_t nent, int k, int vec_per_row,
-                  uint4 *__restrict__ x_perm, float *__restrict__ w_perm)
+                  uint4 *__restrict__ x_perm, float *__restrict__ w_perm, uint32_t *err)
 {
     const int lane = threadIdx.x & 31;
     const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     for (int64_t n = gw; n < nent; n += nw) {
         const int64_t slot = slot_of[n];
+        if (!dbg_ok(slot >= 0 && slot < nent, err))
+            continue;
         const int64_t t = n / k;
         const uint4 *src = x + t * vec_per_row;
         uint4 *dst = x_perm + slot * vec_per_row;
@@ -329,24 +339,28 @@ __global__ void __launch_bounds__(256)
 // Tile table from an offsets array in global memory (the moe_expert_ffn entry point).
 __global__ void __launch_bounds__(kPermThreads)
     chunks_kernel(const int32_t *__restrict__ offsets, int E, int T, int cap, int4 *__restrict__ chunks,
-                  int32_t *__restrict__ hdr, int cap_d, int4 *__restrict__ chunks_d, int32_t *__restrict__ hdr_d)
+                  int32_t *__restrict__ hdr, int cap_d, int4 *__restrict__ chunks_d, int32_t *__restrict__ hdr_d,
+                  int max_chunks, int max_chunks_d, int64_t rows, uint32_t *err)
 {
-    build_chunk_table(offsets, E, T, cap, chunks, hdr);
+    build_chunk_table(offsets, E, T, cap, chunks, hdr, max_chunks, rows, err);
     if (chunks_d)
-        build_chunk_table(offsets, E, T, cap_d, chunks_d, hdr_d);
+        build_chunk_table(offsets, E, T, cap_d, chunks_d, hdr_d, max_chunks_d, rows, err);
 }
 
 // y[t] = sum_{j<k} o_perm[slot_of[t, j]] + o_perm[T*k + t], in that order.
 __global__ void __launch_bounds__(256)
     combine_kernel(const float4 *__restrict__ o_perm, const int32_t *__restrict__ slot_of, int T, int k,
-                   int vec_per_row, float4 *__restrict__ y)
+                   int vec_per_row, float4 *__restrict__ y, uint32_t *err)
 {
     const int t = blockIdx.x;
     const int64_t shared_row = static_cast<int64_t>(T) * k + t;
     for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
-            const float4 o = __ldg(o_perm + static_cast<int64_t>(slot_of[static_cast<int64_t>(t) * k + j]) * vec_per_row + v);
+            int64_t slot = slot_of[static_cast<int64_t>(t) * k + j];
+            if (!dbg_ok(slot >= 0 && slot < static_cast<int64_t>(T) * k, err))
+                continue;
+            const float4 o = __ldg(o_perm + slot * vec_per_row + v);
             acc.x += o.x;
             acc.y += o.y;
             acc.z += o.z;
@@ -392,14 +406,14 @@ cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream)
 }
 
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
-                          uint16_t *x_perm, float *w_perm, int num_sms, cudaStream_t stream)
+                          uint16_t *x_perm, float *w_perm, int num_sms, uint32_t *err, cudaStream_t stream)
 {
     const int64_t nent = static_cast<int64_t>(T) * k;
     const int64_t blocks_needed = (nent + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms) * 8;
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
     gather_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(x), topk_w, slot_of, nent, k, H / 8,
-                                            reinterpret_cast<uint4 *>(x_perm), w_perm);
+                                            reinterpret_cast<uint4 *>(x_perm), w_perm, err);
     return cudaGetLastError();
 }
 
@@ -426,17 +440,19 @@ cudaError_t launch_ep_regroup(const int32_t *counts, int R, int Er, int64_t nrow
 }
 
 cudaError_t launch_chunks(const int32_t *offsets, int E, int T, int cap, int4 *chunks, int32_t *hdr, int cap_d,
-                          int4 *chunks_d, int32_t *hdr_d, cudaStream_t stream)
+                          int4 *chunks_d, int32_t *hdr_d, int max_chunks, int max_chunks_d, int64_t rows,
+                          uint32_t *err, cudaStream_t stream)
 {
-    chunks_kernel<<<1, kPermThreads, 0, stream>>>(offsets, E, T, cap, chunks, hdr, cap_d, chunks_d, hdr_d);
+    chunks_kernel<<<1, kPermThreads, 0, stream>>>(offsets, E, T, cap, chunks, hdr, cap_d, chunks_d, hdr_d, max_chunks,
+                                                  max_chunks_d, rows, err);
     return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const float *o_perm, const int32_t *slot_of, int T, int k, int H, float *y,
-                           cudaStream_t stream)
+                           uint32_t *err, cudaStream_t stream)
 {
     combine_kernel<<<T, 256, 0, stream>>>(reinterpret_cast<const float4 *>(o_perm), slot_of, T, k, H / 4,
-                                          reinterpret_cast<float4 *>(y));
+                                          reinterpret_cast<float4 *>(y), err);
     return cudaGetLastError();
 }
 

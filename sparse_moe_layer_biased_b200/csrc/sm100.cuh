@@ -12,6 +12,24 @@ namespace moe {
 
 // Bits of the library's device error word.
 constexpr uint32_t kDevErrTimeout = 1u;
+constexpr uint32_t kDevErrBounds = 2u;
+
+// Range checks of the debug build (MOE_DEBUG): dbg_ok(cond, err) returns cond and, when
+// it is false, records kDevErrBounds in *err; callers then clamp or skip the access. In
+// the release build it is constant true and the condition is compiled out.
+#ifdef MOE_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool dbg_ok(bool cond, uint32_t *err)
+{
+    if (!kDebugChecks)
+        return true;
+    if (!cond)
+        atomicOr(err, kDevErrBounds);
+    return cond;
+}
 
 // Every device wait gives up after limit_ns nanoseconds of %globaltimer, records
 // kDevErrTimeout in *err and tells the other roles of the CTA through an abort flag.

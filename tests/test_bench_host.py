@@ -35,11 +35,58 @@ def test_gate_up_byte_model_counts_touched_experts_only():
     b, touched = bench.gate_up_bytes(sh, counts)
     assert touched == 10
     w = 10 * 2 * sh.I * sh.H * 2 + 2 * sh.Is * sh.H * 2
-    acts = sh.T * sh.k * sh.H * 2 + sh.T * sh.H * 2
+    acts = sh.T * sh.H * 2  # x read once; the permuted copy is not algorithmic
     out = sh.T * sh.k * sh.I * 2 + sh.T * sh.Is * 2
     assert b == w + acts + out
     b8, _ = bench.gate_up_bytes(sh, counts, fp8=True)
     assert b8 == b - 10 * 2 * sh.I * sh.H + 10 * (2 * sh.I // 128) * (sh.H // 128) * 4
+
+
+PEAKS = {"hbm_gbs": 6541.8, "bf16_tflops": 1662.5, "bf16_tflops_sustained": 1383.5}
+
+
+def _counts(sh, touched):
+    c = np.zeros(sh.E + 1, np.int64)
+    c[:touched] = 1
+    return c
+
+
+def test_roofline_bound_follows_arithmetic_intensity():
+    # skewed Step-5 shape (248 experts touched): 3.71 TFLOP against 6.85 GB -> tensor-bound
+    sh = WORKLOADS["step5_skewed"]
+    r = bench.gate_up_roofline(sh, _counts(sh, 248), 3.0, PEAKS, "measured")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    flops = 4.0 * sh.H * (sh.I * sh.T * sh.k + sh.Is * sh.T)
+    assert r["algorithmic_flops"] == flops
+    assert abs(r["achieved"] - flops / 3e-3 / 1e12) < 1e-9 * r["achieved"]
+    assert abs(r["frac"] - r["achieved"] / 1662.5) < 1e-12
+    # Step-3.5 prefill (242 touched): 141 flop/B, below the ~254 flop/B ridge -> HBM-bound
+    s35 = WORKLOADS["step35_prefill"]
+    r = bench.gate_up_roofline(s35, _counts(s35, 242), 1.0, PEAKS, "measured")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["intensity_flop_per_byte"] < r["ridge_flop_per_byte"]
+    # decode: HBM-bound; FP8 weights are always reported against HBM
+    dec = WORKLOADS["step35_decode"]
+    assert bench.gate_up_roofline(dec, _counts(dec, 159), 0.5, PEAKS, "measured")["bound"] == "hbm"
+    assert bench.gate_up_roofline(sh, _counts(sh, 248), 3.0, PEAKS, "measured", fp8=True)["bound"] == "hbm"
+
+
+def test_decode_sized_workloads_flush_l2():
+    assert bench.decode_sized(WORKLOADS["step35_decode"])
+    assert not bench.decode_sized(WORKLOADS["step5_skewed"])
+
+
+def test_sample_parity_counts_near_tie_tokens_separately():
+    import torch
+
+    rng = np.random.default_rng(0)
+    y = torch.from_numpy(rng.standard_normal((10, 8)).astype(np.float32))
+    idx = torch.from_numpy(np.tile(np.arange(2, dtype=np.int32), (10, 1)))
+    ref = {"y": y.double().numpy()[[1, 4, 7]], "idx": np.array([[1, 0], [0, 1], [0, 5]], np.int32),
+           "margin": np.array([1.0, 1.0, 1e-8], np.float32)}
+    p = bench.sample_parity(y, idx, None, [1, 4, 7], ref)
+    assert p["tokens"] == 3 and p["near_ties"] == 1 and p["near_tie_tokens_routed_differently"] == 1
+    assert p["ids_equal_outside_near_ties"] and p["rel_fro"] == 0.0 and p["max_abs"] == 0.0
 
 
 def test_source_digest_ignores_comments_only():

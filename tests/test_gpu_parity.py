@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import oracle
-from _parity import (check_output, check_routing, gpu_router, oracle_forward_rows, oracle_router, rel_fro)
+from _parity import (check_near_tie_outputs, check_near_ties, check_output, check_routing, chunk_covering_sample,
+                     gpu_router, oracle_forward_rows, oracle_router, rel_fro)
 from sparse_moe_layer_biased_b200 import _abi
 from sparse_moe_layer_biased_b200.inputs import WORKLOADS, LayerShape, bf16_bits, draw, token_sample
 from sparse_moe_layer_biased_b200.layer import MoeLayer
@@ -80,6 +81,7 @@ def test_router_small(name):
     o = oracle_router(sh, inp)
     keep = check_routing(g["idx"], g["w"], o, sh.E, sh.k)
     assert keep.mean() > 0.95
+    check_near_ties(sh, inp, g["idx"], g["w"], o)
     m = np.isfinite(o["margin"]) & keep
     np.testing.assert_allclose(g["margin"][m], o["margin"][m], atol=2e-6)
     if sh.k == sh.E:
@@ -142,6 +144,28 @@ def test_forward_small(name, det):
     o = {"idx": ref["idx"], "w": ref["w"], "margin": ref["margin"]}
     keep = check_routing(idx, w, o, sh.E, sh.k)
     check_output(y[keep], ref["y"][keep], name)
+    check_near_ties(sh, inp, idx, w, o)
+    check_near_tie_outputs(sh, inp, y, idx, w, o)
+
+
+def test_exact_ties_go_to_the_lower_index_and_are_validated():
+    """Experts in identical pairs (same router row, same bias) tie exactly; with k odd the
+    k-th and (k+1)-th ranked experts are the two halves of one pair on every token, so every
+    token is a near tie (margin 0). Both sides break the tie towards the lower index; the
+    near-tie checks validate every token's set and weights and compare every output with the
+    oracle's forward on the GPU's own routing."""
+    sh = LayerShape("ties", T=256, H=256, E=24, k=5, I=64, Is=64, seed=36, limit_routed=0.25)
+    inp = draw(sh)
+    inp["Wr"][1::2] = inp["Wr"][0::2]
+    inp["bias"][1::2] = inp["bias"][0::2]
+    y, idx, w = _forward(sh, _to(inp))
+    ref = oracle.forward_full(inp, sh)
+    o = {"idx": ref["idx"], "w": ref["w"], "margin": ref["margin"]}
+    assert np.all(ref["margin"] == 0.0)
+    check_routing(idx, w, o, sh.E, sh.k)
+    assert check_near_ties(sh, inp, idx, w, o) == sh.T
+    assert check_near_tie_outputs(sh, inp, y, idx, w, o) == sh.T
+    np.testing.assert_array_equal(np.sort(idx, 1), np.sort(ref["idx"], 1))
 
 
 def test_deterministic_matches_atomic_and_repeats():
@@ -251,8 +275,11 @@ def test_full_size_routing_all_tokens(full):
     o = oracle_router(sh, full["inp"])
     keep = check_routing(full["idx"], full["w"], o, sh.E, sh.k)
     excluded = int((~keep).sum())
-    print(f"{sh.name}: near-tie tokens excluded: {excluded} of {sh.T}")
+    validated = check_near_ties(sh, full["inp"], full["idx"], full["w"], o)
+    print(f"{sh.name}: near-tie tokens excluded from the bit-exact comparison: {excluded} of {sh.T}; "
+          f"validated as ties: {validated}")
     assert excluded <= max(4, sh.T // 1000)
+    assert validated == excluded
     counts = np.bincount(full["idx"].ravel(), minlength=sh.E)
     if sh.bias_kind == "zipf":
         share = np.sort(counts)[::-1][:8].sum() / counts.sum()
@@ -268,14 +295,30 @@ def test_full_size_permutation_bit_exact(full):
         np.testing.assert_array_equal(g[key], o[key], err_msg=key)
 
 
+def _caps(sh):
+    """Row caps of the grouped GEMMs' tile tables for the workload: 32-row chunks at decode
+    size (at most 16 rows per expert on average), else 256-row gate_up and 128-row down
+    chunks on CTA pairs."""
+    return (32,) if sh.T * sh.k <= 16 * sh.E else (256, 128)
+
+
 @pytest.mark.slow
 def test_full_size_output_sampled(full):
+    """At least 256 tokens: the last row of every gate_up and down chunk of the 8 hottest
+    experts, the last chunk of every split expert, random tokens up to 256."""
     sh = full["shape"]
-    rows = token_sample(sh.T, 16, sh.seed).numpy()
-    ref = oracle_forward_rows(sh, full["inp"], torch.from_numpy(rows).cuda())
+    rows, covered = chunk_covering_sample(full["idx"], sh.E, caps=_caps(sh), seed=sh.seed)
+    tr = torch.from_numpy(rows).cuda()
+    ref = oracle_forward_rows(sh, full["inp"], tr)
     keep = ref["margin"] >= 1e-6
-    y = full["y"][torch.from_numpy(rows).cuda()].cpu().numpy()
-    check_output(y[keep], ref["y"][keep], sh.name)
+    y = full["y"][tr].cpu().numpy()
+    g_idx, g_w = full["idx"][rows], full["w"][rows]
+    np.testing.assert_array_equal(np.sort(g_idx[keep], 1), np.sort(ref["idx"][keep], 1))
+    rf, ma = check_output(y[keep], ref["y"][keep], sh.name)
+    ties = check_near_tie_outputs(sh, full["inp"], y, g_idx, g_w, ref, rows=rows)
+    print(f"{sh.name}: output sample {len(rows)} tokens covering {covered} chunks; rel_fro {rf:.2e} "
+          f"max_abs {ma:.2e}; near-tie tokens compared on the GPU's routing: {ties}")
+    assert len(rows) >= 256
 
 
 def _with_ids(sh, inp, idx, w, det=False):
