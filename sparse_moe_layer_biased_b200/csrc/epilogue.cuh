@@ -117,10 +117,12 @@ __device__ __forceinline__ void decode_down(const DownArgs &a, int tile, int &g,
 
 // gate_up: accumulator m holds 64 (gate, up) row pairs interleaved by lane (lane 2i gate
 // row i, lane 2i+1 its up row) of features feat0 + 64 m .. feat0 + 64 m + 63. Writes
-// h[row0 + c, feature] = act(gate, up) in bf16 for the ntok columns of the chunk.
+// h[row0 + c, feature] = act(gate, up) in bf16 for the ntok columns of the chunk, in blocks
+// of 32 columns starting at cb0 and cstep apart (several warps may share a lane quarter).
 template <int MT>
 __device__ __forceinline__ void gate_up_epilogue(uint32_t tmem_tile, int bn, int64_t feat0, int ntok,
-                                                 int64_t row0, uint16_t *out, int64_t ld, float L, int q, int lane)
+                                                 int64_t row0, uint16_t *out, int64_t ld, float L, int q, int lane,
+                                                 int cb0 = 0, int cstep = 32)
 {
     const int row = q * 32 + lane;
     const int pair = row >> 1;
@@ -129,7 +131,7 @@ __device__ __forceinline__ void gate_up_epilogue(uint32_t tmem_tile, int bn, int
     for (int m = 0; m < MT; ++m) {
         const int64_t feat = feat0 + m * 64 + pair;
         const uint32_t tb = tmem_tile + m * bn + (static_cast<uint32_t>(q * 32) << 16);
-        for (int cb = 0; cb < ntok; cb += 32) {
+        for (int cb = cb0; cb < ntok; cb += cstep) {
             float v[32];
             tmem_load32(tb + cb, v);
 #pragma unroll

@@ -351,12 +351,13 @@ cudaError_t down_impl(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, cons
 // of <= 32 tokens with one weight tile per stage and a 10-deep ring of 20 KB stages;
 // chunks of <= 128 tokens with two weight tiles per stage (48 KB stages, 4 deep); shapes
 // whose I, Is or H do not split into two tiles use one weight tile and <= 256 tokens.
-cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
-                           const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
-                           const GemmConfig &c, cudaStream_t stream)
+cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const TokMaps &tok,
+                           const GateUpArgs &a, const WaitCfg &wc, int grid, const GemmConfig &c,
+                           cudaStream_t stream)
 {
     if (c.pair)
-        return launch_gate_up_pair(tm_w, tm_wsh, tm_xp, tm_x, a, wc, grid, stream);
+        return launch_gate_up_pair(tm_w, tm_wsh, tok, a, wc, grid, stream);
+    const CUtensorMap &tm_xp = tok.routed, &tm_x = tok.shared;
     if (c.cap == 32)
         return gate_up_impl<32, 10, 1>(tm_w, tm_wsh, tm_xp, tm_x, a, wc, grid, stream);
     if (c.mt == 2)
@@ -364,12 +365,12 @@ cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, c
     return gate_up_impl<256, 4, 1>(tm_w, tm_wsh, tm_xp, tm_x, a, wc, grid, stream);
 }
 
-cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
-                        const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
-                        const GemmConfig &c, cudaStream_t stream)
+cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const TokMaps &tok,
+                        const DownArgs &a, const WaitCfg &wc, int grid, const GemmConfig &c, cudaStream_t stream)
 {
     if (c.pair)
-        return launch_down_pair(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
+        return launch_down_pair(tm_wd, tm_wdsh, tok, a, wc, grid, stream);
+    const CUtensorMap &tm_h = tok.routed, &tm_hsh = tok.shared;
     if (c.cap_d == 32)
         return down_impl<32, 10, 1>(tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc, grid, stream);
     if (c.mt_d == 2)

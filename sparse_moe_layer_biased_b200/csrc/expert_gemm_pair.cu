@@ -26,13 +26,11 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 192;
 constexpr int kBK = 64;
 constexpr uint32_t kATileBytes = 128 * 128;  // 128 weight rows x 64 bf16
 // Token rows reach shared memory in boxes of 64 rows (8 KB per K slice); a stage loads only
 // the boxes that hold rows of its chunk, so a short chunk in a wide tile costs no extra bytes.
-constexpr int kTokBoxRows = 64;
-constexpr uint32_t kTokBoxBytes = kTokBoxRows * 128;
+constexpr int kTokBoxRows = kPairTokBoxRows;
 
 // BN = token rows per pair tile (N of the pair MMA); each CTA holds BN/2 of them.
 // NB = accumulator buffers in TMEM (2: the epilogue of one tile overlaps the next tile's
@@ -48,8 +46,9 @@ struct PairGeo {
     static constexpr uint32_t kStageBytes = NSL * kSliceBytes;
     static constexpr uint32_t kOutOff = S * kStageBytes;
     static constexpr uint32_t kBarOff = kOutOff + OUT;
-    static constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * S + 5);  // holder, abort flag, epilogue flags
-    static constexpr uint32_t kSmemBytes = kMiscOff + 48 + 1024;
+    // misc: TMEM holder, abort flag, then 8 epilogue flags per epilogue group (up to two)
+    static constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * S + 5);
+    static constexpr uint32_t kSmemBytes = kMiscOff + 80 + 1024;
     static constexpr uint32_t kBufCols = MT * BN;
     static constexpr uint32_t kTmemCols = NB * kBufCols <= 32 ? 32 : (NB * kBufCols <= 64 ? 64 : (NB * kBufCols <= 128 ? 128 : (NB * kBufCols <= 256 ? 256 : 512)));
     static_assert(NB * kBufCols <= 512, "accumulators exceed TMEM");
@@ -57,7 +56,7 @@ struct PairGeo {
     static_assert(kSmemBytes <= kMaxDynSmem, "ring exceeds shared memory");
 
     static_assert(BN % 32 == 0 && BN <= 256, "pair token tile");
-    static_assert((BN / 2) % kTokBoxRows == 0, "token rows per CTA are whole boxes");
+    static_assert(BN / 2 <= kPairTokBoxRowsL, "token rows per CTA fit one large box");
 };
 
 struct PairRing {
@@ -69,8 +68,10 @@ struct PairRing {
     uint32_t acce_leader;  // shared::cluster address of the leader's acce[0]
 };
 
+// epi_warps: epilogue warps per CTA (each arrives once per tile on the leader's
+// accumulator-empty barrier, from both CTAs).
 template <class G, int S>
-__device__ __forceinline__ uint8_t *pair_setup(uint8_t *smem_raw, PairRing &r)
+__device__ __forceinline__ uint8_t *pair_setup(uint8_t *smem_raw, PairRing &r, int epi_warps = 4)
 {
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *smem = smem_raw + pad;
@@ -92,7 +93,7 @@ __device__ __forceinline__ uint8_t *pair_setup(uint8_t *smem_raw, PairRing &r)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&r.accf[b], 1);
-            mbar_init(&r.acce[b], 8);  // 4 epilogue warps in each CTA of the pair
+            mbar_init(&r.acce[b], 2 * epi_warps);  // every epilogue warp of both CTAs
         }
         mbar_init(r.drain, 1);
         *r.abort_flag = 0;
@@ -218,16 +219,20 @@ __device__ __forceinline__ void decode_gate_up_pair(const GateUpArgs &a, int nrc
     ntok = c.z;
 }
 
-template <int BN, int S, int MT, int NB, int NSL>
-__global__ void __launch_bounds__(kThreads, 1)
+// EW epilogue warps (4 or 8): with 8, two warps share each TMEM lane quarter and take
+// alternate 32-column blocks of the tile.
+template <int BN, int S, int MT, int NB, int NSL, int EW>
+__global__ void __launch_bounds__(64 + 32 * EW, 1)
     gate_up_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_wsh,
                         const __grid_constant__ CUtensorMap tm_xp, const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ CUtensorMap tm_xp_l, const __grid_constant__ CUtensorMap tm_x_l,
                         const GateUpArgs a, const WaitCfg wc)
 {
+    static_assert(EW == 4 || EW == 8, "one or two groups of four epilogue warps");
     using G = PairGeo<BN, S, MT, NB, 0, NSL>;
     extern __shared__ uint8_t smem_raw[];
     PairRing r;
-    uint8_t *smem = pair_setup<G, S>(smem_raw, r);
+    uint8_t *smem = pair_setup<G, S>(smem_raw, r, EW);
     const uint32_t tmem = *r.holder;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -245,6 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_map(&tm_wsh);
             tma_prefetch_map(&tm_xp);
             tma_prefetch_map(&tm_x);
+            tma_prefetch_map(&tm_xp_l);
+            tma_prefetch_map(&tm_x_l);
             int it = 0;
             bool stop = false;
             for (int tile = first; tile < tiles && !stop; tile += stride) {
@@ -252,9 +259,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_gate_up_pair<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
                 const bool sh = g == a.E;
                 const int half = ((ntok + 15) & ~15) >> 1;  // token rows used from each CTA
-                const int nbox = (half + kTokBoxRows - 1) / kTokBoxRows;
+                // one token box per K slice: 64 rows, or 128 when the half is larger
+                const bool large = half > kTokBoxRows;
+                const uint32_t tok_bytes = (large ? kPairTokBoxRowsL : kTokBoxRows) * 128;
                 const CUtensorMap *mw = sh ? &tm_wsh : &tm_w;
-                const CUtensorMap *mb = sh ? &tm_x : &tm_xp;
+                const CUtensorMap *mb = large ? (sh ? &tm_x_l : &tm_xp_l) : (sh ? &tm_x : &tm_xp);
                 const int ge = sh ? 0 : g;
                 const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
                 const int brow = row0 + static_cast<int>(r.rank) * half;
@@ -265,17 +274,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (r.rank == 0)
-                        mbar_arrive_expect_tx(&r.full[s], 2 * NSL * (G::kABytes + nbox * kTokBoxBytes));
+                        mbar_arrive_expect_tx(&r.full[s], 2 * NSL * (G::kABytes + tok_bytes));
                     const uint32_t bar = r.full_leader + 8 * s;
-                    // per K slice: one box with this CTA's MT weight tiles, then the token
-                    // boxes that cover its half of the chunk (rows past the half are loaded
-                    // and ignored)
+                    // per K slice: one box with this CTA's MT weight tiles, then one box of
+                    // token rows covering its half of the chunk (rows past the half are
+                    // loaded and ignored)
                     for (int c = 0; c < NSL; ++c) {
                         uint8_t *A = smem + s * G::kStageBytes + c * G::kSliceBytes;
                         const int k0 = (kb * NSL + c) * kBK;
                         tma_load_4d_pair(A, mw, bar, k0, 0, wt0 * 64, ge);
-                        for (int b = 0; b < nbox; ++b)
-                            tma_load_2d_pair(A + G::kABytes + b * kTokBoxBytes, mb, bar, k0, brow + b * kTokBoxRows);
+                        tma_load_2d_pair(A + G::kABytes, mb, bar, k0, brow);
                     }
                 }
             }
@@ -292,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         const int q = warp & 3;
+        const int grp = (warp - 2) / 4;
         int tc = 0;
         for (int tile = first; tile < tiles; tile += stride, ++tc) {
             int g, row0, ntok, fb;
@@ -303,7 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool sh = g == a.E;
             const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
             gate_up_epilogue<MT>(tmem + buf * G::kBufCols, BN, static_cast<int64_t>(wt0) * 64, ntok, row0,
-                                 sh ? a.h_sh : a.h, sh ? a.Is : a.I, sh ? a.lim_s : a.lim_r, q, lane);
+                                 sh ? a.h_sh : a.h, sh ? a.Is : a.I, sh ? a.lim_s : a.lim_r, q, lane, grp * 32,
+                                 (EW / 4) * 32);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -317,23 +327,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 // down on pairs: a pair tile covers 2 * MT * 128 output features.
 //
 // Epilogue through shared memory and TMA bulk reductions: per block of 16 token columns,
-// the four epilogue warps write the weighted outputs of this CTA's MT * 128 features as 16
-// rows of MT * 512 bytes (one row per token) into a staging buffer; then one lane per token
-// issues a bulk reduce-add of its row into y[token] (or, in deterministic mode, a bulk store
-// into o_perm[slot]). Each output row thus takes one MT * 512-byte reduction at L2 instead
-// of MT * 4 reductions of 128 bytes. NOB staging buffers rotate so a block's reductions
-// overlap the next block's TMEM loads; a buffer is rewritten only after its bulk reads are
-// done. Named barrier 1 joins the 4 epilogue warps.
+// the four warps of an epilogue group write the weighted outputs of this CTA's MT * 128
+// features as 16 rows of MT * 512 bytes (one row per token) into a staging buffer; then one
+// lane per token issues a bulk reduce-add of its row into y[token] (or, in deterministic
+// mode, a bulk store into o_perm[slot]). Each output row thus takes one MT * 512-byte
+// reduction at L2 instead of MT * 4 reductions of 128 bytes. NOB staging buffers per group
+// rotate so a block's reductions overlap the next block's TMEM loads; a buffer is
+// rewritten only after its bulk reads are done. With EW = 8 epilogue warps, two groups of
+// four (each covering all 128 TMEM lanes) take alternate 16-token blocks of a tile, with
+// their own staging buffers and named barrier (id 1 + group).
 constexpr int kOutTok = 16;
 
 template <int MT, int NOB>
 __device__ __forceinline__ void down_epilogue_bulk(uint32_t tmem_tile, int bn, int64_t feat0, int ntok, int64_t row0,
                                                    bool sh, const DownArgs &a, int q, int lane, uint8_t *stage,
-                                                   int &ob)
+                                                   int &ob, int grp, int ngrp)
 {
     constexpr uint32_t kRowBytes = MT * 128 * 4;
     constexpr uint32_t kBufBytes = kOutTok * kRowBytes;
-    for (int cb = 0; cb < ntok; cb += kOutTok, ++ob) {
+    const int bar_id = 1 + grp;
+    for (int cb = grp * kOutTok; cb < ntok; cb += ngrp * kOutTok, ++ob) {
         uint8_t *buf = stage + (ob % NOB) * kBufBytes;
         // lane l (and l + 16) fetch the destination row and weight of column cb + l % 16
         // (-1: no column)
@@ -356,7 +369,7 @@ __device__ __forceinline__ void down_epilogue_bulk(uint32_t tmem_tile, int bn, i
                 col[i * (kRowBytes / 4)] = __shfl_sync(0xFFFFFFFFu, wgt, i) * v[i];
         }
         fence_proxy_async_smem();
-        named_bar_sync(1, 128);
+        named_bar_sync(bar_id, 128);
         if (q == 0 && lane < kOutTok) {
             if (dst_row >= 0) {
                 float *dst = a.out + dst_row * a.H + feat0;
@@ -370,7 +383,7 @@ __device__ __forceinline__ void down_epilogue_bulk(uint32_t tmem_tile, int bn, i
             }
             bulk_wait_read<NOB - 1>();  // the buffer written next is no longer being read
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(bar_id, 128);
     }
 }
 template <int MT>
@@ -385,16 +398,22 @@ __device__ __forceinline__ void decode_down_pair(const DownArgs &a, int tile, in
     ntok = c.z;
 }
 
-template <int BN, int S, int MT, int NB, int NOB>
-__global__ void __launch_bounds__(kThreads, 1)
+// BN token rows per tile (BN / 2 per CTA), S stages of NSL 64-wide K slices, MT weight
+// tiles of 128 rows per CTA and slice, NB TMEM accumulators, NOB staging buffers per
+// epilogue group, EW epilogue warps (4 or 8).
+template <int BN, int S, int MT, int NB, int NOB, int NSL, int EW>
+__global__ void __launch_bounds__(64 + 32 * EW, 1)
     down_pair_kernel(const __grid_constant__ CUtensorMap tm_wd, const __grid_constant__ CUtensorMap tm_wdsh,
                      const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_hsh,
+                     const __grid_constant__ CUtensorMap tm_h_l, const __grid_constant__ CUtensorMap tm_hsh_l,
                      const DownArgs a, const WaitCfg wc)
 {
-    using G = PairGeo<BN, S, MT, NB, NOB * kOutTok * MT * 512>;
+    static_assert(EW == 4 || EW == 8, "one or two groups of four epilogue warps");
+    constexpr int kGroups = EW / 4;
+    using G = PairGeo<BN, S, MT, NB, kGroups * NOB * kOutTok * MT * 512, NSL>;
     extern __shared__ uint8_t smem_raw[];
     PairRing r;
-    uint8_t *smem = pair_setup<G, S>(smem_raw, r);
+    uint8_t *smem = pair_setup<G, S>(smem_raw, r, EW);
     const uint32_t tmem = *r.holder;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -410,17 +429,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_map(&tm_wdsh);
             tma_prefetch_map(&tm_h);
             tma_prefetch_map(&tm_hsh);
+            tma_prefetch_map(&tm_h_l);
+            tma_prefetch_map(&tm_hsh_l);
             int it = 0;
             bool stop = false;
             for (int tile = first; tile < tiles && !stop; tile += stride) {
                 int g, row0, ntok, fb;
                 decode_down_pair<MT>(a, tile, g, row0, ntok, fb);
                 const bool sh = g == a.E;
-                const int nkb = (sh ? a.Is : a.I) / kBK;
+                const int nkb = (sh ? a.Is : a.I) / (kBK * NSL);
                 const int half = ((ntok + 15) & ~15) >> 1;
-                const int nbox = (half + kTokBoxRows - 1) / kTokBoxRows;
+                const bool large = half > kTokBoxRows;
+                const uint32_t tok_bytes = (large ? kPairTokBoxRowsL : kTokBoxRows) * 128;
                 const CUtensorMap *mw = sh ? &tm_wdsh : &tm_wd;
-                const CUtensorMap *mb = sh ? &tm_hsh : &tm_h;
+                const CUtensorMap *mb = large ? (sh ? &tm_hsh_l : &tm_h_l) : (sh ? &tm_hsh : &tm_h);
                 const int wrow = (sh ? 0 : g * a.H) + (fb * 2 + static_cast<int>(r.rank)) * MT * 128;
                 const int brow = row0 + static_cast<int>(r.rank) * half;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
@@ -430,12 +452,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (r.rank == 0)
-                        mbar_arrive_expect_tx(&r.full[s], 2 * (G::kABytes + nbox * kTokBoxBytes));
+                        mbar_arrive_expect_tx(&r.full[s], 2 * NSL * (G::kABytes + tok_bytes));
                     const uint32_t bar = r.full_leader + 8 * s;
-                    uint8_t *A = smem + s * G::kStageBytes;
-                    tma_load_2d_pair(A, mw, bar, kb * kBK, wrow);
-                    for (int b = 0; b < nbox; ++b)
-                        tma_load_2d_pair(A + G::kABytes + b * kTokBoxBytes, mb, bar, kb * kBK, brow + b * kTokBoxRows);
+                    for (int c = 0; c < NSL; ++c) {
+                        uint8_t *A = smem + s * G::kStageBytes + c * G::kSliceBytes;
+                        const int k0 = (kb * NSL + c) * kBK;
+                        tma_load_2d_pair(A, mw, bar, k0, wrow);
+                        tma_load_2d_pair(A + G::kABytes, mb, bar, k0, brow);
+                    }
                 }
             }
             pair_producer_drain<S>(r, it, stop || *r.abort_flag, wc);
@@ -445,32 +469,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto info = [&](int tile, int &ntok, int &nk) {
                 int g, row0, fb;
                 decode_down_pair<MT>(a, tile, g, row0, ntok, fb);
-                nk = (g == a.E ? a.Is : a.I) / kBK;
+                nk = (g == a.E ? a.Is : a.I) / (kBK * NSL);
             };
-            pair_mma_role<G, S, BN, MT, NB, 1>(r, smem, tmem, first, tiles, stride, info, wc);
+            pair_mma_role<G, S, BN, MT, NB, NSL>(r, smem, tmem, first, tiles, stride, info, wc);
         }
     } else {
         const int q = warp & 3;
+        const int grp = (warp - 2) / 4;
+        const int bar_id = 1 + grp;
         int tc = 0, ob = 0;
-        volatile int *epi_ok = reinterpret_cast<volatile int *>(smem + G::kMiscOff + 16);
+        volatile int *epi_ok = reinterpret_cast<volatile int *>(smem + G::kMiscOff + 16) + grp * 8;
+        uint8_t *stage = smem + G::kOutOff + grp * (NOB * kOutTok * MT * 512);
         for (int tile = first; tile < tiles; tile += stride, ++tc) {
             int g, row0, ntok, fb;
             decode_down_pair<MT>(a, tile, g, row0, ntok, fb);
             const int buf = tc % NB;
-            // The four warps agree on the wait's outcome before the barrier-synchronised
-            // epilogue, so a wait that expires in one warp cannot strand the others at a
-            // named barrier (flags double-buffered by tile parity).
+            // The four warps of a group agree on the wait's outcome before the
+            // barrier-synchronised epilogue, so a wait that expires in one warp cannot
+            // strand the others at a named barrier (flags double-buffered by tile parity).
             const bool ok = warp_wait(&r.accf[buf], (tc / NB) & 1, wc, r.abort_flag);
             if (lane == 0)
                 epi_ok[(tc & 1) * 4 + q] = ok ? 1 : 0;
-            named_bar_sync(1, 128);
+            named_bar_sync(bar_id, 128);
             const volatile int *f = epi_ok + (tc & 1) * 4;
             if (!(f[0] && f[1] && f[2] && f[3]))
                 break;
             tc_fence_after();
             const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
             down_epilogue_bulk<MT, NOB>(tmem + buf * G::kBufCols, BN, static_cast<int64_t>(wt0) * 128, ntok, row0,
-                                        g == a.E, a, q, lane, smem + G::kOutOff, ob);
+                                        g == a.E, a, q, lane, stage, ob, grp, kGroups);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -483,14 +510,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <class Kernel, class... Args>
-cudaError_t launch_pairs(Kernel kernel, int smem, int grid, cudaStream_t stream, Args... args)
+cudaError_t launch_pairs(Kernel kernel, int smem, int grid, int threads, cudaStream_t stream, Args... args)
 {
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid & ~1, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -509,31 +536,37 @@ cudaError_t launch_pairs(Kernel kernel, int smem, int grid, cudaStream_t stream,
 // gate_up: pair tiles of up to 256 token rows (128 per CTA) x 128 features, one weight
 // tile per CTA and K slice, two 64-wide K slices per stage (8 pair MMAs per barrier test
 // and commit of the MMA thread), three 64 KB stages. Most experts of a prefill batch then
-// need one pass over their weights. down: 128 token rows x 512 output features, two weight
-// tiles per CTA and stage (40 KB stages, 4 deep) and two 16 KB output staging buffers for
-// the bulk reductions. Both keep two TMEM accumulators.
-constexpr int kGateUpStages = 3, kGateUpSlices = 2;
-using GateUpPair = PairGeo<kPairCapGateUp, kGateUpStages, kPairMtGateUp, 2, 0, kGateUpSlices>;
-constexpr int kDownStages = 4, kDownOutBufs = 2;  // 4 x 40 KB ring + 2 x 16 KB output staging
-using DownPair = PairGeo<kPairCapDown, kDownStages, kPairMtDown, 2, kDownOutBufs * kOutTok * kPairMtDown * 512>;
+// need one pass over their weights. down: the same 256-row chunks x 256 output features, one
+// weight tile per CTA and K slice, two K slices per stage (three 64 KB stages), eight
+// epilogue warps in two groups, each with two 8 KB output staging buffers for the bulk
+// reductions (measured against 128-row chunks with two weight tiles per CTA and four
+// epilogue warps: 5% faster on the Step-5 prefill down GEMM, equal on the other shapes; with
+// four epilogue warps the 256-row chunks were 20-35% slower: the reductions of a 256-column
+// tile then outlast its mainloop). Both keep two TMEM accumulators.
+constexpr int kGateUpStages = 3, kGateUpSlices = 2, kGateUpBufs = 2, kGateUpEpiWarps = 4;
+using GateUpPair = PairGeo<kPairCapGateUp, kGateUpStages, kPairMtGateUp, kGateUpBufs, 0, kGateUpSlices>;
+constexpr int kDownStages = 3, kDownSlices = 2, kDownOutBufs = 2, kDownEpiWarps = 8;
+using DownPair = PairGeo<kPairCapDown, kDownStages, kPairMtDown, 2,
+                         (kDownEpiWarps / 4) * kDownOutBufs * kOutTok * kPairMtDown * 512, kDownSlices>;
 
 }  // namespace
 
-cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
-                                const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
-                                cudaStream_t stream)
+cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const TokMaps &tok,
+                                const GateUpArgs &a, const WaitCfg &wc, int grid, cudaStream_t stream)
 {
-    return launch_pairs(gate_up_pair_kernel<kPairCapGateUp, kGateUpStages, kPairMtGateUp, 2, kGateUpSlices>,
-                        static_cast<int>(GateUpPair::kSmemBytes), grid, stream, tm_w, tm_wsh, tm_xp, tm_x, a, wc);
+    return launch_pairs(gate_up_pair_kernel<kPairCapGateUp, kGateUpStages, kPairMtGateUp, kGateUpBufs, kGateUpSlices,
+                                            kGateUpEpiWarps>,
+                        static_cast<int>(GateUpPair::kSmemBytes), grid, 64 + 32 * kGateUpEpiWarps, stream, tm_w,
+                        tm_wsh, tok.routed, tok.shared, tok.routed_l, tok.shared_l, a, wc);
 }
 
-cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
-                             const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
-                             cudaStream_t stream)
+cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const TokMaps &tok,
+                             const DownArgs &a, const WaitCfg &wc, int grid, cudaStream_t stream)
 {
-    return launch_pairs(down_pair_kernel<kPairCapDown, kDownStages, kPairMtDown, 2, kDownOutBufs>,
-                        static_cast<int>(DownPair::kSmemBytes),
-                        grid, stream, tm_wd, tm_wdsh, tm_h, tm_hsh, a, wc);
+    return launch_pairs(
+        down_pair_kernel<kPairCapDown, kDownStages, kPairMtDown, 2, kDownOutBufs, kDownSlices, kDownEpiWarps>,
+        static_cast<int>(DownPair::kSmemBytes), grid, 64 + 32 * kDownEpiWarps, stream, tm_wd, tm_wdsh, tok.routed,
+        tok.shared, tok.routed_l, tok.shared_l, a, wc);
 }
 
 }  // namespace moe

@@ -63,11 +63,26 @@ cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t 
 // weight tiles per pipeline stage and CTA; `pair` = tiles run on CTA pairs (cta_group::2).
 // Decode-sized calls (at most 16 tokens per expert on average) use 32-row chunks with one
 // weight tile and a deep ring. Larger calls run on CTA pairs when I and Is split into
-// 128-feature gate_up pair tiles and H into 512-feature down pair tiles: gate_up on chunks
-// of up to 256 rows (so most experts of a prefill batch stream their weights once), down on
-// 128-row chunks with two weight tiles. Otherwise single CTAs take two weight tiles per
-// stage (I, Is multiples of 128, H of 256), else one weight tile and 256-row chunks.
-constexpr int kPairCapGateUp = 256, kPairMtGateUp = 1, kPairCapDown = 128, kPairMtDown = 2;
+// 128-feature gate_up pair tiles and H into 512-feature blocks: both GEMMs on chunks of up to
+// 256 rows (so most experts of a prefill batch stream their weights once) with one weight
+// tile per CTA (gate_up 128 features, down 256 output features per pair tile). Otherwise
+// single CTAs take two weight tiles per stage (I, Is multiples of 128, H of 256), else one
+// weight tile and 256-row chunks.
+constexpr int kPairCapGateUp = 256, kPairMtGateUp = 1, kPairCapDown = 256, kPairMtDown = 1;
+// Token rows per TMA box on CTA pairs: the token tensor maps of the pair kernels are encoded
+// with 64-row boxes, and a second set with 128-row boxes; a tile whose CTA half holds up to
+// 64 rows loads one 64-row box per K slice, a larger one one 128-row box. 16-row boxes (at
+// most 15 unused rows per K slice) measured 20-30% slower on gate_up: the single producer
+// thread then issues up to 18 TMA copies per stage and becomes the bound.
+constexpr int kPairTokBoxRows = 64;
+constexpr int kPairTokBoxRowsL = 128;
+
+// Token-row tensor maps of one grouped GEMM: routed rows (x_perm or h) and shared rows (x or
+// h_sh), boxes of the chunk cap rows on single CTAs or kPairTokBoxRows on pairs, and for the
+// pair kernels the same rows with kPairTokBoxRowsL-row boxes (routed_l, shared_l).
+struct TokMaps {
+    CUtensorMap routed, shared, routed_l, shared_l;
+};
 struct GemmConfig {
     int cap;
     int mt;
@@ -123,9 +138,9 @@ struct GateUpArgs {
     int max_chunks, cap;
     uint32_t *err;  // device error word
 };
-cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
-                           const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
-                           const GemmConfig &c, cudaStream_t stream);
+cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const TokMaps &tok,
+                           const GateUpArgs &a, const WaitCfg &wc, int grid, const GemmConfig &c,
+                           cudaStream_t stream);
 
 struct DownArgs {
     const int4 *chunks;
@@ -139,16 +154,13 @@ struct DownArgs {
     int max_chunks, cap;   // tile-table capacity and rows per tile (debug-build range checks)
     uint32_t *err;         // device error word
 };
-cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
-                        const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
-                        const GemmConfig &c, cudaStream_t stream);
+cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const TokMaps &tok,
+                        const DownArgs &a, const WaitCfg &wc, int grid, const GemmConfig &c, cudaStream_t stream);
 
-cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
-                                const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
-                                cudaStream_t stream);
-cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
-                             const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
-                             cudaStream_t stream);
+cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const TokMaps &tok,
+                                const GateUpArgs &a, const WaitCfg &wc, int grid, cudaStream_t stream);
+cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const TokMaps &tok,
+                             const DownArgs &a, const WaitCfg &wc, int grid, cudaStream_t stream);
 
 // FP8 E4M3 routed experts (128x128 block scales, shared expert BF16): tm_w / tm_wd map
 // the E4M3 codes (gate_up: 4-D (H, half, row, expert) bytes; down: 2-D (I, E*H) bytes).

@@ -219,12 +219,13 @@ WsLayout ws_layout(const moe_layer_desc &d)
     L.h = take(T * k * I * 2);
     L.h_sh = take(T * Is * 2);
     // chunk tables of gate_up and (when its cap differs) of down, sized for both weight
-    // formats; hdr holds both headers
+    // formats; the second region also holds the shared expert's two tables when FP8 routed
+    // experts run with the BF16 shared expert on the pair kernels; hdr holds three headers
     const moe::GemmConfig cfg = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
     const moe::GemmConfig cfg8 = moe::gemm_config_fp8(d.T, d.k, d.E);
     const int cap_min = cfg.cap < cfg8.cap ? cfg.cap : cfg8.cap;
     L.chunks = take(static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, cap_min)) * 16);
-    L.chunks_d = take(cfg.cap_d != cfg.cap ? static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, cfg.cap_d)) * 16 : 0);
+    L.chunks_d = take(static_cast<size_t>(moe::max_chunks(d.T, d.k, d.E, cfg.cap_d)) * 16);
     L.hdr = take(64);
     L.o_perm = take(d.deterministic ? (T * k + T) * H * 4 : 0);
     L.idx = take(T * k * 4);
@@ -302,19 +303,23 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
 
     // One TMA box per weight operand and pipeline stage: all weight tiles of a stage (64 * mt
     // gate/up feature pairs, or 128 * mt_d down rows). Token rows come in one box of the
-    // chunk cap on single CTAs, in 64-row boxes on CTA pairs.
-    const uint32_t brows = static_cast<uint32_t>(cfg.pair ? 64 : cfg.cap);
+    // chunk cap on single CTAs, in one 64- or 128-row box per K slice on CTA pairs.
+    const uint32_t brows = static_cast<uint32_t>(cfg.pair ? moe::kPairTokBoxRows : cfg.cap);
+    const uint32_t brows_l = static_cast<uint32_t>(moe::kPairTokBoxRowsL);
     const uint32_t feats = static_cast<uint32_t>(64 * cfg.mt);
     const uint32_t drows = static_cast<uint32_t>(128 * cfg.mt_d);
-    CUtensorMap tm_w, tm_wsh, tm_xp, tm_x, tm_wd, tm_wdsh, tm_h, tm_hsh;
+    CUtensorMap tm_w, tm_wsh, tm_wd, tm_wdsh;
+    moe::TokMaps tok_gu, tok_d;  // token rows of gate_up (x_perm, x) and down (h, h_sh)
     const int64_t EH = static_cast<int64_t>(d.E) * d.H;
     const uint32_t inner8 = 128;  // one 128-wide scale block of E4M3 codes per stage
     bool ok = (fp8 ? map_gate_up_u8(&tm_w, W.gu, d.H, d.I, d.E, feats, inner8)
                    : map_gate_up(&tm_w, W.gu, d.H, d.I, d.E, feats)) &&
               (fp8 ? map_rows_u8(&tm_wd, W.d, d.I, EH, drows, inner8) : map_rows(&tm_wd, W.d, d.I, EH, drows)) &&
-              map_gate_up(&tm_wsh, W.sh_gu, d.H, d.Is, 1, feats) && map_rows(&tm_xp, x_perm, d.H, Tk, brows) &&
-              map_rows(&tm_x, x, d.H, d.T, brows) && map_rows(&tm_wdsh, W.sh_d, d.Is, d.H, drows) &&
-              map_rows(&tm_h, h, d.I, Tk, brows) && map_rows(&tm_hsh, h_sh, d.Is, d.T, brows);
+              map_gate_up(&tm_wsh, W.sh_gu, d.H, d.Is, 1, feats) && map_rows(&tm_wdsh, W.sh_d, d.Is, d.H, drows) &&
+              map_rows(&tok_gu.routed, x_perm, d.H, Tk, brows) && map_rows(&tok_gu.shared, x, d.H, d.T, brows) &&
+              map_rows(&tok_gu.routed_l, x_perm, d.H, Tk, brows_l) && map_rows(&tok_gu.shared_l, x, d.H, d.T, brows_l) &&
+              map_rows(&tok_d.routed, h, d.I, Tk, brows) && map_rows(&tok_d.shared, h_sh, d.Is, d.T, brows) &&
+              map_rows(&tok_d.routed_l, h, d.I, Tk, brows_l) && map_rows(&tok_d.shared_l, h_sh, d.Is, d.T, brows_l);
     if (!ok)
         return MOE_ERR_CUDA;
 
@@ -325,20 +330,26 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     // cap_d), and headers at hdr + 4 / hdr + 8.
     const moe::GemmConfig cfg_sh = moe::gemm_config(d.T, d.k, d.E, d.H, d.I, d.Is);
     const bool split = fp8 && groups == FfnGroups::kBoth && cfg.cap > 32 && cfg_sh.pair;
-    CUtensorMap tm_wsh2, tm_x2, tm_wdsh2, tm_hsh2;
+    CUtensorMap tm_wsh2, tm_wdsh2;
+    moe::TokMaps tok_gu2, tok_d2;  // the shared expert's token rows as routed-position maps
     int4 *chunks_s = nullptr, *chunks_sd = nullptr;
     if (split) {
         const int64_t n_gu = (d.T + cfg_sh.cap - 1) / cfg_sh.cap + 1;
         const int64_t n_d = (d.T + cfg_sh.cap_d - 1) / cfg_sh.cap_d + 1;
-        if (cfg_sh.cap_d == cfg_sh.cap || n_gu + n_d > moe::max_chunks(d.T, d.k, d.E, cfg_sh.cap_d))
+        if (n_gu + n_d > moe::max_chunks(d.T, d.k, d.E, cfg_sh.cap_d))
             return MOE_ERR_WORKSPACE;
         chunks_s = at<int4>(ws, L.chunks_d);
         chunks_sd = chunks_s + n_gu;
+        const uint32_t b = moe::kPairTokBoxRows;
         if (!(map_gate_up(&tm_wsh2, W.sh_gu, d.H, d.Is, 1, static_cast<uint32_t>(64 * cfg_sh.mt)) &&
-              map_rows(&tm_x2, x, d.H, d.T, 64) &&
               map_rows(&tm_wdsh2, W.sh_d, d.Is, d.H, static_cast<uint32_t>(128 * cfg_sh.mt_d)) &&
-              map_rows(&tm_hsh2, h_sh, d.Is, d.T, 64)))
+              map_rows(&tok_gu2.routed, x, d.H, d.T, b) && map_rows(&tok_gu2.routed_l, x, d.H, d.T, brows_l) &&
+              map_rows(&tok_d2.routed, h_sh, d.Is, d.T, b) && map_rows(&tok_d2.routed_l, h_sh, d.Is, d.T, brows_l)))
             return MOE_ERR_CUDA;
+        tok_gu2.shared = tok_gu2.routed;
+        tok_gu2.shared_l = tok_gu2.routed_l;
+        tok_d2.shared = tok_d2.routed;
+        tok_d2.shared_l = tok_d2.routed_l;
     }
 
     if (!stage_mark(2, s))
@@ -369,12 +380,12 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
                        Tk, d.T, nch, cfg.cap, di.err};
     if (!stage_mark(3, s))
         return MOE_ERR_CUDA;
-    e = fp8 ? moe::launch_gate_up_fp8(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s)
-            : moe::launch_gate_up(tm_w, tm_wsh, tm_xp, tm_x, ga, wc, di.num_sms, cfg, s);
+    e = fp8 ? moe::launch_gate_up_fp8(tm_w, tm_wsh, tok_gu.routed, tok_gu.shared, ga, wc, di.num_sms, cfg, s)
+            : moe::launch_gate_up(tm_w, tm_wsh, tok_gu, ga, wc, di.num_sms, cfg, s);
     if (e == cudaSuccess && split) {
         const moe::GateUpArgs gs{chunks_s, hdr + 4, h, h_sh, 0, d.H, d.I, d.Is, d.limit_routed, d.limit_shared,
                                  nullptr, Tk, d.T, nch_s, cfg_sh.cap, di.err};
-        e = moe::launch_gate_up(tm_wsh2, tm_wsh2, tm_x2, tm_x2, gs, wc, di.num_sms, cfg_sh, s);
+        e = moe::launch_gate_up(tm_wsh2, tm_wsh2, tok_gu2, gs, wc, di.num_sms, cfg_sh, s);
     }
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -382,12 +393,12 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
                      W.d_scale, cfg.cap_d != cfg.cap ? nch_d : nch, cfg.cap_d, di.err};
     if (!stage_mark(4, s))
         return MOE_ERR_CUDA;
-    e = fp8 ? moe::launch_down_fp8(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s)
-            : moe::launch_down(tm_wd, tm_wdsh, tm_h, tm_hsh, da, wc, di.num_sms, cfg, s);
+    e = fp8 ? moe::launch_down_fp8(tm_wd, tm_wdsh, tok_d.routed, tok_d.shared, da, wc, di.num_sms, cfg, s)
+            : moe::launch_down(tm_wd, tm_wdsh, tok_d, da, wc, di.num_sms, cfg, s);
     if (e == cudaSuccess && split) {
         const moe::DownArgs ds{chunks_sd, hdr + 8, perm_token, w_perm, out, 0, d.H, d.I, d.Is, d.T, d.k,
                                d.deterministic, nullptr, nch_sd, cfg_sh.cap_d, di.err};
-        e = moe::launch_down(tm_wdsh2, tm_wdsh2, tm_hsh2, tm_hsh2, ds, wc, di.num_sms, cfg_sh, s);
+        e = moe::launch_down(tm_wdsh2, tm_wdsh2, tok_d2, ds, wc, di.num_sms, cfg_sh, s);
     }
     if (e != cudaSuccess || !stage_mark(5, s))
         return MOE_ERR_CUDA;
