@@ -154,13 +154,16 @@ __device__ __forceinline__ void gate_up_epilogue(uint32_t tmem_tile, int bn, int
 // down: accumulator m holds output features feat0 + 128 m + (lane row). Routed columns
 // add w_slot * o into y[token] (fp32 atomics) or store it in o_perm[slot]
 // (deterministic mode); shared-expert columns (sh) add o with weight 1.
+// Columns are taken in blocks of 32 starting at cb0, cstep apart (several warps may share a
+// lane quarter).
 template <int MT>
 __device__ __forceinline__ void down_epilogue(uint32_t tmem_tile, int bn, int64_t feat0, int ntok, int64_t row0,
-                                              bool sh, const DownArgs &a, int q, int lane)
+                                              bool sh, const DownArgs &a, int q, int lane, int cb0 = 0,
+                                              int cstep = 32)
 {
     const int64_t f = q * 32 + lane;
     const int64_t H = a.H;
-    for (int cb = 0; cb < ntok; cb += 32) {
+    for (int cb = cb0; cb < ntok; cb += cstep) {
         // lane l fetches the destination row and weight of column cb + l (-1: no column)
         const int mycol = cb + lane;
         int64_t dst_row = -1;

@@ -30,7 +30,6 @@ constexpr int kBK = 64;
 constexpr uint32_t kATileBytes = 128 * 128;  // 128 weight rows x 64 bf16
 // Token rows reach shared memory in boxes of 64 rows (8 KB per K slice); a stage loads only
 // the boxes that hold rows of its chunk, so a short chunk in a wide tile costs no extra bytes.
-constexpr int kTokBoxRows = kPairTokBoxRows;
 
 // BN = token rows per pair tile (N of the pair MMA); each CTA holds BN/2 of them.
 // NB = accumulator buffers in TMEM (2: the epilogue of one tile overlaps the next tile's
@@ -46,9 +45,9 @@ struct PairGeo {
     static constexpr uint32_t kStageBytes = NSL * kSliceBytes;
     static constexpr uint32_t kOutOff = S * kStageBytes;
     static constexpr uint32_t kBarOff = kOutOff + OUT;
-    // misc: TMEM holder, abort flag, then 8 epilogue flags per epilogue group (up to two)
+    // misc: TMEM holder, abort flag, then 8 epilogue flags per epilogue group (up to four)
     static constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * S + 5);
-    static constexpr uint32_t kSmemBytes = kMiscOff + 80 + 1024;
+    static constexpr uint32_t kSmemBytes = kMiscOff + 144 + 1024;
     static constexpr uint32_t kBufCols = MT * BN;
     static constexpr uint32_t kTmemCols = NB * kBufCols <= 32 ? 32 : (NB * kBufCols <= 64 ? 64 : (NB * kBufCols <= 128 ? 128 : (NB * kBufCols <= 256 ? 256 : 512)));
     static_assert(NB * kBufCols <= 512, "accumulators exceed TMEM");
@@ -56,7 +55,7 @@ struct PairGeo {
     static_assert(kSmemBytes <= kMaxDynSmem, "ring exceeds shared memory");
 
     static_assert(BN % 32 == 0 && BN <= 256, "pair token tile");
-    static_assert(BN / 2 <= kPairTokBoxRowsL, "token rows per CTA fit one large box");
+    static_assert(BN / 2 <= kPairTokBoxStep * kPairTokBoxes, "token rows per CTA fit the largest box");
 };
 
 struct PairRing {
@@ -224,11 +223,9 @@ __device__ __forceinline__ void decode_gate_up_pair(const GateUpArgs &a, int nrc
 template <int BN, int S, int MT, int NB, int NSL, int EW>
 __global__ void __launch_bounds__(64 + 32 * EW, 1)
     gate_up_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_wsh,
-                        const __grid_constant__ CUtensorMap tm_xp, const __grid_constant__ CUtensorMap tm_x,
-                        const __grid_constant__ CUtensorMap tm_xp_l, const __grid_constant__ CUtensorMap tm_x_l,
-                        const GateUpArgs a, const WaitCfg wc)
+                        const __grid_constant__ PairTokMaps tok, const GateUpArgs a, const WaitCfg wc)
 {
-    static_assert(EW == 4 || EW == 8, "one or two groups of four epilogue warps");
+    static_assert(EW % 4 == 0 && EW >= 4 && EW <= 16, "one to four groups of four epilogue warps");
     using G = PairGeo<BN, S, MT, NB, 0, NSL>;
     extern __shared__ uint8_t smem_raw[];
     PairRing r;
@@ -248,10 +245,10 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
         if (lane == 0) {
             tma_prefetch_map(&tm_w);
             tma_prefetch_map(&tm_wsh);
-            tma_prefetch_map(&tm_xp);
-            tma_prefetch_map(&tm_x);
-            tma_prefetch_map(&tm_xp_l);
-            tma_prefetch_map(&tm_x_l);
+            for (int i = 0; i < kPairTokBoxes; ++i) {
+                tma_prefetch_map(&tok.routed_b[i]);
+                tma_prefetch_map(&tok.shared_b[i]);
+            }
             int it = 0;
             bool stop = false;
             for (int tile = first; tile < tiles && !stop; tile += stride) {
@@ -259,11 +256,11 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
                 decode_gate_up_pair<MT>(a, nrc, tiles_r, tile, g, row0, ntok, fb);
                 const bool sh = g == a.E;
                 const int half = ((ntok + 15) & ~15) >> 1;  // token rows used from each CTA
-                // one token box per K slice: 64 rows, or 128 when the half is larger
-                const bool large = half > kTokBoxRows;
-                const uint32_t tok_bytes = (large ? kPairTokBoxRowsL : kTokBoxRows) * 128;
+                // one token box per K slice: the smallest box height covering the half
+                const int bi = (half + kPairTokBoxStep - 1) / kPairTokBoxStep - 1;
+                const uint32_t tok_bytes = (bi + 1) * kPairTokBoxStep * 128;
                 const CUtensorMap *mw = sh ? &tm_wsh : &tm_w;
-                const CUtensorMap *mb = large ? (sh ? &tm_x_l : &tm_xp_l) : (sh ? &tm_x : &tm_xp);
+                const CUtensorMap *mb = sh ? &tok.shared_b[bi] : &tok.routed_b[bi];
                 const int ge = sh ? 0 : g;
                 const int wt0 = (fb * 2 + static_cast<int>(r.rank)) * MT;
                 const int brow = row0 + static_cast<int>(r.rank) * half;
@@ -404,11 +401,9 @@ __device__ __forceinline__ void decode_down_pair(const DownArgs &a, int tile, in
 template <int BN, int S, int MT, int NB, int NOB, int NSL, int EW>
 __global__ void __launch_bounds__(64 + 32 * EW, 1)
     down_pair_kernel(const __grid_constant__ CUtensorMap tm_wd, const __grid_constant__ CUtensorMap tm_wdsh,
-                     const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_hsh,
-                     const __grid_constant__ CUtensorMap tm_h_l, const __grid_constant__ CUtensorMap tm_hsh_l,
-                     const DownArgs a, const WaitCfg wc)
+                     const __grid_constant__ PairTokMaps tok, const DownArgs a, const WaitCfg wc)
 {
-    static_assert(EW == 4 || EW == 8, "one or two groups of four epilogue warps");
+    static_assert(EW % 4 == 0 && EW >= 4 && EW <= 16, "one to four groups of four epilogue warps");
     constexpr int kGroups = EW / 4;
     using G = PairGeo<BN, S, MT, NB, kGroups * NOB * kOutTok * MT * 512, NSL>;
     extern __shared__ uint8_t smem_raw[];
@@ -427,10 +422,10 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
         if (lane == 0) {
             tma_prefetch_map(&tm_wd);
             tma_prefetch_map(&tm_wdsh);
-            tma_prefetch_map(&tm_h);
-            tma_prefetch_map(&tm_hsh);
-            tma_prefetch_map(&tm_h_l);
-            tma_prefetch_map(&tm_hsh_l);
+            for (int i = 0; i < kPairTokBoxes; ++i) {
+                tma_prefetch_map(&tok.routed_b[i]);
+                tma_prefetch_map(&tok.shared_b[i]);
+            }
             int it = 0;
             bool stop = false;
             for (int tile = first; tile < tiles && !stop; tile += stride) {
@@ -439,10 +434,10 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
                 const bool sh = g == a.E;
                 const int nkb = (sh ? a.Is : a.I) / (kBK * NSL);
                 const int half = ((ntok + 15) & ~15) >> 1;
-                const bool large = half > kTokBoxRows;
-                const uint32_t tok_bytes = (large ? kPairTokBoxRowsL : kTokBoxRows) * 128;
+                const int bi = (half + kPairTokBoxStep - 1) / kPairTokBoxStep - 1;
+                const uint32_t tok_bytes = (bi + 1) * kPairTokBoxStep * 128;
                 const CUtensorMap *mw = sh ? &tm_wdsh : &tm_wd;
-                const CUtensorMap *mb = large ? (sh ? &tm_hsh_l : &tm_h_l) : (sh ? &tm_hsh : &tm_h);
+                const CUtensorMap *mb = sh ? &tok.shared_b[bi] : &tok.routed_b[bi];
                 const int wrow = (sh ? 0 : g * a.H) + (fb * 2 + static_cast<int>(r.rank)) * MT * 128;
                 const int brow = row0 + static_cast<int>(r.rank) * half;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
@@ -509,6 +504,16 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
     pair_teardown<G>(tmem);
 }
 
+PairTokMaps pair_maps(const TokMaps &t)
+{
+    PairTokMaps p;
+    for (int i = 0; i < kPairTokBoxes; ++i) {
+        p.routed_b[i] = t.routed_b[i];
+        p.shared_b[i] = t.shared_b[i];
+    }
+    return p;
+}
+
 template <class Kernel, class... Args>
 cudaError_t launch_pairs(Kernel kernel, int smem, int grid, int threads, cudaStream_t stream, Args... args)
 {
@@ -557,7 +562,7 @@ cudaError_t launch_gate_up_pair(const CUtensorMap &tm_w, const CUtensorMap &tm_w
     return launch_pairs(gate_up_pair_kernel<kPairCapGateUp, kGateUpStages, kPairMtGateUp, kGateUpBufs, kGateUpSlices,
                                             kGateUpEpiWarps>,
                         static_cast<int>(GateUpPair::kSmemBytes), grid, 64 + 32 * kGateUpEpiWarps, stream, tm_w,
-                        tm_wsh, tok.routed, tok.shared, tok.routed_l, tok.shared_l, a, wc);
+                        tm_wsh, pair_maps(tok), a, wc);
 }
 
 cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const TokMaps &tok,
@@ -565,8 +570,8 @@ cudaError_t launch_down_pair(const CUtensorMap &tm_wd, const CUtensorMap &tm_wds
 {
     return launch_pairs(
         down_pair_kernel<kPairCapDown, kDownStages, kPairMtDown, 2, kDownOutBufs, kDownSlices, kDownEpiWarps>,
-        static_cast<int>(DownPair::kSmemBytes), grid, 64 + 32 * kDownEpiWarps, stream, tm_wd, tm_wdsh, tok.routed,
-        tok.shared, tok.routed_l, tok.shared_l, a, wc);
+        static_cast<int>(DownPair::kSmemBytes), grid, 64 + 32 * kDownEpiWarps, stream, tm_wd, tm_wdsh, pair_maps(tok),
+        a, wc);
 }
 
 }  // namespace moe

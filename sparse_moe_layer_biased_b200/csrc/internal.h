@@ -69,19 +69,24 @@ cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t 
 // single CTAs take two weight tiles per stage (I, Is multiples of 128, H of 256), else one
 // weight tile and 256-row chunks.
 constexpr int kPairCapGateUp = 256, kPairMtGateUp = 1, kPairCapDown = 256, kPairMtDown = 1;
-// Token rows per TMA box on CTA pairs: the token tensor maps of the pair kernels are encoded
-// with 64-row boxes, and a second set with 128-row boxes; a tile whose CTA half holds up to
-// 64 rows loads one 64-row box per K slice, a larger one one 128-row box. 16-row boxes (at
-// most 15 unused rows per K slice) measured 20-30% slower on gate_up: the single producer
-// thread then issues up to 18 TMA copies per stage and becomes the bound.
-constexpr int kPairTokBoxRows = 64;
-constexpr int kPairTokBoxRowsL = 128;
+// Token rows per TMA box on CTA pairs: the pair kernels get token tensor maps with boxes of
+// 32, 64, 96 and 128 rows, and a tile loads one box per K slice, the smallest that covers
+// the rows of its CTA half (at most 31 unused rows). Several smaller boxes per slice (16-row
+// boxes: up to 18 TMA copies per stage) measured 20-30% slower on gate_up: the single
+// producer thread became the bound.
+constexpr int kPairTokBoxStep = 32;
+constexpr int kPairTokBoxes = 4;  // box heights kPairTokBoxStep * (i + 1)
 
 // Token-row tensor maps of one grouped GEMM: routed rows (x_perm or h) and shared rows (x or
-// h_sh), boxes of the chunk cap rows on single CTAs or kPairTokBoxRows on pairs, and for the
-// pair kernels the same rows with kPairTokBoxRowsL-row boxes (routed_l, shared_l).
+// h_sh) with boxes of the chunk cap on single CTAs, and for the pair kernels the same rows
+// with boxes of kPairTokBoxStep * (i + 1) rows (routed_b[i], shared_b[i]).
 struct TokMaps {
-    CUtensorMap routed, shared, routed_l, shared_l;
+    CUtensorMap routed, shared;
+    CUtensorMap routed_b[kPairTokBoxes], shared_b[kPairTokBoxes];
+};
+// The pair kernels take their token maps by value in one parameter block.
+struct PairTokMaps {
+    CUtensorMap routed_b[kPairTokBoxes], shared_b[kPairTokBoxes];
 };
 struct GemmConfig {
     int cap;

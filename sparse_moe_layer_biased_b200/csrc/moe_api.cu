@@ -238,6 +238,20 @@ WsLayout ws_layout(const moe_layer_desc &d)
     return L;
 }
 
+// Token-row maps of the pair kernels: routed rows [rows_r, cols] and shared rows [rows_s,
+// cols_s] (cols_s = cols unless given), boxes of 32, 64, 96 and 128 rows.
+bool pair_token_maps(moe::TokMaps *t, const void *routed, const void *shared, int64_t cols, int64_t rows_r,
+                     int64_t rows_s, int64_t cols_s = 0)
+{
+    for (int i = 0; i < moe::kPairTokBoxes; ++i) {
+        const uint32_t b = static_cast<uint32_t>(moe::kPairTokBoxStep * (i + 1));
+        if (!map_rows(&t->routed_b[i], routed, cols, rows_r, b) ||
+            !map_rows(&t->shared_b[i], shared, cols_s ? cols_s : cols, rows_s, b))
+            return false;
+    }
+    return true;
+}
+
 template <typename P>
 P *at(void *ws, size_t off)
 {
@@ -304,8 +318,7 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     // One TMA box per weight operand and pipeline stage: all weight tiles of a stage (64 * mt
     // gate/up feature pairs, or 128 * mt_d down rows). Token rows come in one box of the
     // chunk cap on single CTAs, in one 64- or 128-row box per K slice on CTA pairs.
-    const uint32_t brows = static_cast<uint32_t>(cfg.pair ? moe::kPairTokBoxRows : cfg.cap);
-    const uint32_t brows_l = static_cast<uint32_t>(moe::kPairTokBoxRowsL);
+    const uint32_t brows = static_cast<uint32_t>(cfg.cap);
     const uint32_t feats = static_cast<uint32_t>(64 * cfg.mt);
     const uint32_t drows = static_cast<uint32_t>(128 * cfg.mt_d);
     CUtensorMap tm_w, tm_wsh, tm_wd, tm_wdsh;
@@ -317,9 +330,9 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
               (fp8 ? map_rows_u8(&tm_wd, W.d, d.I, EH, drows, inner8) : map_rows(&tm_wd, W.d, d.I, EH, drows)) &&
               map_gate_up(&tm_wsh, W.sh_gu, d.H, d.Is, 1, feats) && map_rows(&tm_wdsh, W.sh_d, d.Is, d.H, drows) &&
               map_rows(&tok_gu.routed, x_perm, d.H, Tk, brows) && map_rows(&tok_gu.shared, x, d.H, d.T, brows) &&
-              map_rows(&tok_gu.routed_l, x_perm, d.H, Tk, brows_l) && map_rows(&tok_gu.shared_l, x, d.H, d.T, brows_l) &&
-              map_rows(&tok_d.routed, h, d.I, Tk, brows) && map_rows(&tok_d.shared, h_sh, d.Is, d.T, brows) &&
-              map_rows(&tok_d.routed_l, h, d.I, Tk, brows_l) && map_rows(&tok_d.shared_l, h_sh, d.Is, d.T, brows_l);
+              map_rows(&tok_d.routed, h, d.I, Tk, brows) && map_rows(&tok_d.shared, h_sh, d.Is, d.T, brows);
+    if (ok && cfg.pair)
+        ok = pair_token_maps(&tok_gu, x_perm, x, d.H, Tk, d.T) && pair_token_maps(&tok_d, h, h_sh, d.I, Tk, d.T, d.Is);
     if (!ok)
         return MOE_ERR_CUDA;
 
@@ -340,16 +353,11 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
             return MOE_ERR_WORKSPACE;
         chunks_s = at<int4>(ws, L.chunks_d);
         chunks_sd = chunks_s + n_gu;
-        const uint32_t b = moe::kPairTokBoxRows;
+        // the shared expert runs as the only group: its rows are the "shared" maps
         if (!(map_gate_up(&tm_wsh2, W.sh_gu, d.H, d.Is, 1, static_cast<uint32_t>(64 * cfg_sh.mt)) &&
               map_rows(&tm_wdsh2, W.sh_d, d.Is, d.H, static_cast<uint32_t>(128 * cfg_sh.mt_d)) &&
-              map_rows(&tok_gu2.routed, x, d.H, d.T, b) && map_rows(&tok_gu2.routed_l, x, d.H, d.T, brows_l) &&
-              map_rows(&tok_d2.routed, h_sh, d.Is, d.T, b) && map_rows(&tok_d2.routed_l, h_sh, d.Is, d.T, brows_l)))
+              pair_token_maps(&tok_gu2, x, x, d.H, d.T, d.T) && pair_token_maps(&tok_d2, h_sh, h_sh, d.Is, d.T, d.T)))
             return MOE_ERR_CUDA;
-        tok_gu2.shared = tok_gu2.routed;
-        tok_gu2.shared_l = tok_gu2.routed_l;
-        tok_d2.shared = tok_d2.routed;
-        tok_d2.shared_l = tok_d2.routed_l;
     }
 
     if (!stage_mark(2, s))

@@ -236,6 +236,28 @@ __device__ __forceinline__ void tma_load_4d_pair(void *dst, const CUtensorMap *m
         : "memory");
 }
 
+// The same pair loads with an L2 eviction-priority policy (from l2_policy_evict_first /
+// l2_policy_evict_last) for the loaded lines.
+__device__ __forceinline__ void tma_load_2d_pair_hint(void *dst, const CUtensorMap *m, uint32_t bar_cluster, int32_t c0,
+                                                      int32_t c1, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d_pair_hint(void *dst, const CUtensorMap *m, uint32_t bar_cluster, int32_t c0,
+                                                      int32_t c1, int32_t c2, int32_t c3, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+        : "memory");
+}
+
 // TMEM allocation shared by the pair: one warp of each CTA issues it (same warp, same
 // holder offset); both CTAs receive the same address.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *holder, uint32_t ncols)
@@ -468,6 +490,15 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last()
 {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// L2 eviction-priority policy for the whole access: lines are evicted first (streamed data
+// read once).
+__device__ __forceinline__ uint64_t l2_policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
 
