@@ -36,7 +36,9 @@ constexpr uint32_t kATileBytes = 128 * 128;  // 128 weight rows x 64 bf16
 // mainloop; 1: larger tiles, the MMA waits for the epilogue between tiles).
 // OUT = bytes of output staging after the ring (the down epilogue's bulk-reduction buffers).
 // NSL = 64-wide K slices per stage, each laid out as [MT weight tiles][token rows]: more MMAs
-// per barrier wait and commit of the single MMA-issuing thread, fewer stages.
+// per barrier wait of the single MMA-issuing thread, fewer stages. Each slice has its own
+// empty barrier: the MMA thread commits after each slice's MMAs, so the producer refills
+// the first slice of a stage while the MMAs of the second are still running.
 template <int BN, int S, int MT, int NB, int OUT = 0, int NSL = 1>
 struct PairGeo {
     static constexpr uint32_t kABytes = MT * kATileBytes;
@@ -45,8 +47,10 @@ struct PairGeo {
     static constexpr uint32_t kStageBytes = NSL * kSliceBytes;
     static constexpr uint32_t kOutOff = S * kStageBytes;
     static constexpr uint32_t kBarOff = kOutOff + OUT;
+    // barriers: S full, S * NSL empty, 2 accumulator-full, 2 accumulator-empty, drain;
     // misc: TMEM holder, abort flag, then 8 epilogue flags per epilogue group (up to four)
-    static constexpr uint32_t kMiscOff = kBarOff + 8 * (2 * S + 5);
+    static constexpr int kNsl = NSL;
+    static constexpr uint32_t kMiscOff = kBarOff + 8 * (S + S * NSL + 5);
     static constexpr uint32_t kSmemBytes = kMiscOff + 144 + 1024;
     static constexpr uint32_t kBufCols = MT * BN;
     static constexpr uint32_t kTmemCols = NB * kBufCols <= 32 ? 32 : (NB * kBufCols <= 64 ? 64 : (NB * kBufCols <= 128 ? 128 : (NB * kBufCols <= 256 ? 256 : 512)));
@@ -76,7 +80,7 @@ __device__ __forceinline__ uint8_t *pair_setup(uint8_t *smem_raw, PairRing &r, i
     uint8_t *smem = smem_raw + pad;
     r.full = reinterpret_cast<uint64_t *>(smem + G::kBarOff);
     r.empty = r.full + S;
-    r.accf = r.empty + S;
+    r.accf = r.empty + S * G::kNsl;
     r.acce = r.accf + 2;
     r.drain = r.acce + 2;
     r.holder = reinterpret_cast<uint32_t *>(smem + G::kMiscOff);
@@ -86,10 +90,10 @@ __device__ __forceinline__ uint8_t *pair_setup(uint8_t *smem_raw, PairRing &r, i
     r.acce_leader = dsmem_addr(smem_u32(r.acce), 0);
     const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
+        for (int s = 0; s < S; ++s)
             mbar_init(&r.full[s], 1);
+        for (int s = 0; s < S * G::kNsl; ++s)
             mbar_init(&r.empty[s], 1);
-        }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&r.accf[b], 1);
             mbar_init(&r.acce[b], 2 * epi_warps);  // every epilogue warp of both CTAs
@@ -164,8 +168,8 @@ __device__ __forceinline__ bool pair_mma_tile(const PairRing &r, uint8_t *smem, 
                     umma_bf16_pair(d + m * BN, ad + 2 * kk, bd + 2 * kk, idesc, (kb | c | kk) != 0);
                 }
             }
+            umma_commit_pair_mc(&r.empty[s * NSL + c], 0x3);  // this slice's buffers are free
         }
-        umma_commit_pair_mc(&r.empty[s], 0x3);
     }
     return true;
 }
@@ -266,21 +270,30 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
                 const int brow = row0 + static_cast<int>(r.rank) * half;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % S;
-                    if (!mbar_wait(&r.empty[s], ((it / S) & 1) ^ 1, wc, r.abort_flag)) {
+                    const uint32_t par = ((it / S) & 1) ^ 1;
+                    if (!mbar_wait(&r.empty[s * NSL], par, wc, r.abort_flag)) {
                         stop = true;
                         break;
                     }
                     if (r.rank == 0)
                         mbar_arrive_expect_tx(&r.full[s], 2 * NSL * (G::kABytes + tok_bytes));
                     const uint32_t bar = r.full_leader + 8 * s;
-                    // per K slice: one box with this CTA's MT weight tiles, then one box of
-                    // token rows covering its half of the chunk (rows past the half are
-                    // loaded and ignored)
+                    // per K slice, once its buffers are free: one box with this CTA's MT
+                    // weight tiles, then one box of token rows covering its half of the chunk
+                    // (rows past the half are loaded and ignored)
                     for (int c = 0; c < NSL; ++c) {
+                        if (c > 0 && !mbar_wait(&r.empty[s * NSL + c], par, wc, r.abort_flag)) {
+                            stop = true;
+                            break;
+                        }
                         uint8_t *A = smem + s * G::kStageBytes + c * G::kSliceBytes;
                         const int k0 = (kb * NSL + c) * kBK;
                         tma_load_4d_pair(A, mw, bar, k0, 0, wt0 * 64, ge);
                         tma_load_2d_pair(A + G::kABytes, mb, bar, k0, brow);
+                    }
+                    if (stop) {
+                        ++it;  // a partly issued stage: the drain also waits for its copies
+                        break;
                     }
                 }
             }
@@ -442,7 +455,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
                 const int brow = row0 + static_cast<int>(r.rank) * half;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % S;
-                    if (!mbar_wait(&r.empty[s], ((it / S) & 1) ^ 1, wc, r.abort_flag)) {
+                    const uint32_t par = ((it / S) & 1) ^ 1;
+                    if (!mbar_wait(&r.empty[s * NSL], par, wc, r.abort_flag)) {
                         stop = true;
                         break;
                     }
@@ -450,10 +464,18 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
                         mbar_arrive_expect_tx(&r.full[s], 2 * NSL * (G::kABytes + tok_bytes));
                     const uint32_t bar = r.full_leader + 8 * s;
                     for (int c = 0; c < NSL; ++c) {
+                        if (c > 0 && !mbar_wait(&r.empty[s * NSL + c], par, wc, r.abort_flag)) {
+                            stop = true;
+                            break;
+                        }
                         uint8_t *A = smem + s * G::kStageBytes + c * G::kSliceBytes;
                         const int k0 = (kb * NSL + c) * kBK;
                         tma_load_2d_pair(A, mw, bar, k0, wrow);
                         tma_load_2d_pair(A + G::kABytes, mb, bar, k0, brow);
+                    }
+                    if (stop) {
+                        ++it;  // a partly issued stage: the drain also waits for its copies
+                        break;
                     }
                 }
             }
@@ -542,15 +564,18 @@ cudaError_t launch_pairs(Kernel kernel, int smem, int grid, int threads, cudaStr
 // tile per CTA and K slice, two 64-wide K slices per stage (8 pair MMAs per barrier test
 // and commit of the MMA thread), three 64 KB stages. Most experts of a prefill batch then
 // need one pass over their weights. down: the same 256-row chunks x 256 output features, one
-// weight tile per CTA and K slice, two K slices per stage (three 64 KB stages), eight
-// epilogue warps in two groups, each with two 8 KB output staging buffers for the bulk
-// reductions (measured against 128-row chunks with two weight tiles per CTA and four
-// epilogue warps: 5% faster on the Step-5 prefill down GEMM, equal on the other shapes; with
-// four epilogue warps the 256-row chunks were 20-35% slower: the reductions of a 256-column
-// tile then outlast its mainloop). Both keep two TMEM accumulators.
+// weight tile per CTA and K slice, two K slices per stage (three 64 KB stages), sixteen
+// epilogue warps in four groups, each with one 8 KB output staging buffer for the bulk
+// reductions. The down epilogue is bound by the reductions it keeps in flight: a 256-column
+// tile's K loop (I = 1536) is short against its 128 KB of fp32 output per CTA. Measured on
+// the Step-5 shapes against 128-row chunks with two weight tiles per CTA and four epilogue
+// warps: 256-row chunks with 4 warps 20-35% slower, with 8 warps (two buffers each) 5%
+// faster, with 16 warps 10-14% faster; 12 or 16 warps adding straight from registers
+// (coalesced fp32 reductions, no staging) 5-11%; 24 warps on a 5 x 32 KB ring slower. Both
+// keep two TMEM accumulators.
 constexpr int kGateUpStages = 3, kGateUpSlices = 2, kGateUpBufs = 2, kGateUpEpiWarps = 4;
 using GateUpPair = PairGeo<kPairCapGateUp, kGateUpStages, kPairMtGateUp, kGateUpBufs, 0, kGateUpSlices>;
-constexpr int kDownStages = 3, kDownSlices = 2, kDownOutBufs = 2, kDownEpiWarps = 8;
+constexpr int kDownStages = 3, kDownSlices = 2, kDownOutBufs = 1, kDownEpiWarps = 16;
 using DownPair = PairGeo<kPairCapDown, kDownStages, kPairMtDown, 2,
                          (kDownEpiWarps / 4) * kDownOutBufs * kOutTok * kPairMtDown * 512, kDownSlices>;
 
