@@ -266,13 +266,16 @@ def run_reference(args, shape):
     print(json.dumps(line), flush=True)
 
 
-# DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu capture
-# (profiles/dram_gate_up_down_step35_prefill.md). A figure holds only for the kernel sources
-# it was taken from: the lookup returns None once any file under csrc/ changes.
+# DRAM traffic (read + write) of one launch of the dominant kernel, as a ratio to the launch's
+# algorithmic bytes, from one ncu capture of a reduced case of the same shape per expert
+# (profiles/dram_gate_up_down_step5_skewed_T2048_E44.md: T=2048, E=44, the skewed Step-5
+# layer): the full launch's traffic is that ratio times its own algorithmic bytes. A figure
+# holds only for the kernel sources it was taken from: the lookup returns None once the code
+# of any file under csrc/ changes.
 PROFILED_TRAFFIC = {
-    ("step35_prefill", "bf16"): {"bytes": 5612357632 + 86688000,
-                                 "csrc_sha256": "d6cb41040b51603f6888922b17e4c7241d03419a061e0a4a38b91331f6d9907f",
-                                 "source": "profiles/dram_gate_up_down_step35_prefill.md"},
+    ("step5_skewed", "bf16"): {"ratio": (1454216448 + 51585536) / 1205862400,
+                               "csrc_sha256": "15dd272b4b2f1d6627764df2eefab03b2fbf8ca60330c169e378abb3d500b721",
+                               "source": "profiles/dram_gate_up_down_step5_skewed_T2048_E44.md"},
 }
 
 
@@ -312,11 +315,13 @@ def csrc_digest() -> str:
     return h.hexdigest()
 
 
-def profiled_traffic(shape_name: str, weights: str):
+def profiled_traffic(shape_name: str, weights: str, algorithmic_bytes: float):
+    """Per-launch DRAM traffic of gate_up for this workload (None without a capture of the
+    current sources)."""
     e = PROFILED_TRAFFIC.get((shape_name, weights))
     if e is None or e["csrc_sha256"] != csrc_digest():
         return None
-    return e["bytes"]
+    return e["ratio"] * algorithmic_bytes
 
 
 def kernels_per_step(shape, fp8=False, deterministic=False, router=True):
@@ -544,8 +549,8 @@ def run_b200(args, shape):
                "h2d_bytes_per_step": shape.T * shape.H * 2, "d2h_bytes_per_step": shape.T * shape.H * 4}
 
     peaks, peak_kind = load_peaks()
-    roofline = gate_up_roofline(shape, counts, stage_ms["gate_up"], peaks, peak_kind, fp8,
-                                profiled_traffic(shape.name, args.weights))
+    roofline = gate_up_roofline(shape, counts, stage_ms["gate_up"], peaks, peak_kind, fp8)
+    roofline["traffic"] = profiled_traffic(shape.name, args.weights, roofline["algorithmic_bytes"])
     flops = shape.flops_per_token * shape.T
     step_ms = ms / args.steps
     value = job_tokens_per_s(world, shape.T, args.steps, ms)
