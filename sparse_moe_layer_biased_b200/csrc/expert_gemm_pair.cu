@@ -536,6 +536,9 @@ PairTokMaps pair_maps(const TokMaps &t)
     return p;
 }
 
+// Launches `grid` CTAs (rounded down to pairs) as clusters of 2, but no more pairs than can be
+// resident at once (cudaOccupancyMaxActiveClusters): the kernels are persistent, so a pair that
+// could only start after another one exits would run its whole tile share as a tail.
 template <class Kernel, class... Args>
 cudaError_t launch_pairs(Kernel kernel, int smem, int grid, int threads, cudaStream_t stream, Args... args)
 {
@@ -554,6 +557,14 @@ cudaError_t launch_pairs(Kernel kernel, int smem, int grid, int threads, cudaStr
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    int resident = 0;
+    err = cudaOccupancyMaxActiveClusters(&resident, kernel, &cfg);
+    if (err != cudaSuccess)
+        return err;
+    if (resident < 1)
+        return cudaErrorInvalidConfiguration;
+    if (2 * resident < static_cast<int>(cfg.gridDim.x))
+        cfg.gridDim.x = 2 * resident;
     err = cudaLaunchKernelEx(&cfg, kernel, args...);
     if (err != cudaSuccess)
         return err;
