@@ -249,7 +249,12 @@ __global__ void __launch_bounds__(256)
         d[i] = z;
 }
 
-// dWr[e][h] = Σ over group e's rows of dl_pad[row] * x_pad[row][h]; block (e, 512 columns).
+// dWr[e][h] = Σ over group e's rows of dl_pad[row] * x_pad[row][h]. Block (e, 512 columns,
+// split z of kDwrSplit) sums rows r0 + z, r0 + z + kDwrSplit, ... (four rows of loads in flight)
+// and adds its partial sums into dWr, which the launch zeroes first: a hot expert's thousands
+// of rows no longer run as one block's serial loop.
+constexpr int kDwrSplit = 8;
+
 __global__ void __launch_bounds__(256)
     bwd_dwr_kernel(const uint16_t *__restrict__ x_pad, const float *__restrict__ dl_pad,
                    const int32_t *__restrict__ poff, const int32_t *__restrict__ counts, int E, int H,
@@ -257,17 +262,35 @@ __global__ void __launch_bounds__(256)
 {
     const int e = blockIdx.x;
     const int h = blockIdx.y * 512 + threadIdx.x * 2;
-    if (h >= H)
-        return;
     const int64_t r0 = poff[e], r1 = r0 + counts[e];
+    if (h >= H || r0 + blockIdx.z >= r1)
+        return;
     float a0 = 0.0f, a1 = 0.0f;
-    for (int64_t r = r0; r < r1; ++r) {
+    const int64_t step = kDwrSplit;
+    int64_t r = r0 + blockIdx.z;
+    for (; r + 3 * step < r1; r += 4 * step) {
+        float d[4];
+        float2 xf[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            d[u] = dl_pad[r + u * step];
+            xf[u] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(x_pad + (r + u * step) * H + h));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            a0 = fmaf(d[u], xf[u].x, a0);
+            a1 = fmaf(d[u], xf[u].y, a1);
+        }
+    }
+    for (; r < r1; r += step) {
         const float d = dl_pad[r];
         const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(x_pad + r * H + h));
         a0 = fmaf(d, xf.x, a0);
         a1 = fmaf(d, xf.y, a1);
     }
-    *reinterpret_cast<float2 *>(dWr + static_cast<int64_t>(e) * H + h) = make_float2(a0, a1);
+    float *out = dWr + static_cast<int64_t>(e) * H + h;
+    atomicAdd(out, a0);
+    atomicAdd(out + 1, a1);
 }
 
 }  // namespace
@@ -311,24 +334,31 @@ cudaError_t launch_bwd_zero_untouched(const int32_t *counts, int E, int H, int I
 cudaError_t launch_bwd_dwr(const uint16_t *x_pad, const float *dl_pad, const int32_t *poff, const int32_t *counts,
                            int E, int H, float *dWr, cudaStream_t stream)
 {
-    bwd_dwr_kernel<<<dim3(E, (H + 511) / 512), 256, 0, stream>>>(x_pad, dl_pad, poff, counts, E, H, dWr);
+    cudaError_t err = cudaMemsetAsync(dWr, 0, static_cast<size_t>(E) * H * 4, stream);
+    if (err != cudaSuccess)
+        return err;
+    bwd_dwr_kernel<<<dim3(E, (H + 511) / 512, kDwrSplit), 256, 0, stream>>>(x_pad, dl_pad, poff, counts, E, H, dWr);
     return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------------------------
 // Grouped GEMMs of the backward pass. One persistent kernel per mode, one CTA per SM, 192
 // threads (warp 0 TMA producer, warp 1 MMA issuer and TMEM owner, warps 2..5 epilogue).
-// A tile is 128 rows of the output's M side x up to 128 columns (N); a pipeline stage holds
-// one 64-wide K slice of A (16 KB) and B (16 KB). A and B are K-major (128-byte rows of K)
-// or MN-major (two 8 KB chunks of 64 MN elements x 64 K rows), as the mode's global layout
-// gives them; two TMEM accumulators of 128 columns let the epilogue of one tile overlap the
-// next tile's mainloop.
+// A tile is 128 rows of the output's M side x N columns: up to kBwdCap = 256 token rows in the
+// row-streaming modes (GU, DH, DX), kBwdBN = 128 output columns in the weight-gradient modes
+// (WD, WGU). A pipeline stage holds one 64-wide K slice of A (16 KB) and B (32 KB of token rows,
+// or 16 KB MN-major); a chunk of at most 128 rows loads a 128-row token box. A and B are
+// K-major (128-byte rows of K) or MN-major (two 8 KB chunks of 64 MN elements x 64 K rows), as
+// the mode's global layout gives them; two TMEM accumulators of 256 columns let the epilogue
+// of one tile overlap the next tile's mainloop. 256-row tiles halve the bytes each MMA column
+// needs from L2 against 128-row ones (each weight tile streams once per 256 rows).
 namespace {
 
 constexpr int kBwdThreads = 192;
-constexpr int kBwdStages = 6;
-constexpr int kBwdBN = 128;
-constexpr uint32_t kBwdTile = 16384;  // one operand per stage
+constexpr int kBwdStages = 6;  // stages of 32 KB (the ring region's size in those units)
+constexpr int kBwdBN = 128;    // output columns of a weight-gradient tile
+constexpr int kBwdAcc = kBwdCap;  // TMEM columns of one accumulator buffer
+constexpr uint32_t kBwdTile = 16384;  // A operand (or MN-major B) per K slice
 constexpr uint32_t kBwdStage = 2 * kBwdTile;
 constexpr uint32_t kBwdBarOff = kBwdStages * kBwdStage;
 constexpr uint32_t kBwdMiscOff = kBwdBarOff + 8 * (2 * kBwdStages + 5);
@@ -438,7 +468,7 @@ __device__ __forceinline__ void bwd_load(const BwdArgs &a, const CUtensorMap *ma
         tma_load_4d(A, ma, bar, k0, 0, t.mb * 64, t.sh ? 0 : t.g);
         tma_load_2d(B, mb, bar, k0, t.row0);
     } else if (MODE == kBwdDH) {
-        const int wrow = (t.sh ? 0 : t.g * a.H) + k0;
+        const int wrow = (t.sh ? 0 : t.g * a.H) + k0;  // B: mb is the map of the tile's box height
         tma_load_2d(A, ma, bar, t.mb * 128, wrow);
         tma_load_2d(A + 8192, ma, bar, t.mb * 128 + 64, wrow);
         tma_load_2d(B, mb, bar, k0, t.row0);
@@ -617,9 +647,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 {
     constexpr bool kAmn = MODE != kBwdGU;
     constexpr bool kBmn = MODE == kBwdWD || MODE == kBwdWGU;
-    constexpr int S = kBwdStages / NSL;
-    constexpr uint32_t kStage = NSL * kBwdStage;
-    static_assert(S * kStage <= kBwdBarOff, "ring exceeds its region");
+    // K slice: A, then B (MN-major 16 KB, or kBwdCap token rows of 128 bytes)
+    constexpr uint32_t kSlice = kBwdTile + (kBmn ? kBwdTile : static_cast<uint32_t>(kBwdCap) * 128);
+    constexpr uint32_t kStage = NSL * kSlice;
+    constexpr int S = static_cast<int>(kBwdBarOff / kStage);
+    static_assert(S >= 2 && S <= kBwdStages, "ring depth");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *smem = smem_raw + pad;
@@ -646,7 +678,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(holder, 2 * kBwdBN);
+        tmem_alloc(holder, 2 * kBwdAcc);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -665,17 +697,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bool stop = false;
             for (int tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x) {
                 const BTile t = bwd_tile<MODE>(a, tile);
+                // row-streaming modes: a chunk of at most 128 rows takes the 128-row token box
+                const bool small = !kBmn && t.ntok <= 128;
+                const CUtensorMap *mb = small ? (t.sh ? &o_s : &o_r) : (t.sh ? &b_s : &b_r);
+                const uint32_t bbytes = kBmn ? kBwdTile : (small ? 128u : static_cast<uint32_t>(kBwdCap)) * 128u;
                 for (int k0 = 0; k0 < t.K; k0 += 64 * NSL, ++it) {
                     const int s = it % S;
                     if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, wc, abort_flag)) {
                         stop = true;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], kStage);
+                    mbar_arrive_expect_tx(&full[s], NSL * (kBwdTile + bbytes));
                     for (int c = 0; c < NSL; ++c) {
-                        uint8_t *A = smem + s * kStage + c * kBwdStage;
-                        bwd_load<MODE>(a, t.sh ? &a_s : &a_r, t.sh ? &b_s : &b_r, A, A + kBwdTile, &full[s], t,
-                                       k0 + 64 * c);
+                        uint8_t *A = smem + s * kStage + c * kSlice;
+                        bwd_load<MODE>(a, t.sh ? &a_s : &a_r, mb, A, A + kBwdTile, &full[s], t, k0 + 64 * c);
                     }
                 }
             }
@@ -692,7 +727,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!mbar_wait(&acce[buf], ((tc >> 1) & 1) ^ 1, wc, abort_flag))
                     break;
                 tc_fence_after();
-                const uint32_t d = tmem + buf * kBwdBN;
+                const uint32_t d = tmem + buf * kBwdAcc;
                 const uint32_t idesc = idesc_bf16_f32(128, (t.ntok + 15) & ~15) | (kAmn ? 1u << 15 : 0u) |
                                        (kBmn ? 1u << 16 : 0u);
                 for (int k0 = 0; k0 < t.K; k0 += 64 * NSL, ++it) {
@@ -704,7 +739,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < NSL; ++c) {
-                        const uint32_t sa = smem_u32(smem + s * kStage + c * kBwdStage);
+                        const uint32_t sa = smem_u32(smem + s * kStage + c * kSlice);
                         const uint32_t sb = sa + kBwdTile;
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks) {
@@ -732,7 +767,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!warp_wait(&accf[buf], (tc >> 1) & 1, wc, abort_flag))
                 break;
             tc_fence_after();
-            bwd_epilogue<MODE>(a, tmem + buf * kBwdBN, t, q, lane,
+            bwd_epilogue<MODE>(a, tmem + buf * kBwdAcc, t, q, lane,
                                reinterpret_cast<float *>(smem + kBwdEpiOff + q * kBwdEpiWarp), t.sh ? &o_s : &o_r);
             tc_fence_before();
             __syncwarp();
@@ -746,7 +781,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 2 * kBwdBN);
+        tmem_dealloc(tmem, 2 * kBwdAcc);
     }
 }
 
@@ -769,18 +804,15 @@ cudaError_t launch_bwd_gemm(int mode, const CUtensorMap &a_r, const CUtensorMap 
                             const CUtensorMap &b_s, const CUtensorMap &o_r, const CUtensorMap &o_s, const BwdArgs &a,
                             const WaitCfg &wc, int grid, cudaStream_t stream)
 {
-    // weight-streaming modes take two K slices per stage when K (H for GU and DH, 2 I for
-    // DX) is a multiple of 128; the weight-gradient modes reduce over 64-row padded groups
-    const bool h2 = a.H % 128 == 0;
+    // row-streaming modes: one K slice per stage (48 KB stages, four deep); the
+    // weight-gradient modes reduce over 64-row padded groups (32 KB stages, six deep)
     switch (mode) {
     case kBwdGU:
-        return h2 ? launch_mode<kBwdGU, 2>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream)
-                  : launch_mode<kBwdGU, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
+        return launch_mode<kBwdGU, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
     case kBwdDH:
-        return h2 ? launch_mode<kBwdDH, 2>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream)
-                  : launch_mode<kBwdDH, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
+        return launch_mode<kBwdDH, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
     case kBwdDX:
-        return launch_mode<kBwdDX, 2>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
+        return launch_mode<kBwdDX, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
     case kBwdWD:
         return launch_mode<kBwdWD, 1>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc, grid, stream);
     case kBwdWGU:

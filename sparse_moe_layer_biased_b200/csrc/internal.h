@@ -183,7 +183,7 @@ cudaError_t launch_down_fp8(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh
 // x_pad / dy_pad, so the weight-gradient GEMMs reduce over whole 64-row K slices. chunks: tiles of <= kBwdCap valid rows (group, first
 // row, rows); wgroups: (group, first row, padded rows). hdr: [0] routed chunks, [1] all
 // chunks, [2] routed wgroups, [3] all wgroups.
-constexpr int kBwdCap = 128;
+constexpr int kBwdCap = 256;
 constexpr int kBwdPad = 64;
 struct BwdArgs {
     int T, H, E, k, I, Is;
@@ -208,9 +208,11 @@ enum BwdMode { kBwdGU = 0, kBwdDH = 1, kBwdDX = 2, kBwdWD = 3, kBwdWGU = 4 };
 //   DX : W_gate_up / Wsh_gate_up as (H, rows) MN-major, dgu_r, dgu_s (K-major)
 //   WD : dy_pad (H, rows) MN-major (both), hw_r / hw_s (I, rows) MN-major
 //   WGU: dgu_r / dgu_s (2I, rows) MN-major, x_pad (H, rows) MN-major (both)
-// and output maps (routed, shared) of the weight-gradient modes, fp32 32 x 32 boxes with
-// 128-byte swizzle: WD dW_down (I, E*H) / dWsh_down (Is, H), WGU dW_gate_up (H, E*2I) /
-// dWsh_gate_up (H, 2Is); the other modes ignore them.
+// and, last, two more maps (routed, shared): for the weight-gradient modes their fp32 outputs,
+// 32 x 32 boxes with 128-byte swizzle (WD dW_down (I, E*H) / dWsh_down (Is, H), WGU
+// dW_gate_up (H, E*2I) / dWsh_gate_up (H, 2Is)); for GU, DH and DX the same token rows as
+// their B maps with 128-row boxes (the B maps have kBwdCap-row boxes; a chunk of at most 128
+// rows loads the smaller box).
 cudaError_t launch_bwd_gemm(int mode, const CUtensorMap &a_r, const CUtensorMap &a_s, const CUtensorMap &b_r,
                             const CUtensorMap &b_s, const CUtensorMap &o_r, const CUtensorMap &o_s, const BwdArgs &a,
                             const WaitCfg &wc, int grid, cudaStream_t stream);

@@ -958,6 +958,7 @@ moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const u
     const int64_t E = d.E, H = d.H, I = d.I, Is = d.Is, P = L.P_max, Pr = L.P_r_max, Ps = L.P_s;
 
     // tensor maps (rows of the padded buffers are upper bounds; tiles only touch filled rows)
+    CUtensorMap gu_b2, dh_b2, dx_b2_r, dx_b2_s;  // the same token rows with 128-row boxes
     CUtensorMap gu_a_r, gu_a_s, gu_b, dh_a_r, dh_a_s, dh_b, dx_a_r, dx_a_s, dx_b_r, dx_b_s, wd_a, wd_b_r, wd_b_s,
         wg_a_r, wg_a_s, wg_b, wd_o_r, wd_o_s, wg_o_r, wg_o_s;
     const bool ok = map_gate_up(&gu_a_r, W_gate_up, H, I, E, 64) && map_gate_up(&gu_a_s, Wsh_gate_up, H, Is, 1, 64) &&
@@ -971,7 +972,9 @@ moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const u
                     map_rows(&wg_b, x_pad, H, P, 64) && map_rows_f32_store(&wd_o_r, dW_down, I, E * H) &&
                     map_rows_f32_store(&wd_o_s, dWsh_down, Is, H) &&
                     map_rows_f32_store(&wg_o_r, dW_gate_up, H, E * 2 * I) &&
-                    map_rows_f32_store(&wg_o_s, dWsh_gate_up, H, 2 * Is);
+                    map_rows_f32_store(&wg_o_s, dWsh_gate_up, H, 2 * Is) &&
+                    map_rows(&gu_b2, x_pad, H, P, 128) && map_rows(&dh_b2, dy_pad, H, P, 128) &&
+                    map_rows(&dx_b2_r, dgu_r, 2 * I, Pr, 128) && map_rows(&dx_b2_s, dgu_s, 2 * Is, Ps, 128);
     if (!ok)
         return MOE_ERR_CUDA;
     const moe::WaitCfg wc = wait_cfg(di);
@@ -989,14 +992,14 @@ moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const u
     if (e == cudaSuccess)
         e = cudaMemsetAsync(dw_pad, 0, static_cast<size_t>(P) * 4, s);
     if (e == cudaSuccess)
-        e = moe::launch_bwd_gemm(moe::kBwdGU, gu_a_r, gu_a_s, gu_b, gu_b, gu_b, gu_b, ba, wc, di.num_sms, s);
+        e = moe::launch_bwd_gemm(moe::kBwdGU, gu_a_r, gu_a_s, gu_b, gu_b, gu_b2, gu_b2, ba, wc, di.num_sms, s);
     if (e == cudaSuccess)
-        e = moe::launch_bwd_gemm(moe::kBwdDH, dh_a_r, dh_a_s, dh_b, dh_b, dh_b, dh_b, ba, wc, di.num_sms, s);
+        e = moe::launch_bwd_gemm(moe::kBwdDH, dh_a_r, dh_a_s, dh_b, dh_b, dh_b2, dh_b2, ba, wc, di.num_sms, s);
     if (e == cudaSuccess)
         e = moe::launch_bwd_router(x, Wr, topk_idx, slot_of, offsets, poff, dw_pad, d.T, d.k, d.E, d.H, d.scale,
                                    d.norm_expert_weight, dx, dl_pad, s);
     if (e == cudaSuccess)
-        e = moe::launch_bwd_gemm(moe::kBwdDX, dx_a_r, dx_a_s, dx_b_r, dx_b_s, dx_b_r, dx_b_s, ba, wc, di.num_sms, s);
+        e = moe::launch_bwd_gemm(moe::kBwdDX, dx_a_r, dx_a_s, dx_b_r, dx_b_s, dx_b2_r, dx_b2_s, ba, wc, di.num_sms, s);
     if (e == cudaSuccess)
         e = moe::launch_bwd_zero_untouched(counts, d.E, d.H, d.I, dW_gate_up, dW_down, s);
     if (e == cudaSuccess)

@@ -10,19 +10,22 @@ One forward on each rank (one process per GPU):
   1. moe_router and moe_permute over the global E experts: routed slots in global expert
      order, which is (owner rank, local expert) order;
   2. moe_ep_pack: the send rows x_send[slot] = x[token] and their routing weights;
-  3. dispatch: an all-to-all of the [R, Er] per-(owner, local expert) row counts, then of the
+  3. moe_shared_expert writes rows [T*k, T*k + T) of o_perm: it needs no routing, so it is
+     enqueued before the host waits for the counts below and keeps the GPU busy meanwhile;
+  4. dispatch: an all-to-all of the [R, Er] per-(owner, local expert) row counts, then of the
      rows and weights, which arrive source-major (source 0's rows for its local expert 0, 1,
      ..., then source 1's);
-  4. moe_ep_experts: this rank's experts on the received rows, one weighted fp32 output row
+  5. moe_ep_experts: this rank's experts on the received rows, one weighted fp32 output row
      per received row, in received order;
-  5. return: the reverse all-to-all puts every output row back at its slot, rows [0, T*k)
-     of o_perm; moe_shared_expert writes rows [T*k, T*k + T);
-  6. moe_combine: y[t] = sum over j of o_perm[slot_of[t, j]] + o_perm[T*k + t], in a fixed
+  6. return: the reverse all-to-all puts every output row back at its slot, rows [0, T*k)
+     of o_perm;
+  7. moe_combine: y[t] = sum over j of o_perm[slot_of[t, j]] + o_perm[T*k + t], in a fixed
      order, so the result does not depend on R.
 
 The all-to-alls are NCCL collectives issued through torch.distributed (plumbing); every
 arithmetic step runs in libmoe_b200.so. The counts are read on the host once per forward
-to size the row exchange. Only routed BF16 experts are supported here.
+to size the row exchange (torch.distributed's all-to-all takes host split sizes), after
+the shared expert has been enqueued. Only routed BF16 experts are supported here.
 """
 from __future__ import annotations
 
@@ -107,10 +110,12 @@ class EPMoeLayer:
         slot_of = torch.empty((T, k), dtype=torch.int32, device=dev)
         x_send = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
         w_send = torch.empty((T * k,), dtype=torch.float32, device=dev)
+        o_perm = torch.empty((T * k + T, H), dtype=torch.float32, device=dev)
         if T > 0:
             _abi.moe_router(d, x, W["Wr"], W["bias"], idx, w)
             _abi.moe_permute(d, idx, counts, offsets, perm_token, slot_of)
             _abi.moe_ep_pack(d, x, w, slot_of, x_send, w_send)
+            _abi.moe_shared_expert(d, x, W["Wsh_gate_up"], W["Wsh_down"], o_perm[T * k:], self.ws)
         else:
             counts.zero_()
         x_recv, w_recv, recv_ce, send_rows, recv_rows = dispatch(x_send, w_send, ep_counts(counts, self.R),
@@ -123,10 +128,8 @@ class EPMoeLayer:
         out_recv = torch.empty((n, H), dtype=torch.float32, device=dev)
         _abi.moe_ep_experts(dl, self.R, recv_ce, x_recv, w_recv, W["W_gate_up"], W["W_down"], out_recv,
                             self.ws_experts)
-        o_perm = torch.empty((T * k + T, H), dtype=torch.float32, device=dev)
         combine_back(out_recv, o_perm[: T * k], send_rows, recv_rows, self.group)
         y = torch.empty((T, H), dtype=torch.float32, device=dev)
         if T > 0:
-            _abi.moe_shared_expert(d, x, W["Wsh_gate_up"], W["Wsh_down"], o_perm[T * k:], self.ws)
             _abi.moe_combine(d, o_perm, slot_of, y)
         return (y, idx, w) if routing else y

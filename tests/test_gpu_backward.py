@@ -25,9 +25,15 @@ SHAPES = {
                        seed=71, weight_std=0.08),
     # more groups than tokens per group, experts without tokens (zeroed gradients), H = 3 x 128
     "sparse": LayerShape("bwd_sparse", T=40, H=384, E=24, k=2, I=128, Is=256, seed=72, weight_std=0.05),
-    # chunks above the 128-row cap and padding to 64 rows, no clip, no normalisation
+    # chunks of more than 128 rows (256-row token boxes) and padding to 64 rows, the shared group
+    # split in two chunks, no clip, no normalisation
     "big_groups": LayerShape("bwd_big", T=300, H=256, E=3, k=2, I=128, Is=128, scale=2.5,
                              norm_expert_weight=False, seed=73, weight_std=0.05),
+    # groups above the 256-row chunk cap (~400 rows per routed group, the shared group in three
+    # chunks); k = 2 of 3 experts, so the normalised weights depend on the logits (with k = 1
+    # they would be the constant scale and the router-weight gradient exactly zero)
+    "huge_groups": LayerShape("bwd_huge", T=600, H=256, E=3, k=2, I=128, Is=256, limit_routed=0.5, seed=74,
+                              weight_std=0.05),
     "tiny": WORKLOADS["tiny"],
 }
 

@@ -107,3 +107,17 @@ def test_backward_is_linear_in_dy_and_bias_free():
     b3 = oracle.backward(*args2, dy, **kw)
     for key in ("dx", "dWr", "dW_gate_up", "dW_down", "dWsh_gate_up", "dWsh_down"):
         np.testing.assert_array_equal(b3[key], b1[key])
+
+
+def test_single_normalised_expert_sends_no_gradient_to_the_router():
+    """k = 1 with normalisation: the weight is scale * s / s, the constant scale, so no
+    gradient reaches the logits (dWr = 0 and the router part of dx vanishes) while the expert
+    weights still get theirs (closed form of the chain rule for this case)."""
+    sh = LayerShape("bw_k1", T=9, H=32, E=3, k=1, I=8, Is=16, limit_routed=0.5, seed=64, weight_std=0.25)
+    inp = draw(sh)
+    dy = np.random.default_rng(sh.seed).standard_normal((sh.T, sh.H)).astype(np.float32)
+    ob = oracle.backward(bf16_bits(inp["x"]), bf16_bits(inp["Wr"]), inp["bias"].numpy(), bf16_bits(inp["W_gate_up"]),
+                         bf16_bits(inp["W_down"]), bf16_bits(inp["Wsh_gate_up"]), bf16_bits(inp["Wsh_down"]), dy,
+                         k=1, scale=sh.scale, norm=True, limit_routed=sh.limit_routed, limit_shared=sh.limit_shared)
+    assert np.abs(ob["dWr"]).max() <= 1e-12 * max(1.0, np.abs(ob["dW_gate_up"]).max())
+    assert np.abs(ob["dW_gate_up"]).max() > 0 and np.abs(ob["dW_down"]).max() > 0
