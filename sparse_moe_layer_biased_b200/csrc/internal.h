@@ -55,8 +55,11 @@ size_t ep_regroup_smem(int R, int Er);
 cudaError_t launch_ep_regroup(const int32_t *counts, int R, int Er, int64_t nrows, int32_t *offsets,
                               int32_t *perm_token, int32_t *slot_of, int num_sms, cudaStream_t stream);
 
+// x rows into their routed slots of x_perm (and each slot's routing weight into w_perm); when
+// y_zero is not NULL the launch also zeroes its T rows of H fp32 (16-byte aligned).
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
-                          uint16_t *x_perm, float *w_perm, int num_sms, uint32_t *err, cudaStream_t stream);
+                          uint16_t *x_perm, float *w_perm, int num_sms, uint32_t *err, cudaStream_t stream,
+                          float *y_zero = nullptr);
 
 // Grouped-GEMM configuration. gate_up and down each split every group into chunks of at
 // most `cap` / `cap_d` token rows (the N side of one tile) and stage `mt` / `mt_d` 128-row

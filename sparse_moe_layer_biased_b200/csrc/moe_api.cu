@@ -363,8 +363,11 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     if (!stage_mark(2, s))
         return MOE_ERR_CUDA;
     cudaError_t e = cudaSuccess;
+    // the gather also zeroes y (the down GEMM's reduction target) when it runs
+    const bool zero_in_gather = groups != FfnGroups::kSharedOnly && !d.deterministic;
     if (groups != FfnGroups::kSharedOnly)
-        e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, di.err, s);
+        e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, di.err, s,
+                               zero_in_gather ? out : nullptr);
     const int shared_rows = groups == FfnGroups::kRoutedOnly || split ? 0 : d.T;
     const int nch = static_cast<int>(moe::max_chunks(d.T, d.k, d.E, cfg.cap));
     const int nch_d = static_cast<int>(moe::max_chunks(d.T, d.k, d.E, cfg.cap_d));
@@ -379,7 +382,7 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     if (e == cudaSuccess && split)
         e = moe::launch_chunks(offsets, 0, d.T, cfg_sh.cap, chunks_s, hdr + 4, cfg_sh.cap_d, chunks_sd, hdr + 8,
                                nch_s, nch_sd, Tk, di.err, s);
-    if (e == cudaSuccess && !d.deterministic)
+    if (e == cudaSuccess && !d.deterministic && !zero_in_gather)
         e = cudaMemsetAsync(out, 0, static_cast<size_t>(d.T) * d.H * 4, s);
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;

@@ -224,28 +224,60 @@ __global__ void __launch_bounds__(kPermThreads)
     cluster_sync_all();  // no CTA leaves while a peer may still read its totals
 }
 
-// One warp per (token, rank) entry: copies the token's row of x into its slot and
-// records the slot's routing weight.
+// One warp per token: loads the token's row of x once (pieces of up to 512 16-byte vectors,
+// all of a lane's loads in flight) and stores it into each of its k slots; lane j records
+// the routing weight of slot j. x is read once instead of once per selected expert. When
+// y_zero is given, the warp also clears the token's row of it (the output the down GEMM
+// then accumulates into), in place of a separate memset.
+constexpr int kGatherVec = 16;  // 16-byte vectors per lane and piece
+
 __global__ void __launch_bounds__(256)
     gather_kernel(const uint4 *__restrict__ x, const float *__restrict__ topk_w,
-                  const int32_t *__restrict__ slot_of, int64_t nent, int k, int vec_per_row,
-                  uint4 *__restrict__ x_perm, float *__restrict__ w_perm, uint32_t *err)
+                  const int32_t *__restrict__ slot_of, int64_t T, int k, int vec_per_row,
+                  uint4 *__restrict__ x_perm, float *__restrict__ w_perm, uint4 *__restrict__ y_zero,
+                  int yvec_per_row, uint32_t *err)
 {
     const int lane = threadIdx.x & 31;
     const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t n = gw; n < nent; n += nw) {
-        const int64_t slot = slot_of[n];
-        if (!dbg_ok(slot >= 0 && slot < nent, err))
-            continue;
-        const int64_t t = n / k;
+    const int64_t nent = T * k;
+    for (int64_t t = gw; t < T; t += nw) {
+        // lane j < k holds slot j of the token (the warp reads them by shuffle)
+        int64_t my_slot = -1;
+        if (lane < k) {
+            my_slot = slot_of[t * k + lane];
+            if (!dbg_ok(my_slot >= 0 && my_slot < nent, err))
+                my_slot = -1;
+            else
+                w_perm[my_slot] = topk_w[t * k + lane];
+        }
+        if (y_zero) {
+            uint4 *yr = y_zero + t * yvec_per_row;
+            for (int c = lane; c < yvec_per_row; c += 32)
+                yr[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
         const uint4 *src = x + t * vec_per_row;
-        uint4 *dst = x_perm + slot * vec_per_row;
-#pragma unroll 4
-        for (int v = lane; v < vec_per_row; v += 32)
-            dst[v] = __ldg(src + v);
-        if (lane == 0)
-            w_perm[slot] = topk_w[n];
+        for (int p0 = 0; p0 < vec_per_row; p0 += 32 * kGatherVec) {
+            uint4 v[kGatherVec];
+#pragma unroll
+            for (int i = 0; i < kGatherVec; ++i) {
+                const int c = p0 + i * 32 + lane;
+                if (c < vec_per_row)
+                    v[i] = __ldg(src + c);
+            }
+            for (int j = 0; j < k; ++j) {
+                const int64_t slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
+                if (slot < 0)
+                    continue;
+                uint4 *dst = x_perm + slot * vec_per_row;
+#pragma unroll
+                for (int i = 0; i < kGatherVec; ++i) {
+                    const int c = p0 + i * 32 + lane;
+                    if (c < vec_per_row)
+                        dst[c] = v[i];
+                }
+            }
+        }
     }
 }
 
@@ -406,14 +438,16 @@ cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream)
 }
 
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
-                          uint16_t *x_perm, float *w_perm, int num_sms, uint32_t *err, cudaStream_t stream)
+                          uint16_t *x_perm, float *w_perm, int num_sms, uint32_t *err, cudaStream_t stream,
+                          float *y_zero)
 {
-    const int64_t nent = static_cast<int64_t>(T) * k;
-    const int64_t blocks_needed = (nent + 7) / 8;
+    // one warp per token, 8 warps per block, at most 8 blocks per SM
+    const int64_t blocks_needed = (static_cast<int64_t>(T) + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms) * 8;
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-    gather_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(x), topk_w, slot_of, nent, k, H / 8,
-                                            reinterpret_cast<uint4 *>(x_perm), w_perm, err);
+    gather_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(x), topk_w, slot_of, T, k, H / 8,
+                                            reinterpret_cast<uint4 *>(x_perm), w_perm,
+                                            reinterpret_cast<uint4 *>(y_zero), H / 4, err);
     return cudaGetLastError();
 }
 
