@@ -56,10 +56,12 @@ cudaError_t launch_ep_regroup(const int32_t *counts, int R, int Er, int64_t nrow
                               int32_t *perm_token, int32_t *slot_of, int num_sms, cudaStream_t stream);
 
 // x rows into their routed slots of x_perm (and each slot's routing weight into w_perm); when
-// y_zero is not NULL the launch also zeroes its T rows of H fp32 (16-byte aligned).
+// y_zero is not NULL the launch also zeroes its T rows of H fp32 (16-byte aligned). When
+// amax_x is not NULL it receives, per routed slot, the largest |x| of the slot's row (float
+// bits), and amax_h (same length) is zeroed.
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
                           uint16_t *x_perm, float *w_perm, int num_sms, uint32_t *err, cudaStream_t stream,
-                          float *y_zero = nullptr);
+                          float *y_zero = nullptr, uint32_t *amax_x = nullptr, uint32_t *amax_h = nullptr);
 
 // Grouped-GEMM configuration. gate_up and down each split every group into chunks of at
 // most `cap` / `cap_d` token rows (the N side of one tile) and stage `mt` / `mt_d` 128-row
@@ -145,6 +147,10 @@ struct GateUpArgs {
     int64_t rows_r, rows_s;
     int max_chunks, cap;
     uint32_t *err;  // device error word
+    // FP8 tensor-core kernels: largest |x| of each routed row of x_perm (float bits, read)
+    // and of each routed row of h (float bits, raised with atomicMax; zero on entry)
+    const uint32_t *amax_in;
+    uint32_t *amax_out;
 };
 cudaError_t launch_gate_up(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const TokMaps &tok,
                            const GateUpArgs &a, const WaitCfg &wc, int grid, const GemmConfig &c,
@@ -161,6 +167,7 @@ struct DownArgs {
     const float *w_scale;  // FP8 kernels: block scales [E, H/128, I/128]; else unused
     int max_chunks, cap;   // tile-table capacity and rows per tile (debug-build range checks)
     uint32_t *err;         // device error word
+    const uint32_t *amax_in;  // FP8 tensor-core kernels: largest |h| of each routed row (float bits)
 };
 cudaError_t launch_down(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const TokMaps &tok,
                         const DownArgs &a, const WaitCfg &wc, int grid, const GemmConfig &c, cudaStream_t stream);
@@ -178,6 +185,24 @@ cudaError_t launch_gate_up_fp8(const CUtensorMap &tm_w, const CUtensorMap &tm_ws
 cudaError_t launch_down_fp8(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
                             const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
                             const GemmConfig &c, cudaStream_t stream);
+
+// FP8 E4M3 routed experts on the FP8 tensor cores (tcgen05 kind::f8f6f4), decode-sized
+// calls: tiles of two 128-row weight blocks (gate_up: 128 gate rows and their up rows; down:
+// 256 output rows), 32-row chunks, the block scales applied to the token operand. Needs H a
+// multiple of 256 and I, Is multiples of 128. tm_w / tm_wd: the E4M3 codes as 2-D (H, E*2I)
+// / (I, E*H) bytes with 128 x 128 boxes; tm_wsh / tm_wdsh: the BF16 shared expert as (H, 2Is)
+// / (Is, H) with 64 x 128 boxes; token maps with 32-row boxes. GateUpArgs::amax_in /
+// amax_out and DownArgs::amax_in must be set.
+inline bool fp8_mma_config(const GemmConfig &c, int64_t H, int64_t I, int64_t Is)
+{
+    return c.cap == 32 && c.cap_d == 32 && H % 256 == 0 && I % 128 == 0 && Is % 128 == 0;
+}
+cudaError_t launch_gate_up_fp8_mma(const CUtensorMap &tm_w, const CUtensorMap &tm_wsh, const CUtensorMap &tm_xp,
+                                   const CUtensorMap &tm_x, const GateUpArgs &a, const WaitCfg &wc, int grid,
+                                   cudaStream_t stream);
+cudaError_t launch_down_fp8_mma(const CUtensorMap &tm_wd, const CUtensorMap &tm_wdsh, const CUtensorMap &tm_h,
+                                const CUtensorMap &tm_hsh, const DownArgs &a, const WaitCfg &wc, int grid,
+                                cudaStream_t stream);
 
 // ------------------------------------------------------------------------------------
 // Backward pass. Rows live in a padded permuted space: the shared group takes rows [0, T)

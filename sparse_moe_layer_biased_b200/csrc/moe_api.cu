@@ -196,7 +196,8 @@ moe_status_t check_desc(const moe_layer_desc *d)
 }
 
 struct WsLayout {
-    size_t x_perm, w_perm, h, h_sh, chunks, chunks_d, hdr, o_perm, idx, w, counts, offsets, perm_token, slot_of, total;
+    size_t x_perm, w_perm, h, h_sh, chunks, chunks_d, hdr, o_perm, idx, w, counts, offsets, perm_token, slot_of, amax,
+        total;
 };
 
 size_t up256(size_t v)
@@ -234,6 +235,8 @@ WsLayout ws_layout(const moe_layer_desc &d)
     L.offsets = take((E + 2) * 4);
     L.perm_token = take((T * k + T) * 4);
     L.slot_of = take(T * k * 4);
+    // row maxima of x_perm and h (FP8 weights on the FP8 tensor cores)
+    L.amax = take(T * k * 8);
     L.total = off;
     return L;
 }
@@ -325,12 +328,22 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     moe::TokMaps tok_gu, tok_d;  // token rows of gate_up (x_perm, x) and down (h, h_sh)
     const int64_t EH = static_cast<int64_t>(d.E) * d.H;
     const uint32_t inner8 = 128;  // one 128-wide scale block of E4M3 codes per stage
-    bool ok = (fp8 ? map_gate_up_u8(&tm_w, W.gu, d.H, d.I, d.E, feats, inner8)
-                   : map_gate_up(&tm_w, W.gu, d.H, d.I, d.E, feats)) &&
-              (fp8 ? map_rows_u8(&tm_wd, W.d, d.I, EH, drows, inner8) : map_rows(&tm_wd, W.d, d.I, EH, drows)) &&
-              map_gate_up(&tm_wsh, W.sh_gu, d.H, d.Is, 1, feats) && map_rows(&tm_wdsh, W.sh_d, d.Is, d.H, drows) &&
-              map_rows(&tok_gu.routed, x_perm, d.H, Tk, brows) && map_rows(&tok_gu.shared, x, d.H, d.T, brows) &&
+    // FP8 decode on the FP8 tensor cores: weights as plain row-major boxes of 128 rows (E4M3
+    // codes 128 bytes wide, the BF16 shared expert 64 elements wide)
+    const bool f8mma = fp8 && moe::fp8_mma_config(cfg, d.H, d.I, d.Is);
+    bool ok = map_rows(&tok_gu.routed, x_perm, d.H, Tk, brows) && map_rows(&tok_gu.shared, x, d.H, d.T, brows) &&
               map_rows(&tok_d.routed, h, d.I, Tk, brows) && map_rows(&tok_d.shared, h_sh, d.Is, d.T, brows);
+    if (ok && f8mma)
+        ok = map_rows_u8(&tm_w, W.gu, d.H, static_cast<int64_t>(d.E) * 2 * d.I, 128, inner8) &&
+             map_rows_u8(&tm_wd, W.d, d.I, EH, 128, inner8) && map_rows(&tm_wsh, W.sh_gu, d.H, 2 * d.Is, 128) &&
+             map_rows(&tm_wdsh, W.sh_d, d.Is, d.H, 128);
+    else if (ok)
+        ok = (fp8 ? map_gate_up_u8(&tm_w, W.gu, d.H, d.I, d.E, feats, inner8)
+                  : map_gate_up(&tm_w, W.gu, d.H, d.I, d.E, feats)) &&
+             (fp8 ? map_rows_u8(&tm_wd, W.d, d.I, EH, drows, inner8) : map_rows(&tm_wd, W.d, d.I, EH, drows)) &&
+             map_gate_up(&tm_wsh, W.sh_gu, d.H, d.Is, 1, feats) && map_rows(&tm_wdsh, W.sh_d, d.Is, d.H, drows);
+    uint32_t *amax_x = f8mma ? at<uint32_t>(ws, L.amax) : nullptr;
+    uint32_t *amax_h = f8mma ? amax_x + Tk : nullptr;
     if (ok && cfg.pair)
         ok = pair_token_maps(&tok_gu, x_perm, x, d.H, Tk, d.T) && pair_token_maps(&tok_d, h, h_sh, d.I, Tk, d.T, d.Is);
     if (!ok)
@@ -367,7 +380,7 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     const bool zero_in_gather = groups != FfnGroups::kSharedOnly && !d.deterministic;
     if (groups != FfnGroups::kSharedOnly)
         e = moe::launch_gather(x, topk_w, slot_of, d.T, d.k, d.H, x_perm, w_perm, di.num_sms, di.err, s,
-                               zero_in_gather ? out : nullptr);
+                               zero_in_gather ? out : nullptr, amax_x, amax_h);
     const int shared_rows = groups == FfnGroups::kRoutedOnly || split ? 0 : d.T;
     const int nch = static_cast<int>(moe::max_chunks(d.T, d.k, d.E, cfg.cap));
     const int nch_d = static_cast<int>(moe::max_chunks(d.T, d.k, d.E, cfg.cap_d));
@@ -388,11 +401,14 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
         return MOE_ERR_CUDA;
     const moe::WaitCfg wc = wait_cfg(di);
     moe::GateUpArgs ga{chunks, hdr, h, h_sh, d.E, d.H, d.I, d.Is, d.limit_routed, d.limit_shared, W.gu_scale,
-                       Tk, d.T, nch, cfg.cap, di.err};
+                       Tk, d.T, nch, cfg.cap, di.err, amax_x, amax_h};
     if (!stage_mark(3, s))
         return MOE_ERR_CUDA;
-    e = fp8 ? moe::launch_gate_up_fp8(tm_w, tm_wsh, tok_gu.routed, tok_gu.shared, ga, wc, di.num_sms, cfg, s)
-            : moe::launch_gate_up(tm_w, tm_wsh, tok_gu, ga, wc, di.num_sms, cfg, s);
+    if (f8mma)
+        e = moe::launch_gate_up_fp8_mma(tm_w, tm_wsh, tok_gu.routed, tok_gu.shared, ga, wc, di.num_sms, s);
+    else
+        e = fp8 ? moe::launch_gate_up_fp8(tm_w, tm_wsh, tok_gu.routed, tok_gu.shared, ga, wc, di.num_sms, cfg, s)
+                : moe::launch_gate_up(tm_w, tm_wsh, tok_gu, ga, wc, di.num_sms, cfg, s);
     if (e == cudaSuccess && split) {
         const moe::GateUpArgs gs{chunks_s, hdr + 4, h, h_sh, 0, d.H, d.I, d.Is, d.limit_routed, d.limit_shared,
                                  nullptr, Tk, d.T, nch_s, cfg_sh.cap, di.err};
@@ -401,11 +417,14 @@ moe_status_t run_expert_ffn(const moe_layer_desc &d, const DeviceInfo &di, const
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
     moe::DownArgs da{chunks_d, hdr_d, perm_token, w_perm, out, d.E, d.H, d.I, d.Is, d.T, d.k, d.deterministic,
-                     W.d_scale, cfg.cap_d != cfg.cap ? nch_d : nch, cfg.cap_d, di.err};
+                     W.d_scale, cfg.cap_d != cfg.cap ? nch_d : nch, cfg.cap_d, di.err, amax_h};
     if (!stage_mark(4, s))
         return MOE_ERR_CUDA;
-    e = fp8 ? moe::launch_down_fp8(tm_wd, tm_wdsh, tok_d.routed, tok_d.shared, da, wc, di.num_sms, cfg, s)
-            : moe::launch_down(tm_wd, tm_wdsh, tok_d, da, wc, di.num_sms, cfg, s);
+    if (f8mma)
+        e = moe::launch_down_fp8_mma(tm_wd, tm_wdsh, tok_d.routed, tok_d.shared, da, wc, di.num_sms, s);
+    else
+        e = fp8 ? moe::launch_down_fp8(tm_wd, tm_wdsh, tok_d.routed, tok_d.shared, da, wc, di.num_sms, cfg, s)
+                : moe::launch_down(tm_wd, tm_wdsh, tok_d, da, wc, di.num_sms, cfg, s);
     if (e == cudaSuccess && split) {
         const moe::DownArgs ds{chunks_sd, hdr + 8, perm_token, w_perm, out, 0, d.H, d.I, d.Is, d.T, d.k,
                                d.deterministic, nullptr, nch_sd, cfg_sh.cap_d, di.err};

@@ -228,14 +228,25 @@ __global__ void __launch_bounds__(kPermThreads)
 // all of a lane's loads in flight) and stores it into each of its k slots; lane j records
 // the routing weight of slot j. x is read once instead of once per selected expert. When
 // y_zero is given, the warp also clears the token's row of it (the output the down GEMM
-// then accumulates into), in place of a separate memset.
+// then accumulates into), in place of a separate memset. With amax_x, lane j also stores the
+// row's largest |x| (float bits) for slot j and zeroes amax_h of that slot (the FP8
+// tensor-core GEMMs scale each token row by it).
 constexpr int kGatherVec = 16;  // 16-byte vectors per lane and piece
+
+// Largest magnitude among the eight bf16 of v, as bf16 magnitude bits in [0, 0x7fff] (the
+// magnitude bits of non-NaN bf16 values order like the values).
+__device__ __forceinline__ uint32_t bf16x8_absmax(const uint4 &v)
+{
+    const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu),
+                                __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu));
+    return max(m & 0xffffu, m >> 16);
+}
 
 __global__ void __launch_bounds__(256)
     gather_kernel(const uint4 *__restrict__ x, const float *__restrict__ topk_w,
                   const int32_t *__restrict__ slot_of, int64_t T, int k, int vec_per_row,
                   uint4 *__restrict__ x_perm, float *__restrict__ w_perm, uint4 *__restrict__ y_zero,
-                  int yvec_per_row, uint32_t *err)
+                  int yvec_per_row, uint32_t *amax_x, uint32_t *amax_h, uint32_t *err)
 {
     const int lane = threadIdx.x & 31;
     const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -257,13 +268,17 @@ __global__ void __launch_bounds__(256)
                 yr[c] = make_uint4(0u, 0u, 0u, 0u);
         }
         const uint4 *src = x + t * vec_per_row;
+        uint32_t amax = 0;
         for (int p0 = 0; p0 < vec_per_row; p0 += 32 * kGatherVec) {
             uint4 v[kGatherVec];
 #pragma unroll
             for (int i = 0; i < kGatherVec; ++i) {
                 const int c = p0 + i * 32 + lane;
-                if (c < vec_per_row)
+                if (c < vec_per_row) {
                     v[i] = __ldg(src + c);
+                    if (amax_x)
+                        amax = max(amax, bf16x8_absmax(v[i]));
+                }
             }
             for (int j = 0; j < k; ++j) {
                 const int64_t slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
@@ -276,6 +291,13 @@ __global__ void __launch_bounds__(256)
                     if (c < vec_per_row)
                         dst[c] = v[i];
                 }
+            }
+        }
+        if (amax_x) {
+            amax = __reduce_max_sync(0xFFFFFFFFu, amax);
+            if (my_slot >= 0) {
+                amax_x[my_slot] = amax << 16;
+                amax_h[my_slot] = 0u;
             }
         }
     }
@@ -439,7 +461,7 @@ cudaError_t launch_permute(const PermuteArgs &a, cudaStream_t stream)
 
 cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t *slot_of, int T, int k, int H,
                           uint16_t *x_perm, float *w_perm, int num_sms, uint32_t *err, cudaStream_t stream,
-                          float *y_zero)
+                          float *y_zero, uint32_t *amax_x, uint32_t *amax_h)
 {
     // one warp per token, 8 warps per block, at most 8 blocks per SM
     const int64_t blocks_needed = (static_cast<int64_t>(T) + 7) / 8;
@@ -447,7 +469,7 @@ cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t 
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
     gather_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(x), topk_w, slot_of, T, k, H / 8,
                                             reinterpret_cast<uint4 *>(x_perm), w_perm,
-                                            reinterpret_cast<uint4 *>(y_zero), H / 4, err);
+                                            reinterpret_cast<uint4 *>(y_zero), H / 4, amax_x, amax_h, err);
     return cudaGetLastError();
 }
 

@@ -356,6 +356,20 @@ __device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, u
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] · B[smem]^T with E4M3 A and B (tcgen05.mma kind::f8f6f4, both
+// K-major), fp32 accumulation, M = 128 rows. One instruction covers K = 32 (32 bytes of each
+// 128-byte swizzled row).
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Stores 16 consecutive 32-bit TMEM columns of this thread's lane (warp-collective). The
 // stores complete at tmem_store_wait.
 __device__ __forceinline__ void tmem_store16(uint32_t taddr, const uint32_t (&r)[16])
@@ -451,6 +465,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N)
     return (1u << 4)                                     // D format fp32
            | (1u << 7)                                   // A format bf16
            | (1u << 10)                                  // B format bf16
+           | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);      // M / 16
+}
+
+// Instruction descriptor of tcgen05.mma.kind::f8f6f4 with E4M3 A and B (format code 0 in
+// both fields; both K-major), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
+{
+    return (1u << 4)                                     // D format fp32
            | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);      // M / 16
 }

@@ -6,6 +6,11 @@ scale) on the tensor cores. The extra bf16 rounding of each dequantized weight
 (relative <= 2^-9, independent across weights) adds about 2^-9 / sqrt(3) ~ 1.1e-3
 relative error to a dot product whose terms have random signs, inside the layer's
 1e-2 relative-Frobenius / 3e-2 max-abs bar, which the tests keep.
+
+Decode-sized calls with H a multiple of 256 and I, Is multiples of 128 run the routed experts
+on the FP8 tensor cores instead (E4M3 codes straight into the MMA, each block scale and each
+token row's largest |x| applied to the token operand, which is split into two E4M3 parts
+carrying about 8 significant bits: the precision of the bf16 operands above).
 """
 import numpy as np
 import pytest
@@ -28,6 +33,11 @@ SHAPES = {
     # in a half-empty stage that TMA fills with zeros for both operands
     "decode_is192": LayerShape("fp8_decode_is192", T=24, H=512, E=40, k=8, I=256, Is=192, limit_shared=0.25,
                                seed=55, weight_std=0.03),
+    # decode-sized with H a multiple of 256 and I, Is of 128: the FP8 tensor-core kernels
+    # (E4M3 weights straight into the MMA, block scales on the token operand); 6 K blocks of
+    # gate/up, 3 down tiles of 256 rows, 2 shared feature blocks, chunks of 16 and 32 rows
+    "decode_h768": LayerShape("fp8_decode_h768", T=40, H=768, E=24, k=6, I=256, Is=256, limit_routed=0.25,
+                              seed=58, weight_std=0.03),
     # prefill-sized: 128-row chunks, several K blocks, ragged chunk tails, Is not a multiple of 128
     "prefill": LayerShape("fp8_prefill", T=300, H=512, E=12, k=4, I=256, Is=192, limit_routed=0.25,
                           limit_shared=0.125, seed=52, weight_std=0.03),
@@ -148,3 +158,57 @@ def test_fp8_full_size_output_sampled(full):
     np.testing.assert_array_equal(np.sort(full["idx"][rows][keep], 1), np.sort(r["idx"][keep], 1))
     rf, ma = check_output(full["y"][rows][keep], y_ref[keep], sh.name)
     print(f"{sh.name} fp8 sampled: rel_fro {rf:.2e} max_abs {ma:.2e}")
+
+
+def test_fp8_decode_row_and_block_scaling():
+    """FP8 tensor-core decode path: the token operand is scaled per row by its largest |x|
+    and per weight block row by its largest block scale. Rows of very different magnitude
+    (x 8, x 2^-6: the layer's relative bar, row by row; all zero: output exactly 0) and block
+    scales spread over a factor 2^8 within each block row (the layer bar on the other rows)."""
+    sh = SHAPES["decode_h768"].replace(limit_routed=0.0)
+    inp = draw_fp8(sh)
+    x = inp["x"].float()
+    x[0] *= 8.0
+    x[1] *= 2.0 ** -6
+    x[2] = 0.0
+    inp["x"] = x.to(torch.bfloat16)
+    gen = torch.Generator().manual_seed(59)
+    for key in ("W_gate_up_s", "W_down_s"):
+        # factors 2^-4 .. 2^4 along each block row (K blocks), renormalised so the row's
+        # mean square is kept: the outputs stay at the workload's scale, where the absolute
+        # bar applies
+        spread = torch.exp2(torch.randint(-4, 5, inp[key].shape, generator=gen).float())
+        spread = spread / spread.square().mean(-1, keepdim=True).sqrt()
+        inp[key] = inp[key] * spread
+    y, idx, w = _forward(sh, {k: v.cuda() for k, v in inp.items()})
+    ref = _oracle(sh, inp)
+    keep = check_routing(idx, w, ref, sh.E, sh.k)
+    assert np.abs(y[2]).max() == 0.0
+    for r in (0, 1):
+        if not keep[r]:
+            continue  # a near tie: the routing check above covers it
+        rf = rel_fro(y[r], ref["y"][r])
+        print(f"row {r}: rel_fro {rf:.2e}")
+        assert rf <= 1e-2
+    rest = keep.copy()
+    rest[:3] = False
+    rf, ma = check_output(y[rest], ref["y"][rest], "scaled rows")
+    print(f"decode_h768 scaled: rel_fro {rf:.2e} max_abs {ma:.2e}")
+
+
+def test_fp8_decode_scales_are_applied_per_block():
+    """FP8 tensor-core decode path: doubling every down scale of the busiest expert doubles
+    its contribution (the difference matches the oracle's)."""
+    sh = SHAPES["decode_h768"]
+    inp = draw_fp8(sh)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    y1, idx, _ = _forward(sh, dev, det=True)
+    e = int(np.bincount(idx.ravel(), minlength=sh.E).argmax())
+    inp2 = dict(inp)
+    s2 = inp["W_down_s"].clone()
+    s2[e] *= 2.0
+    inp2["W_down_s"] = s2
+    dev["W_down_s"] = s2.cuda()
+    y2, _, _ = _forward(sh, dev, det=True)
+    r1, r2 = _oracle(sh, inp), _oracle(sh, inp2)
+    check_output(y2 - y1, r2["y"] - r1["y"], "decode scale delta")
