@@ -168,9 +168,14 @@ MOE_API moe_status_t moe_forward_with_ids(const moe_layer_desc *desc, const uint
  *   W_gate_up_q [E, 2I, H] uint8 E4M3 codes (rows [0, I) gate, [I, 2I) up),
  *   W_gate_up_scale [E, 2I/128, H/128] fp32, W_down_q [E, H, I] uint8,
  *   W_down_scale [E, H/128, I/128] fp32: weight[r][c] = e4m3(q[r][c]) * scale[r/128][c/128].
- * The kernels stream the codes (half the weight bytes of BF16) and turn them into
- * bf16(e4m3 * scale) in tensor memory for the BF16 tensor-core MMA, so a dequantized weight
- * carries one bf16 rounding (relative 2^-9) besides the BF16 path's arithmetic. Every other
+ * The kernels stream the codes (half the weight bytes of BF16). Decode-sized calls (T * k <=
+ * 16 * E) with H % 256 == 0 and I, Is % 128 == 0 feed the codes unchanged to the FP8 tensor
+ * cores: each block scale, together with a power of two per token row taken from the row's
+ * largest |x| (or |h|), multiplies the token operand, which is split into two E4M3 parts
+ * (hi + lo, about 8 significant bits, the precision of a bf16 operand). Other calls turn the
+ * codes into bf16(e4m3 * scale) in tensor memory for the BF16 tensor-core MMA, so a
+ * dequantized weight carries one bf16 rounding (relative 2^-9) besides the BF16 path's
+ * arithmetic. Every other
  * argument, the workspace (moe_workspace_size covers both formats) and the results are
  * those of moe_forward. Requires I % 128 == 0 (MOE_ERR_UNSUPPORTED otherwise); code arrays
  * 16-byte aligned, scale arrays 4-byte aligned; the library reads the weights only. */
