@@ -357,6 +357,18 @@ def gate_up_flops(shape):
     return 4.0 * shape.H * (shape.I * shape.T * shape.k + shape.Is * shape.T)
 
 
+def gate_up_kernel_name(shape, fp8=False):
+    """The gate_up kernel one call launches (the library's configuration choice)."""
+    decode = shape.T * shape.k <= 16 * shape.E
+    if fp8:
+        if decode and shape.H % 256 == 0 and shape.I % 128 == 0 and shape.Is % 128 == 0:
+            return "gemm_fp8_mma_kernel<GateUpArgs>"
+        return "gemm_fp8_kernel<GateUpArgs>"
+    if not decode and shape.I % 128 == 0 and shape.Is % 128 == 0 and shape.H % 512 == 0:
+        return "gate_up_pair_kernel"
+    return "gate_up_kernel"
+
+
 def gate_up_roofline(shape, counts, launch_ms, peaks, peak_kind, fp8=False, traffic=None):
     """Roofline block of the dominant kernel (gate_up). The bound is the resource whose
     time floor is longer at the measured peaks: algorithmic bytes / HBM copy bandwidth
@@ -368,7 +380,7 @@ def gate_up_roofline(shape, counts, launch_ms, peaks, peak_kind, fp8=False, traf
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     gbs = nbytes / (launch_ms / 1e3) / 1e9
     tfs = flops / (launch_ms / 1e3) / 1e12
-    kernel = "gemm_fp8_kernel<GateUpArgs>" if fp8 else "gate_up_pair_kernel"
+    kernel = gate_up_kernel_name(shape, fp8)
     common = {"kernel": kernel, "traffic": traffic, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
               "intensity_flop_per_byte": flops / nbytes,
               "ridge_flop_per_byte": peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9),

@@ -230,25 +230,6 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// Weight gradients of routed experts that received no tokens (no GEMM tile writes them):
-// block (e, slice) zeroes a 1/64 slice of dW_gate_up[e] and dW_down[e].
-__global__ void __launch_bounds__(256)
-    bwd_zero_untouched_kernel(const int32_t *__restrict__ counts, int H, int I, float *__restrict__ dWgu,
-                              float *__restrict__ dWd)
-{
-    const int e = blockIdx.x;
-    if (counts[e] != 0)
-        return;
-    const int64_t n_gu = static_cast<int64_t>(2) * I * H / 4, n_d = static_cast<int64_t>(H) * I / 4;
-    float4 *gu = reinterpret_cast<float4 *>(dWgu + static_cast<int64_t>(e) * 2 * I * H);
-    float4 *d = reinterpret_cast<float4 *>(dWd + static_cast<int64_t>(e) * H * I);
-    const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int64_t i = static_cast<int64_t>(blockIdx.y) * 256 + threadIdx.x; i < n_gu; i += 256 * gridDim.y)
-        gu[i] = z;
-    for (int64_t i = static_cast<int64_t>(blockIdx.y) * 256 + threadIdx.x; i < n_d; i += 256 * gridDim.y)
-        d[i] = z;
-}
-
 // dWr[e][h] = Σ over group e's rows of dl_pad[row] * x_pad[row][h]. Block (e, 512 columns,
 // split z of kDwrSplit) sums rows r0 + z, r0 + z + kDwrSplit, ... (four rows of loads in flight)
 // and adds its partial sums into dWr, which the launch zeroes first: a hot expert's thousands
@@ -324,13 +305,6 @@ cudaError_t launch_bwd_router(const uint16_t *x, const uint16_t *Wr, const int32
     return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_zero_untouched(const int32_t *counts, int E, int H, int I, float *dWgu, float *dWd,
-                                      cudaStream_t stream)
-{
-    bwd_zero_untouched_kernel<<<dim3(E, 64), 256, 0, stream>>>(counts, H, I, dWgu, dWd);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_bwd_dwr(const uint16_t *x_pad, const float *dl_pad, const int32_t *poff, const int32_t *counts,
                            int E, int H, float *dWr, cudaStream_t stream)
 {
@@ -355,6 +329,10 @@ cudaError_t launch_bwd_dwr(const uint16_t *x_pad, const float *dl_pad, const int
 namespace {
 
 constexpr int kBwdThreads = 192;
+// the DH kernel carries one more warp: it zeroes the weight gradients of routed experts that
+// received no tokens (no weight-gradient tile writes them) while the GEMM streams W_down
+constexpr int kBwdThreadsDH = kBwdThreads + 32;
+constexpr uint32_t kBwdZeroBytes = 2048;  // zero source of those bulk stores
 constexpr int kBwdStages = 6;  // stages of 32 KB (the ring region's size in those units)
 constexpr int kBwdBN = 128;    // output columns of a weight-gradient tile
 constexpr int kBwdAcc = kBwdCap;  // TMEM columns of one accumulator buffer
@@ -368,6 +346,9 @@ constexpr uint32_t kBwdEpiOff = (kBwdMiscOff + 16 + 1023) / 1024 * 1024;
 constexpr uint32_t kBwdEpiBox = 32 * 32 * 4;
 constexpr uint32_t kBwdEpiWarp = 2 * kBwdEpiBox;
 static_assert(32 * 33 * 4 <= kBwdEpiWarp, "transpose buffer");
+// the zero source sits in the unused end of epilogue warp 0's area in the DH mode
+constexpr uint32_t kBwdZeroOff = kBwdEpiOff + kBwdEpiWarp - kBwdZeroBytes;
+static_assert(32 * 33 * 4 <= kBwdEpiWarp - kBwdZeroBytes, "zero source overlaps the transpose buffer");
 constexpr uint32_t kBwdSmem = kBwdEpiOff + 4 * kBwdEpiWarp + 1024;
 static_assert(kBwdSmem <= kMaxDynSmem, "backward ring exceeds shared memory");
 
@@ -537,6 +518,8 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
             float v[32], gg[32], uu[32];
             tmem_load32(tq + cb, v);
             const int ncol = t.ntok - cb < 32 ? t.ntok - cb : 32;
+            // lane c: routing weight of column cb + c (read by shuffle below)
+            const float wl = t.sh || lane >= ncol ? 1.0f : a.w_pad[t.row0 + cb + lane];
             // all 64 pre-activation loads of the block in flight before any use
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
@@ -550,7 +533,9 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
                     break;
                 const int64_t rr = rs + cb + c;
                 const float g = gg[c], u = uu[c];
-                const float sg = 1.0f / (1.0f + expf(-g));
+                // fast exponential and division: a few fp32 ulp, far below the bf16 rounding of
+                // the gradients that follows
+                const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
                 const float act = g * sg;
                 float ac = act, uc = u, ma = 1.0f, mu = 1.0f;
                 if (L > 0.0f) {
@@ -569,7 +554,7 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
                 const float dhu = v[c];
                 if (!t.sh)
                     tr[lane * 33 + c] = ac * uc * dhu;  // this lane's term of h . dhu for column c
-                const float dh = (t.sh ? 1.0f : a.w_pad[t.row0 + cb + c]) * dhu;
+                const float dh = __shfl_sync(0xFFFFFFFFu, wl, c) * dhu;
                 const float dg = dh * uc * ma * sg * (1.0f + g * (1.0f - sg));
                 const float du = dh * ac * mu;
                 dgu[rr * 2 * Iw + i] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
@@ -638,8 +623,35 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
 
 // NSL = 64-wide K slices per stage (2: half as many stages of twice the size, so the MMA
 // thread's barrier test and commit cover 8 MMAs; the tile's K must be a multiple of 128).
+// Zeroes dW_gate_up[e] and dW_down[e] of every routed expert with no rows: each region is cut
+// into kBwdZeroBytes pieces, CTA b stores pieces b, b + grid, ... from a zeroed shared-memory
+// buffer with bulk copies (one issuing thread; the copies only read the constant buffer).
+__device__ __forceinline__ void bwd_zero_untouched(const BwdArgs &a, const uint8_t *zero)
+{
+    const uint64_t gu_bytes = static_cast<uint64_t>(2) * a.I * a.H * 4, d_bytes = static_cast<uint64_t>(a.H) * a.I * 4;
+    int issued = 0;
+    for (int e = 0; e < a.E; ++e) {
+        if (a.counts[e] != 0)
+            continue;
+        for (int r = 0; r < 2; ++r) {
+            uint8_t *base = r == 0 ? reinterpret_cast<uint8_t *>(a.dWgu) + e * gu_bytes
+                                   : reinterpret_cast<uint8_t *>(a.dWd) + e * d_bytes;
+            const uint64_t bytes = r == 0 ? gu_bytes : d_bytes;
+            for (uint64_t off = static_cast<uint64_t>(blockIdx.x) * kBwdZeroBytes; off < bytes;
+                 off += static_cast<uint64_t>(gridDim.x) * kBwdZeroBytes) {
+                const uint64_t n = bytes - off < kBwdZeroBytes ? bytes - off : kBwdZeroBytes;
+                bulk_store(base + off, zero, static_cast<uint32_t>(n));
+                if (++issued % 16 == 0)
+                    bulk_commit();
+            }
+        }
+    }
+    bulk_commit();
+    bulk_wait<0>();  // complete before the CTA (and its shared memory) goes away
+}
+
 template <int MODE, int NSL>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreadsDH, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap a_r, const __grid_constant__ CUtensorMap a_s,
                     const __grid_constant__ CUtensorMap b_r, const __grid_constant__ CUtensorMap b_s,
                     const __grid_constant__ CUtensorMap o_r, const __grid_constant__ CUtensorMap o_s,
@@ -758,6 +770,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             umma_commit(drain);
             mbar_wait_drain(drain, 0, wc);
         }
+    } else if (warp == 6) {
+        // DH only: zero the gradients of untouched experts
+        uint8_t *zero = smem + kBwdZeroOff;
+        for (uint32_t i = lane * 16; i < kBwdZeroBytes; i += 32 * 16)
+            *reinterpret_cast<uint4 *>(zero + i) = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0)
+            bwd_zero_untouched(a, zero);
+        __syncwarp();
     } else {
         const int q = warp & 3;
         int tc = 0;
@@ -794,7 +816,8 @@ cudaError_t launch_mode(const CUtensorMap &a_r, const CUtensorMap &a_s, const CU
                                            static_cast<int>(kBwdSmem));
     if (err != cudaSuccess)
         return err;
-    bwd_gemm_kernel<MODE, NSL><<<grid, kBwdThreads, kBwdSmem, stream>>>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc);
+    const int threads = MODE == kBwdDH ? kBwdThreadsDH : kBwdThreads;
+    bwd_gemm_kernel<MODE, NSL><<<grid, threads, kBwdSmem, stream>>>(a_r, a_s, b_r, b_s, o_r, o_s, a, wc);
     return cudaGetLastError();
 }
 

@@ -228,6 +228,7 @@ struct BwdArgs {
     float *dw_pad;            // [P] dLoss/dw of routed rows (accumulated)
     float *dx;                // [T, H]
     float *dWd, *dWgu, *dWsh_d, *dWsh_gu;
+    const int32_t *counts;    // [E] rows per routed expert (DH zeroes the gradients of those with none)
 };
 enum BwdMode { kBwdGU = 0, kBwdDH = 1, kBwdDX = 2, kBwdWD = 3, kBwdWGU = 4 };
 // Maps per mode (routed A, shared A, routed B, shared B):
@@ -257,9 +258,6 @@ cudaError_t launch_bwd_gather(const uint16_t *x, const float *dy, const int32_t 
 cudaError_t launch_bwd_router(const uint16_t *x, const uint16_t *Wr, const int32_t *topk_idx, const int32_t *slot_of,
                               const int32_t *offsets, const int32_t *poff, const float *dw_pad, int T, int k, int E,
                               int H, float scale, int norm, float *dx, float *dl_pad, cudaStream_t stream);
-// Zeroes dW_gate_up[e] and dW_down[e] of routed experts with no tokens.
-cudaError_t launch_bwd_zero_untouched(const int32_t *counts, int E, int H, int I, float *dWgu, float *dWd,
-                                      cudaStream_t stream);
 // dWr[e] = sum of dl_pad[row] * x_pad[row] over group e's rows.
 cudaError_t launch_bwd_dwr(const uint16_t *x_pad, const float *dl_pad, const int32_t *poff, const int32_t *counts,
                            int E, int H, float *dWr, cudaStream_t stream);

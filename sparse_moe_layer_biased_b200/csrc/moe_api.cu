@@ -1002,7 +1002,7 @@ moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const u
     const moe::WaitCfg wc = wait_cfg(di);
     moe::BwdArgs ba{d.T, d.H, d.E, d.k, d.I, d.Is, d.limit_routed, d.limit_shared, static_cast<int>(Ps), chunks,
                     wgroups, hdr, w_pad, tok_pad, gu_r, gu_s, dgu_r, dgu_s, hw_r, hw_s, dw_pad, dx, dW_down,
-                    dW_gate_up, dWsh_down, dWsh_gate_up};
+                    dW_gate_up, dWsh_down, dWsh_gate_up, counts};
     const moe::PermuteArgs pa{topk_idx, d.T, d.k, d.E, counts, offsets, perm_token, slot_of, nullptr, nullptr,
                               nullptr, nullptr, 0, di.err, 0};
     cudaError_t e = moe::launch_permute(pa, s);
@@ -1022,8 +1022,6 @@ moe_status_t moe_backward(const moe_layer_desc *desc, const uint16_t *x, const u
                                    d.norm_expert_weight, dx, dl_pad, s);
     if (e == cudaSuccess)
         e = moe::launch_bwd_gemm(moe::kBwdDX, dx_a_r, dx_a_s, dx_b_r, dx_b_s, dx_b2_r, dx_b2_s, ba, wc, di.num_sms, s);
-    if (e == cudaSuccess)
-        e = moe::launch_bwd_zero_untouched(counts, d.E, d.H, d.I, dW_gate_up, dW_down, s);
     if (e == cudaSuccess)
         e = moe::launch_bwd_gemm(moe::kBwdWD, wd_a, wd_a, wd_b_r, wd_b_s, wd_o_r, wd_o_s, ba, wc, di.num_sms, s);
     if (e == cudaSuccess)

@@ -224,14 +224,17 @@ __global__ void __launch_bounds__(kPermThreads)
     cluster_sync_all();  // no CTA leaves while a peer may still read its totals
 }
 
-// One warp per token: loads the token's row of x once (pieces of up to 512 16-byte vectors,
-// all of a lane's loads in flight) and stores it into each of its k slots; lane j records
-// the routing weight of slot j. x is read once instead of once per selected expert. When
-// y_zero is given, the warp also clears the token's row of it (the output the down GEMM
-// then accumulates into), in place of a separate memset. With amax_x, lane j also stores the
-// row's largest |x| (float bits) for slot j and zeroes amax_h of that slot (the FP8
-// tensor-core GEMMs scale each token row by it).
-constexpr int kGatherVec = 16;  // 16-byte vectors per lane and piece
+// Per-token mode (large batches): one warp per token loads the token's row of x once (pieces
+// of up to 512 16-byte vectors, all of a lane's loads in flight) and stores it into each of
+// its k slots; lane j records the routing weight of slot j. x is read once instead of once per
+// selected expert. Per-slot mode (small batches, where T warps would leave most of the GPU
+// idle): one warp per (token, slot), x read k times (from L2). When y_zero is given, the
+// warps also clear the token's row of it (the output the down GEMM then accumulates into; in
+// per-slot mode slot j clears the j-th of k column ranges), in place of a separate memset.
+// With amax_x, each slot also gets its row's largest |x| (float bits) and a zeroed amax_h (the
+// FP8 tensor-core GEMMs scale each token row by it).
+constexpr int kGatherVec = 16;        // 16-byte vectors per lane and piece
+constexpr int kGatherPerTokenT = 2048;  // batches of at least this many tokens use per-token mode
 
 // Largest magnitude among the eight bf16 of v, as bf16 magnitude bits in [0, 0x7fff] (the
 // magnitude bits of non-NaN bf16 values order like the values).
@@ -242,6 +245,7 @@ __device__ __forceinline__ uint32_t bf16x8_absmax(const uint4 &v)
     return max(m & 0xffffu, m >> 16);
 }
 
+template <bool kPerSlot>
 __global__ void __launch_bounds__(256)
     gather_kernel(const uint4 *__restrict__ x, const float *__restrict__ topk_w,
                   const int32_t *__restrict__ slot_of, int64_t T, int k, int vec_per_row,
@@ -252,19 +256,26 @@ __global__ void __launch_bounds__(256)
     const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const int64_t nent = T * k;
-    for (int64_t t = gw; t < T; t += nw) {
-        // lane j < k holds slot j of the token (the warp reads them by shuffle)
+    const int64_t units = kPerSlot ? nent : T;
+    for (int64_t u = gw; u < units; u += nw) {
+        const int64_t t = kPerSlot ? u / k : u;
+        const int j0 = kPerSlot ? static_cast<int>(u - t * k) : 0;  // first slot of the unit
+        const int nj = kPerSlot ? 1 : k;                              // slots of the unit
+        // lane j < nj holds slot j0 + j of the token (the warp reads them by shuffle)
         int64_t my_slot = -1;
-        if (lane < k) {
-            my_slot = slot_of[t * k + lane];
+        if (lane < nj) {
+            my_slot = slot_of[t * k + j0 + lane];
             if (!dbg_ok(my_slot >= 0 && my_slot < nent, err))
                 my_slot = -1;
             else
-                w_perm[my_slot] = topk_w[t * k + lane];
+                w_perm[my_slot] = topk_w[t * k + j0 + lane];
         }
         if (y_zero) {
             uint4 *yr = y_zero + t * yvec_per_row;
-            for (int c = lane; c < yvec_per_row; c += 32)
+            const int c0 = kPerSlot ? static_cast<int>(static_cast<int64_t>(yvec_per_row) * j0 / k) : 0;
+            const int c1 = kPerSlot ? static_cast<int>(static_cast<int64_t>(yvec_per_row) * (j0 + 1) / k)
+                                    : yvec_per_row;
+            for (int c = c0 + lane; c < c1; c += 32)
                 yr[c] = make_uint4(0u, 0u, 0u, 0u);
         }
         const uint4 *src = x + t * vec_per_row;
@@ -280,7 +291,7 @@ __global__ void __launch_bounds__(256)
                         amax = max(amax, bf16x8_absmax(v[i]));
                 }
             }
-            for (int j = 0; j < k; ++j) {
+            for (int j = 0; j < nj; ++j) {
                 const int64_t slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
                 if (slot < 0)
                     continue;
@@ -463,13 +474,16 @@ cudaError_t launch_gather(const uint16_t *x, const float *topk_w, const int32_t 
                           uint16_t *x_perm, float *w_perm, int num_sms, uint32_t *err, cudaStream_t stream,
                           float *y_zero, uint32_t *amax_x, uint32_t *amax_h)
 {
-    // one warp per token, 8 warps per block, at most 8 blocks per SM
-    const int64_t blocks_needed = (static_cast<int64_t>(T) + 7) / 8;
+    // one warp per token (or per slot), 8 warps per block, at most 8 blocks per SM
+    const bool per_slot = T < kGatherPerTokenT;
+    const int64_t units = per_slot ? static_cast<int64_t>(T) * k : T;
+    const int64_t blocks_needed = (units + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms) * 8;
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-    gather_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(x), topk_w, slot_of, T, k, H / 8,
-                                            reinterpret_cast<uint4 *>(x_perm), w_perm,
-                                            reinterpret_cast<uint4 *>(y_zero), H / 4, amax_x, amax_h, err);
+    auto kernel = per_slot ? gather_kernel<true> : gather_kernel<false>;
+    kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(x), topk_w, slot_of, T, k, H / 8,
+                                     reinterpret_cast<uint4 *>(x_perm), w_perm, reinterpret_cast<uint4 *>(y_zero),
+                                     H / 4, amax_x, amax_h, err);
     return cudaGetLastError();
 }
 

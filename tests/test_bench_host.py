@@ -117,3 +117,12 @@ def test_kernels_per_step():
     assert bench.kernels_per_step(s35, router=False) == 5
     assert bench.kernels_per_step(s35, fp8=True) == 9  # shared expert on the BF16 pair kernels
     assert bench.kernels_per_step(dec, fp8=True) == 6
+
+
+def test_gate_up_kernel_name_follows_the_library_configuration():
+    assert bench.gate_up_kernel_name(WORKLOADS["step5_skewed"]) == "gate_up_pair_kernel"
+    assert bench.gate_up_kernel_name(WORKLOADS["step35_decode"]) == "gate_up_kernel"
+    assert bench.gate_up_kernel_name(WORKLOADS["step35_decode"], fp8=True) == "gemm_fp8_mma_kernel<GateUpArgs>"
+    assert bench.gate_up_kernel_name(WORKLOADS["step35_prefill"], fp8=True) == "gemm_fp8_kernel<GateUpArgs>"
+    odd = WORKLOADS["step35_decode"].replace(Is=192)
+    assert bench.gate_up_kernel_name(odd, fp8=True) == "gemm_fp8_kernel<GateUpArgs>"
