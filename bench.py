@@ -302,16 +302,23 @@ def _strip_comments(src: str) -> str:
     return "\n".join(l.strip() for l in "".join(out).splitlines() if l.strip())
 
 
+# Sources of the BF16 forward path up to and including the grouped GEMMs (launch sequence and
+# configuration, permutation and gather, GEMM kernels and their helpers): the files whose
+# code decides the gate_up kernel's DRAM traffic. The router, the FP8 kernels and the
+# backward pass are not among them.
+TRAFFIC_SOURCES = ("moe_api.cu", "internal.h", "permute.cu", "expert_gemm.cu", "expert_gemm_pair.cu",
+                   "epilogue.cuh", "gemm_common.cuh", "sm100.cuh")
+
+
 def csrc_digest() -> str:
-    """Digest of the kernel sources' code (comments excluded), which the profiled traffic
+    """Digest of the code (comments excluded) of TRAFFIC_SOURCES, which the profiled traffic
     figures are tied to."""
     import hashlib
     d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "sparse_moe_layer_biased_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(d, name), encoding="utf-8") as f:
-                h.update(name.encode() + b"\0" + _strip_comments(f.read()).encode())
+    for name in sorted(TRAFFIC_SOURCES):
+        with open(os.path.join(d, name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + _strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

@@ -126,3 +126,9 @@ def test_gate_up_kernel_name_follows_the_library_configuration():
     assert bench.gate_up_kernel_name(WORKLOADS["step35_prefill"], fp8=True) == "gemm_fp8_kernel<GateUpArgs>"
     odd = WORKLOADS["step35_decode"].replace(Is=192)
     assert bench.gate_up_kernel_name(odd, fp8=True) == "gemm_fp8_kernel<GateUpArgs>"
+
+
+def test_traffic_sources_exist():
+    d = os.path.join(ROOT, "sparse_moe_layer_biased_b200", "csrc")
+    for name in bench.TRAFFIC_SOURCES:
+        assert os.path.exists(os.path.join(d, name)), name
