@@ -212,3 +212,25 @@ def test_fp8_decode_scales_are_applied_per_block():
     y2, _, _ = _forward(sh, dev, det=True)
     r1, r2 = _oracle(sh, inp), _oracle(sh, inp2)
     check_output(y2 - y1, r2["y"] - r1["y"], "decode scale delta")
+
+
+def test_fp8_decode_extreme_codes():
+    """FP8 tensor-core decode path on codes at the ends of the E4M3 range: the largest
+    finite magnitudes (448, codes 0x7e / 0xfe), every subnormal code (0x01..0x07 and their
+    negatives) and zeros, mixed into the drawn weights, against the oracle's exact decode."""
+    sh = SHAPES["decode_h768"]
+    inp = draw_fp8(sh)
+    gen = torch.Generator().manual_seed(60)
+    special = torch.tensor([0x7E, 0xFE, 0x00, 0x80] + list(range(0x01, 0x08)) + list(range(0x81, 0x88)),
+                           dtype=torch.uint8)
+    for key in ("W_gate_up_q", "W_down_q"):
+        q = inp[key].clone()
+        mask = torch.rand(q.shape, generator=gen) < 0.05
+        pick = torch.randint(0, special.numel(), q.shape, generator=gen)
+        q[mask] = special[pick[mask]]
+        inp[key] = q
+    y, idx, w = _forward(sh, {k: v.cuda() for k, v in inp.items()})
+    ref = _oracle(sh, inp)
+    keep = check_routing(idx, w, ref, sh.E, sh.k)
+    rf, ma = check_output(y[keep], ref["y"][keep], "extreme codes")
+    print(f"decode_h768 extreme codes: rel_fro {rf:.2e} max_abs {ma:.2e}")
