@@ -329,9 +329,13 @@ cudaError_t launch_bwd_dwr(const uint16_t *x_pad, const float *dl_pad, const int
 namespace {
 
 constexpr int kBwdThreads = 192;
-// the DH kernel carries one more warp: it zeroes the weight gradients of routed experts that
-// received no tokens (no weight-gradient tile writes them) while the GEMM streams W_down
-constexpr int kBwdThreadsDH = kBwdThreads + 32;
+// The DH kernel has eight epilogue warps (its per-element SwiGLU derivative work is the
+// longest epilogue; the two warps of a lane quarter take alternate 16-column blocks) and one
+// more warp that zeroes the weight gradients of routed experts that received no tokens (no
+// weight-gradient tile writes them) while the GEMM streams W_down.
+constexpr int kBwdDhHalves = 2;
+constexpr int kBwdDhEpiWarps = 4 * kBwdDhHalves;
+constexpr int kBwdThreadsDH = 32 * (2 + kBwdDhEpiWarps + 1);
 constexpr uint32_t kBwdZeroBytes = 2048;  // zero source of those bulk stores
 constexpr int kBwdStages = 6;  // stages of 32 KB (the ring region's size in those units)
 constexpr int kBwdBN = 128;    // output columns of a weight-gradient tile
@@ -345,10 +349,12 @@ constexpr uint32_t kBwdMiscOff = kBwdBarOff + 8 * (2 * kBwdStages + 5);
 constexpr uint32_t kBwdEpiOff = (kBwdMiscOff + 16 + 1023) / 1024 * 1024;
 constexpr uint32_t kBwdEpiBox = 32 * 32 * 4;
 constexpr uint32_t kBwdEpiWarp = 2 * kBwdEpiBox;
-static_assert(32 * 33 * 4 <= kBwdEpiWarp, "transpose buffer");
-// the zero source sits in the unused end of epilogue warp 0's area in the DH mode
-constexpr uint32_t kBwdZeroOff = kBwdEpiOff + kBwdEpiWarp - kBwdZeroBytes;
-static_assert(32 * 33 * 4 <= kBwdEpiWarp - kBwdZeroBytes, "zero source overlaps the transpose buffer");
+// DH: a 32 x 17 fp32 transpose buffer per epilogue warp, and the zero source at the end of
+// the epilogue area
+constexpr uint32_t kBwdDhTr = 2304;
+constexpr uint32_t kBwdZeroOff = kBwdEpiOff + 4 * kBwdEpiWarp - kBwdZeroBytes;
+static_assert(32 * 17 * 4 <= kBwdDhTr, "transpose buffer");
+static_assert(kBwdDhEpiWarps * kBwdDhTr <= 4 * kBwdEpiWarp - kBwdZeroBytes, "zero source overlaps the transpose buffers");
 constexpr uint32_t kBwdSmem = kBwdEpiOff + 4 * kBwdEpiWarp + 1024;
 static_assert(kBwdSmem <= kMaxDynSmem, "backward ring exceeds shared memory");
 
@@ -471,12 +477,12 @@ __device__ __forceinline__ void bwd_load(const BwdArgs &a, const CUtensorMap *ma
     }
 }
 
-// Epilogue of one tile for one warp (TMEM lane quarter q; lane row = q*32 + lane of M).
-// om = tensor map of the tile's weight-gradient output (WD / WGU), 32 x 32 fp32 boxes with
+// Epilogue of one tile for one warp (TMEM lane quarter q; lane row = q*32 + lane of M; in DH
+// the warp's half of the column blocks). om = tensor map of the tile's weight-gradient output (WD / WGU), 32 x 32 fp32 boxes with
 // 128-byte swizzle; tr = this warp's staging area (kBwdEpiWarp bytes, 1024-byte aligned).
 template <int MODE>
-__device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, const BTile &t, int q, int lane,
-                                             float *tr, const CUtensorMap *om)
+__device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, const BTile &t, int q, int half,
+                                             int lane, float *tr, const CUtensorMap *om)
 {
     const int row = q * 32 + lane;
     const uint32_t tq = tacc + (static_cast<uint32_t>(q * 32) << 16);
@@ -510,25 +516,26 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
             }
         }
     } else if (MODE == kBwdDH) {
+        // blocks of 16 columns; the two warps of a lane quarter take alternate blocks
         const int64_t i = t.mb * 128 + row;
         const float *gu = t.sh ? a.gu_s : a.gu_r;
         uint16_t *dgu = t.sh ? a.dgu_s : a.dgu_r;
         const float L = t.sh ? a.lim_s : a.lim_r;
-        for (int cb = 0; cb < t.ntok; cb += 32) {
-            float v[32], gg[32], uu[32];
-            tmem_load32(tq + cb, v);
-            const int ncol = t.ntok - cb < 32 ? t.ntok - cb : 32;
-            // lane c: routing weight of column cb + c (read by shuffle below)
+        for (int cb = 16 * half; cb < t.ntok; cb += 16 * kBwdDhHalves) {
+            float v[16], gg[16], uu[16];
+            tmem_load16(tq + cb, v);
+            const int ncol = t.ntok - cb < 16 ? t.ntok - cb : 16;
+            // lane c < 16: routing weight of column cb + c (read by shuffle below)
             const float wl = t.sh || lane >= ncol ? 1.0f : a.w_pad[t.row0 + cb + lane];
-            // all 64 pre-activation loads of the block in flight before any use
+            // all 32 pre-activation loads of the block in flight before any use
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int c = 0; c < 16; ++c) {
                 const int64_t rr = rs + cb + (c < ncol ? c : 0);
                 gg[c] = gu[rr * 2 * Iw + i];
                 uu[c] = gu[rr * 2 * Iw + Iw + i];
             }
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int c = 0; c < 16; ++c) {
                 if (c >= ncol)  // uniform across the warp
                     break;
                 const int64_t rr = rs + cb + c;
@@ -553,7 +560,7 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
                 }
                 const float dhu = v[c];
                 if (!t.sh)
-                    tr[lane * 33 + c] = ac * uc * dhu;  // this lane's term of h . dhu for column c
+                    tr[lane * 17 + c] = ac * uc * dhu;  // this lane's term of h . dhu for column c
                 const float dh = __shfl_sync(0xFFFFFFFFu, wl, c) * dhu;
                 const float dg = dh * uc * ma * sg * (1.0f + g * (1.0f - sg));
                 const float du = dh * ac * mu;
@@ -569,7 +576,7 @@ __device__ __forceinline__ void bwd_epilogue(const BwdArgs &a, uint32_t tacc, co
                     float sum = 0.0f;
 #pragma unroll
                     for (int r = 0; r < 32; ++r)
-                        sum += tr[r * 33 + lane];
+                        sum += tr[r * 17 + lane];
                     atomicAdd(a.dw_pad + t.row0 + cb + lane, sum);
                 }
                 __syncwarp();
@@ -651,7 +658,7 @@ __device__ __forceinline__ void bwd_zero_untouched(const BwdArgs &a, const uint8
 }
 
 template <int MODE, int NSL>
-__global__ void __launch_bounds__(kBwdThreadsDH, 1)
+__global__ void __launch_bounds__(MODE == kBwdDH ? kBwdThreadsDH : kBwdThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap a_r, const __grid_constant__ CUtensorMap a_s,
                     const __grid_constant__ CUtensorMap b_r, const __grid_constant__ CUtensorMap b_s,
                     const __grid_constant__ CUtensorMap o_r, const __grid_constant__ CUtensorMap o_s,
@@ -683,7 +690,7 @@ __global__ void __launch_bounds__(kBwdThreadsDH, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accf[b], 1);
-            mbar_init(&acce[b], 4);
+            mbar_init(&acce[b], MODE == kBwdDH ? kBwdDhEpiWarps : 4);  // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -770,7 +777,7 @@ __global__ void __launch_bounds__(kBwdThreadsDH, 1)
             umma_commit(drain);
             mbar_wait_drain(drain, 0, wc);
         }
-    } else if (warp == 6) {
+    } else if (MODE == kBwdDH && warp == 2 + kBwdDhEpiWarps) {
         // DH only: zero the gradients of untouched experts
         uint8_t *zero = smem + kBwdZeroOff;
         for (uint32_t i = lane * 16; i < kBwdZeroBytes; i += 32 * 16)
@@ -782,6 +789,9 @@ __global__ void __launch_bounds__(kBwdThreadsDH, 1)
         __syncwarp();
     } else {
         const int q = warp & 3;
+        const int half = (warp - 2) >> 2;  // DH: which of the lane quarter's two warps
+        float *tr = reinterpret_cast<float *>(smem + kBwdEpiOff +
+                                              (MODE == kBwdDH ? (warp - 2) * kBwdDhTr : q * kBwdEpiWarp));
         int tc = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
             const BTile t = bwd_tile<MODE>(a, tile);
@@ -789,8 +799,7 @@ __global__ void __launch_bounds__(kBwdThreadsDH, 1)
             if (!warp_wait(&accf[buf], (tc >> 1) & 1, wc, abort_flag))
                 break;
             tc_fence_after();
-            bwd_epilogue<MODE>(a, tmem + buf * kBwdAcc, t, q, lane,
-                               reinterpret_cast<float *>(smem + kBwdEpiOff + q * kBwdEpiWarp), t.sh ? &o_s : &o_r);
+            bwd_epilogue<MODE>(a, tmem + buf * kBwdAcc, t, q, half, lane, tr, t.sh ? &o_s : &o_r);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
