@@ -217,8 +217,9 @@ def test_fp8_decode_scales_are_applied_per_block():
 def test_fp8_decode_extreme_codes():
     """FP8 tensor-core decode path on codes at the ends of the E4M3 range: the largest
     finite magnitudes (448, codes 0x7e / 0xfe), every subnormal code (0x01..0x07 and their
-    negatives) and zeros, mixed into the drawn weights, against the oracle's exact decode."""
-    sh = SHAPES["decode_h768"]
+    negatives) and zeros, mixed into the drawn weights, against the oracle's exact decode
+    (routed clip off, so the routed experts carry most of the output)."""
+    sh = SHAPES["decode_h768"].replace(limit_routed=0.0)
     inp = draw_fp8(sh)
     gen = torch.Generator().manual_seed(60)
     special = torch.tensor([0x7E, 0xFE, 0x00, 0x80] + list(range(0x01, 0x08)) + list(range(0x81, 0x88)),
