@@ -25,11 +25,15 @@
 // The shared expert (BF16) runs in the same kernel: its stages are 64 K of bf16 weights for
 // both blocks and one bf16 token slice, multiplied by kind::f16 MMAs as they land.
 //
+// Each stage's token slices and weight boxes land on barriers of their own, and the token
+// slices are requested first: the prep warps start on a stage as soon as its token rows are
+// in, while its weights are still on the way.
+//
 // Roles per CTA (persistent, one CTA per SM, static round-robin over tiles):
-//   warp 0       producer: two weight boxes + token slices per stage
+//   warp 0       producer: token slices + two weight boxes per stage
 //   warp 1       MMA issuer and TMEM owner (2 accumulator buffers x 2 blocks x 64 columns)
 //   warps 2..5   epilogue (TMEM lane quarter warp % 4)
-//   warps 6..9   token prep: the E4M3 hi/lo B operands of routed stages
+//   warps 6..    token prep (kF8Prep warps): the E4M3 hi/lo B operands of routed stages
 // Every wait is bounded; on expiry the CTA drains its own copies and MMAs, frees TMEM and
 // returns with the device error word set.
 #include <cuda_bf16.h>
@@ -41,7 +45,8 @@
 namespace moe {
 namespace {
 
-constexpr int kF8Threads = 320;
+constexpr int kF8Prep = 8;                                    // token-prep warps (4 or 8)
+constexpr int kF8Threads = 32 * (6 + kF8Prep);
 constexpr int kF8BN = 32;                                     // token rows per chunk (decode cap)
 constexpr int kF8S = 4;                                       // ring stages
 constexpr uint32_t kF8WBox = 128 * 128;                       // weight box: 128 rows x 128 bytes
@@ -51,19 +56,20 @@ constexpr uint32_t kF8TokOff = 2 * kF8WBox;                   // slot: weight bo
 constexpr uint32_t kF8BOff = kF8TokOff + 2 * kF8TokSl;
 constexpr uint32_t kF8Slot = kF8BOff + 2 * kF8BOp;
 constexpr uint32_t kF8BarOff = kF8S * kF8Slot;
-constexpr uint32_t kF8NumBars = 3 * kF8S + 5;
+constexpr uint32_t kF8NumBars = 4 * kF8S + 5;
 constexpr uint32_t kF8MiscOff = kF8BarOff + 8 * kF8NumBars;
 constexpr uint32_t kF8Smem = kF8MiscOff + 16 + 1024;
 constexpr uint32_t kF8AccCols = 2 * kF8BN;                    // one block's accumulator (hi, lo columns)
 constexpr uint32_t kF8BufCols = 2 * kF8AccCols;               // one buffer: two blocks
 constexpr uint32_t kF8TmemCols = 2 * kF8BufCols;
-constexpr int kF8Prep = 4;                                    // token-prep warps
+static_assert(kF8Prep == 4 || kF8Prep == 8, "one or two prep warps per lane quarter");
 static_assert(kF8Slot % 1024 == 0 && kF8BOff % 1024 == 0, "operands stay 1024-byte aligned");
 static_assert(kF8Smem <= static_cast<uint32_t>(kMaxDynSmem), "ring exceeds shared memory");
 static_assert(kF8TmemCols == 256, "TMEM allocation is a power of two");
 
 struct RingF8 {
-    uint64_t *full, *empty, *conv, *accf, *acce, *drain;
+    uint64_t *wfull, *tfull;  // a stage's weight boxes / token slices landed
+    uint64_t *empty, *conv, *accf, *acce, *drain;
     uint32_t *holder;
     volatile int *abort_flag;
 };
@@ -72,8 +78,9 @@ __device__ __forceinline__ uint8_t *ringf8_setup(uint8_t *smem_raw, RingF8 &r)
 {
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *smem = smem_raw + pad;
-    r.full = reinterpret_cast<uint64_t *>(smem + kF8BarOff);
-    r.empty = r.full + kF8S;
+    r.wfull = reinterpret_cast<uint64_t *>(smem + kF8BarOff);
+    r.tfull = r.wfull + kF8S;
+    r.empty = r.tfull + kF8S;
     r.conv = r.empty + kF8S;
     r.accf = r.conv + kF8S;
     r.acce = r.accf + 2;
@@ -82,7 +89,8 @@ __device__ __forceinline__ uint8_t *ringf8_setup(uint8_t *smem_raw, RingF8 &r)
     r.abort_flag = reinterpret_cast<volatile int *>(smem + kF8MiscOff + 4);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kF8S; ++s) {
-            mbar_init(&r.full[s], 1);
+            mbar_init(&r.wfull[s], 1);
+            mbar_init(&r.tfull[s], 1);
             mbar_init(&r.empty[s], 1);
             mbar_init(&r.conv[s], kF8Prep);  // one arrival per prep warp
         }
@@ -411,20 +419,23 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                     uint8_t *slot = smem + s * kF8Slot;
                     const int nsl = t.sh ? 1 : 2;  // 64-wide token slices of the stage
                     const int k0 = st * (t.sh ? 64 : 128);
-                    mbar_arrive_expect_tx(&r.full[s], 2 * kF8WBox + nsl * kF8TokSl);
-                    for (int b = 0; b < 2; ++b)
-                        load_wbox(a, t.sh ? &m_wsh : &m_w, slot + b * kF8WBox, &r.full[s], t, b, k0);
+                    mbar_arrive_expect_tx(&r.tfull[s], nsl * kF8TokSl);
                     for (int sl = 0; sl < nsl; ++sl)
-                        tma_load_2d(slot + kF8TokOff + sl * kF8TokSl, t.sh ? &m_tok_sh : &m_tok, &r.full[s],
+                        tma_load_2d(slot + kF8TokOff + sl * kF8TokSl, t.sh ? &m_tok_sh : &m_tok, &r.tfull[s],
                                     k0 + sl * 64, t.row0);
+                    mbar_arrive_expect_tx(&r.wfull[s], 2 * kF8WBox);
+                    for (int b = 0; b < 2; ++b)
+                        load_wbox(a, t.sh ? &m_wsh : &m_w, slot + b * kF8WBox, &r.wfull[s], t, b, k0);
                 }
             }
-            drain_f8(r.full, kF8S, it, wc);
+            drain_f8(r.tfull, kF8S, it, wc);
+            drain_f8(r.wfull, kF8S, it, wc);
         }
     } else if (warp == 1) {
         // MMA: routed stages multiply the E4M3 weight boxes by the hi/lo B operands (N = 2n),
         // shared stages the bf16 weight boxes by the bf16 token slice (N = n). The prep warps
-        // arrive on conv after the stage's bytes landed, so conv alone gates the stage.
+        // arrive on conv after the stage's token rows landed; the weights have a barrier of
+        // their own.
         if (lane == 0) {
             int it = 0, tc = 0;
             bool ok = true;
@@ -440,7 +451,8 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                 const int nst = t.stages();
                 for (int st = 0; st < nst; ++st, ++it) {
                     const int s = it % kF8S;
-                    if (!mbar_wait(&r.conv[s], (it / kF8S) & 1, wc, r.abort_flag)) {
+                    if (!mbar_wait(&r.conv[s], (it / kF8S) & 1, wc, r.abort_flag) ||
+                        !mbar_wait(&r.wfull[s], (it / kF8S) & 1, wc, r.abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -483,25 +495,28 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                 mbar_arrive(&r.acce[buf]);
         }
     } else {
-        // token prep: warps 6..9; thread p handles 16-K chunk c = p % 8 of rows p / 8 and
-        // p / 8 + 16 for both blocks
+        // token prep: warps 6 ..; thread p handles 16-K chunk c = p % 8 of rows j0 = (p / 8) % 16
+        // and j0 + 16, for both blocks (four prep warps) or for block p / 128 (eight)
         const int p = threadIdx.x - 6 * 32;
-        const int c = p & 7, j0 = p >> 3;
+        const int c = p & 7, j0 = (p >> 3) & 15;
+        constexpr int kBlocksPer = 8 / kF8Prep;
+        const int bfirst = kF8Prep == 8 ? (p >> 7) : 0;
         int it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
             const TileF8 t = tile_f8(a, tile);
             const int n = t.npad();
             const int nst = t.stages();
-            // per tile: 2^-e_b of both blocks, 2^(6 - e_j) of this thread's rows (0 past the chunk)
-            float pb0 = 0.0f, pb1 = 0.0f, f0 = 0.0f, f1 = 0.0f;
-            const float *s0 = nullptr, *s1 = nullptr;
+            // per tile: 2^-e_b of this thread's blocks, 2^(6 - e_j) of its rows (0 past the chunk)
+            float pb[kBlocksPer], f0 = 0.0f, f1 = 0.0f;
+            const float *sr[kBlocksPer];
             if (!t.sh) {
                 const int nkb = t.K / 128;
-                s0 = scale_row(a, t, 0);
-                s1 = scale_row(a, t, 1);
-                pb0 = pow2i(-block_exp(s0, nkb, lane));
-                pb1 = pow2i(-block_exp(s1, nkb, lane));
+#pragma unroll
+                for (int q = 0; q < kBlocksPer; ++q) {
+                    sr[q] = scale_row(a, t, bfirst + q);
+                    pb[q] = pow2i(-block_exp(sr[q], nkb, lane));
+                }
                 const uint32_t *am = row_amax(a);
                 if (j0 < t.ntok)
                     f0 = pow2i(6 - exp_of(am[t.row0 + j0]));
@@ -510,20 +525,20 @@ __global__ void __launch_bounds__(kF8Threads, 1)
             }
             for (int st = 0; st < nst; ++st, ++it) {
                 const int s = it % kF8S;
-                if (!warp_wait(&r.full[s], (it / kF8S) & 1, wc, r.abort_flag)) {
+                if (!warp_wait(&r.tfull[s], (it / kF8S) & 1, wc, r.abort_flag)) {
                     ok = false;
                     break;
                 }
                 if (!t.sh) {
                     uint8_t *slot = smem + s * kF8Slot;
                     const uint8_t *tok = slot + kF8TokOff;
-                    const float sb0 = __ldg(s0 + st) * pb0;
-                    const float sb1 = __ldg(s1 + st) * pb1;
-                    prep_chunk(tok, j0, c, sb0 * f0, slot + kF8BOff, n);
-                    prep_chunk(tok, j0, c, sb1 * f0, slot + kF8BOff + kF8BOp, n);
-                    if (n > 16) {
-                        prep_chunk(tok, j0 + 16, c, sb0 * f1, slot + kF8BOff, n);
-                        prep_chunk(tok, j0 + 16, c, sb1 * f1, slot + kF8BOff + kF8BOp, n);
+#pragma unroll
+                    for (int q = 0; q < kBlocksPer; ++q) {
+                        const float sb = __ldg(sr[q] + st) * pb[q];
+                        uint8_t *bop = slot + kF8BOff + (bfirst + q) * kF8BOp;
+                        prep_chunk(tok, j0, c, sb * f0, bop, n);
+                        if (n > 16)
+                            prep_chunk(tok, j0 + 16, c, sb * f1, bop, n);
                     }
                     fence_proxy_async_smem();  // the B operands are read by the tensor cores
                 }
