@@ -486,7 +486,8 @@ cudaError_t launch8(int grid, cudaStream_t stream, const CUtensorMap &m0, const 
 
 }  // namespace
 
-// Decode-sized calls: 32-row chunks; stages of two scale blocks (256 K: 16 MMAs per barrier
+// Decode-sized calls whose shapes the FP8 tensor-core kernels do not take (H not a multiple of
+// 256, or I, Is not multiples of 128): 32-row chunks; stages of two scale blocks (256 K: 16 MMAs per barrier
 // test and commit of the MMA thread), staging slots of 48 KB (32 KB weights + four 4 KB token
 // slices), 4 deep; 3 TMEM operand slots of 128 columns.
 // Prefill: 128-row chunks; stages of one scale block, 48 KB staging slots, 4 deep; 4 TMEM
