@@ -117,7 +117,7 @@ def _worker(rank, world, port, out):
 @pytest.mark.parametrize("world", [2, 4])
 def test_ep_exchange_reproduces_the_layer(world):
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
