@@ -38,6 +38,11 @@ SHAPES = {
     # gate/up, 3 down tiles of 256 rows, 2 shared feature blocks, chunks of 16 and 32 rows
     "decode_h768": LayerShape("fp8_decode_h768", T=40, H=768, E=24, k=6, I=256, Is=256, limit_routed=0.25,
                               seed=58, weight_std=0.03),
+    # FP8 tensor-core edge cases: a single token (every chunk one row, 15 padding rows of the
+    # 16-row operand), and every expert selected by every token (k = E)
+    "one_token": LayerShape("fp8_one_token", T=1, H=256, E=8, k=2, I=128, Is=128, seed=61, weight_std=0.03),
+    "all_experts": LayerShape("fp8_all_experts", T=5, H=512, E=8, k=8, I=256, Is=128, limit_routed=0.25,
+                              seed=62, weight_std=0.03),
     # prefill-sized: 128-row chunks, several K blocks, ragged chunk tails, Is not a multiple of 128
     "prefill": LayerShape("fp8_prefill", T=300, H=512, E=12, k=4, I=256, Is=192, limit_routed=0.25,
                           limit_shared=0.125, seed=52, weight_std=0.03),
