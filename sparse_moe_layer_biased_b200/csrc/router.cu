@@ -13,9 +13,11 @@
 // memory (the idle ring). After a cluster barrier each CTA takes a share of the tile's tokens:
 // one warp per token sums the S partials of each expert through distributed shared memory in
 // rank order (a fixed order: the logits do not depend on timing), applies the sigmoid and the
-// bias, and selects the top k by k+1 rounds of a warp-wide maximum over sortable keys (biased
-// score, then lower expert index), which also gives the (k+1)-th for the margin. No logits
-// reach global memory. S (1, 2, 4 or 8) is chosen so the grid covers the SMs about once.
+// bias, and selects the top k by k+1 rounds of a warp-wide maximum over sortable 32-bit score
+// keys (ties to the lower expert index: first within a lane, then across lanes by a second
+// reduction that runs only when two lanes hold the maximum), which also gives the (k+1)-th for
+// the margin. Lane l holds experts l, l + 32, ... (KPL of them, E <= 32 KPL). No logits reach
+// global memory. S (1, 2, 4 or 8) is chosen so the grid covers the SMs about once.
 #include "internal.h"
 
 namespace moe {
@@ -29,7 +31,6 @@ constexpr int kTileM = 128;
 constexpr int kBK = 64;                         // bf16 elements per 128-byte swizzled row
 constexpr uint32_t kABytes = kTileM * kBK * 2;  // 16 KB
 constexpr int kMaxStages = 8;
-constexpr int kMaxKeysPerLane = 16;             // E <= 512 experts over 32 lanes
 
 // Shared-memory layout for E_pad experts (a multiple of 16): a ring of stages (x tile +
 // Wr rows of every expert), its barriers, and after the main loop the partial logits
@@ -58,42 +59,26 @@ struct Layout {
     }
 };
 
-// Rank key of a biased score: larger key = ranked earlier. Order: value descending
-// (-0 equal to +0), a NaN below every number, ties to the lower expert index. Key 0
-// (an empty list entry) ranks below every real entry.
-__device__ __forceinline__ uint64_t rank_key(float b, int e)
+// Rank key of a biased score: larger key = ranked earlier. Order: value descending (-0 equal
+// to +0), a NaN below every number; key 0 is an empty entry (an expert past E, or one already
+// selected) and ranks below every real entry. A number's key is its order-preserving unsigned
+// image plus one (at most 0xFF800001 for +inf), a NaN's key is 1.
+__device__ __forceinline__ uint32_t rank_key(float b)
 {
-    uint32_t u;
-    if (b != b) {
-        u = 0u;
-    } else {
-        u = (b == 0.0f) ? 0u : __float_as_uint(b);
-        u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    }
-    return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
+    if (b != b)
+        return 1u;
+    uint32_t u = (b == 0.0f) ? 0u : __float_as_uint(b);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return u + 1u;
 }
 
-__device__ __forceinline__ float key_value(uint64_t key)
+__device__ __forceinline__ float key_value(uint32_t key)
 {
-    const uint32_t u = static_cast<uint32_t>(key >> 32);
+    const uint32_t u = key - 1u;
     return __uint_as_float((u & 0x80000000u) ? (u ^ 0x80000000u) : ~u);
 }
 
-__device__ __forceinline__ int key_expert(uint64_t key)
-{
-    return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
-}
-
-// Warp-wide maximum of 64-bit rank keys (unique per expert): the larger high word (biased
-// score), then among lanes holding it the larger low word (lower expert index).
-__device__ __forceinline__ uint64_t warp_max_key(uint64_t key)
-{
-    const uint32_t hi = static_cast<uint32_t>(key >> 32), lo = static_cast<uint32_t>(key);
-    const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
-    const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
-    return (static_cast<uint64_t>(mhi) << 32) | mlo;
-}
-
+template <int KPL>
 __global__ void __launch_bounds__(kThreads, 1)
     router_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wr,
                   const RouterArgs a, const int e_pad, const WaitCfg wc)
@@ -236,17 +221,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int p = 0; p < 8; ++p)
             peer[p] = peer_ptr(part, static_cast<uint32_t>(p < S ? p : 0));
         const int rounds = a.k < a.E ? a.k + 1 : a.k;
+        // this lane's experts' biases, the same for every token
+        float bias_r[KPL];
+#pragma unroll
+        for (int i = 0; i < KPL; ++i)
+            bias_r[i] = lane + 32 * i < a.E ? a.bias[lane + 32 * i] : 0.0f;
         for (int tt = rank * per + warp; tt < t_hi; tt += kWarps) {
             const int t = m0 + tt;
             if (t >= a.T)
                 break;
             // lane l holds experts l, l + 32, ...: logit = sum of the S partials in rank order
-            uint64_t key[kMaxKeysPerLane];
-            float sc[kMaxKeysPerLane];
+            uint32_t key[KPL];
+            float sc[KPL];
 #pragma unroll
-            for (int i = 0; i < kMaxKeysPerLane; ++i) {
+            for (int i = 0; i < KPL; ++i) {
                 const int e = lane + 32 * i;
-                key[i] = 0;
+                key[i] = 0u;
                 sc[i] = 0.0f;
                 if (e < a.E) {
                     const int off = tt * static_cast<int>(L.part_stride) + e;
@@ -256,44 +246,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (p < S)
                             l += peer[p][off];
                     const float s = 1.0f / (1.0f + expf(-l));
-                    key[i] = rank_key(s + a.bias[e], e);
+                    key[i] = rank_key(s + bias_r[i]);
                     sc[i] = s;
                 }
             }
             // k (+1 for the margin) rounds of a warp-wide maximum: lane j keeps round j's
-            // expert and score (lane 0 also round 32's key); the normalisation sum and the
-            // margin keys are warp-uniform, accumulated in rank order
+            // expert and score; the normalisation sum and the margin keys are warp-uniform,
+            // accumulated in rank order
             const int k = a.k;
-            uint64_t my_key = 0, key_k = 0, key_k1 = 0;
+            int my_e = 0;
+            uint32_t key_k = 0u, key_k1 = 0u;
             float my_s = 0.0f, sum = 0.0f;
             for (int j = 0; j < rounds; ++j) {
-                uint64_t best = 0;
-                float best_s = 0.0f;
+                // this lane's best entry: highest key, lowest index among equal keys
+                uint32_t best = 0u;
+                int bi = 0;
 #pragma unroll
-                for (int i = 0; i < kMaxKeysPerLane; ++i) {
+                for (int i = 0; i < KPL; ++i) {
                     const bool gt = key[i] > best;
                     best = gt ? key[i] : best;
-                    best_s = gt ? sc[i] : best_s;
+                    bi = gt ? i : bi;
                 }
-                const uint64_t m = warp_max_key(best);
-                const unsigned owner = __ballot_sync(0xFFFFFFFFu, best == m && m != 0);
-                const float ms = __shfl_sync(0xFFFFFFFFu, best_s, owner ? __ffs(owner) - 1 : 0);
-                if (best == m) {
+                const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, best);
+                const unsigned holders = __ballot_sync(0xFFFFFFFFu, best == m && m != 0u);
+                int win = holders ? __ffs(holders) - 1 : 0;
+                if (__popc(holders) > 1) {
+                    // equal keys in several lanes: the lowest expert index wins
+                    const uint32_t ex = (holders >> lane) & 1u ? static_cast<uint32_t>(lane + 32 * bi) : 0xFFFFFFFFu;
+                    const uint32_t emin = __reduce_min_sync(0xFFFFFFFFu, ex);
+                    win = static_cast<int>(emin & 31u);
+                }
+                const int we = __shfl_sync(0xFFFFFFFFu, lane + 32 * bi, win);
+                float ws = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < kMaxKeysPerLane; ++i)
-                        key[i] = key[i] == m ? 0ull : key[i];
+                for (int i = 0; i < KPL; ++i)
+                    ws = i == bi ? sc[i] : ws;
+                ws = __shfl_sync(0xFFFFFFFFu, ws, win);
+                ws = m != 0u ? ws : 0.0f;  // no entry left (cannot happen with k + 1 <= E rounds)
+                if (lane == win && m != 0u) {
+#pragma unroll
+                    for (int i = 0; i < KPL; ++i)
+                        key[i] = i == bi ? 0u : key[i];
                 }
                 if (lane == (j & 31) && j < k) {
-                    my_key = m;
-                    my_s = ms;
+                    my_e = we;
+                    my_s = ws;
                 }
                 if (j < k)
-                    sum += ms;
+                    sum += ws;
                 key_k = j + 1 == k ? m : key_k;
                 key_k1 = j == k ? m : key_k1;
             }
             if (lane < k) {
-                int e = key_expert(my_key);
+                int e = my_e;
                 e = e < 0 ? 0 : (e > a.E - 1 ? a.E - 1 : e);
                 float w;
                 if (a.norm)
@@ -325,7 +330,10 @@ cudaError_t launch_impl(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const
     const RouterSplit sp = router_split(a.E, a.T, a.H, a.num_sms);
     const Layout L(sp.e_pad);
     const int smem = static_cast<int>(L.total) + 1024;
-    cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // keys per lane: the smallest of 4, 8, 12, 16 covering E_pad experts over 32 lanes
+    const int kpl = (sp.e_pad + 31) / 32;
+    auto kernel = kpl <= 4 ? router_kernel<4> : (kpl <= 8 ? router_kernel<8> : (kpl <= 12 ? router_kernel<12> : router_kernel<16>));
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
     cudaLaunchConfig_t cfg = {};
@@ -340,7 +348,7 @@ cudaError_t launch_impl(const CUtensorMap &tm_x, const CUtensorMap &tm_wr, const
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, router_kernel, tm_x, tm_wr, a, sp.e_pad, wc);
+    err = cudaLaunchKernelEx(&cfg, kernel, tm_x, tm_wr, a, sp.e_pad, wc);
     if (err != cudaSuccess)
         return err;
     return cudaGetLastError();
