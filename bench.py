@@ -56,6 +56,8 @@ def parse():
                          "router: time moe_router alone (profiling)")
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
                     help="ep: expert parallelism, E/N routed experts per rank, T tokens per rank")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the forward captured once in a CUDA graph and replayed (key 'graph')")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling runs)")
     return ap.parse_args()
@@ -364,6 +366,35 @@ def gate_up_flops(shape):
     return 4.0 * shape.H * (shape.I * shape.T * shape.k + shape.Is * shape.T)
 
 
+def graph_replay(args, shape, step, x, y, flush_buf, stream, world):
+    """The step captured once in a CUDA graph (the library only enqueues: no allocation or
+    synchronisation inside a call) and replayed K times, each replay between its own CUDA events
+    (the L2 flush of decode-sized workloads stays outside them). Returns the per-step time and
+    the throughput; the launches of the graph are the step's kernels."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        step(x, y)
+    torch.cuda.synchronize()
+    for _ in range(max(1, args.warmup)):
+        g.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    for i in range(args.steps):
+        if flush_buf is not None:
+            flush_buf.fill_(i & 0xFF)
+        evs[i][0].record(cur)
+        g.replay()
+        evs[i][1].record(cur)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), "cuda")
+    del g
+    return {"value": job_tokens_per_s(world, shape.T, args.steps, ms), "unit": UNIT,
+            "ms_per_step": ms / args.steps, "api": "moe_forward captured in one CUDA graph, replayed"}
+
+
 def gate_up_kernel_name(shape, fp8=False):
     """The gate_up kernel one call launches (the library's configuration choice)."""
     decode = shape.T * shape.k <= 16 * shape.E
@@ -592,6 +623,8 @@ def run_b200(args, shape):
         "e2e": e2e,
         "gpu_launches": kernels_per_step(shape, fp8, args.deterministic, args.routing != "balanced") * args.steps,
     }
+    if args.graph:
+        line["graph"] = graph_replay(args, shape, step, x, y, flush_buf, stream, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         # one more forward in the timed launch configuration: the oracle's sample doubles
         # as a parity check of the timed path
