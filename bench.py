@@ -278,6 +278,9 @@ PROFILED_TRAFFIC = {
     ("step5_skewed", "bf16"): {"ratio": (1451889152 + 53718016) / 1205862400,
                                "csrc_sha256": "f484c73fd3a47ce5ddf47b43a5d825b0623c71bff92437973550e4d645de4ca8",
                                "source": "profiles/dram_gate_up_down_step5_skewed_T2048_E44.md"},
+    ("step35_prefill", "bf16"): {"ratio": (1624338432 + 23043328) / 1562902528,
+                                 "csrc_sha256": "f484c73fd3a47ce5ddf47b43a5d825b0623c71bff92437973550e4d645de4ca8",
+                                 "source": "profiles/dram_gate_up_down_step35_prefill_T1024_E72.md"},
 }
 
 
