@@ -81,7 +81,11 @@ class ClockSampler:
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
                ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
-               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+               # informative only (a clock lock or an application-clock setting shows here)
+               ("applications_clocks_setting", "nvmlClocksEventReasonApplicationsClocksSetting"),
+               ("sync_boost", "nvmlClocksEventReasonSyncBoost"),
+               ("display_clock_setting", "nvmlClocksEventReasonDisplayClockSetting"))
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -101,7 +105,7 @@ class ClockSampler:
             pynvml.nvmlInit()
             handle = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
             smax = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
-            masks = [(name, getattr(pynvml, attr)) for name, attr in self.REASONS]
+            masks = [(name, getattr(pynvml, attr, 0)) for name, attr in self.REASONS]
         except Exception:
             self._start_smi()
             return
