@@ -200,8 +200,9 @@ MOE_API moe_status_t moe_host_workspace_size(const moe_layer_desc *desc, size_t 
  *   the E4M3 codes, as in moe_forward_fp8); both NULL or both given.
  *   Other weights, desc and the routing as in moe_forward; ws of at least
  *   moe_host_workspace_size.
- * The copies run on two internal streams, double-buffered in ws: batch i+1's input copy
- * and batch i-1's output copy overlap batch i's forward on `stream`. The call only enqueues
+ * The copies run on internal streams, double-buffered in ws: batch i+1's input copy (one
+ * stream) and batch i-1's output copy (two halves on two streams) overlap batch i's forward
+ * on `stream`. The call only enqueues
  * work; when `stream` has completed, every output row is in y_host. n_batches = 0 or T = 0
  * is a no-op. */
 MOE_API moe_status_t moe_forward_host(const moe_layer_desc *desc, int32_t n_batches, const uint16_t *x_host,

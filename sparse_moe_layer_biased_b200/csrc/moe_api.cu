@@ -693,24 +693,30 @@ moe_status_t moe_forward_host(const moe_layer_desc *desc, int32_t n_batches, con
     float *yd[2] = {at<float>(ws, L.y0), at<float>(ws, L.y1)};
 
     // copy streams and the events that order them against the compute stream s; streams and
-    // events are released by the runtime once their pending work completes
-    cudaStream_t h2d = nullptr, d2h = nullptr;
-    cudaEvent_t ev[7] = {};  // start, h2d done x2, compute done x2, d2h done x2
+    // events are released by the runtime once their pending work completes. The output copy
+    // of a batch is split in two halves on two streams: one device-to-host copy ran at ~44 GB/s
+    // on a B200, two concurrent halves at ~57 GB/s (host-to-device: ~55 GB/s either way).
+    cudaStream_t h2d = nullptr, d2h[2] = {nullptr, nullptr};
+    cudaEvent_t ev[9] = {};  // start, h2d done x2, compute done x2, d2h done x2 per half
     bool ok = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) == cudaSuccess;
-    for (int i = 0; ok && i < 7; ++i)
+              cudaStreamCreateWithFlags(&d2h[0], cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&d2h[1], cudaStreamNonBlocking) == cudaSuccess;
+    for (int i = 0; ok && i < 9; ++i)
         ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
-    cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_comp = ev + 3, *ev_out = ev + 5;
+    cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_comp = ev + 3, *ev_out = ev + 5;  // ev_out[2 * b + half]
     // the copies start after the work already queued on s
     ok = ok && cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(h2d, ev_start, 0) == cudaSuccess &&
-         cudaStreamWaitEvent(d2h, ev_start, 0) == cudaSuccess;
+         cudaStreamWaitEvent(d2h[0], ev_start, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(d2h[1], ev_start, 0) == cudaSuccess;
+    const size_t rows0 = static_cast<size_t>(desc->T) / 2;  // rows of the first output half
     st = ok ? MOE_OK : MOE_ERR_CUDA;
     for (int i = 0; st == MOE_OK && i < n_batches; ++i) {
         const int b = i & 1;
         // input buffer b was last read by batch i - 2's forward; output buffer b last copied
         // out by batch i - 2's transfer
         if (i >= 2 && (cudaStreamWaitEvent(h2d, ev_comp[b], 0) != cudaSuccess ||
-                       cudaStreamWaitEvent(s, ev_out[b], 0) != cudaSuccess)) {
+                       cudaStreamWaitEvent(s, ev_out[2 * b], 0) != cudaSuccess ||
+                       cudaStreamWaitEvent(s, ev_out[2 * b + 1], 0) != cudaSuccess)) {
             st = MOE_ERR_CUDA;
             break;
         }
@@ -728,15 +734,25 @@ moe_status_t moe_forward_host(const moe_layer_desc *desc, int32_t n_batches, con
                                ws, L.x0, stream);
         if (st != MOE_OK)
             break;
-        if (cudaEventRecord(ev_comp[b], s) != cudaSuccess || cudaStreamWaitEvent(d2h, ev_comp[b], 0) != cudaSuccess ||
-            cudaMemcpyAsync(y_host + static_cast<size_t>(i) * xe, yd[b], xe * 4, cudaMemcpyDeviceToHost, d2h) !=
-                cudaSuccess ||
-            cudaEventRecord(ev_out[b], d2h) != cudaSuccess)
+        if (cudaEventRecord(ev_comp[b], s) != cudaSuccess) {
             st = MOE_ERR_CUDA;
+            break;
+        }
+        for (int hf = 0; hf < 2 && st == MOE_OK; ++hf) {
+            const size_t r0 = hf ? rows0 : 0, nr = hf ? desc->T - rows0 : rows0;
+            const size_t off = static_cast<size_t>(i) * xe + r0 * desc->H;
+            if (nr > 0 && (cudaStreamWaitEvent(d2h[hf], ev_comp[b], 0) != cudaSuccess ||
+                           cudaMemcpyAsync(y_host + off, yd[b] + r0 * desc->H, nr * desc->H * 4,
+                                           cudaMemcpyDeviceToHost, d2h[hf]) != cudaSuccess))
+                st = MOE_ERR_CUDA;
+            if (st == MOE_OK && cudaEventRecord(ev_out[2 * b + hf], d2h[hf]) != cudaSuccess)
+                st = MOE_ERR_CUDA;
+        }
     }
     // s completes after every transfer issued above (the copy streams are in order)
-    if (d2h && ev[0] && cudaEventRecord(ev_out[0], d2h) == cudaSuccess)
-        cudaStreamWaitEvent(s, ev_out[0], 0);
+    for (int hf = 0; hf < 2; ++hf)
+        if (d2h[hf] && ev[0] && cudaEventRecord(ev_out[hf], d2h[hf]) == cudaSuccess)
+            cudaStreamWaitEvent(s, ev_out[hf], 0);
     if (h2d && ev[0] && cudaEventRecord(ev_in[0], h2d) == cudaSuccess)
         cudaStreamWaitEvent(s, ev_in[0], 0);
     for (cudaEvent_t e : ev)
@@ -744,8 +760,9 @@ moe_status_t moe_forward_host(const moe_layer_desc *desc, int32_t n_batches, con
             cudaEventDestroy(e);
     if (h2d)
         cudaStreamDestroy(h2d);
-    if (d2h)
-        cudaStreamDestroy(d2h);
+    for (cudaStream_t d : d2h)
+        if (d)
+            cudaStreamDestroy(d);
     return st;
 }
 
