@@ -273,11 +273,11 @@ def run_reference(args, shape):
 
 
 # DRAM traffic (read + write) of one launch of the dominant kernel, as a ratio to the launch's
-# algorithmic bytes, from one ncu capture of a reduced case of the same shape per expert
-# (profiles/dram_gate_up_down_step5_skewed_T2048_E44.md: T=2048, E=44, the skewed Step-5
-# layer): the full launch's traffic is that ratio times its own algorithmic bytes. A figure
-# holds only for the kernel sources it was taken from: the lookup returns None once the code
-# of any file under csrc/ changes.
+# algorithmic bytes, from one ncu capture of a reduced case of the same shape per expert (the
+# profile named in each entry: T=2048, E=44 for the skewed Step-5 layer; T=1024, E=72 for the
+# Step-3.5 prefill layer): the full launch's traffic is that ratio times its own algorithmic
+# bytes. A figure holds only for the sources it was taken from: the lookup returns None once
+# the code of any file in TRAFFIC_SOURCES changes.
 PROFILED_TRAFFIC = {
     ("step5_skewed", "bf16"): {"ratio": (1450539008 + 51255552) / 1205862400,
                                "csrc_sha256": "f5dad4ee22b697d3d812c89b0052aa624b354519758885a58a935909f9ac4fde",
